@@ -1,0 +1,232 @@
+"""CPU oracle of one HARD-KV Cascade Cache decode step (numpy in, numpy out).
+
+TEST INFRASTRUCTURE ONLY. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg import this package. The CUDA library and its
+Python binding never import it; the two implementations share no code.
+
+The arithmetic lives in ``hkv_oracle.c`` (plain C, IEEE double); this module
+only marshals arrays. bf16 tensors travel as their raw 16-bit patterns
+(``numpy.uint16``); fp32 tensors as ``numpy.float32``.
+"""
+from __future__ import annotations
+
+import ctypes as C
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+
+from . import build as _build
+
+BF16, F32 = 0, 1
+PAD_MAX, FLAT_SUM = 0, 1
+
+_lib = None
+
+
+def lib(path: Optional[str] = None):
+    """Load (building first if needed) the oracle shared library."""
+    global _lib
+    if path is not None:
+        return _bind(C.CDLL(path))
+    if _lib is None:
+        _lib = _bind(C.CDLL(_build.build()))
+    return _lib
+
+
+class _Tier(C.Structure):
+    _fields_ = [
+        ("k", C.c_void_p), ("v", C.c_void_p),
+        ("sb", C.c_int64), ("sh", C.c_int64), ("st", C.c_int64),
+        ("cap", C.c_int32), ("len", C.c_void_p),
+    ]
+
+
+class _Dims(C.Structure):
+    _fields_ = [
+        ("B", C.c_int32), ("Hq", C.c_int32), ("Hkv", C.c_int32), ("D", C.c_int32),
+        ("dtype", C.c_int32), ("scale", C.c_double),
+    ]
+
+
+def _bind(L):
+    P = C.c_void_p
+    i32 = C.c_int32
+    L.hkvo_score.argtypes = [P, P, P, P, i32]
+    L.hkvo_calibrate.argtypes = [i32, P, i32, P, P, P, P, P]
+    L.hkvo_topp.argtypes = [i32, P, i32, P, P, C.c_float, P, i32, i32, P, P, P, P]
+    L.hkvo_compact.argtypes = [i32, P, i32, P, P, i32, i32, P, P]
+    L.hkvo_gather.argtypes = [P, P, P, P, i32, P, P]
+    L.hkvo_attend.argtypes = [P, P, P, P, P, P, i32, P, P, P]
+    L.hkvo_step.argtypes = [P, P, P, P, P, P, C.c_float, P, i32, i32, P, P, P, P, P]
+    for f in ("hkvo_score", "hkvo_calibrate", "hkvo_topp", "hkvo_compact", "hkvo_gather",
+              "hkvo_attend", "hkvo_step", "hkvo_num_threads"):
+        getattr(L, f).restype = C.c_int
+    return L
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data
+
+
+def _dtype_code(a: np.ndarray) -> int:
+    if a.dtype == np.uint16:
+        return BF16
+    if a.dtype == np.float32:
+        return F32
+    raise TypeError(f"oracle takes uint16 (bf16 bits) or float32, got {a.dtype}")
+
+
+@dataclass
+class Tier:
+    """One cache tier: K, V of shape [B, Hkv, cap, D] (D contiguous) and len[B*Hkv]."""
+
+    k: np.ndarray
+    v: np.ndarray
+    len: np.ndarray
+
+    def c(self, keep: list) -> _Tier:
+        k, v = self.k, self.v
+        assert k.shape == v.shape and k.strides == v.strides and k.ndim == 4
+        assert k.strides[3] == k.itemsize, "D must be contiguous"
+        ln = np.ascontiguousarray(self.len, dtype=np.int32)
+        keep += [k, v, ln]
+        es = k.itemsize
+        return _Tier(k.ctypes.data, v.ctypes.data, k.strides[0] // es, k.strides[1] // es,
+                     k.strides[2] // es, k.shape[2], ln.ctypes.data)
+
+
+def _dims(q: np.ndarray, Hkv: int, scale: float) -> _Dims:
+    B, Hq, D = q.shape
+    return _Dims(B, Hq, Hkv, D, _dtype_code(q), float(scale))
+
+
+def _ck(r: int, what: str):
+    if r != 0:
+        raise ValueError(f"oracle {what} failed with code {r}")
+
+
+def score(q: np.ndarray, sparse: Tier, scale: float) -> np.ndarray:
+    """S1: z[B*Hkv, cap] (entries past len are left at 0)."""
+    keep: list = []
+    q = np.ascontiguousarray(q)
+    t = sparse.c(keep)
+    d = _dims(q, sparse.k.shape[1], scale)
+    z = np.zeros((d.B * d.Hkv, t.cap), np.float32)
+    _ck(lib().hkvo_score(C.byref(d), _ptr(q), C.byref(t), _ptr(z), t.cap), "score")
+    return z
+
+
+def calibrate(z: np.ndarray, length: np.ndarray, beta: Optional[np.ndarray] = None,
+              want_P: bool = True):
+    """S2: (P or None, m, logZ) per unit."""
+    z = np.ascontiguousarray(z, np.float32)
+    ln = np.ascontiguousarray(length, np.int32)
+    units, zcap = z.shape
+    be = None if beta is None else np.ascontiguousarray(beta, np.float32)
+    P = np.zeros_like(z) if want_P else None
+    m = np.zeros(units, np.float32)
+    lz = np.zeros(units, np.float32)
+    _ck(lib().hkvo_calibrate(units, _ptr(z), zcap, _ptr(ln), _ptr(be), _ptr(P), _ptr(m),
+                             _ptr(lz)), "calibrate")
+    return P, m, lz
+
+
+def topp(z: np.ndarray, length: np.ndarray, p: float, bmin: int, bmax: int,
+         beta: Optional[np.ndarray] = None, p_unit: Optional[np.ndarray] = None) -> dict:
+    """S3: dict(k, kstar, c_before, c_at) per unit."""
+    z = np.ascontiguousarray(z, np.float32)
+    ln = np.ascontiguousarray(length, np.int32)
+    units, zcap = z.shape
+    be = None if beta is None else np.ascontiguousarray(beta, np.float32)
+    pu = None if p_unit is None else np.ascontiguousarray(p_unit, np.float32)
+    k = np.zeros(units, np.int32)
+    ks = np.zeros(units, np.int32)
+    cb = np.zeros(units, np.float64)
+    ca = np.zeros(units, np.float64)
+    _ck(lib().hkvo_topp(units, _ptr(z), zcap, _ptr(ln), _ptr(be), float(p), _ptr(pu), int(bmin),
+                        int(bmax), _ptr(k), _ptr(ks), _ptr(cb), _ptr(ca)), "topp")
+    return {"k": k, "kstar": ks, "c_before": cb, "c_at": ca}
+
+
+def compact(z: np.ndarray, length: np.ndarray, sel_len: np.ndarray, bmax: int,
+            layout: int = PAD_MAX):
+    """S4: PAD_MAX -> idx[units, bmax]; FLAT_SUM -> (flat idx, offsets[units+1])."""
+    z = np.ascontiguousarray(z, np.float32)
+    ln = np.ascontiguousarray(length, np.int32)
+    k = np.ascontiguousarray(sel_len, np.int32)
+    units, zcap = z.shape
+    if layout == PAD_MAX:
+        idx = np.zeros((units, bmax), np.int32)
+        off = None
+    else:
+        idx = np.full(max(int(k.sum()), 1), -7, np.int32)
+        off = np.zeros(units + 1, np.int32)
+    _ck(lib().hkvo_compact(units, _ptr(z), zcap, _ptr(ln), _ptr(k), int(bmax), int(layout),
+                           _ptr(idx), _ptr(off)), "compact")
+    if layout == PAD_MAX:
+        return idx
+    return idx[: int(off[-1])], off
+
+
+def gather(sparse: Tier, idx: np.ndarray, sel_len: np.ndarray, bmax: int, Hq: int = 1):
+    """S4 Rewrite Cache: (Kc, Vc) of shape [units, bmax, D] (rows past sel_len are 0)."""
+    keep: list = []
+    t = sparse.c(keep)
+    B, Hkv, _, D = sparse.k.shape
+    d = _Dims(B, Hkv * Hq, Hkv, D, _dtype_code(sparse.k), 1.0)
+    idx = np.ascontiguousarray(idx, np.int32)
+    k = np.ascontiguousarray(sel_len, np.int32)
+    kc = np.zeros((B * Hkv, bmax, D), sparse.k.dtype)
+    vc = np.zeros((B * Hkv, bmax, D), sparse.k.dtype)
+    _ck(lib().hkvo_gather(C.byref(d), C.byref(t), _ptr(idx), _ptr(k), int(bmax), _ptr(kc),
+                          _ptr(vc)), "gather")
+    return kc, vc
+
+
+def attend(q: np.ndarray, dense: Optional[Tier], sparse: Optional[Tier],
+           idx: Optional[np.ndarray], sel_len: Optional[np.ndarray], bmax: int,
+           condensed: Optional[Tier], scale: float, Hkv: Optional[int] = None):
+    """S5: (out[B, Hq, D] fp32, lse[B, Hq] fp32)."""
+    keep: list = []
+    q = np.ascontiguousarray(q)
+    tiers = [t for t in (dense, sparse, condensed) if t is not None]
+    if Hkv is None:
+        Hkv = tiers[0].k.shape[1]
+    d = _dims(q, Hkv, scale)
+    ct = [None if t is None else t.c(keep) for t in (dense, sparse, condensed)]
+    idx = None if idx is None else np.ascontiguousarray(idx, np.int32)
+    k = None if sel_len is None else np.ascontiguousarray(sel_len, np.int32)
+    out = np.zeros(q.shape, np.float32)
+    lse = np.zeros(q.shape[:2], np.float32)
+    refs = [None if t is None else C.byref(t) for t in ct]
+    _ck(lib().hkvo_attend(C.byref(d), _ptr(q), refs[0], refs[1], _ptr(idx), _ptr(k), int(bmax),
+                          refs[2], _ptr(out), _ptr(lse)), "attend")
+    return out, lse
+
+
+def step(q: np.ndarray, dense: Optional[Tier], sparse: Tier, condensed: Optional[Tier],
+         scale: float, p: float, bmin: int, bmax: int, beta: Optional[np.ndarray] = None,
+         p_unit: Optional[np.ndarray] = None) -> dict:
+    """S1..S5: dict(z, k, idx, out, lse)."""
+    keep: list = []
+    q = np.ascontiguousarray(q)
+    d = _dims(q, sparse.k.shape[1], scale)
+    ct = [None if t is None else t.c(keep) for t in (dense, sparse, condensed)]
+    units = d.B * d.Hkv
+    z = np.zeros((units, ct[1].cap), np.float32)
+    k = np.zeros(units, np.int32)
+    idx = np.zeros((units, bmax), np.int32)
+    out = np.zeros(q.shape, np.float32)
+    lse = np.zeros(q.shape[:2], np.float32)
+    be = None if beta is None else np.ascontiguousarray(beta, np.float32)
+    pu = None if p_unit is None else np.ascontiguousarray(p_unit, np.float32)
+    refs = [None if t is None else C.byref(t) for t in ct]
+    _ck(lib().hkvo_step(C.byref(d), _ptr(q), refs[0], refs[1], refs[2], _ptr(be), float(p),
+                        _ptr(pu), int(bmin), int(bmax), _ptr(z), _ptr(k), _ptr(idx), _ptr(out),
+                        _ptr(lse)), "step")
+    return {"z": z, "k": k, "idx": idx, "out": out, "lse": lse}
+
+
+def num_threads() -> int:
+    return int(lib().hkvo_num_threads())

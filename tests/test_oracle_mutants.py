@@ -1,0 +1,78 @@
+"""Planted mistakes in the CPU oracle must each break at least one pin.
+
+Each mutant is a copy of ``oracle/hkv_oracle.c`` with one plausible mistake
+(a dropped term, a wrong sign, index or comparison), compiled on the CPU into a
+temporary library. The pins of ``tests/pins.py`` run against it; at least one
+must fail, which shows the pins constrain that part of the oracle.
+"""
+import os
+import shutil
+
+import pytest
+
+import oracle
+from oracle import build as obuild
+from tests import pins
+
+MUTANTS = {
+    "gqa_group_mapping": ("h * G + g, sp, h, j)", "g * d->Hkv + h, sp, h, j)"),
+    "score_scale_dropped": ("double s = d->scale * dot_qk(d, q, b, h * G + g, sp, h, j);",
+                            "double s = dot_qk(d, q, b, h * G + g, sp, h, j);"),
+    "pool_min_not_max": ("if (s > best)\n                    best = s;",
+                         "if (s < best || best == -INFINITY)\n                    best = s;"),
+    "bf16_widen_shift": ("(uint32_t)bits << 16", "(uint32_t)bits << 15"),
+    "calib_beta_dropped": ("return exp(beta * ((double)zj - (double)m));",
+                           "return exp(((double)zj - (double)m));"),
+    "calib_sign": ("return exp(beta * ((double)zj - (double)m));",
+                   "return exp(beta * ((double)m - (double)zj));"),
+    "calib_not_normalised": ("(float)(calib_weight(zu[j], mu, bu) / Z)",
+                             "(float)(calib_weight(zu[j], mu, bu))"),
+    "tie_higher_index_first": ("return (x->j > y->j) - (x->j < y->j);",
+                               "return (x->j < y->j) - (x->j > y->j);"),
+    "order_ascending": ("if (x->z > y->z)\n        return -1;\n    if (x->z < y->z)\n        return 1;",
+                        "if (x->z > y->z)\n        return 1;\n    if (x->z < y->z)\n        return -1;"),
+    "mass_strictly_above_p": ("if (C >= (double)p) {", "if (C > (double)p) {"),
+    "kstar_off_by_one": ("kstar = i + 1;", "kstar = i;"),
+    "no_cap_at_n": ("if (k > n)\n        k = n;", "if (k > n + 1000000)\n        k = n;"),
+    "bmin_ignored": ("if (k < bmin)\n        k = bmin;", "if (k < 0)\n        k = bmin;"),
+    "bmax_ignored": ("int32_t k = kstar < bmax ? kstar : bmax;", "int32_t k = kstar;"),
+    "rows_not_index_sorted": ("qsort(row, (size_t)k, sizeof(int32_t), by_index);", ";"),
+    "flat_offsets_not_scanned": ("offsets[u + 1] = offsets[u] + sel_len[u];",
+                                 "offsets[u + 1] = sel_len[u];"),
+    "condensed_tier_dropped": [("int32_t T = W + k + C;", "int32_t T = W + k;"),
+                               ("for (int32_t j = 0; j < C; ++j)\n            toks[t++] = (token_ref){condensed, j};",
+                                "for (int32_t j = 0; j < 0; ++j)\n            toks[t++] = (token_ref){condensed, j};")],
+    "lse_missing_max": ("(float)(M + log(L))", "(float)(log(L))"),
+    "attention_v_from_k": ("elem(toks[i].t->v, d->dtype, vo + x)", "elem(toks[i].t->k, d->dtype, vo + x)"),
+}
+
+
+@pytest.fixture(scope="module")
+def src_text():
+    with open(obuild.SRC) as f:
+        return f.read()
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, src_text, tmp_path, monkeypatch):
+    edits = MUTANTS[name]
+    if isinstance(edits, tuple):
+        edits = [edits]
+    mutated = src_text
+    for old, new in edits:
+        assert mutated.count(old) >= 1, f"mutation site for {name} not found"
+        mutated = mutated.replace(old, new)
+    src = tmp_path / "hkv_oracle.c"
+    src.write_text(mutated)
+    shutil.copy(os.path.join(obuild.HERE, "hkv_oracle.h"), tmp_path / "hkv_oracle.h")
+    so = str(tmp_path / f"libhkv_oracle_{name}.so")
+    obuild.build(force=True, src=str(src), out=so, extra=("-I", str(tmp_path)))
+    monkeypatch.setattr(oracle, "_lib", oracle.lib(so))
+    caught = []
+    for pin in pins.ALL_PINS:
+        try:
+            pin()
+        except (AssertionError, ValueError) as e:  # a pin failed or the oracle refused
+            caught.append((pin.__name__, type(e).__name__))
+            break
+    assert caught, f"mutant {name} passed every pin"
