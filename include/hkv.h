@@ -1,0 +1,238 @@
+/*
+ * hkv.h -- C ABI of the B200 (sm_100a) library for the decode-time hot path of
+ * HARD-KV's Cascade Cache.
+ *
+ * Sources named in the comments:
+ *   [Abstract] arXiv abstract on the mlsanity.com page "HARD-KV: Head-Adaptive
+ *              Regularization for Decoding-time KV Compression".
+ *   [TS 2.A]   gist.science Technical Summary of that paper, section 2.A
+ *              "Cascade Cache Hierarchy"; [TS 2.B] "Logits Calibration
+ *              Mechanism"; [TS 2.C] "System-Aware Index Regularization";
+ *              [TS 3] "Key Contributions"; [TS 5] "Significance and Claims".
+ *
+ * Conventions shared by every entry point
+ * ----------------------------------------
+ * - Memory: the caller owns all memory. Pointers marked "device" must be
+ *   device-accessible (cudaMalloc or torch CUDA tensors) on the current device;
+ *   pointers marked "host" are host memory. The library never allocates, frees
+ *   or synchronises on the compute path (hkv_get_status is the one call that
+ *   synchronises). Every compute call is asynchronous on `stream` and can be
+ *   captured in a CUDA graph: shapes are static and every length, budget and
+ *   temperature that changes from step to step is read on the device
+ *   ([TS 2.C] Head-wise Block Manager: static tensor shapes and persistent
+ *   pointers; [TS 5] CUDA Graph compatibility over many decoding steps).
+ * - A *unit* is one KV head of one sequence, u = b*Hkv + h. Per-unit arrays are
+ *   length B*Hkv in that order.
+ * - Query head h*G + g (g < G = Hq/Hkv) attends through KV head h.
+ * - A tier stores K and V as [B, Hkv, cap, D] with D contiguous and element
+ *   strides (stride_b, stride_h, stride_t); rows must start on 16-byte
+ *   boundaries (base pointers 16-byte aligned, strides multiples of 8 bf16 or
+ *   4 fp32 elements).
+ * - Return codes report host-side validation and CUDA launch errors only; a
+ *   call that returns an error has launched nothing unless it says otherwise.
+ *   Conditions found on the device (a length above its capacity, a bounded
+ *   wait that ran out, a negative temperature) set bits in a status word in
+ *   the workspace, read by hkv_get_status. No exception crosses the ABI.
+ * - Scores and Top-p selection follow one fixed rule: tokens are ordered by
+ *   score descending, ties by lower token index (-0 equals +0); the budget is
+ *   the fewest tokens whose calibrated mass is at least p, clamped to
+ *   [bmin, bmax] and to the tokens present.
+ */
+#ifndef HKV_H
+#define HKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *hkv_stream_t;
+
+typedef enum {
+    HKV_OK = 0,
+    HKV_ERR_INVALID_ARG = 1,  /* a pointer, shape, stride, alignment or value is invalid */
+    HKV_ERR_UNSUPPORTED = 2,  /* valid but not built: D not in {64,128}, G not in {1,2,4,8} */
+    HKV_ERR_CUDA = 3,         /* a CUDA runtime call failed (launch, copy, attribute) */
+    HKV_ERR_TIMEOUT = 4,      /* hkv_get_status: a bounded device wait ran out */
+    HKV_ERR_DEVICE = 5,       /* hkv_get_status: another device-side condition (see flags) */
+    HKV_ERR_WORKSPACE = 6     /* workspace pointer missing, misaligned or too small */
+} hkv_status;
+
+typedef enum { HKV_BF16 = 0, HKV_F32 = 1 } hkv_dtype;
+
+/* [TS 2.C] Flatten Index: indices regularised to the maximum length or to the
+ * sum of the lengths. */
+typedef enum {
+    HKV_LAYOUT_PAD_MAX = 0,   /* idx[u*bmax + i], rows padded with -1 */
+    HKV_LAYOUT_FLAT_SUM = 1   /* idx[offsets[u] + i], offsets[B*Hkv+1] */
+} hkv_layout;
+
+/* Device status-word bits (hkv_get_status). */
+#define HKV_DEV_LEN_CLAMPED  0x1u  /* a per-unit length exceeded its capacity; clamped */
+#define HKV_DEV_TIMEOUT      0x2u  /* a bounded wait ran out; outputs of that call invalid */
+#define HKV_DEV_BAD_TEMP     0x4u  /* a negative or NaN inverse temperature; 1 used */
+#define HKV_DEV_BAD_INDEX    0x8u  /* an index or budget outside its range; row 0 / a clamp used */
+#define HKV_DEV_BAD_P        0x10u /* a NaN per-unit p; p = 1 used */
+
+/* One cache tier ([TS 2.A]: dense recent window, sparse tier, condensed slots). */
+typedef struct {
+    const void *k;            /* device, [B, Hkv, cap, D] */
+    const void *v;            /* device, same shape and strides as k (may be NULL for
+                                 calls that read only keys: hkv_score, hkv_compact without
+                                 rewrite) */
+    int64_t stride_b, stride_h, stride_t;  /* element strides; D is contiguous */
+    int32_t cap;              /* token capacity per unit (0 <= len <= cap) */
+    const int32_t *len;       /* device [B*Hkv], valid tokens per unit */
+} hkv_tier;
+
+/* The problem statement of one decode step of one layer. */
+typedef struct {
+    int32_t B, Hq, Hkv, D;    /* sequences, query heads, KV heads, head dim (64 or 128) */
+    hkv_dtype dtype;          /* element type of q, K, V */
+    float scale;              /* logit scale; 0 selects 1/sqrt(D) */
+    float p;                  /* Top-p mass ([Abstract]); used when p_unit is NULL */
+    int32_t bmin, bmax;       /* budget clamps, 0 <= bmin <= bmax ([TS 2.A] hard limits) */
+    hkv_layout layout;        /* compacted index layout */
+    const float *inv_temp;    /* device [B*Hkv] Logits Calibration inverse temperature
+                                 beta ([TS 2.B]); NULL = 1 everywhere */
+    const float *p_unit;      /* device [B*Hkv] per-unit p; NULL = use p */
+} hkv_problem;
+
+/* Per-unit cut of the Top-p selection, produced by hkv_topp_select and read by
+ * hkv_compact. The selected set is every token whose score is above z_cut, plus
+ * the first n_tie tokens (in index order) whose score equals z_cut. */
+typedef struct {
+    float z_cut;              /* score of the last selected token (0 if k = 0) */
+    int32_t n_above;          /* selected tokens scoring above z_cut */
+    int32_t n_tie;            /* selected tokens scoring exactly z_cut */
+    int32_t kstar;            /* unclamped Top-p budget, or -1 when the clamp decided
+                                 k without computing it */
+} hkv_cut;
+
+/* Outputs of hkv_step. Optional pointers may be NULL. */
+typedef struct {
+    int32_t *sel_len;         /* device [B*Hkv], budget k per unit (required) */
+    int32_t *idx;             /* device, layout of problem.layout (required):
+                                 PAD_MAX [B*Hkv*bmax]; FLAT_SUM [B*Hkv*bmax] capacity */
+    int32_t *offsets;         /* device [B*Hkv+1], FLAT_SUM only (required there) */
+    float *out;               /* device [B, Hq, D] fp32 attention output (required) */
+    float *lse;               /* device [B, Hq] fp32 natural-log sum of exp (optional) */
+    float *z;                 /* device [B*Hkv, sparse.cap] fp32 scores (optional) */
+    hkv_cut *cut;             /* device [B*Hkv] (optional) */
+    float *m;                 /* device [B*Hkv] max score (optional) */
+    float *logZ;              /* device [B*Hkv] log of the calibration normaliser (optional) */
+    void *k_out, *v_out;      /* device Rewrite Cache rows in the idx layout:
+                                 PAD_MAX [B*Hkv, bmax, D]; FLAT_SUM [B*Hkv*bmax, D] (optional,
+                                 both or neither) */
+} hkv_step_out;
+
+/* Size in bytes of the workspace the calls below need for this problem and
+ * these tier capacities (it depends on shapes only, never on lengths). Host
+ * pointers; tiers may be NULL for an empty tier. */
+hkv_status hkv_workspace_size(const hkv_problem *prob, const hkv_tier *dense,
+                              const hkv_tier *sparse, const hkv_tier *condensed,
+                              size_t *bytes);
+
+/* Zero a workspace (asynchronous memset on `stream`). Required once before its
+ * first use, and again after a call whose status reported HKV_DEV_TIMEOUT. */
+hkv_status hkv_workspace_init(void *ws, size_t bytes, hkv_stream_t stream);
+
+/* S1 Score ([TS 2.B] max-pooled attention logits; [TS 2.A] Tier 2):
+ * z[u*z_stride + j] = scale * max_g q[b, h*G+g, :] . K_sparse[b, h, j, :] for
+ * j < len[u], fp32 accumulation from bf16/fp32 inputs. q: device [B, Hq, D].
+ * z: device, 4-byte aligned; z_stride >= sparse->cap. Entries past len[u] are
+ * not written. */
+hkv_status hkv_score(const hkv_problem *prob, const void *q, const hkv_tier *sparse,
+                     float *z, int64_t z_stride, void *ws, size_t ws_bytes,
+                     hkv_stream_t stream);
+
+/* S2 Logits Calibration ([TS 2.B], [TS 3]): per unit m = max_j z_j,
+ * Z = sum_j exp(beta (z_j - m)), logZ = ln Z, and optionally
+ * P[u*z_stride + j] = exp(beta (z_j - m)) / Z. sparse supplies the lengths
+ * (its K/V are not read). m, logZ: device [B*Hkv]; P may be NULL. An empty unit
+ * gives m = -inf, logZ = -inf. Z is summed in exact fixed point, as in
+ * hkv_topp_select. */
+hkv_status hkv_calibrate(const hkv_problem *prob, const float *z, int64_t z_stride,
+                         const hkv_tier *sparse, float *P, float *m, float *logZ,
+                         void *ws, size_t ws_bytes, hkv_stream_t stream);
+
+/* S3 Top-p budget ([Abstract], [TS 2.A], [TS 2.B]): per unit the budget
+ * sel_len[u] = min(n, max(bmin, min(k*, bmax))), k* the fewest tokens (score
+ * descending, lower index first) whose calibrated mass is at least p, and the
+ * cut that identifies the set. Masses are summed as exact 40-bit fixed-point
+ * weights, so the result is deterministic. sparse supplies the lengths.
+ * sel_len, cut: device [B*Hkv]. */
+hkv_status hkv_topp_select(const hkv_problem *prob, const float *z, int64_t z_stride,
+                           const hkv_tier *sparse, int32_t *sel_len, hkv_cut *cut,
+                           void *ws, size_t ws_bytes, hkv_stream_t stream);
+
+/* S4 Index Regularization ([TS 2.C] Flatten Index, Rewrite Cache): writes the
+ * selected tokens of each unit in ascending index order into idx (layout of
+ * prob->layout; PAD_MAX rows padded with -1; FLAT_SUM offsets = exclusive scan
+ * of sel_len over units). If k_out and v_out are given, also copies the selected
+ * K/V rows bit for bit into them, in the same layout (rows of D elements).
+ * sparse supplies len (and K/V for the rewrite). */
+hkv_status hkv_compact(const hkv_problem *prob, const float *z, int64_t z_stride,
+                       const hkv_tier *sparse, const int32_t *sel_len, const hkv_cut *cut,
+                       int32_t *idx, int32_t *offsets, void *k_out, void *v_out,
+                       void *ws, size_t ws_bytes, hkv_stream_t stream);
+
+/* S5 Cascade decode attention ([TS 2.A] three tiers; [Abstract]): for each
+ * query head, softmax attention (scale * q.k) over dense[0, len) ++
+ * sparse[idx_0 .. idx_{k-1}] ++ condensed[0, len), split across CTAs and merged
+ * by online softmax. out: device [B, Hq, D] fp32; lse: device [B, Hq] fp32 or
+ * NULL. idx/offsets in prob->layout with k = sel_len[u]. An empty token list
+ * gives out = 0, lse = -inf. Any tier may be NULL (empty). ws: workspace of
+ * hkv_workspace_size bytes, zeroed once by hkv_workspace_init. */
+hkv_status hkv_cascade_decode(const hkv_problem *prob, const void *q,
+                              const hkv_tier *dense, const hkv_tier *sparse,
+                              const int32_t *idx, const int32_t *offsets,
+                              const int32_t *sel_len, const hkv_tier *condensed,
+                              float *out, float *lse, void *ws, size_t ws_bytes,
+                              hkv_stream_t stream);
+
+/* S1..S5 fused ([TS 2.A] pipeline steps 2 and 3 plus decoding): one persistent
+ * kernel scores every sparse token, calibrates, takes the Top-p budget and
+ * compacts each unit as soon as its last score tile lands, and runs the split
+ * attention tiles of the units whose selection is published; the last tile of
+ * a unit merges it. Attention reads the selected rows through the indices
+ * ([TS 2.C] Sparse Loading); k_out/v_out add the Rewrite Cache copy. ws as for
+ * hkv_cascade_decode. */
+hkv_status hkv_step(const hkv_problem *prob, const void *q, const hkv_tier *dense,
+                    const hkv_tier *sparse, const hkv_tier *condensed,
+                    const hkv_step_out *out, void *ws, size_t ws_bytes,
+                    hkv_stream_t stream);
+
+/* Every compute call takes a workspace `ws` of at least hkv_workspace_size
+ * bytes (256-byte aligned, zeroed once by hkv_workspace_init); its first word
+ * is the device status word. Calls that overlap on the GPU need separate
+ * workspaces. */
+
+/* Read and clear the device status word of a workspace. Synchronises `stream`.
+ * *flags (host, may be NULL) receives the HKV_DEV_* bits. Returns HKV_OK when
+ * no bit is set, HKV_ERR_TIMEOUT when HKV_DEV_TIMEOUT is set, else
+ * HKV_ERR_DEVICE. */
+hkv_status hkv_get_status(void *ws, uint32_t *flags, hkv_stream_t stream);
+
+/* Upper bound, in nanoseconds, of every spin-wait inside the library's kernels
+ * (default 1e9). Takes effect at the next launch. */
+hkv_status hkv_set_wait_limit_ns(uint64_t ns);
+
+/* Fault injection for tests: when nonzero, the fused step never publishes a
+ * unit's selection, so every attention tile's bounded wait runs out and the
+ * status word gets HKV_DEV_TIMEOUT. Takes effect at the next launch. */
+hkv_status hkv_debug_withhold_publish(int32_t on);
+
+/* Kernel launches this library has issued in this process (all devices). */
+uint64_t hkv_launch_count(void);
+
+/* Human-readable name of a status code (static string). */
+const char *hkv_status_string(hkv_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HKV_H */

@@ -1,0 +1,124 @@
+"""Helpers of the GPU parity tests: inputs on the device, the same inputs on the
+host for the oracle, and the acceptance rules of the selection."""
+from __future__ import annotations
+
+import math
+from typing import Optional
+
+import numpy as np
+import scipy.special as sps
+import torch
+
+import oracle
+from head_adaptive_kv_b200 import hkv
+from head_adaptive_kv_b200.workloads import TierTensors, Workload, make_inputs, to_host_bits
+
+# Attention outputs: fp32 accumulation from bf16/fp32 inputs against the fp64
+# oracle, elementwise |a - b| <= ATOL + RTOL |b|.
+ATOL, RTOL = 2e-3, 1e-2
+# Ambiguous cut: the oracle's prefix mass is this close to p on either side of k*.
+AMBIG = 1e-5
+# End to end a token may flip only if its calibrated probability is this close
+# to the probability of the oracle's last selected token.
+P_FLIP = 1e-6
+
+
+def dev():
+    return torch.device("cuda:0")
+
+
+def tiers_of(x):
+    return [hkv.Tier(t.k, t.v, t.len) for t in (x.dense, x.sparse, x.condensed)]
+
+
+def problem_of(wl: Workload, p=None, bmin=None, bmax=None, layout=hkv.PAD_MAX, inv_temp=None, p_unit=None):
+    return hkv.Problem(wl.B, wl.Hq, wl.Hkv, wl.D, wl.dtype, wl.p if p is None else p,
+                       wl.bmin if bmin is None else bmin, wl.bmax if bmax is None else bmax,
+                       layout=layout, inv_temp=inv_temp, p_unit=p_unit)
+
+
+def host_tier(t: TierTensors, b: Optional[slice] = None) -> oracle.Tier:
+    k, v, ln = t.k, t.v, t.len
+    if b is not None:
+        Hkv = k.shape[1]
+        k, v = k[b], v[b]
+        ln = ln.view(-1, Hkv)[b].reshape(-1)
+    return oracle.Tier(to_host_bits(k), to_host_bits(v), ln.cpu().numpy().astype(np.int32))
+
+
+def score_bound(q: np.ndarray, k: np.ndarray, ln: np.ndarray, G: int, scale: float) -> np.ndarray:
+    """Worst-case error of an fp32 dot product of length D with exact products:
+    D * 2^-24 * scale * max_g sum_d |q_gd k_jd| (plus one final rounding)."""
+    from tests.helpers import as_f64
+
+    qa = np.abs(as_f64(q))
+    ka = np.abs(as_f64(k))
+    B, Hkv, cap, D = ka.shape
+    qa = qa.reshape(B, Hkv, G, D)
+    s = np.einsum("bhgd,bhnd->bhgn", qa, ka).max(axis=2) * scale
+    return (D * 2.0 ** -24 * s + 2.0 ** -22 * s).reshape(B * Hkv, cap)
+
+
+def selection_ok(z_ref: np.ndarray, n: int, k_gpu: int, idx_gpu: np.ndarray, p: float, bmin: int, bmax: int,
+                 beta: float = 1.0) -> tuple:
+    """End-to-end rule: budgets equal except at an ambiguous cut; every token in
+    the symmetric difference of the sets has |P_j - P_cut| <= P_FLIP."""
+    z = z_ref[:n].astype(np.float64)
+    r = oracle.topp(z_ref[None, :n].astype(np.float32), np.array([n], np.int32), p, bmin, bmax,
+                    np.array([beta], np.float32))
+    k_ref = int(r["k"][0])
+    amb = (abs(r["c_before"][0] - p) < AMBIG) or (abs(r["c_at"][0] - p) < AMBIG)
+    if k_gpu != k_ref and not (amb and abs(k_gpu - k_ref) <= 1):
+        return False, f"k {k_gpu} vs oracle {k_ref} (not an ambiguous cut)"
+    if n == 0:
+        return True, ""
+    P = sps.softmax(beta * z)
+    order = np.lexsort((np.arange(n), -(z + 0.0)))
+    ref_set = set(order[:k_ref].tolist())
+    gpu_set = set(int(j) for j in idx_gpu[:k_gpu])
+    if len(gpu_set) != k_gpu or any(j < 0 or j >= n for j in gpu_set):
+        return False, "GPU row has repeats or out-of-range tokens"
+    if list(idx_gpu[:k_gpu]) != sorted(gpu_set):
+        return False, "GPU row not in ascending token order"
+    if k_ref == 0:
+        return (len(gpu_set) <= 1), "k_ref = 0"
+    p_cut = P[order[k_ref - 1]]
+    diff = ref_set ^ gpu_set
+    bad = [j for j in diff if abs(P[j] - p_cut) > P_FLIP]
+    if bad:
+        return False, f"{len(bad)} tokens flipped away from the cut (e.g. {bad[:3]})"
+    return True, f"{len(diff)} flipped at the cut"
+
+
+def attn_close(out, ref):
+    out = np.asarray(out, np.float64)
+    ref = np.asarray(ref, np.float64)
+    fin = np.isfinite(ref)
+    same_inf = np.array_equal(np.isneginf(out), np.isneginf(ref))
+    err = np.abs(out[fin] - ref[fin])
+    ok = same_inf and bool(np.all(err <= ATOL + RTOL * np.abs(ref[fin])))
+    return ok, (float(err.max()) if err.size else 0.0)
+
+
+def run_step(wl: Workload, x, p=None, bmin=None, bmax=None, layout=hkv.PAD_MAX, with_z=True,
+             with_cut=True, rewrite=False, inv_temp=None, p_unit=None):
+    prob = problem_of(wl, p, bmin, bmax, layout, inv_temp, p_unit)
+    tiers = tiers_of(x)
+    ws = hkv.Workspace(prob, *tiers)
+    out = hkv.StepOutputs.allocate(prob, tiers[1], dev(), with_z=with_z, with_cut=with_cut,
+                                   with_stats=True, rewrite=rewrite)
+    hkv.step(prob, x.q, *tiers, out, ws)
+    torch.cuda.synchronize()
+    return prob, out, ws
+
+
+def scale_of(wl: Workload) -> float:
+    return 1.0 / math.sqrt(wl.D)
+
+
+def small(wl: Workload, **kw) -> Workload:
+    return wl.with_(**kw)
+
+
+def inputs(wl: Workload, layer: int = 0):
+    return make_inputs(wl, dev(), layer)

@@ -1,0 +1,108 @@
+"""The C ABI library loads, exports every entry point of include/hkv.h and
+validates arguments on the host (these calls launch nothing, so no GPU is used)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+import torch
+
+from head_adaptive_kv_b200 import build as hbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def hk():
+    hbuild.build()
+    from head_adaptive_kv_b200 import hkv
+
+    return hkv
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "hkv.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(hkv_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(hk):
+    names = declared_symbols()
+    assert len(names) == 13, names
+    for n in names:
+        assert hasattr(hk.lib, n), n
+    nm = os.popen(f"nm -D --defined-only {hk.LIB_PATH}").read()
+    for n in names:
+        assert re.search(rf"\bT {n}\b", nm), f"{n} not exported"
+
+
+def _prob(hk, **kw):
+    d = dict(B=2, Hq=8, Hkv=2, D=128, dtype=torch.bfloat16, p=0.9, bmin=4, bmax=64)
+    d.update(kw)
+    return hk.Problem(**d)
+
+
+def _tier(hk, cap, addr=0x10000):
+    t = hk._Tier(addr, addr + 0x100000, 2 * 128 * cap, 128 * cap, 128, cap, 0x2000)
+    return t
+
+
+def _ws_size(hk, prob, dense, sparse, cond):
+    n = C.c_size_t(0)
+    code = hk.lib.hkv_workspace_size(C.byref(prob.c()), dense and C.byref(dense), C.byref(sparse),
+                                     cond and C.byref(cond), C.byref(n))
+    return code, n.value
+
+
+def test_workspace_size_and_validation(hk):
+    d, s, c = _tier(hk, 64), _tier(hk, 1000), _tier(hk, 16)
+    code, n = _ws_size(hk, _prob(hk), d, s, c)
+    assert code == 0 and n > 0 and n % 256 == 0
+    # the workspace depends on capacities only and grows with them
+    code2, n2 = _ws_size(hk, _prob(hk), d, _tier(hk, 4000), c)
+    assert code2 == 0 and n2 > n
+    cases = {
+        "bmin > bmax": (_prob(hk, bmin=10, bmax=5), 1),
+        "Hq % Hkv": (_prob(hk, Hq=7), 1),
+        "D 96": (_prob(hk, D=96), 2),
+        "G 3": (_prob(hk, Hq=6), 2),
+        "p NaN": (_prob(hk, p=float("nan")), 1),
+        "negative scale": (_prob(hk, scale=-1.0), 1),
+    }
+    for what, (prob, want) in cases.items():
+        assert _ws_size(hk, prob, d, s, c)[0] == want, what
+    assert hk.lib.hkv_workspace_size(None, None, None, None, None) == 1
+    bad = _tier(hk, 64, addr=0x10008)  # misaligned base
+    assert _ws_size(hk, _prob(hk), bad, s, c)[0] == 1
+    odd = hk._Tier(0x10000, 0x20000, 1, 1, 130, 64, 0x2000)  # stride_t not a 16-byte multiple
+    assert _ws_size(hk, _prob(hk), odd, s, c)[0] == 1
+
+
+def test_compute_calls_reject_bad_workspace_without_launching(hk):
+    prob = _prob(hk)
+    s = _tier(hk, 1000)
+    before = hk.launch_count()
+    z = 0x40000
+    # workspace missing / misaligned / too small -> HKV_ERR_WORKSPACE
+    assert hk.lib.hkv_score(C.byref(prob.c()), 0x1000, C.byref(s), z, 1000, None, 0, None) == 6
+    assert hk.lib.hkv_score(C.byref(prob.c()), 0x1000, C.byref(s), z, 1000, 0x100010, 1 << 30, None) == 6
+    assert hk.lib.hkv_score(C.byref(prob.c()), 0x1000, C.byref(s), z, 1000, 0x100000, 256, None) == 6
+    # z row stride below capacity -> invalid
+    assert hk.lib.hkv_score(C.byref(prob.c()), 0x1000, C.byref(s), z, 999, 0x100000, 1 << 30, None) == 1
+    # misaligned q
+    assert hk.lib.hkv_score(C.byref(prob.c()), 0x1008, C.byref(s), z, 1000, 0x100000, 1 << 30, None) == 1
+    assert hk.launch_count() == before
+
+
+def test_status_strings(hk):
+    assert hk.status_string(0) == "HKV_OK"
+    assert hk.status_string(4) == "HKV_ERR_TIMEOUT"
+    assert hk.status_string(99) == "HKV_ERR_UNKNOWN"
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
+def test_valid_call_without_gpu_fails_cleanly(hk):
+    prob = _prob(hk)
+    s = _tier(hk, 1000)
+    code = hk.lib.hkv_score(C.byref(prob.c()), 0x1000, C.byref(s), 0x40000, 1000, 0x100000, 1 << 30, None)
+    assert code == 3  # HKV_ERR_CUDA, not a crash

@@ -1,0 +1,201 @@
+"""End-to-end parity of the fused decode step (hkv_step) against the CPU oracle,
+on small cases and on the full-size workloads."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from head_adaptive_kv_b200 import hkv
+from head_adaptive_kv_b200.workloads import WORKLOADS, make_inputs, to_host_bits
+from tests import gpu_helpers as H
+from tests.test_gpu_stages import CASES
+
+pytestmark = pytest.mark.gpu
+
+
+def check_step(wl, x, out, p, bmin, bmax, b_sel=None, beta=None, tag=""):
+    """z within the fp32 bound, selection by the end-to-end rule, attention over
+    the GPU's selection within tolerance. b_sel: sequences to check (all)."""
+    bs = range(wl.B) if b_sel is None else b_sel
+    scale = H.scale_of(wl)
+    z_all = out.z.cpu().numpy() if out.z is not None else None
+    k_all = out.sel_len.cpu().numpy()
+    idx_all = out.idx.cpu().numpy().reshape(wl.units, wl.bmax if bmax is None else bmax)
+    o_all = out.out.cpu().numpy()
+    l_all = out.lse.cpu().numpy()
+    for b in bs:
+        sl = slice(b, b + 1)
+        q = to_host_bits(x.q[sl])
+        sp = H.host_tier(x.sparse, sl)
+        zr = oracle.score(q, sp, scale)
+        ln = sp.len
+        units = range(b * wl.Hkv, (b + 1) * wl.Hkv)
+        if z_all is not None:
+            bound = H.score_bound(q, sp.k, ln, wl.G, scale)
+            for i, u in enumerate(units):
+                n = ln[i]
+                err = np.abs(z_all[u, :n].astype(np.float64) - zr[i, :n])
+                assert np.all(err <= bound[i, :n]), (tag, b, u, err.max())
+        for i, u in enumerate(units):
+            be = 1.0 if beta is None else float(beta[u])
+            ok, why = H.selection_ok(zr[i], int(ln[i]), int(k_all[u]), idx_all[u], p, bmin, bmax, be)
+            assert ok, (tag, b, u, why)
+        bm = idx_all.shape[1]
+        o_ref, l_ref = oracle.attend(q, H.host_tier(x.dense, sl), sp, idx_all[list(units)],
+                                     k_all[list(units)], bm, H.host_tier(x.condensed, sl), scale)
+        ok, err = H.attn_close(o_all[sl], o_ref)
+        assert ok, (tag, b, "out", err)
+        ok, err = H.attn_close(l_all[sl], l_ref)
+        assert ok, (tag, b, "lse", err)
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_step_small(name):
+    wl = CASES[name]
+    x = H.inputs(wl)
+    for p in (wl.p, 0.5, 1.0):
+        prob, out, ws = H.run_step(wl, x, p=p)
+        assert ws.status() == 0
+        check_step(wl, x, out, p, wl.bmin, wl.bmax, tag=f"{name} p={p}")
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_step_equals_stage_chain(name):
+    """The fused kernel and the five separate calls give bit-identical results."""
+    wl = CASES[name]
+    x = H.inputs(wl)
+    prob, out, ws = H.run_step(wl, x)
+    U = wl.units
+    dense, sparse, cond = H.tiers_of(x)
+    z = torch.zeros(U, sparse.cap, device=H.dev())
+    hkv.score(prob, x.q, sparse, z, ws)
+    sel = torch.zeros(U, dtype=torch.int32, device=H.dev())
+    cut = torch.zeros(U, 4, dtype=torch.int32, device=H.dev())
+    hkv.topp_select(prob, z, sparse, sel, cut, ws)
+    idx = torch.zeros(U * wl.bmax, dtype=torch.int32, device=H.dev())
+    hkv.compact(prob, z, sparse, sel, cut, idx, ws)
+    o = torch.zeros(wl.B, wl.Hq, wl.D, device=H.dev())
+    lse = torch.zeros(wl.B, wl.Hq, device=H.dev())
+    hkv.cascade_decode(prob, x.q, dense, sparse, idx, sel, cond, o, ws, lse=lse)
+    m = torch.zeros(U, device=H.dev())
+    lz = torch.zeros(U, device=H.dev())
+    hkv.calibrate(prob, z, sparse, m, lz, ws)
+    torch.cuda.synchronize()
+    assert ws.status() == 0
+    ln = x.sparse.len.cpu().numpy()
+    zs, zf = z.cpu().numpy(), out.z.cpu().numpy()
+    for u in range(U):
+        assert np.array_equal(zs[u, : ln[u]], zf[u, : ln[u]])
+    assert torch.equal(sel, out.sel_len)
+    assert torch.equal(cut, out.cut)
+    assert torch.equal(idx, out.idx)
+    assert torch.equal(o, out.out)
+    assert torch.equal(lse, out.lse)
+    assert torch.equal(m, out.m)
+    assert torch.equal(lz, out.logZ)
+
+
+@pytest.mark.parametrize("name", ["bf16_b2_n3000", "bf16_ragged"])
+def test_step_flat_sum_and_rewrite(name):
+    wl = CASES[name]
+    x = H.inputs(wl)
+    _, pad, _ = H.run_step(wl, x, rewrite=True)
+    _, flat, ws = H.run_step(wl, x, layout=hkv.FLAT_SUM, rewrite=True)
+    assert ws.status() == 0
+    U = wl.units
+    k = pad.sel_len.cpu().numpy()
+    assert np.array_equal(k, flat.sel_len.cpu().numpy())
+    offs = flat.offsets.cpu().numpy()
+    assert list(offs) == [0] + list(np.cumsum(k))
+    rows = pad.idx.cpu().numpy().reshape(U, wl.bmax)
+    fl = flat.idx.cpu().numpy()
+    kp = to_host_bits(pad.k_out).reshape(U, wl.bmax, wl.D)
+    kf = to_host_bits(flat.k_out)
+    vp = to_host_bits(pad.v_out).reshape(U, wl.bmax, wl.D)
+    vf = to_host_bits(flat.v_out)
+    ks = to_host_bits(x.sparse.k).reshape(U, -1, wl.D)
+    vs = to_host_bits(x.sparse.v).reshape(U, -1, wl.D)
+    for u in range(U):
+        r = rows[u, : k[u]]
+        assert np.array_equal(fl[offs[u]: offs[u + 1]], r)
+        assert np.all(rows[u, k[u]:] == -1)
+        assert np.array_equal(kp[u, : k[u]], ks[u, r]) and np.array_equal(vp[u, : k[u]], vs[u, r])
+        assert np.array_equal(kf[offs[u]: offs[u + 1]], ks[u, r])
+        assert np.array_equal(vf[offs[u]: offs[u + 1]], vs[u, r])
+    assert torch.equal(pad.out, flat.out)
+
+
+def test_step_per_unit_p_and_temperature():
+    wl = CASES["bf16_hetero"]
+    x = H.inputs(wl)
+    U = wl.units
+    beta = np.linspace(0.25, 3.0, U).astype(np.float32)
+    pu = np.linspace(0.6, 0.99, U).astype(np.float32)
+    prob, out, ws = H.run_step(wl, x, inv_temp=torch.from_numpy(beta).to(H.dev()),
+                               p_unit=torch.from_numpy(pu).to(H.dev()))
+    assert ws.status() == 0
+    k = out.sel_len.cpu().numpy()
+    idx = out.idx.cpu().numpy().reshape(U, wl.bmax)
+    z = out.z.cpu().numpy()
+    ln = x.sparse.len.cpu().numpy()
+    r = oracle.topp(z, ln, 0.0, wl.bmin, wl.bmax, beta, pu)
+    for u in range(U):
+        if k[u] != r["k"][u]:
+            amb = abs(r["c_before"][u] - pu[u]) < H.AMBIG or abs(r["c_at"][u] - pu[u]) < H.AMBIG
+            assert amb and abs(int(k[u]) - int(r["k"][u])) <= 1
+    want = oracle.compact(z, ln, k, wl.bmax)
+    assert np.array_equal(idx, want)
+
+
+# ---- full-size workloads -----------------------------------------------------------
+
+
+@pytest.mark.slow
+def test_workload1_full():
+    wl = WORKLOADS[1]
+    x = H.inputs(wl)
+    prob, out, ws = H.run_step(wl, x)
+    assert ws.status() == 0
+    check_step(wl, x, out, wl.p, wl.bmin, wl.bmax, tag="w1")
+
+
+@pytest.mark.slow
+def test_workload2_full():
+    wl = WORKLOADS[2]
+    x = H.inputs(wl)
+    prob, out, ws = H.run_step(wl, x)
+    assert ws.status() == 0
+    check_step(wl, x, out, wl.p, wl.bmin, wl.bmax, tag="w2")
+
+
+@pytest.mark.slow
+def test_workload3_full_sampled():
+    wl = WORKLOADS[3]
+    x = H.inputs(wl)
+    prob, out, ws = H.run_step(wl, x)
+    assert ws.status() == 0
+    check_step(wl, x, out, wl.p, wl.bmin, wl.bmax, b_sel=[0, 9, 22, 37, 50, 63], tag="w3")
+    k = out.sel_len.cpu().numpy()
+    assert k.min() >= wl.bmin and k.max() <= wl.bmax
+
+
+@pytest.mark.slow
+def test_workload4_full_p_sweep():
+    wl = WORKLOADS[4]
+    x = H.inputs(wl)
+    for p in wl.p_sweep:
+        prob, out, ws = H.run_step(wl, x, p=p)
+        assert ws.status() == 0
+        check_step(wl, x, out, p, wl.bmin, wl.bmax, b_sel=[0, 5, 15], tag=f"w4 p={p}")
+
+
+@pytest.mark.slow
+def test_workload5_sampled_layers():
+    wl = WORKLOADS[5]
+    for layer in (0, 35):
+        x = make_inputs(wl, H.dev(), layer)
+        prob, out, ws = H.run_step(wl, x)
+        assert ws.status() == 0
+        check_step(wl, x, out, wl.p, wl.bmin, wl.bmax, b_sel=[1, 3], tag=f"w5 layer {layer}")
+        del x
+        torch.cuda.empty_cache()
