@@ -1,0 +1,444 @@
+"""Benchmark of one HARD-KV Cascade Cache decode step on B200.
+
+A *step* is one pass of the whole hot path (score, Logits Calibration, Top-p
+budget, compaction, cascade decode attention) over one batch of the
+``bf16_b8_ctx16k`` workload (batch 8, 32/8 heads, head dim 128, context 16384 =
+dense 256 + condensed 64 + sparse 16064, p = 0.95, clamp [64, 2048]).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs its own batch (weak scaling, no data-path
+collective); the device time is the max over ranks. Prints one JSON line on
+rank 0. ``--impl reference`` times the CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from head_adaptive_kv_b200.workloads import WORKLOADS, make_inputs, to_host_bits  # noqa: E402
+
+WORKLOAD_ID = 2
+NSETS = 3  # distinct decode states rotated so that no step re-reads the previous one from L2
+METRIC = "decode steps/sec and KV GB/s at 1 B200 (fraction of 8 TB/s HBM roofline)"
+NORTH_STAR_HBM_GBS = 8000.0
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def csrc_hash() -> str:
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "head_adaptive_kv_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profile(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d.get(kernel)
+        if e and e.get("csrc_hash") == csrc_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ---- distributed plumbing ----------------------------------------------------------
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def init_dist(world: int, backend: str):
+    if world <= 1:
+        return None
+    import datetime
+
+    import torch.distributed as dist
+
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist, device):
+    if dist is not None:
+        if device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def whole_job_value(units_per_rank: int, units_per_step: int, world: int, seconds_max: float, steps: int):
+    """Steps/s of the whole job: units all ranks processed / max-over-ranks time."""
+    total_units = units_per_rank * world * steps
+    return total_units / units_per_step / seconds_max
+
+
+# ---- algorithmic bytes --------------------------------------------------------------
+
+
+def step_bytes(wl, sparse_len, dense_len, cond_len, sel_len) -> int:
+    """Bytes the method must move in one step: every sparse key is scored once;
+    dense, selected and condensed K and V rows are attended once; plus q, the
+    outputs and the compacted rows."""
+    e = 2 if wl.dtype == torch.bfloat16 else 4
+    D = wl.D
+    scored = int(np.sum(sparse_len)) * D * e
+    attended = int(np.sum(dense_len) + np.sum(cond_len) + np.sum(sel_len)) * 2 * D * e
+    q = wl.B * wl.Hq * D * e
+    out = wl.B * wl.Hq * (D + 1) * 4
+    idx = wl.units * wl.bmax * 4 + wl.units * 4
+    return scored + attended + q + out + idx
+
+
+# ---- clocks -------------------------------------------------------------------------
+
+SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    def __init__(self, local_rank: int):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        try:
+            self.index = int(vis.split(",")[local_rank]) if vis else local_rank
+        except ValueError:
+            self.index = local_rank
+        self.proc = None
+        self.path = os.path.join("/tmp", f"hkv_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={SMI_FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                c = [x.strip() for x in line.split(",")]
+                if len(c) < 9 or not c[0].isdigit() or int(c[0]) != self.index:
+                    continue
+                try:
+                    sm.append(float(c[1]))
+                    smax.append(float(c[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, c[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.remove(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---- CPU oracle timing ----------------------------------------------------------------
+
+
+def host_state(x):
+    import oracle
+
+    def tier(t):
+        return oracle.Tier(to_host_bits(t.k), to_host_bits(t.v), t.len.cpu().numpy())
+
+    return to_host_bits(x.q), tier(x.dense), tier(x.sparse), tier(x.condensed)
+
+
+def oracle_units(wl, hs, units: list):
+    """Run the oracle step on a subset of units (one sub-problem per sequence)."""
+    import oracle
+
+    q, dense, sparse, cond = hs
+    by_b = {}
+    for u in units:
+        by_b.setdefault(u // wl.Hkv, []).append(u % wl.Hkv)
+    for b, hs_ in by_b.items():
+        h0, h1 = min(hs_), max(hs_) + 1
+        G = wl.G
+
+        def sub(t):
+            ln = t.len.reshape(wl.B, wl.Hkv)[b, h0:h1].copy()
+            return oracle.Tier(t.k[b:b + 1, h0:h1], t.v[b:b + 1, h0:h1], ln)
+
+        oracle.step(q[b:b + 1, h0 * G:h1 * G], sub(dense), sub(sparse), sub(cond), 1 / math.sqrt(wl.D),
+                    wl.p, wl.bmin, wl.bmax)
+
+
+def cpu_baseline(wl, hs, min_seconds=10.0):
+    """The oracle as it stands on the host cores: whole steps repeated for at
+    least min_seconds (at least one)."""
+    import oracle
+
+    units = list(range(wl.units))
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle_units(wl, hs, units)
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= min_seconds:
+            break
+    return {"value": reps / dt, "unit": "steps/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{reps} whole step(s) of {wl.name} ({wl.units} units), {dt:.1f} s"}
+
+
+# ---- our arm ----------------------------------------------------------------------------
+
+
+def run_ours(args):
+    from head_adaptive_kv_b200 import hkv
+
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device for --impl ours")
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist = init_dist(world, "nccl")
+    wl = WORKLOADS[WORKLOAD_ID]
+
+    sets = []
+    for s in range(NSETS):
+        x = make_inputs(wl, device, layer=100 * rank + s)
+        prob = hkv.Problem(wl.B, wl.Hq, wl.Hkv, wl.D, wl.dtype, wl.p, wl.bmin, wl.bmax)
+        tiers = [hkv.Tier(t.k, t.v, t.len) for t in (x.dense, x.sparse, x.condensed)]
+        out = hkv.StepOutputs.allocate(prob, tiers[1], device)
+        sets.append((x, prob, tiers, out))
+    ws = hkv.Workspace(sets[0][1], *sets[0][2])
+    stream = torch.cuda.current_stream()
+
+    # one CUDA graph per input set, each holding one hkv_step launch
+    for x, prob, tiers, out in sets:
+        hkv.step(prob, x.q, *tiers, out, ws)
+    torch.cuda.synchronize()
+    graphs = []
+    captured0 = hkv.launch_count()
+    for x, prob, tiers, out in sets:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            hkv.step(prob, x.q, *tiers, out, ws)
+        graphs.append(g)
+    torch.cuda.synchronize()
+    launches_per_step = (hkv.launch_count() - captured0) // NSETS
+
+    for i in range(args.warmup):
+        graphs[i % NSETS].replay()
+    torch.cuda.synchronize()
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.15)
+    launches0 = hkv.launch_count()
+    barrier(dist, device)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        starts[i].record(stream)
+        graphs[i % NSETS].replay()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier(dist, device)
+    clk = clocks.stop()
+    region_ms = starts[0].elapsed_time(ends[-1])
+    per_launch_ms = float(np.mean([s.elapsed_time(e) for s, e in zip(starts, ends)]))
+    # launches inside the timed region: the library's own kernels recorded in
+    # each replayed graph (counted at capture) plus any launched directly
+    gpu_launches = args.steps * launches_per_step + (hkv.launch_count() - launches0)
+    assert ws.status() == 0, "device status word set during the benchmark"
+
+    region_ms_max = max_over_ranks(region_ms, dist, device)
+    launch_ms_max = max_over_ranks(per_launch_ms, dist, device)
+    value = whole_job_value(wl.units, wl.units, world, region_ms_max / 1e3, args.steps)
+
+    # algorithmic bytes of one step, from the measured budgets of each set
+    nbytes = []
+    for x, prob, tiers, out in sets:
+        nbytes.append(step_bytes(wl, x.sparse.len.cpu().numpy(), x.dense.len.cpu().numpy(),
+                                 x.condensed.len.cpu().numpy(), out.sel_len.cpu().numpy()))
+    bytes_per_step = float(np.mean(nbytes))
+    achieved_gbs = bytes_per_step / (launch_ms_max / 1e3) / 1e9
+    peak, peak_kind = peaks()
+    kernel = f"k_step<2,{wl.D},{wl.G}>"
+    roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved_gbs / peak, 4), "traffic": traffic_from_profile(kernel),
+                "peak_kind": peak_kind, "kernel": kernel, "bytes_per_launch": int(bytes_per_step)}
+
+    # end to end through the public API: per step, copy the step's query and the
+    # per-unit lengths from pinned host memory, run, and read the outputs back
+    x, prob, tiers, out = sets[0]
+    q_host = x.q.cpu().pin_memory()
+    lens_host = [t.len.cpu().pin_memory() for t in (x.dense, x.sparse, x.condensed)]
+    out_host = torch.empty_like(out.out, device="cpu").pin_memory()
+    lse_host = torch.empty_like(out.lse, device="cpu").pin_memory()
+    k_host = torch.empty_like(out.sel_len, device="cpu").pin_memory()
+    e2e_steps = min(args.steps, 500)
+    barrier(dist, device)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        x.q.copy_(q_host, non_blocking=True)
+        for t, h in zip((x.dense, x.sparse, x.condensed), lens_host):
+            t.len.copy_(h, non_blocking=True)
+        hkv.step(prob, x.q, *tiers, out, ws)
+        out_host.copy_(out.out, non_blocking=True)
+        lse_host.copy_(out.lse, non_blocking=True)
+        k_host.copy_(out.sel_len, non_blocking=True)
+        stream.synchronize()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
+    h2d = x.q.numel() * x.q.element_size() + sum(h.numel() * 4 for h in lens_host)
+    d2h = out_host.numel() * 4 + lse_host.numel() * 4 + k_host.numel() * 4
+    e2e = {"value": round(whole_job_value(wl.units, wl.units, world, e2e_ms / 1e3, e2e_steps), 2),
+           "unit": "steps/s", "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+           "steps": e2e_steps}
+
+    base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        base = cpu_baseline(wl, host_state(sets[0][0]), args.cpu_seconds)
+
+    for g in graphs:
+        del g
+    graphs.clear()
+    if rank == 0:
+        ms = region_ms_max / args.steps
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "steps/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded Gaussian decode states with planted heavy hitters)",
+            "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "D": wl.D,
+                       "ctx": wl.w_cap + wl.c_cap + wl.n_cap, "dense": wl.w_cap, "condensed": wl.c_cap,
+                       "sparse": wl.n_cap, "p": wl.p, "clamp": [wl.bmin, wl.bmax], "layout": "pad_max",
+                       "l2": f"inputs larger than L2 ({wl.units * wl.n_cap * wl.D * 2 / 1e6:.0f} MB of sparse "
+                             f"keys per set), {NSETS} distinct sets rotated",
+                       "parallelism": f"replicas x{world}", "timing": "CUDA graph replay per step"},
+            "kv_gbs": round(bytes_per_step * world / (region_ms_max / args.steps / 1e3) / 1e9, 1),
+            "frac_of_8tbs": round(bytes_per_step / (ms / 1e3) / 1e9 / NORTH_STAR_HBM_GBS, 4),
+            "roofline": roofline,
+            "cpu_baseline": base,
+            "e2e": e2e,
+            "gpu_launches": int(gpu_launches),
+            "clocks": clk,
+            "impl": "ours",
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+# ---- reference arm: the CPU oracle ---------------------------------------------------------
+
+
+def run_reference(args):
+    import oracle
+
+    world, rank, local = dist_env()
+    if rank != 0:
+        return  # rank 0 alone times the oracle
+    wl = WORKLOADS[WORKLOAD_ID]
+    x = make_inputs(wl, "cpu", layer=0)
+    hs = host_state(x)
+    # size each step's sample so that warm-up + timed steps take about two minutes
+    t0 = time.perf_counter()
+    oracle_units(wl, hs, [0])
+    t_unit = max(time.perf_counter() - t0, 1e-4)
+    per_step = int(max(1, min(wl.units, 120.0 / max(1, args.steps + args.warmup) / t_unit)))
+    units = list(range(per_step))
+    for _ in range(args.warmup):
+        oracle_units(wl, hs, units)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_units(wl, hs, units)
+    dt = time.perf_counter() - t0
+    value = args.steps * per_step / wl.units / dt
+    sample = f"{per_step} of {wl.units} units of {wl.name} per step"
+    line = {
+        "metric": METRIC, "value": round(value, 4), "unit": "steps/s", "n_gpus": 0, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 / value, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name}, "impl": "reference",
+        "cpu_baseline": {"value": round(value, 4), "unit": "steps/s", "cores": oracle.num_threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -87,9 +87,13 @@ class Tier:
 
     def c(self, keep: list) -> _Tier:
         k, v = self.k, self.v
+        ln = np.ascontiguousarray(self.len, dtype=np.int32)
+        if k.size == 0:  # an empty tier (numpy gives empty arrays arbitrary strides)
+            keep += [k, ln]
+            B, H, _, D = k.shape
+            return _Tier(k.ctypes.data, k.ctypes.data, H * D, D, D, 0, ln.ctypes.data)
         assert k.shape == v.shape and k.strides == v.strides and k.ndim == 4
         assert k.strides[3] == k.itemsize, "D must be contiguous"
-        ln = np.ascontiguousarray(self.len, dtype=np.int32)
         keep += [k, v, ln]
         es = k.itemsize
         return _Tier(k.ctypes.data, v.ctypes.data, k.strides[0] // es, k.strides[1] // es,

@@ -20,7 +20,8 @@ def check_step(wl, x, out, p, bmin, bmax, b_sel=None, beta=None, tag=""):
     scale = H.scale_of(wl)
     z_all = out.z.cpu().numpy() if out.z is not None else None
     k_all = out.sel_len.cpu().numpy()
-    idx_all = out.idx.cpu().numpy().reshape(wl.units, wl.bmax if bmax is None else bmax)
+    row = max(1, wl.bmax if bmax is None else bmax)  # a bmax of 0 still allocates one slot per unit
+    idx_all = out.idx.cpu().numpy()[: wl.units * row].reshape(wl.units, row)
     o_all = out.out.cpu().numpy()
     l_all = out.lse.cpu().numpy()
     for b in bs:
