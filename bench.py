@@ -132,6 +132,39 @@ def step_bytes(wl, sparse_len, dense_len, cond_len, sel_len) -> int:
     return scored + attended + q + out + idx
 
 
+def score_bytes_of(wl, sparse_len) -> int:
+    """Bytes the scoring kernel must move: every sparse key read once, the
+    queries read, one fp32 score written per key."""
+    e = 2 if wl.dtype == torch.bfloat16 else 4
+    n = int(np.sum(sparse_len))
+    return n * wl.D * e + wl.B * wl.Hq * wl.D * e + n * 4
+
+
+def kernel_ms(launch_round, launches_per_round: int, stream, args) -> float:
+    """Average device time of one launch: rounds of launches captured in one
+    CUDA graph, replayed between CUDA events on the launching stream."""
+    rounds = 64
+    launch_round()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(rounds):
+            launch_round()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    reps = max(1, min(20, args.steps // (rounds * launches_per_round)))
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    del g
+    return e0.elapsed_time(e1) / (reps * rounds * launches_per_round)
+
+
 # ---- clocks -------------------------------------------------------------------------
 
 SMI_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -312,12 +345,30 @@ def run_ours(args):
         nbytes.append(step_bytes(wl, x.sparse.len.cpu().numpy(), x.dense.len.cpu().numpy(),
                                  x.condensed.len.cpu().numpy(), out.sel_len.cpu().numpy()))
     bytes_per_step = float(np.mean(nbytes))
-    achieved_gbs = bytes_per_step / (launch_ms_max / 1e3) / 1e9
+    step_gbs = bytes_per_step / (launch_ms_max / 1e3) / 1e9
+
+    # The dominant kernel, the scorer, timed on its own: R rounds of one launch
+    # per input set, captured in one graph and replayed on the launching stream.
+    zbuf = torch.empty(wl.units, sets[0][2][1].cap, dtype=torch.float32, device=device)
+    score_ms = kernel_ms(lambda: [hkv.score(prob, x.q, tiers[1], zbuf, ws) for x, prob, tiers, out in sets],
+                         NSETS, stream, args)
+    score_ms = max_over_ranks(score_ms, dist, device)
+    attn_ms = kernel_ms(lambda: [hkv.cascade_decode(prob, x.q, *tiers[:2], out.idx, out.sel_len, tiers[2],
+                                                    out.out, ws, lse=out.lse) for x, prob, tiers, out in sets],
+                        NSETS, stream, args)
+    attn_ms = max_over_ranks(attn_ms, dist, device)
+    assert ws.status() == 0, "device status word set during the kernel timing"
+    score_bytes = float(np.mean([score_bytes_of(wl, x.sparse.len.cpu().numpy()) for x, *_ in sets]))
+    achieved_gbs = score_bytes / (score_ms / 1e3) / 1e9
     peak, peak_kind = peaks()
-    kernel = f"k_step<2,{wl.D},{wl.G}>"
+    kernel = f"k_score_stream<2,{wl.D},{wl.G}>"
     roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved_gbs / peak, 4), "traffic": traffic_from_profile(kernel),
-                "peak_kind": peak_kind, "kernel": kernel, "bytes_per_launch": int(bytes_per_step)}
+                "peak_kind": peak_kind, "kernel": kernel, "bytes_per_launch": int(score_bytes),
+                "launch_us": round(score_ms * 1e3, 2)}
+    kernels = {"step_us": round(launch_ms_max * 1e3, 2), "step_gbs": round(step_gbs, 1),
+               "score_us": round(score_ms * 1e3, 2), "attn_us": round(attn_ms * 1e3, 2),
+               "select_compact_us_remainder": round((launch_ms_max - score_ms - attn_ms) * 1e3, 2)}
 
     # end to end through the public API: per step, copy the step's query and the
     # per-unit lengths from pinned host memory, run, and read the outputs back
@@ -374,6 +425,7 @@ def run_ours(args):
             "kv_gbs": round(bytes_per_step * world / (region_ms_max / args.steps / 1e3) / 1e9, 1),
             "frac_of_8tbs": round(bytes_per_step / (ms / 1e3) / 1e9 / NORTH_STAR_HBM_GBS, 4),
             "roofline": roofline,
+            "kernels": kernels,
             "cpu_baseline": base,
             "e2e": e2e,
             "gpu_launches": int(gpu_launches),

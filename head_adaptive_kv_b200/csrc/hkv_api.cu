@@ -5,6 +5,17 @@
 // [TS 2.B], [TS 2.C] = sections of the gist.science Technical Summary of that
 // paper ("Cascade Cache Hierarchy", "Logits Calibration Mechanism",
 // "System-Aware Index Regularization").
+//
+// One decode step (hkv_step) is three kernels on the caller's stream, the last
+// two launched as programmatic dependents so that their launch and prologue
+// overlap the previous kernel's tail:
+//   1. k_score_stream -- S1: every sparse-tier key scored once (streaming);
+//   2. k_unit         -- S2-S4: per unit, calibration + Top-p budget + cut,
+//                        then the order-preserving compaction of the indices;
+//   3. k_attn_stream  -- S5: attention over dense ++ selected ++ condensed,
+//                        per-tile online softmax, the last tile merges the unit.
+// FLAT_SUM layouts and the Rewrite Cache copy add k_flatten.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstring>
@@ -14,83 +25,55 @@
 
 namespace hkv {
 
-// Work per tile: 256 KiB of sparse keys per score tile, 64 KiB of keys (and as
-// much of values) per attention tile.
-constexpr int SCORE_TILE_BYTES = 256 * 1024;
-constexpr int ATTN_TILE_BYTES = 64 * 1024;
+// Trace slots (builds with -DHKV_TRACE only): per unit u of the per-unit
+// kernel, TR_SEL + 8u + i: 0 start, 1 sweep 1 done, 2 sweep 2 done, 3 cut
+// found, 4 range known, 5 compacted.
+[[maybe_unused]] constexpr int TR_SEL = 250000;
 
 // =============================================================================
 // Kernels
 // =============================================================================
 
-// S1 standalone: one score tile per CTA.
-template <int ES, int D, int G>
-__global__ void __launch_bounds__(NTHREADS) k_score(const __grid_constant__ Params P)
+template <int ES, int D, int G, template <int, int, int> class Tile, bool ATTN>
+__device__ __forceinline__ void stream_kernel_body(const Params &P, int n_tiles)
 {
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    Smem &sm = *reinterpret_cast<Smem *>(smem_raw);
+    using SM = SSmem<ES, D, G>;
+    SM &sm = *reinterpret_cast<SM *>(smem_raw);
     const Ctl c = make_ctl(P);
-    const int u = blockIdx.x / P.score_tiles, t = blockIdx.x % P.score_tiles;
-    const int n = tier_len(P.sparse, u, c);
-    const int r0 = t * P.score_rows, r1 = min(n, r0 + P.score_rows);
-    if (r0 >= r1)
-        return;
-    ring_init(sm);
-    uint32_t seq = 0;
-    score_tile<ES, D, G>(P, u, r0, r1, sm, seq, c, evict_first_policy());
-}
-
-// S2 standalone: one unit per CTA.
-__global__ void __launch_bounds__(NTHREADS) k_calibrate(const __grid_constant__ Params P)
-{
-    __shared__ unsigned long long red[16];
-    __shared__ float redf[16];
-    const Ctl c = make_ctl(P);
-    const int u = blockIdx.x;
-    const int n = tier_len(P.sparse, u, c);
-    const float *zu = P.z + (int64_t)u * P.z_stride;
-    float mx = -INFINITY;
-    for (int j = threadIdx.x; j < n; j += NTHREADS)
-        mx = fmaxf(mx, __ldcg(zu + j));
-    const float m = block_max(mx, redf);
-    const float beta = unit_beta(P, u, c);
-    unsigned long long part = 0;
-    for (int j = threadIdx.x; j < n; j += NTHREADS)
-        part += wfix(__ldcg(zu + j), m, beta);
-    const unsigned long long Z = block_sum_u64(part, red);
-    if (P.P_out != nullptr && n > 0) {
-        const float inv = (float)(1099511627776.0 / (double)Z);
-        float *Pu = P.P_out + (int64_t)u * P.z_stride;
-        for (int j = threadIdx.x; j < n; j += NTHREADS) {
-            const float zj = __ldcg(zu + j);
-            const float w = (zj == m || beta == 0.0f) ? 1.0f : expf(beta * (zj - m));
-            Pu[j] = w * inv;
+    stream_init(sm);
+    allow_dependents();
+    wait_prior_grid();  // the previous kernel's results are visible from here on
+    if ((threadIdx.x >> 5) == S_PROD)
+        producer_loop<Tile<ES, D, G>>(P, sm, c, n_tiles, evict_first_policy());
+    else
+        consumer_loop<ES, D, G, ATTN>(P, sm, c);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        // The last CTA to leave resets the ticket counter for the next launch.
+        // Every other CTA has stopped claiming tickets by then.
+        __threadfence();
+        const uint32_t prev = atomicAdd(P.ctl + 2, 1u);
+        if (prev == gridDim.x - 1) {
+            P.ctl[1] = 0;
+            P.ctl[2] = 0;
         }
     }
-    if (threadIdx.x == 0) {
-        P.m_out[u] = m;
-        P.logZ_out[u] = n > 0 ? (float)(log((double)Z) - WFIX_BITS * 0.6931471805599453) : -INFINITY;
-    }
 }
 
-// S3 standalone: one unit per CTA.
-__global__ void __launch_bounds__(NTHREADS) k_select(const __grid_constant__ Params P)
+// S1 ([TS 2.B] max-pooled logits over the query group; [TS 2.A] Tier 2):
+// persistent streaming scorer; also records each tile's score range.
+template <int ES, int D, int G>
+__global__ void __launch_bounds__(S_THREADS, 1) k_score_stream(const __grid_constant__ Params P)
 {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    Smem &sm = *reinterpret_cast<Smem *>(smem_raw);
-    const Ctl c = make_ctl(P);
-    const int u = blockIdx.x;
-    const int n = tier_len(P.sparse, u, c);
-    const float *zu = P.z + (int64_t)u * P.z_stride;
-    float mx = -INFINITY;
-    for (int j = threadIdx.x; j < n; j += NTHREADS)
-        mx = fmaxf(mx, __ldcg(zu + j));
-    const float m = block_max(mx, sm.redf);
-    const Selection s = select_unit(zu, n, m, unit_beta(P, u, c), unit_p(P, u, c), P.bmin, P.bmax, sm);
-    if (threadIdx.x == 0) {
-        P.sel_len[u] = s.k;
-        P.cut[u] = s.cut;
-    }
+    stream_kernel_body<ES, D, G, ScoreTile, false>(P, P.units * P.score_tiles);
+}
+
+// S5 ([TS 2.A] cascade decode over the three tiers; [TS 2.C] Sparse Loading).
+template <int ES, int D, int G>
+__global__ void __launch_bounds__(S_THREADS, 1) k_attn_stream(const __grid_constant__ Params P)
+{
+    stream_kernel_body<ES, D, G, AttnTile, true>(P, P.units * P.attn_tiles);
 }
 
 // Rewrite Cache ([TS 2.C]): copy the k selected K/V rows of unit u, listed in
@@ -101,7 +84,7 @@ __device__ void rewrite_rows(const Params &P, int u, const int32_t *row, int k, 
     const int b = u / P.Hkv, h = u % P.Hkv;
     const int vec_per_row = P.D * es / 16;
     const int64_t total = (int64_t)k * vec_per_row;
-    for (int64_t i = threadIdx.x; i < total; i += NTHREADS) {
+    for (int64_t i = threadIdx.x; i < total; i += NT) {
         const int r = (int)(i / vec_per_row), x = (int)(i % vec_per_row);
         int j = __ldcg(row + r);
         if (j < 0 || j >= n_sparse) {
@@ -115,244 +98,156 @@ __device__ void rewrite_rows(const Params &P, int u, const int32_t *row, int k, 
     }
 }
 
-// Exclusive scan position of unit u in the FLAT_SUM layout.
+// Start of unit u in the FLAT_SUM layout: the budgets of the units before it.
 __device__ int64_t flat_offset(const Params &P, int u, unsigned long long *red)
 {
     unsigned long long part = 0;
-    for (int i = threadIdx.x; i < u; i += NTHREADS)
+    for (int i = threadIdx.x; i < u; i += NT)
         part += (unsigned long long)max(0, __ldcg(P.sel_len + i));
-    return (int64_t)block_sum_u64(part, red);
+    return (int64_t)block_sum_u64<NT>(part, red);
 }
 
-// S4 standalone ([TS 2.C]): compaction of one unit per CTA from its cut, into
-// the caller's layout, plus the optional Rewrite Cache copy.
-template <int ES>
-__global__ void __launch_bounds__(NTHREADS) k_compact(const __grid_constant__ Params P)
+__device__ __forceinline__ void write_offsets(const Params &P, int u, int64_t off)
 {
-    __shared__ unsigned long long red[16];
+    if (threadIdx.x == 0) {
+        P.offsets[u] = (int32_t)off;
+        if (u == P.units - 1)
+            P.offsets[P.units] = (int32_t)(off + max(0, __ldcg(P.sel_len + u)));
+    }
+}
+
+// S2-S4 per unit, one CTA per (sequence, KV head).
+//  do_select  ([TS 2.B] calibration, [Abstract]/[TS 2.A] Top-p budget with the
+//             hard limits): writes sel_len, cut, m, logZ. With have_range the
+//             unit's score range comes from the scorer's tile records.
+//  do_compact ([TS 2.C] Flatten Index): writes the unit's indices in score
+//             order from the cut -- PAD_MAX rows, or FLAT_SUM (standalone) --
+//             and, standalone, the Rewrite Cache copy when k_out is given.
+template <int ES>
+__global__ void __launch_bounds__(NT) k_unit(const __grid_constant__ Params P)
+{
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    USmem &sm = *reinterpret_cast<USmem *>(smem_raw);
     const Ctl c = make_ctl(P);
     const int u = blockIdx.x;
+    allow_dependents();
+    wait_prior_grid();
+    HKV_TRACE_AT(TR_SEL + 8 * u);
     const int n = tier_len(P.sparse, u, c);
     const float *zu = P.z + (int64_t)u * P.z_stride;
-    int k = __ldcg(P.sel_len + u);
-    const hkv_cut ct = P.cut[u];
-    if (k < 0 || k > n || k > P.bmax || ct.n_above < 0 || ct.n_tie < 0 || ct.n_above + ct.n_tie != k) {
-        raise_flag(c, HKV_DEV_BAD_INDEX);
-        k = 0;
-    }
-    int64_t off;
-    if (P.layout == HKV_LAYOUT_FLAT_SUM) {
-        off = flat_offset(P, u, red);
+    int k, n_tie;
+    uint32_t key;
+    if (P.do_select) {
+        float m, zlo;
+        if (P.have_range) {
+            float mx = -INFINITY, mn = INFINITY;
+            const int64_t t0 = (int64_t)u * P.score_tiles;
+            for (int i = threadIdx.x; i < P.score_tiles; i += NT) {
+                mx = fmaxf(mx, __ldcg(P.tile_max + t0 + i));
+                mn = fminf(mn, __ldcg(P.tile_min + t0 + i));
+            }
+            m = block_max<NT>(mx, sm.redf);
+            zlo = -block_max<NT>(-mn, sm.redf);
+        } else {
+            unit_range(zu, n, &m, &zlo, sm);
+        }
+        HKV_TRACE_AT(TR_SEL + 8 * u + 4);
+        const Selection s = select_unit(zu, n, m, zlo, unit_beta(P, u, c), unit_p(P, u, c), P.bmin, P.bmax, sm,
+                                        TR_SEL + 8 * u);
+        k = s.k;
+        key = s.key;
+        n_tie = s.cut.n_tie;
         if (threadIdx.x == 0) {
-            P.offsets[u] = (int32_t)off;
-            if (u == P.units - 1)
-                P.offsets[P.units] = (int32_t)(off + max(0, __ldcg(P.sel_len + u)));
+            P.sel_len[u] = k;
+            if (P.cut)
+                P.cut[u] = s.cut;
+            if (P.m_out)
+                P.m_out[u] = m;
+            if (P.logZ_out)
+                P.logZ_out[u] = n > 0 ? (float)log(s.Z) : -INFINITY;
         }
     } else {
-        off = (int64_t)u * P.bmax;
+        k = __ldcg(P.sel_len + u);
+        const hkv_cut ct = P.cut[u];
+        if (k < 0 || k > n || k > P.bmax || ct.n_above < 0 || ct.n_tie < 0 || ct.n_above + ct.n_tie != k) {
+            raise_flag(c, HKV_DEV_BAD_INDEX);
+            k = 0;
+        }
+        key = k > 0 ? score_key(ct.z_cut) : 0u;
+        n_tie = ct.n_tie;
+    }
+    if (!P.do_compact)
+        return;
+    const bool flat = P.layout == HKV_LAYOUT_FLAT_SUM && !P.do_select;
+    int64_t off = (int64_t)u * P.bmax;
+    if (flat) {
+        off = flat_offset(P, u, sm.red);
+        write_offsets(P, u, off);
     }
     int32_t *row = P.idx + off;
-    compact_unit(zu, n, k > 0 ? score_key(ct.z_cut) : 0u, ct.n_tie, k, row,
-                 P.layout == HKV_LAYOUT_PAD_MAX ? P.bmax : k, red);
-    if (P.k_out != nullptr) {
+    compact_unit(zu, n, key, n_tie, k, row, flat ? k : P.bmax, sm.red);
+    HKV_TRACE_AT(TR_SEL + 8 * u + 5);
+    if (P.k_out != nullptr && !P.do_select) {
         __syncthreads();
         rewrite_rows(P, u, row, k, off, ES, c, n);
     }
 }
 
-// S5 standalone: one attention tile per CTA; the last tile of a unit merges it.
-template <int ES, int D, int G>
-__global__ void __launch_bounds__(NTHREADS) k_decode(const __grid_constant__ Params P)
+// S2 standalone ([TS 2.B]): m, logZ and optionally the calibrated
+// probabilities of each unit. Z is summed exactly as the selection sums it,
+// so m and logZ match hkv_step's bit for bit.
+__global__ void __launch_bounds__(NT) k_calibrate(const __grid_constant__ Params P)
 {
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    Smem &sm = *reinterpret_cast<Smem *>(smem_raw);
+    USmem &sm = *reinterpret_cast<USmem *>(smem_raw);
     const Ctl c = make_ctl(P);
-    const int u = blockIdx.x / P.attn_tiles, s = blockIdx.x % P.attn_tiles;
-    const int W = tier_len(P.dense, u, c), Cn = tier_len(P.cond, u, c);
+    const int u = blockIdx.x;
     const int n = tier_len(P.sparse, u, c);
-    int k = P.sparse.len ? __ldcg(P.sel_len + u) : 0;
-    if (k < 0 || k > n || k > P.bmax) {
-        raise_flag(c, HKV_DEV_BAD_INDEX);
-        k = max(0, min(k, min(n, P.bmax)));
-    }
-    const int32_t *idx_row =
-        P.layout == HKV_LAYOUT_FLAT_SUM ? P.idx + __ldcg(P.offsets + u) : P.idx + (int64_t)u * P.bmax;
-    const int total = W + k + Cn;
-    const int t0 = s * P.attn_toks, t1 = min(total, t0 + P.attn_toks);
-    float *parts = P.part + (int64_t)u * P.attn_tiles * G * (D + 2);
-    ring_init(sm);
-    if (t0 < t1) {
-        uint32_t seq = 0;
-        attn_tile<ES, D, G>(P, u, t0, t1, idx_row, W, k, Cn, n, parts + (int64_t)s * G * (D + 2), sm, seq, c,
-                            evict_first_policy());
+    const float *zu = P.z + (int64_t)u * P.z_stride;
+    float m, zlo;
+    unit_range(zu, n, &m, &zlo, sm);
+    const float bl2 = unit_beta(P, u, c) * LOG2E;
+    double part = 0.0;
+    sweep_scores(zu, n, [&](float z, int, bool valid) {
+        if (valid)
+            part += (double)wcal(z, m, bl2);
+    });
+    const double Z = block_sum_f64<NT>(part, sm.redd);
+    if (P.P_out != nullptr && n > 0) {
+        const float inv = (float)(1.0 / Z);
+        float *Pu = P.P_out + (int64_t)u * P.z_stride;
+        sweep_scores(zu, n, [&](float z, int j, bool valid) {
+            if (valid)
+                Pu[j] = wcal(z, m, bl2) * inv;
+        });
     }
     if (threadIdx.x == 0) {
-        __threadfence();
-        const uint32_t prev = atomicAdd(P.attn_done + u, 1u);
-        sm.bc[0] = (prev == (uint32_t)P.attn_tiles - 1) ? 1 : 0;
-    }
-    __syncthreads();
-    if (sm.bc[0]) {
-        __threadfence();
-        merge_unit<D, G>(P, u, parts, (total + P.attn_toks - 1) / P.attn_toks);
-        if (threadIdx.x == 0)
-            P.attn_done[u] = 0;
+        P.m_out[u] = m;
+        P.logZ_out[u] = n > 0 ? (float)log(Z) : -INFINITY;
     }
 }
 
-// FLAT_SUM rows and Rewrite Cache copies after the fused step: one unit per CTA.
+// FLAT_SUM rows and Rewrite Cache copies after the step's PAD_MAX compaction
+// (one unit per CTA).
 template <int ES>
-__global__ void __launch_bounds__(NTHREADS) k_flatten(const __grid_constant__ Params P)
+__global__ void __launch_bounds__(NT) k_flatten(const __grid_constant__ Params P)
 {
+    __shared__ unsigned long long red[NT / 32];
     const Ctl c = make_ctl(P);
     const int u = blockIdx.x;
+    wait_prior_grid();
     const int n = tier_len(P.sparse, u, c);
     const int k = max(0, min(__ldcg(P.sel_len + u), min(n, P.bmax)));
     const int32_t *src = P.idx + (int64_t)u * P.bmax;
     int64_t off = (int64_t)u * P.bmax;
     if (P.layout == HKV_LAYOUT_FLAT_SUM) {
-        __shared__ unsigned long long red[16];
         off = flat_offset(P, u, red);
-        for (int i = threadIdx.x; i < k; i += NTHREADS)
+        for (int i = threadIdx.x; i < k; i += NT)
             P.idx_user[off + i] = __ldcg(src + i);
-        if (threadIdx.x == 0) {
-            P.offsets[u] = (int32_t)off;
-            if (u == P.units - 1)
-                P.offsets[P.units] = (int32_t)(off + k);
-        }
+        write_offsets(P, u, off);
     }
     if (P.k_out != nullptr)
         rewrite_rows(P, u, src, k, off, ES, c, n);
-}
-
-// S1..S5 fused: persistent CTAs take tickets in order -- every score tile
-// first (unit-major), then every attention tile. The CTA finishing a unit's
-// last score tile selects and compacts that unit and publishes it; attention
-// tiles of the unit wait (bounded) for that. A unit's last attention tile
-// merges the unit. Tickets only wait on tickets issued before them, whose
-// CTAs are running, so the schedule cannot deadlock.
-template <int ES, int D, int G>
-__global__ void __launch_bounds__(NTHREADS) k_step(const __grid_constant__ Params P)
-{
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    Smem &sm = *reinterpret_cast<Smem *>(smem_raw);
-    const Ctl c = make_ctl(P);
-    const uint64_t policy = evict_first_policy();
-    const int n_score = P.units * P.score_tiles;
-    const int n_total = n_score + P.units * P.attn_tiles;
-    ring_init(sm);
-    uint32_t seq = 0;
-    for (;;) {
-        if (threadIdx.x == 0)
-            sm.bc[1] = (int32_t)atomicAdd(P.ctl + 1, 1u);
-        __syncthreads();
-        const int t = sm.bc[1];
-        __syncthreads();
-        if (t >= n_total)
-            break;
-        if (t < n_score) {
-            const int u = t / P.score_tiles, ct = t % P.score_tiles;
-            const int n = tier_len(P.sparse, u, c);
-            const int r0 = ct * P.score_rows, r1 = min(n, r0 + P.score_rows);
-            float tmax = -INFINITY;
-            if (r0 < r1) {
-                score_tile<ES, D, G>(P, u, r0, r1, sm, seq, c, policy);
-                tmax = sm.redf[NCW];
-            }
-            if (threadIdx.x == 0) {
-                P.tile_max[(int64_t)u * P.score_tiles + ct] = tmax;
-                __threadfence();
-                const uint32_t prev = atomicAdd(P.score_done + u, 1u);
-                sm.bc[2] = (prev == (uint32_t)P.score_tiles - 1) ? 1 : 0;
-            }
-            __syncthreads();
-            if (!sm.bc[2])
-                continue;
-            // Last score tile of unit u: Logits Calibration, Top-p, compaction.
-            __threadfence();
-            if (threadIdx.x == 0) {
-                float m = -INFINITY;
-                for (int i = 0; i < P.score_tiles; ++i)
-                    m = fmaxf(m, __ldcg(P.tile_max + (int64_t)u * P.score_tiles + i));
-                sm.redf[8] = m;
-            }
-            __syncthreads();
-            const float m = sm.redf[8];
-            const float *zu = P.z + (int64_t)u * P.z_stride;
-            const Selection s = select_unit(zu, n, m, unit_beta(P, u, c), unit_p(P, u, c), P.bmin, P.bmax, sm);
-            compact_unit(zu, n, s.key, s.cut.n_tie, s.k, P.idx + (int64_t)u * P.bmax, P.bmax, sm.red);
-            if (threadIdx.x == 0) {
-                P.sel_len[u] = s.k;
-                if (P.cut)
-                    P.cut[u] = s.cut;
-                if (P.m_out)
-                    P.m_out[u] = m;
-                if (P.logZ_out)
-                    P.logZ_out[u] = n > 0 ? (float)(log((double)s.Z) - WFIX_BITS * 0.6931471805599453) : -INFINITY;
-            }
-            __syncthreads();
-            if (threadIdx.x == 0) {
-                __threadfence();
-                P.score_done[u] = 0;
-                if (!P.withhold)
-                    st_release(P.ready + u, 1u);
-            }
-        } else {
-            const int a = t - n_score;
-            const int u = a / P.attn_tiles, st = a % P.attn_tiles;
-            if (threadIdx.x == 0) {
-                bool ok = ld_acquire(P.ready + u) != 0;
-                if (!ok) {
-                    const uint64_t t0 = global_ns();
-                    while (!ok) {
-                        __nanosleep(200);
-                        ok = ld_acquire(P.ready + u) != 0;
-                        if (ok || timed_out(c))
-                            break;
-                        if (global_ns() - t0 > c.wait_ns) {
-                            raise_flag(c, HKV_DEV_TIMEOUT);
-                            break;
-                        }
-                    }
-                }
-                sm.bc[3] = ok ? 1 : 0;
-            }
-            __syncthreads();
-            const bool ready = sm.bc[3] != 0;
-            const int W = tier_len(P.dense, u, c), Cn = tier_len(P.cond, u, c);
-            const int n = tier_len(P.sparse, u, c);
-            const int k = ready ? max(0, min(__ldcg(P.sel_len + u), min(n, P.bmax))) : 0;
-            const int total = W + k + Cn;
-            const int t0 = st * P.attn_toks, t1 = min(total, t0 + P.attn_toks);
-            float *parts = P.part + (int64_t)u * P.attn_tiles * G * (D + 2);
-            if (t0 < t1)
-                attn_tile<ES, D, G>(P, u, t0, t1, P.idx + (int64_t)u * P.bmax, W, k, Cn, n,
-                                    parts + (int64_t)st * G * (D + 2), sm, seq, c, policy);
-            if (threadIdx.x == 0) {
-                __threadfence();
-                const uint32_t prev = atomicAdd(P.attn_done + u, 1u);
-                sm.bc[4] = (prev == (uint32_t)P.attn_tiles - 1) ? 1 : 0;
-            }
-            __syncthreads();
-            if (sm.bc[4]) {
-                __threadfence();
-                merge_unit<D, G>(P, u, parts, (total + P.attn_toks - 1) / P.attn_toks);
-                __syncthreads();
-                if (threadIdx.x == 0) {
-                    P.attn_done[u] = 0;
-                    P.ready[u] = 0;
-                }
-            }
-        }
-    }
-    if (threadIdx.x == 0) {
-        __threadfence();
-        const uint32_t prev = atomicAdd(P.ctl + 2, 1u);
-        if (prev == gridDim.x - 1) {
-            P.ctl[1] = 0;
-            P.ctl[2] = 0;
-        }
-    }
 }
 
 // =============================================================================
@@ -364,7 +259,7 @@ std::atomic<uint64_t> g_wait_ns{1000000000ull};
 std::atomic<int32_t> g_withhold{0};
 
 struct WsLayout {
-    size_t ctl, score_done, attn_done, ready, tile_max, zbuf, idxbuf, part, cutbuf, total;
+    size_t ctl, attn_done, tile_max, tile_min, part, idxbuf, zbuf, total;
     int64_t z_stride;
     int score_tiles, attn_tiles, score_rows, attn_toks;
 };
@@ -427,8 +322,9 @@ static WsLayout layout_of(const hkv_problem *p, const hkv_tier *dense, const hkv
     const int ncap = sparse ? sparse->cap : 0;
     const int wcap = dense ? dense->cap : 0;
     const int ccap = cond ? cond->cap : 0;
-    L.score_rows = SCORE_TILE_BYTES / (p->D * es);
-    L.attn_toks = ATTN_TILE_BYTES / (p->D * es);
+    const int rowb = p->D * es;
+    L.score_rows = SCORE_TILE_STAGES * (S_SLOT / rowb);
+    L.attn_toks = ATTN_TILE_STAGES * ((S_SLOT / 2) / rowb);
     L.score_tiles = std::max(1, (ncap + L.score_rows - 1) / L.score_rows);
     const int64_t max_tokens = (int64_t)wcap + std::min<int64_t>(p->bmax, ncap) + ccap;
     L.attn_tiles = (int)std::max<int64_t>(1, (max_tokens + L.attn_toks - 1) / L.attn_toks);
@@ -440,13 +336,11 @@ static WsLayout layout_of(const hkv_problem *p, const hkv_tier *dense, const hkv
         return at;
     };
     L.ctl = take(256);
-    L.score_done = take(units * 4);
     L.attn_done = take(units * 4);
-    L.ready = take(units * 4);
     L.tile_max = take(units * L.score_tiles * 4);
-    L.cutbuf = take(units * sizeof(hkv_cut));
+    L.tile_min = take(units * L.score_tiles * 4);
+    L.part = take((size_t)units * L.attn_tiles * part_stride(p->D, G) * 4);
     L.idxbuf = take(units * (size_t)std::max(p->bmax, 1) * 4);
-    L.part = take((size_t)units * L.attn_tiles * G * (p->D + 2) * 4);
     L.zbuf = take((size_t)units * L.z_stride * 4);
     L.total = o;
     return L;
@@ -475,22 +369,12 @@ static Params base_params(const hkv_problem *p, const WsLayout &L, char *ws)
     P.z_stride = L.z_stride;
     P.wait_ns = g_wait_ns.load();
     P.withhold = g_withhold.load();
-    if (ws) {
-        P.ctl = reinterpret_cast<uint32_t *>(ws + L.ctl);
-        P.score_done = reinterpret_cast<uint32_t *>(ws + L.score_done);
-        P.attn_done = reinterpret_cast<uint32_t *>(ws + L.attn_done);
-        P.ready = reinterpret_cast<uint32_t *>(ws + L.ready);
-        P.tile_max = reinterpret_cast<float *>(ws + L.tile_max);
-        P.part = reinterpret_cast<float *>(ws + L.part);
-    }
+    P.ctl = reinterpret_cast<uint32_t *>(ws + L.ctl);
+    P.attn_done = reinterpret_cast<uint32_t *>(ws + L.attn_done);
+    P.tile_max = reinterpret_cast<float *>(ws + L.tile_max);
+    P.tile_min = reinterpret_cast<float *>(ws + L.tile_min);
+    P.part = reinterpret_cast<float *>(ws + L.part);
     return P;
-}
-
-static hkv_status check_ws(void *ws, size_t ws_bytes, const WsLayout &L)
-{
-    if (ws == nullptr || ((uintptr_t)ws & 255) || ws_bytes < L.total)
-        return HKV_ERR_WORKSPACE;
-    return HKV_OK;
 }
 
 static TierP tier_p(const hkv_tier *t)
@@ -508,7 +392,15 @@ static TierP tier_p(const hkv_tier *t)
     return r;
 }
 
-// Per-device cache of kernel attributes (dynamic smem opt-in, occupancy).
+static hkv_status check_ws(void *ws, size_t ws_bytes, const WsLayout &L)
+{
+    if (ws == nullptr || ((uintptr_t)ws & 255) || ws_bytes < L.total)
+        return HKV_ERR_WORKSPACE;
+    return HKV_OK;
+}
+
+// Per-device cache of kernel attributes (dynamic shared memory opt-in and
+// resident CTAs per SM).
 struct KernelInfo {
     const void *fn;
     int device;
@@ -518,7 +410,7 @@ static std::mutex g_mu;
 static KernelInfo g_info[256];
 static int g_ninfo = 0;
 
-static hkv_status prepare(const void *fn, size_t smem, int *blocks_per_sm)
+static hkv_status prepare(const void *fn, int threads, size_t smem, int *blocks_per_sm)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess)
@@ -534,7 +426,7 @@ static hkv_status prepare(const void *fn, size_t smem, int *blocks_per_sm)
         cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return HKV_ERR_CUDA;
     int bps = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, fn, NTHREADS, smem) != cudaSuccess)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, fn, threads, smem) != cudaSuccess)
         return HKV_ERR_CUDA;
     if (g_ninfo < 256)
         g_info[g_ninfo++] = KernelInfo{fn, dev, bps};
@@ -543,17 +435,56 @@ static hkv_status prepare(const void *fn, size_t smem, int *blocks_per_sm)
     return HKV_OK;
 }
 
+static int sm_count()
+{
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    return sms;
+}
+
+// Launch `kernel` over `grid` CTAs. With pdl the launch is a programmatic
+// dependent of the previous kernel on the stream: it may start early, and the
+// kernel calls wait_prior_grid() before it reads that kernel's results.
 template <typename K>
-static hkv_status launch(K kernel, int grid, size_t smem, cudaStream_t stream, const Params &P)
+static hkv_status launch(K kernel, int grid, int threads, size_t smem, cudaStream_t stream, const Params &P,
+                         bool pdl)
 {
     if (grid <= 0)
         return HKV_OK;
-    hkv_status s = prepare((const void *)kernel, smem, nullptr);
+    hkv_status s = prepare((const void *)kernel, threads, smem, nullptr);
     if (s != HKV_OK)
         return s;
-    kernel<<<grid, NTHREADS, smem, stream>>>(P);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, kernel, P) != cudaSuccess)
+        return HKV_ERR_CUDA;
     g_launches.fetch_add(1);
-    return cudaGetLastError() == cudaSuccess ? HKV_OK : HKV_ERR_CUDA;
+    return HKV_OK;
+}
+
+// Streaming kernels: as many CTAs as are resident at once (one per SM), at
+// most one per tile.
+template <typename K>
+static hkv_status launch_stream(K kernel, size_t smem, int tiles, cudaStream_t stream, const Params &P, bool pdl)
+{
+    int bps = 0;
+    hkv_status s = prepare((const void *)kernel, S_THREADS, smem, &bps);
+    if (s != HKV_OK)
+        return s;
+    const int sms = sm_count();
+    if (sms <= 0 || bps <= 0)
+        return HKV_ERR_CUDA;
+    return launch(kernel, std::min(tiles, bps * sms), S_THREADS, smem, stream, P, pdl);
 }
 
 // Dispatch over the compile-time (element size, head dim, group size).
@@ -576,40 +507,57 @@ static hkv_status dispatch(const hkv_problem *p, A &&...args)
 
 template <int ES, int D, int G>
 struct RunScore {
-    static hkv_status run(const Params &P, int grid, cudaStream_t s)
+    static hkv_status run(const Params &P, cudaStream_t s, bool pdl)
     {
-        return launch(k_score<ES, D, G>, grid, sizeof(Smem), s, P);
+        return launch_stream(k_score_stream<ES, D, G>, sizeof(SSmem<ES, D, G>), P.units * P.score_tiles, s, P,
+                             pdl);
     }
 };
 
 template <int ES, int D, int G>
-struct RunDecode {
-    static hkv_status run(const Params &P, int grid, cudaStream_t s)
+struct RunAttn {
+    static hkv_status run(const Params &P, cudaStream_t s, bool pdl)
     {
-        return launch(k_decode<ES, D, G>, grid, sizeof(Smem), s, P);
+        return launch_stream(k_attn_stream<ES, D, G>, sizeof(SSmem<ES, D, G>), P.units * P.attn_tiles, s, P, pdl);
     }
 };
 
-template <int ES, int D, int G>
-struct RunStep {
-    static hkv_status run(const Params &P, int max_grid, cudaStream_t s)
-    {
-        int bps = 0;
-        hkv_status st = prepare((const void *)k_step<ES, D, G>, sizeof(Smem), &bps);
-        if (st != HKV_OK)
-            return st;
-        int dev = 0, sms = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return HKV_ERR_CUDA;
-        const int grid = std::min(max_grid, std::max(1, bps) * sms);
-        return launch(k_step<ES, D, G>, grid, sizeof(Smem), s, P);
-    }
-};
+static hkv_status launch_unit(const hkv_problem *prob, const Params &P, cudaStream_t s, bool pdl)
+{
+    if (prob->dtype == HKV_BF16)
+        return launch(k_unit<2>, P.units, NT, sizeof(USmem), s, P, pdl);
+    return launch(k_unit<4>, P.units, NT, sizeof(USmem), s, P, pdl);
+}
 
 }  // namespace hkv
 
 using namespace hkv;
+
+namespace {
+
+// Common validation of a compute call; fills the layout and the parameters.
+hkv_status prologue(const hkv_problem *prob, const hkv_tier *dense, const hkv_tier *sparse, const hkv_tier *cond,
+                    bool need_v, void *ws, size_t ws_bytes, WsLayout *L, Params *P)
+{
+    hkv_status s = check_problem(prob);
+    if (s != HKV_OK)
+        return s;
+    if ((s = check_tier(dense, prob, true)) != HKV_OK || (s = check_tier(sparse, prob, need_v)) != HKV_OK ||
+        (s = check_tier(cond, prob, true)) != HKV_OK)
+        return s;
+    *L = layout_of(prob, dense, sparse, cond);
+    if ((s = check_ws(ws, ws_bytes, *L)) != HKV_OK)
+        return s;
+    *P = base_params(prob, *L, static_cast<char *>(ws));
+    P->dense = tier_p(dense);
+    P->sparse = tier_p(sparse);
+    P->cond = tier_p(cond);
+    return HKV_OK;
+}
+
+bool aligned(const void *p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
+
+}  // namespace
 
 extern "C" {
 
@@ -681,36 +629,6 @@ hkv_status hkv_get_status(void *ws, uint32_t *flags, hkv_stream_t stream)
     return (word & HKV_DEV_TIMEOUT) ? HKV_ERR_TIMEOUT : HKV_ERR_DEVICE;
 }
 
-}  // extern "C"
-
-namespace {
-
-// Common validation of a compute call; fills the layout and the parameters.
-hkv_status prologue(const hkv_problem *prob, const hkv_tier *dense, const hkv_tier *sparse, const hkv_tier *cond,
-                    bool need_v, void *ws, size_t ws_bytes, WsLayout *L, Params *P)
-{
-    hkv_status s = check_problem(prob);
-    if (s != HKV_OK)
-        return s;
-    if ((s = check_tier(dense, prob, true)) != HKV_OK || (s = check_tier(sparse, prob, need_v)) != HKV_OK ||
-        (s = check_tier(cond, prob, true)) != HKV_OK)
-        return s;
-    *L = layout_of(prob, dense, sparse, cond);
-    if ((s = check_ws(ws, ws_bytes, *L)) != HKV_OK)
-        return s;
-    *P = base_params(prob, *L, static_cast<char *>(ws));
-    P->dense = tier_p(dense);
-    P->sparse = tier_p(sparse);
-    P->cond = tier_p(cond);
-    return HKV_OK;
-}
-
-bool aligned(const void *p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0; }
-
-}  // namespace
-
-extern "C" {
-
 hkv_status hkv_score(const hkv_problem *prob, const void *q, const hkv_tier *sparse, float *z, int64_t z_stride,
                      void *ws, size_t ws_bytes, hkv_stream_t stream)
 {
@@ -728,7 +646,7 @@ hkv_status hkv_score(const hkv_problem *prob, const void *q, const hkv_tier *spa
     P.q = static_cast<const char *>(q);
     P.z = z;
     P.z_stride = z_stride;
-    return dispatch<RunScore>(prob, P, P.units * P.score_tiles, (cudaStream_t)stream);
+    return dispatch<RunScore>(prob, P, (cudaStream_t)stream, false);
 }
 
 hkv_status hkv_calibrate(const hkv_problem *prob, const float *z, int64_t z_stride, const hkv_tier *sparse,
@@ -749,7 +667,7 @@ hkv_status hkv_calibrate(const hkv_problem *prob, const float *z, int64_t z_stri
     P.P_out = Pout;
     P.m_out = m;
     P.logZ_out = logZ;
-    return launch(k_calibrate, P.units, 0, (cudaStream_t)stream, P);
+    return launch(k_calibrate, P.units, NT, sizeof(USmem), (cudaStream_t)stream, P, false);
 }
 
 hkv_status hkv_topp_select(const hkv_problem *prob, const float *z, int64_t z_stride, const hkv_tier *sparse,
@@ -768,7 +686,8 @@ hkv_status hkv_topp_select(const hkv_problem *prob, const float *z, int64_t z_st
     P.z_stride = z_stride;
     P.sel_len = sel_len;
     P.cut = cut;
-    return launch(k_select, P.units, sizeof(Smem), (cudaStream_t)stream, P);
+    P.do_select = 1;
+    return launch_unit(prob, P, (cudaStream_t)stream, false);
 }
 
 hkv_status hkv_compact(const hkv_problem *prob, const float *z, int64_t z_stride, const hkv_tier *sparse,
@@ -799,9 +718,8 @@ hkv_status hkv_compact(const hkv_problem *prob, const float *z, int64_t z_stride
     P.offsets = offsets;
     P.k_out = static_cast<char *>(k_out);
     P.v_out = static_cast<char *>(v_out);
-    if (prob->dtype == HKV_BF16)
-        return launch(k_compact<2>, P.units, 0, (cudaStream_t)stream, P);
-    return launch(k_compact<4>, P.units, 0, (cudaStream_t)stream, P);
+    P.do_compact = 1;
+    return launch_unit(prob, P, (cudaStream_t)stream, false);
 }
 
 hkv_status hkv_cascade_decode(const hkv_problem *prob, const void *q, const hkv_tier *dense,
@@ -822,13 +740,15 @@ hkv_status hkv_cascade_decode(const hkv_problem *prob, const void *q, const hkv_
         if (prob->layout == HKV_LAYOUT_FLAT_SUM && offsets == nullptr)
             return HKV_ERR_INVALID_ARG;
     }
+    if (P.units == 0)
+        return HKV_OK;
     P.q = static_cast<const char *>(q);
     P.idx = const_cast<int32_t *>(idx);
     P.offsets = const_cast<int32_t *>(offsets);
     P.sel_len = const_cast<int32_t *>(sel_len);
     P.out = out;
     P.lse = lse;
-    return dispatch<RunDecode>(prob, P, P.units * P.attn_tiles, (cudaStream_t)stream);
+    return dispatch<RunAttn>(prob, P, (cudaStream_t)stream, false);
 }
 
 hkv_status hkv_step(const hkv_problem *prob, const void *q, const hkv_tier *dense, const hkv_tier *sparse,
@@ -855,12 +775,13 @@ hkv_status hkv_step(const hkv_problem *prob, const void *q, const hkv_tier *dens
     if (P.units == 0)
         return HKV_OK;
     char *wsb = static_cast<char *>(ws);
+    const cudaStream_t st = (cudaStream_t)stream;
     P.q = static_cast<const char *>(q);
     P.z = o->z ? o->z : reinterpret_cast<float *>(wsb + L.zbuf);
     P.z_stride = o->z ? sparse->cap : L.z_stride;
     P.sel_len = o->sel_len;
     P.cut = o->cut;
-    P.idx = flat ? reinterpret_cast<int32_t *>(wsb + L.idxbuf) : o->idx;
+    P.idx = flat ? reinterpret_cast<int32_t *>(wsb + L.idxbuf) : o->idx;  // PAD_MAX rows for the attention
     P.idx_user = o->idx;
     P.offsets = o->offsets;
     P.out = o->out;
@@ -869,13 +790,27 @@ hkv_status hkv_step(const hkv_problem *prob, const void *q, const hkv_tier *dens
     P.logZ_out = o->logZ;
     P.k_out = static_cast<char *>(o->k_out);
     P.v_out = static_cast<char *>(o->v_out);
-    const int tickets = P.units * (P.score_tiles + P.attn_tiles);
-    s = dispatch<RunStep>(prob, P, tickets, (cudaStream_t)stream);
-    if (s != HKV_OK || (!flat && !rewrite))
+    P.layout = HKV_LAYOUT_PAD_MAX;  // the three kernels work on PAD_MAX rows
+    // 1. scores, and each scoring tile's score range
+    const bool scored = sparse->cap > 0;
+    if (scored && (s = dispatch<RunScore>(prob, P, st, false)) != HKV_OK)
         return s;
+    // 2. calibration, Top-p budget, cut and compaction, per unit
+    Params U = P;
+    U.have_range = scored;
+    U.do_select = 1;
+    U.do_compact = 1;
+    if ((s = launch_unit(prob, U, st, scored)) != HKV_OK)
+        return s;
+    // 3. attention over the three tiers and the merge of each unit
+    if ((s = dispatch<RunAttn>(prob, P, st, true)) != HKV_OK)
+        return s;
+    if (!flat && !rewrite)
+        return HKV_OK;
+    P.layout = prob->layout;
     if (prob->dtype == HKV_BF16)
-        return launch(k_flatten<2>, P.units, 0, (cudaStream_t)stream, P);
-    return launch(k_flatten<4>, P.units, 0, (cudaStream_t)stream, P);
+        return launch(k_flatten<2>, P.units, NT, 0, st, P, true);
+    return launch(k_flatten<4>, P.units, NT, 0, st, P, true);
 }
 
 }  // extern "C"

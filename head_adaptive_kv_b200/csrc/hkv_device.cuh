@@ -1,6 +1,7 @@
 // hkv_device.cuh -- sm_100a device primitives shared by the HARD-KV kernels:
-// mbarrier + bulk-copy (TMA) staging, packed fp32x2 FMA, bf16 widening, warp
-// and block reductions, the order key of a score, bounded waits.
+// mbarriers, bulk copies (TMA) and cp.async, packed fp32x2 FMA, bf16
+// widening, warp and block reductions, the order key of a score, the
+// fixed-point calibrated weight, bounded waits and an optional device trace.
 #pragma once
 
 #include <cstdint>
@@ -9,21 +10,6 @@
 #include "hkv.h"
 
 namespace hkv {
-
-// ---------------------------------------------------------------------------
-// CTA shape shared by every kernel: NCW consumer warps and one producer warp.
-// The producer issues bulk copies into a ring of NSLOT slots (one per consumer
-// warp); the consumers turn staged rows into scores or attention partials.
-constexpr int NCW = 4;
-constexpr int NSLOT = NCW;
-constexpr int NTHREADS = (NCW + 1) * 32;
-constexpr int PRODUCER_WARP = NCW;
-constexpr int SLOT_BYTES = 16384;
-constexpr int SC_FLOATS = 512;  // per-warp logits scratch of an attention stage
-
-// Select histograms: 11 + 11 + 10 bits of the 32-bit order key.
-constexpr int L1_BITS = 11, L2_BITS = 11, L3_BITS = 10;
-constexpr int HBINS = 1 << 11;
 
 // Calibrated weights exp(beta (z - m)) <= 1 are summed as unsigned fixed-point
 // integers with 40 fractional bits: exact, order-free and deterministic.
@@ -47,6 +33,25 @@ __device__ __forceinline__ bool timed_out(const Ctl &c)
 {
     return (*reinterpret_cast<volatile const uint32_t *>(c.status) & HKV_DEV_TIMEOUT) != 0;
 }
+
+// Optional device trace (build with -DHKV_TRACE): thread 0 of a CTA (or lane 0
+// of a warp, HKV_TRACE_WARP) stores the global timer at a numbered slot.
+#ifdef HKV_TRACE
+constexpr int HKV_TRACE_SLOTS = 1 << 18;
+__device__ unsigned long long hkv_trace_buf[HKV_TRACE_SLOTS];  // one translation unit per trace build
+#define HKV_TRACE_IF(cond, slot)                                                   \
+    do {                                                                           \
+        const int hkv_slot_ = (slot);                                              \
+        if ((cond) && hkv_slot_ >= 0 && hkv_slot_ < HKV_TRACE_SLOTS)               \
+            hkv_trace_buf[hkv_slot_] = global_ns();                                \
+    } while (0)
+#else
+#define HKV_TRACE_IF(cond, slot) \
+    do {                         \
+    } while (0)
+#endif
+#define HKV_TRACE_AT(slot) HKV_TRACE_IF(threadIdx.x == 0, slot)
+#define HKV_TRACE_WARP(slot) HKV_TRACE_IF((threadIdx.x & 31) == 0, slot)
 
 __device__ __forceinline__ uint32_t smem_addr(const void *p)
 {
@@ -89,31 +94,53 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
-// Wait for the phase of `bar` with the given parity to complete, at most
-// c.wait_ns nanoseconds. On expiry the status word gets HKV_DEV_TIMEOUT and
-// every later wait in any CTA returns false at once.
-__device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const Ctl &c)
+// Non-blocking test of a phase.
+__device__ __forceinline__ bool mbar_test(uint64_t *bar, uint32_t parity)
 {
-    if (mbar_try_wait(bar, parity))
-        return true;
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Slow path of mbar_wait: spin at most wait_ns nanoseconds. On expiry the
+// status word gets HKV_DEV_TIMEOUT and every later wait in any CTA returns
+// false at once.
+__device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parity, uint32_t *status, uint64_t wait_ns)
+{
     const uint64_t t0 = global_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity))
             return true;
         if ((it & 15u) == 0) {
-            if (timed_out(c))
+            if ((*reinterpret_cast<volatile const uint32_t *>(status) & HKV_DEV_TIMEOUT) != 0)
                 return false;
-            if (global_ns() - t0 > c.wait_ns) {
-                raise_flag(c, HKV_DEV_TIMEOUT);
+            if (global_ns() - t0 > wait_ns) {
+                atomicOr(status, HKV_DEV_TIMEOUT);
                 return false;
             }
         }
     }
 }
 
+// Wait for the phase of `bar` with the given parity to complete (bounded).
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const Ctl &c)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    return mbar_wait_slow(bar, parity, c.status, c.wait_ns);
+}
+
+// ---- copies -------------------------------------------------------------------
+
 // 1-D bulk copy (TMA) global -> this CTA's shared memory, completing `bytes`
 // on `bar`. Both addresses 16-byte aligned, bytes a multiple of 16. Keys and
-// values are streamed once per step, so the lines are marked evict-first in L2.
+// values are streamed once per step, so the lines are marked evict-first.
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
                                          uint64_t policy)
 {
@@ -124,12 +151,41 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         : "memory");
 }
 
+// 16-byte asynchronous copy global -> shared, cached in L2 only.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
+}
+
+// Arrive on `bar` once this thread's earlier cp.async copies have landed (the
+// pending count is raised first, so the phase waits for them).
+__device__ __forceinline__ void cp_async_arrive(uint64_t *bar)
+{
+    asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+// Order earlier ordinary (generic-proxy) shared-memory accesses before later
+// bulk copies (async proxy) into the same memory.
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ uint64_t evict_first_policy()
 {
     uint64_t pol;
     asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
     return pol;
 }
+
+// Programmatic dependent launch: wait for the preceding kernel's results
+// (its completion and the visibility of its writes).
+__device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Let the next kernel on the stream, if launched as a programmatic dependent,
+// start its CTAs now; it still waits for this grid's completion before it
+// reads anything this grid writes.
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ---- arithmetic -------------------------------------------------------------
 
@@ -170,15 +226,38 @@ __device__ __forceinline__ float key_score(uint32_t key)
     return __uint_as_float(u);
 }
 
-// Calibrated weight exp(beta (z - m)) in fixed point (1.0 = 2^40); exactly 1.0
-// at the maximum and everywhere when beta = 0.
-__device__ __forceinline__ unsigned long long wfix(float z, float m, float beta)
+// 2^x on the SFU (ex2.approx, relative error below 2^-22).
+__device__ __forceinline__ float ex2(float x)
 {
-    if (z == m || beta == 0.0f)
-        return 1ull << WFIX_BITS;
-    const float w = expf(beta * (z - m));
-    return __float2ull_rn(w * 1099511627776.0f);
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
+
+// Calibrated weight exp(beta (z - m)) = 2^((z - m) beta log2 e), exactly 1 at
+// the maximum and everywhere when beta = 0. bl2 = beta * log2(e).
+__device__ __forceinline__ float wcal(float z, float m, float bl2)
+{
+    if (z == m || bl2 == 0.0f)
+        return 1.0f;
+    return ex2((z - m) * bl2);
+}
+
+// floor(w * 2^40) of a weight 0 <= w <= 1, from its bits (exact integer ops):
+// w = mant * 2^(e - 23) with a 24-bit mant, so w * 2^40 = mant * 2^(e + 17).
+__device__ __forceinline__ unsigned long long wq(float w)
+{
+    const uint32_t bits = __float_as_uint(w);
+    const int e = (int)((bits >> 23) & 0xffu) - 127;
+    if (e < -41)  // below 2^-41 (including 0 and subnormals) contributes nothing
+        return 0ull;
+    const unsigned long long mant = (unsigned long long)((bits & 0x7fffffu) | 0x800000u);
+    const int sh = e + 17;
+    return sh >= 0 ? (mant << sh) : (mant >> (-sh));
+}
+
+// Calibrated weight in fixed point (1.0 = 2^WFIX_BITS).
+__device__ __forceinline__ unsigned long long wfix(float z, float m, float bl2) { return wq(wcal(z, m, bl2)); }
 
 // ---- warp / block reductions ------------------------------------------------
 
@@ -198,15 +277,15 @@ __device__ __forceinline__ float warp_sum(float v)
     return v;
 }
 
-// Exclusive prefix sum over the CTA (NTHREADS threads) of a 64-bit value.
-// `scratch` holds at least NTHREADS/32 + 1 words. *total receives the sum.
-// Contains __syncthreads(); every thread must call it.
-__device__ __forceinline__ unsigned long long block_exclusive_scan(unsigned long long v,
-                                                                   unsigned long long *scratch,
+// Exclusive prefix sum over a CTA of NT threads of a 64-bit value. `scratch`
+// holds at least NT/32 words. *total receives the sum. Contains
+// __syncthreads(); every thread must call it.
+template <int NT>
+__device__ __forceinline__ unsigned long long block_exclusive_scan(unsigned long long v, unsigned long long *scratch,
                                                                    unsigned long long *total)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    constexpr int NW = NTHREADS / 32;
+    constexpr int NW = NT / 32;
     unsigned long long x = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -235,10 +314,19 @@ __device__ __forceinline__ unsigned long long block_exclusive_scan(unsigned long
     return before_warp + x - v;
 }
 
+template <int NT>
+__device__ __forceinline__ unsigned long long block_sum_u64(unsigned long long v, unsigned long long *scratch)
+{
+    unsigned long long total;
+    block_exclusive_scan<NT>(v, scratch, &total);
+    return total;
+}
+
+template <int NT>
 __device__ __forceinline__ float block_max(float v, float *scratch)
 {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    constexpr int NW = NTHREADS / 32;
+    constexpr int NW = NT / 32;
     v = warp_max(v);
     if (lane == 0)
         scratch[warp] = v;
@@ -251,24 +339,24 @@ __device__ __forceinline__ float block_max(float v, float *scratch)
     return r;
 }
 
-__device__ __forceinline__ unsigned long long block_sum_u64(unsigned long long v, unsigned long long *scratch)
+// Sum of a double over the CTA in a fixed order (deterministic).
+template <int NT>
+__device__ __forceinline__ double block_sum_f64(double v, double *scratch)
 {
-    unsigned long long total;
-    block_exclusive_scan(v, scratch, &total);
-    return total;
-}
-
-// Acquire / release flags between CTAs (published selections).
-__device__ __forceinline__ uint32_t ld_acquire(const uint32_t *p)
-{
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void st_release(uint32_t *p, uint32_t v)
-{
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int NW = NT / 32;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0)
+        scratch[warp] = v;
+    __syncthreads();
+    double r = 0.0;
+#pragma unroll
+    for (int i = 0; i < NW; ++i)
+        r += scratch[i];
+    __syncthreads();
+    return r;
 }
 
 }  // namespace hkv

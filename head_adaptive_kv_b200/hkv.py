@@ -14,7 +14,7 @@ from typing import Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libhkv.so")
+LIB_PATH = os.environ.get("HKV_LIBRARY") or os.path.join(_HERE, "libhkv.so")
 
 HKV_BF16, HKV_F32 = 0, 1
 PAD_MAX, FLAT_SUM = 0, 1

@@ -153,8 +153,8 @@ hkv_status hkv_score(const hkv_problem *prob, const void *q, const hkv_tier *spa
  * Z = sum_j exp(beta (z_j - m)), logZ = ln Z, and optionally
  * P[u*z_stride + j] = exp(beta (z_j - m)) / Z. sparse supplies the lengths
  * (its K/V are not read). m, logZ: device [B*Hkv]; P may be NULL. An empty unit
- * gives m = -inf, logZ = -inf. Z is summed in exact fixed point, as in
- * hkv_topp_select. */
+ * gives m = -inf, logZ = -inf. Z is summed in double precision in a fixed
+ * order, exactly as hkv_topp_select and hkv_step sum it. */
 hkv_status hkv_calibrate(const hkv_problem *prob, const float *z, int64_t z_stride,
                          const hkv_tier *sparse, float *P, float *m, float *logZ,
                          void *ws, size_t ws_bytes, hkv_stream_t stream);
@@ -162,8 +162,9 @@ hkv_status hkv_calibrate(const hkv_problem *prob, const float *z, int64_t z_stri
 /* S3 Top-p budget ([Abstract], [TS 2.A], [TS 2.B]): per unit the budget
  * sel_len[u] = min(n, max(bmin, min(k*, bmax))), k* the fewest tokens (score
  * descending, lower index first) whose calibrated mass is at least p, and the
- * cut that identifies the set. Masses are summed as exact 40-bit fixed-point
- * weights, so the result is deterministic. sparse supplies the lengths.
+ * cut that identifies the set. Prefix masses are exact sums of 40-bit
+ * fixed-point weights and Z a fixed-order double sum, so the result is
+ * deterministic. sparse supplies the lengths.
  * sel_len, cut: device [B*Hkv]. */
 hkv_status hkv_topp_select(const hkv_problem *prob, const float *z, int64_t z_stride,
                            const hkv_tier *sparse, int32_t *sel_len, hkv_cut *cut,
@@ -194,12 +195,17 @@ hkv_status hkv_cascade_decode(const hkv_problem *prob, const void *q,
                               float *out, float *lse, void *ws, size_t ws_bytes,
                               hkv_stream_t stream);
 
-/* S1..S5 fused ([TS 2.A] pipeline steps 2 and 3 plus decoding): one persistent
- * kernel scores every sparse token, calibrates, takes the Top-p budget and
- * compacts each unit as soon as its last score tile lands, and runs the split
- * attention tiles of the units whose selection is published; the last tile of
- * a unit merges it. Attention reads the selected rows through the indices
- * ([TS 2.C] Sparse Loading); k_out/v_out add the Rewrite Cache copy. ws as for
+/* S1..S5 in one call ([TS 2.A] pipeline steps 2 and 3 plus decoding): three
+ * kernels on `stream`, the second and third launched as programmatic
+ * dependents of the one before. (1) A persistent streaming kernel scores every
+ * sparse token (the same kernel as hkv_score) and records each scoring tile's
+ * score range; (2) one CTA per unit calibrates, takes the Top-p budget and the
+ * cut, and compacts the unit's indices into PAD_MAX rows; (3) a persistent
+ * streaming kernel runs the split attention tiles (the same kernel as
+ * hkv_cascade_decode), reading the selected rows through the indices
+ * ([TS 2.C] Sparse Loading); the last tile of a unit merges it. A FLAT_SUM
+ * layout or k_out/v_out (the Rewrite Cache copy) adds a fourth kernel. The
+ * results equal those of the five separate calls bit for bit. ws as for
  * hkv_cascade_decode. */
 hkv_status hkv_step(const hkv_problem *prob, const void *q, const hkv_tier *dense,
                     const hkv_tier *sparse, const hkv_tier *condensed,
@@ -221,9 +227,11 @@ hkv_status hkv_get_status(void *ws, uint32_t *flags, hkv_stream_t stream);
  * (default 1e9). Takes effect at the next launch. */
 hkv_status hkv_set_wait_limit_ns(uint64_t ns);
 
-/* Fault injection for tests: when nonzero, the fused step never publishes a
- * unit's selection, so every attention tile's bounded wait runs out and the
- * status word gets HKV_DEV_TIMEOUT. Takes effect at the next launch. */
+/* Fault injection for tests: when nonzero, the streaming kernels (scoring and
+ * attention, hkv_step included) never arm their copy stages, so each consumer's
+ * bounded wait runs out, the kernel returns, and the status word gets
+ * HKV_DEV_TIMEOUT; results of such a call are undefined. Takes effect at the
+ * next launch. */
 hkv_status hkv_debug_withhold_publish(int32_t on);
 
 /* Kernel launches this library has issued in this process (all devices). */
