@@ -814,3 +814,103 @@ hkv_status hkv_step(const hkv_problem *prob, const void *q, const hkv_tier *dens
 }
 
 }  // extern "C"
+
+// =============================================================================
+// No-allocation cascade decode
+//
+// For callers that cannot allocate device memory where they decode (an engine
+// that gives nearly all HBM to its KV pool up front and forbids allocation on
+// the decode path, or a plugin hook with no workspace to hand over). The
+// kernel and its arguments are those of hkv_cascade_decode; only the scratch
+// moves from the caller's workspace into a fixed array of this library.
+// =============================================================================
+
+namespace hkv {
+
+// The scratch, one copy per device that loads the library. In host code this
+// name is only a stand-in for the symbol, never a device address: kernels get
+// the address that cudaGetSymbolAddress returns for the current device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[HKV_NOALLOC_SCRATCH_BYTES];
+
+constexpr int NOALLOC_MAX_DEVICES = 64;
+static std::mutex g_noalloc_mu;
+static void *g_noalloc_ptr[NOALLOC_MAX_DEVICES];
+
+// Device address of the scratch on the current device, looked up once per
+// device (the first call on a device does this; it must not run under stream
+// capture).
+static hkv_status noalloc_scratch(void **ptr)
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= NOALLOC_MAX_DEVICES)
+        return HKV_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+            return HKV_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *ptr = g_noalloc_ptr[dev];
+    return HKV_OK;
+}
+
+}  // namespace hkv
+
+extern "C" hkv_status hkv_cascade_decode_noalloc(const hkv_problem *prob, const void *q, const hkv_tier *dense,
+                                                 const hkv_tier *sparse, const int32_t *idx,
+                                                 const int32_t *offsets, const int32_t *sel_len,
+                                                 const hkv_tier *condensed, float *out, float *lse,
+                                                 uint32_t *status, hkv_stream_t stream)
+{
+    // host validation, as for hkv_cascade_decode
+    hkv_status s = check_problem(prob);
+    if (s != HKV_OK)
+        return s;
+    if ((s = check_tier(dense, prob, true)) != HKV_OK || (s = check_tier(sparse, prob, true)) != HKV_OK ||
+        (s = check_tier(condensed, prob, true)) != HKV_OK)
+        return s;
+    if (q == nullptr || !aligned(q, 16) || out == nullptr || (status != nullptr && !aligned(status, 4)))
+        return HKV_ERR_INVALID_ARG;
+    if (sparse != nullptr && sparse->cap > 0) {
+        if (idx == nullptr || sel_len == nullptr)
+            return HKV_ERR_INVALID_ARG;
+        if (prob->layout == HKV_LAYOUT_FLAT_SUM && offsets == nullptr)
+            return HKV_ERR_INVALID_ARG;
+    }
+    // The attention uses the front of the workspace layout: the status and
+    // counter words, the score ranges and the tile records (everything before
+    // the index and score buffers, which only hkv_step uses).
+    const WsLayout L = layout_of(prob, dense, sparse, condensed);
+    const size_t need = L.idxbuf;
+    if (need > HKV_NOALLOC_SCRATCH_BYTES)
+        return HKV_ERR_WORKSPACE;
+    const cudaStream_t st = (cudaStream_t)stream;
+    if ((int64_t)prob->B * prob->Hkv == 0)
+        return status ? (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) == cudaSuccess ? HKV_OK : HKV_ERR_CUDA)
+                      : HKV_OK;
+    void *scratch = nullptr;
+    if ((s = noalloc_scratch(&scratch)) != HKV_OK)
+        return s;
+    char *base = static_cast<char *>(scratch);
+    Params P = base_params(prob, L, base);
+    P.dense = tier_p(dense);
+    P.sparse = tier_p(sparse);
+    P.cond = tier_p(condensed);
+    P.q = static_cast<const char *>(q);
+    P.idx = const_cast<int32_t *>(idx);
+    P.offsets = const_cast<int32_t *>(offsets);
+    P.sel_len = const_cast<int32_t *>(sel_len);
+    P.out = out;
+    P.lse = lse;
+    // the status word, the ticket and exit counters and the per-unit tile
+    // counters must start at zero; the previous call may have left them set
+    if (cudaMemsetAsync(base, 0, L.tile_max, st) != cudaSuccess)
+        return HKV_ERR_CUDA;
+    if ((s = dispatch<RunAttn>(prob, P, st, false)) != HKV_OK)
+        return s;
+    if (status != nullptr &&
+        cudaMemcpyAsync(status, base, sizeof(uint32_t), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return HKV_ERR_CUDA;
+    return HKV_OK;
+}

@@ -66,6 +66,7 @@ def _load():
         "hkv_compact": [P, P, i64, P, P, P, P, P, P, P, P, sz, P],
         "hkv_cascade_decode": [P, P, P, P, P, P, P, P, P, P, P, sz, P],
         "hkv_step": [P, P, P, P, P, P, P, sz, P],
+        "hkv_cascade_decode_noalloc": [P, P, P, P, P, P, P, P, P, P, P, P],
         "hkv_get_status": [P, C.POINTER(C.c_uint32), P],
         "hkv_set_wait_limit_ns": [C.c_uint64],
         "hkv_debug_withhold_publish": [i32],
@@ -274,6 +275,21 @@ def step(prob: Problem, q: torch.Tensor, dense: Optional[Tier], sparse: Tier, co
          out: StepOutputs, ws: Workspace, stream=None):
     _check(lib.hkv_step(C.byref(prob.c()), _ptr(q), _tref(dense), C.byref(sparse.c()), _tref(condensed),
                         C.byref(out.c()), ws.ptr, ws.nbytes, _stream(stream)), "hkv_step")
+
+
+def cascade_decode_noalloc(prob: Problem, q: torch.Tensor, dense: Optional[Tier], sparse: Optional[Tier],
+                           idx: Optional[torch.Tensor], sel_len: Optional[torch.Tensor],
+                           condensed: Optional[Tier], out: torch.Tensor, lse: Optional[torch.Tensor] = None,
+                           offsets: Optional[torch.Tensor] = None, status: Optional[torch.Tensor] = None,
+                           stream=None):
+    """cascade_decode for callers that cannot allocate device memory: no
+    workspace argument; the library's fixed scratch array is used instead
+    (see hkv_cascade_decode_noalloc in include/hkv.h for its limit and for why
+    overlapping calls must be serialised). status: optional device int32/uint32
+    tensor of one element that receives the call's device status bits."""
+    _check(lib.hkv_cascade_decode_noalloc(C.byref(prob.c()), _ptr(q), _tref(dense), _tref(sparse), _ptr(idx),
+                                          _ptr(offsets), _ptr(sel_len), _tref(condensed), _ptr(out), _ptr(lse),
+                                          _ptr(status), _stream(stream)), "hkv_cascade_decode_noalloc")
 
 
 def set_wait_limit_ns(ns: int):

@@ -212,6 +212,45 @@ hkv_status hkv_step(const hkv_problem *prob, const void *q, const hkv_tier *dens
                     const hkv_step_out *out, void *ws, size_t ws_bytes,
                     hkv_stream_t stream);
 
+/* Capacity, in bytes, of the device scratch array behind
+ * hkv_cascade_decode_noalloc (one array per GPU that loads the library, held
+ * until the process exits). */
+#define HKV_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/* S5 without a caller-supplied workspace. No counterpart in the paper: this is
+ * an integration aid. Some callers cannot allocate device memory at the point
+ * where they decode: a serving engine that hands nearly all HBM to its KV-cache
+ * pool at start-up and forbids allocation on the decode path, or a plugin
+ * whose enqueue hook may not allocate and has no workspace to offer. This call
+ * computes exactly what hkv_cascade_decode computes, with the same kernel and
+ * the same arguments minus ws/ws_bytes, and allocates nothing (no cudaMalloc,
+ * no cudaFree, no allocating library routine): its scratch is a fixed device
+ * array of HKV_NOALLOC_SCRATCH_BYTES bytes inside the library.
+ * - Size limit: the scratch is the front of the layout hkv_workspace_size
+ *   describes (status and counter words, per-tile score ranges, attention
+ *   tile records): about 2.6 MB for bf16, D = 128, G = 4, 64 units of up to
+ *   2368 attended tokens. A problem that needs more than the array holds is
+ *   refused with HKV_ERR_WORKSPACE before anything is launched; use
+ *   hkv_cascade_decode with a workspace for those.
+ * - Set-up: the first call on each device looks up the array's device address
+ *   and sets the kernel's shared-memory attribute. Make that first call outside
+ *   any stream capture.
+ * - Sharing: every call on a device uses the same array, which keeps the last
+ *   call's contents. Each call zeroes the words that must start at zero (status
+ *   and counters) on `stream` before its kernel runs; the tile records are
+ *   always written before they are read. Calls that overlap on the GPU (other
+ *   streams, other host threads) race on the array and give undefined results:
+ *   serialise them.
+ * - status: device pointer to one uint32 or NULL; when given it receives this
+ *   call's HKV_DEV_* bits (stream-ordered copy after the kernel).
+ * Other arguments, layouts and return codes as for hkv_cascade_decode. */
+hkv_status hkv_cascade_decode_noalloc(const hkv_problem *prob, const void *q,
+                                      const hkv_tier *dense, const hkv_tier *sparse,
+                                      const int32_t *idx, const int32_t *offsets,
+                                      const int32_t *sel_len, const hkv_tier *condensed,
+                                      float *out, float *lse, uint32_t *status,
+                                      hkv_stream_t stream);
+
 /* Every compute call takes a workspace `ws` of at least hkv_workspace_size
  * bytes (256-byte aligned, zeroed once by hkv_workspace_init); its first word
  * is the device status word. Calls that overlap on the GPU need separate

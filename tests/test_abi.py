@@ -28,7 +28,7 @@ def declared_symbols():
 
 def test_every_declared_symbol_is_exported(hk):
     names = declared_symbols()
-    assert len(names) == 13, names
+    assert len(names) == 14, names
     for n in names:
         assert hasattr(hk.lib, n), n
     nm = os.popen(f"nm -D --defined-only {hk.LIB_PATH}").read()
