@@ -34,46 +34,46 @@ namespace hkv {
 // Kernels
 // =============================================================================
 
-template <int ES, int D, int G, template <int, int, int> class Tile, bool ATTN>
-__device__ __forceinline__ void stream_kernel_body(const Params &P, int n_tiles)
+// S1 ([TS 2.B] max-pooled logits over the query group; [TS 2.A] Tier 2):
+// persistent streaming scorer over the capacity rows of all units.
+template <int ES, int D, int G>
+__global__ void __launch_bounds__(sc_nw(G) * 32, 1) k_score_stream(const __grid_constant__ Params P)
 {
     extern __shared__ __align__(128) unsigned char smem_raw[];
-    using SM = SSmem<ES, D, G>;
-    SM &sm = *reinterpret_cast<SM *>(smem_raw);
+    using Job = ScoreJob<ES, D, G>;
+    auto &ring = *reinterpret_cast<typename Job::RingT *>(smem_raw);
     const Ctl c = make_ctl(P);
-    stream_init(sm);
+    ring_init(ring);
     allow_dependents();
     wait_prior_grid();  // the previous kernel's results are visible from here on
-    if ((threadIdx.x >> 5) == S_PROD)
-        producer_loop<Tile<ES, D, G>>(P, sm, c, n_tiles, evict_first_policy());
-    else
-        consumer_loop<ES, D, G, ATTN>(P, sm, c);
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        // The last CTA to leave resets the ticket counter for the next launch.
-        // Every other CTA has stopped claiming tickets by then.
-        __threadfence();
-        const uint32_t prev = atomicAdd(P.ctl + 2, 1u);
-        if (prev == gridDim.x - 1) {
-            P.ctl[1] = 0;
-            P.ctl[2] = 0;
-        }
+    const int64_t R = (int64_t)P.units * P.sparse.cap;
+    const int64_t NW = (int64_t)gridDim.x * Job::NW;
+    const int64_t g = (int64_t)blockIdx.x * Job::NW + (threadIdx.x >> 5);
+    Job job(P, c, ring, share_begin(g, NW, R), share_begin(g + 1, NW, R));
+    warp_pipeline(job, ring, c);
+}
+
+// S5 ([TS 2.A] cascade decode over the three tiers; [TS 2.C] Sparse Loading):
+// persistent streaming attention over the tokens of all units.
+template <int ES, int D, int G>
+__global__ void __launch_bounds__(AT_NW * 32, 1) k_attn_stream(const __grid_constant__ Params P)
+{
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    __shared__ unsigned long long red[AT_NW];
+    using SM = AttnSmem<ES, D, G>;
+    SM &sm = *reinterpret_cast<SM *>(smem_raw);
+    const Ctl c = make_ctl(P);
+    ring_init(sm.ring);
+    allow_dependents();
+    wait_prior_grid();
+    const int64_t T = attn_prologue<ES, D, G>(P, sm, c, red);
+    // every warp that takes part gets a non-empty share
+    const int64_t NW = min((int64_t)gridDim.x * AT_NW, T);
+    const int64_t g = (int64_t)blockIdx.x * AT_NW + (threadIdx.x >> 5);
+    if (g < NW) {
+        AttnJob<ES, D, G> job(P, c, sm, NW, T, g);
+        warp_pipeline(job, sm.ring, c);
     }
-}
-
-// S1 ([TS 2.B] max-pooled logits over the query group; [TS 2.A] Tier 2):
-// persistent streaming scorer; also records each tile's score range.
-template <int ES, int D, int G>
-__global__ void __launch_bounds__(S_THREADS, 1) k_score_stream(const __grid_constant__ Params P)
-{
-    stream_kernel_body<ES, D, G, ScoreTile, false>(P, P.units * P.score_tiles);
-}
-
-// S5 ([TS 2.A] cascade decode over the three tiers; [TS 2.C] Sparse Loading).
-template <int ES, int D, int G>
-__global__ void __launch_bounds__(S_THREADS, 1) k_attn_stream(const __grid_constant__ Params P)
-{
-    stream_kernel_body<ES, D, G, AttnTile, true>(P, P.units * P.attn_tiles);
 }
 
 // Rewrite Cache ([TS 2.C]): copy the k selected K/V rows of unit u, listed in
@@ -140,14 +140,19 @@ __global__ void __launch_bounds__(NT) k_unit(const __grid_constant__ Params P)
     if (P.do_select) {
         float m, zlo;
         if (P.have_range) {
-            float mx = -INFINITY, mn = INFINITY;
-            const int64_t t0 = (int64_t)u * P.score_tiles;
-            for (int i = threadIdx.x; i < P.score_tiles; i += NT) {
-                mx = fmaxf(mx, __ldcg(P.tile_max + t0 + i));
-                mn = fminf(mn, __ldcg(P.tile_min + t0 + i));
+            // the scorer's range words of the unit (key 0: no score), reset
+            // for the next step once read
+            if (threadIdx.x == 0) {
+                const uint32_t kmax = __ldcg(P.urange + 2 * u), kmin = __ldcg(P.urange + 2 * u + 1);
+                sm.redf[0] = kmax ? ord_val(kmax) : -INFINITY;
+                sm.redf[1] = kmin ? ord_val(~kmin) : INFINITY;
+                P.urange[2 * u] = 0;
+                P.urange[2 * u + 1] = 0;
             }
-            m = block_max<NT>(mx, sm.redf);
-            zlo = -block_max<NT>(-mn, sm.redf);
+            __syncthreads();
+            m = sm.redf[0];
+            zlo = sm.redf[1];
+            __syncthreads();
         } else {
             unit_range(zu, n, &m, &zlo, sm);
         }
@@ -259,9 +264,9 @@ std::atomic<uint64_t> g_wait_ns{1000000000ull};
 std::atomic<int32_t> g_withhold{0};
 
 struct WsLayout {
-    size_t ctl, attn_done, tile_max, tile_min, part, idxbuf, zbuf, total;
+    size_t ctl, attn_cnt, urange, part, idxbuf, zbuf, total;
     int64_t z_stride;
-    int score_tiles, attn_tiles, score_rows, attn_toks;
+    int part_slots;
 };
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -312,22 +317,33 @@ static hkv_status check_problem(const hkv_problem *p)
     return HKV_OK;
 }
 
+static int sm_count()
+{
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    return sms;
+}
+
+// Streaming CTAs the attention records are sized for: one per SM of the
+// current device (148 on B200, also assumed when no device can be queried).
+static int stream_ctas()
+{
+    const int sms = sm_count();
+    return sms > 0 ? sms : 148;
+}
+
 static WsLayout layout_of(const hkv_problem *p, const hkv_tier *dense, const hkv_tier *sparse,
                           const hkv_tier *cond)
 {
+    (void)dense;
+    (void)cond;
     WsLayout L{};
-    const int es = es_of(p->dtype);
     const int64_t units = (int64_t)p->B * p->Hkv;
     const int G = p->Hq / p->Hkv;
     const int ncap = sparse ? sparse->cap : 0;
-    const int wcap = dense ? dense->cap : 0;
-    const int ccap = cond ? cond->cap : 0;
-    const int rowb = p->D * es;
-    L.score_rows = SCORE_TILE_STAGES * (S_SLOT / rowb);
-    L.attn_toks = ATTN_TILE_STAGES * ((S_SLOT / 2) / rowb);
-    L.score_tiles = std::max(1, (ncap + L.score_rows - 1) / L.score_rows);
-    const int64_t max_tokens = (int64_t)wcap + std::min<int64_t>(p->bmax, ncap) + ccap;
-    L.attn_tiles = (int)std::max<int64_t>(1, (max_tokens + L.attn_toks - 1) / L.attn_toks);
+    L.part_slots = (int)(stream_ctas() * (int64_t)AT_NW + units);
     L.z_stride = (int64_t)align_up((size_t)std::max(ncap, 1), 4);
     size_t o = 0;
     auto take = [&](size_t bytes) {
@@ -335,18 +351,19 @@ static WsLayout layout_of(const hkv_problem *p, const hkv_tier *dense, const hkv
         o = align_up(o + bytes, 256);
         return at;
     };
+    // what must start at zero comes first: status word, counters, range words
     L.ctl = take(256);
-    L.attn_done = take(units * 4);
-    L.tile_max = take(units * L.score_tiles * 4);
-    L.tile_min = take(units * L.score_tiles * 4);
-    L.part = take((size_t)units * L.attn_tiles * part_stride(p->D, G) * 4);
+    L.attn_cnt = take(units * 4);
+    L.urange = take(units * 8);
+    L.part = take((size_t)L.part_slots * part_stride(p->D, G) * 4);
     L.idxbuf = take(units * (size_t)std::max(p->bmax, 1) * 4);
     L.zbuf = take((size_t)units * L.z_stride * 4);
     L.total = o;
     return L;
 }
 
-static Params base_params(const hkv_problem *p, const WsLayout &L, char *ws)
+static Params base_params(const hkv_problem *p, const WsLayout &L, char *ws, const hkv_tier *dense,
+                          const hkv_tier *sparse, const hkv_tier *cond)
 {
     Params P{};
     P.B = p->B;
@@ -362,18 +379,16 @@ static Params base_params(const hkv_problem *p, const WsLayout &L, char *ws)
     P.layout = p->layout;
     P.inv_temp = p->inv_temp;
     P.p_unit = p->p_unit;
-    P.score_tiles = L.score_tiles;
-    P.attn_tiles = L.attn_tiles;
-    P.score_rows = L.score_rows;
-    P.attn_toks = L.attn_toks;
     P.z_stride = L.z_stride;
     P.wait_ns = g_wait_ns.load();
     P.withhold = g_withhold.load();
     P.ctl = reinterpret_cast<uint32_t *>(ws + L.ctl);
-    P.attn_done = reinterpret_cast<uint32_t *>(ws + L.attn_done);
-    P.tile_max = reinterpret_cast<float *>(ws + L.tile_max);
-    P.tile_min = reinterpret_cast<float *>(ws + L.tile_min);
+    P.attn_cnt = reinterpret_cast<uint32_t *>(ws + L.attn_cnt);
     P.part = reinterpret_cast<float *>(ws + L.part);
+    P.part_slots = L.part_slots;
+    P.attn_prefix = P.units <= PREFIX_CAP;
+    const int ncap = sparse ? sparse->cap : 0;
+    P.attn_span = (dense ? dense->cap : 0) + std::min(p->bmax, ncap) + (cond ? cond->cap : 0);
     return P;
 }
 
@@ -435,15 +450,6 @@ static hkv_status prepare(const void *fn, int threads, size_t smem, int *blocks_
     return HKV_OK;
 }
 
-static int sm_count()
-{
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return 0;
-    return sms;
-}
-
 // Launch `kernel` over `grid` CTAs. With pdl the launch is a programmatic
 // dependent of the previous kernel on the stream: it may start early, and the
 // kernel calls wait_prior_grid() before it reads that kernel's results.
@@ -473,18 +479,19 @@ static hkv_status launch(K kernel, int grid, int threads, size_t smem, cudaStrea
 }
 
 // Streaming kernels: as many CTAs as are resident at once (one per SM), at
-// most one per tile.
+// most max_ctas.
 template <typename K>
-static hkv_status launch_stream(K kernel, size_t smem, int tiles, cudaStream_t stream, const Params &P, bool pdl)
+static hkv_status launch_stream(K kernel, int threads, size_t smem, int max_ctas, cudaStream_t stream,
+                                const Params &P, bool pdl)
 {
     int bps = 0;
-    hkv_status s = prepare((const void *)kernel, S_THREADS, smem, &bps);
+    hkv_status s = prepare((const void *)kernel, threads, smem, &bps);
     if (s != HKV_OK)
         return s;
     const int sms = sm_count();
     if (sms <= 0 || bps <= 0)
         return HKV_ERR_CUDA;
-    return launch(kernel, std::min(tiles, bps * sms), S_THREADS, smem, stream, P, pdl);
+    return launch(kernel, std::max(1, std::min(max_ctas, bps * sms)), threads, smem, stream, P, pdl);
 }
 
 // Dispatch over the compile-time (element size, head dim, group size).
@@ -509,8 +516,8 @@ template <int ES, int D, int G>
 struct RunScore {
     static hkv_status run(const Params &P, cudaStream_t s, bool pdl)
     {
-        return launch_stream(k_score_stream<ES, D, G>, sizeof(SSmem<ES, D, G>), P.units * P.score_tiles, s, P,
-                             pdl);
+        return launch_stream(k_score_stream<ES, D, G>, sc_nw(G) * 32, sizeof(typename ScoreJob<ES, D, G>::RingT),
+                             1 << 20, s, P, pdl);
     }
 };
 
@@ -518,7 +525,10 @@ template <int ES, int D, int G>
 struct RunAttn {
     static hkv_status run(const Params &P, cudaStream_t s, bool pdl)
     {
-        return launch_stream(k_attn_stream<ES, D, G>, sizeof(SSmem<ES, D, G>), P.units * P.attn_tiles, s, P, pdl);
+        // the records hold (CTAs x warps + units) slots
+        const int max_ctas = (P.part_slots - P.units) / AT_NW;
+        return launch_stream(k_attn_stream<ES, D, G>, AT_NW * 32, sizeof(AttnSmem<ES, D, G>), max_ctas, s, P,
+                             pdl);
     }
 };
 
@@ -548,7 +558,7 @@ hkv_status prologue(const hkv_problem *prob, const hkv_tier *dense, const hkv_ti
     *L = layout_of(prob, dense, sparse, cond);
     if ((s = check_ws(ws, ws_bytes, *L)) != HKV_OK)
         return s;
-    *P = base_params(prob, *L, static_cast<char *>(ws));
+    *P = base_params(prob, *L, static_cast<char *>(ws), dense, sparse, cond);
     P->dense = tier_p(dense);
     P->sparse = tier_p(sparse);
     P->cond = tier_p(cond);
@@ -791,12 +801,14 @@ hkv_status hkv_step(const hkv_problem *prob, const void *q, const hkv_tier *dens
     P.k_out = static_cast<char *>(o->k_out);
     P.v_out = static_cast<char *>(o->v_out);
     P.layout = HKV_LAYOUT_PAD_MAX;  // the three kernels work on PAD_MAX rows
-    // 1. scores, and each scoring tile's score range
+    // 1. scores, and the score range of each unit
     const bool scored = sparse->cap > 0;
-    if (scored && (s = dispatch<RunScore>(prob, P, st, false)) != HKV_OK)
+    Params S = P;
+    S.urange = reinterpret_cast<uint32_t *>(wsb + L.urange);
+    if (scored && (s = dispatch<RunScore>(prob, S, st, false)) != HKV_OK)
         return s;
     // 2. calibration, Top-p budget, cut and compaction, per unit
-    Params U = P;
+    Params U = S;
     U.have_range = scored;
     U.do_select = 1;
     U.do_compact = 1;
@@ -879,12 +891,15 @@ extern "C" hkv_status hkv_cascade_decode_noalloc(const hkv_problem *prob, const 
             return HKV_ERR_INVALID_ARG;
     }
     // The attention uses the front of the workspace layout: the status and
-    // counter words, the score ranges and the tile records (everything before
-    // the index and score buffers, which only hkv_step uses).
+    // counter words, the range words and the records. It needs at least the
+    // records of one CTA (a record per warp and per unit); when the array
+    // holds fewer than a full grid needs, fewer CTAs run.
     const WsLayout L = layout_of(prob, dense, sparse, condensed);
-    const size_t need = L.idxbuf;
-    if (need > HKV_NOALLOC_SCRATCH_BYTES)
+    const size_t rec = (size_t)part_stride(prob->D, prob->Hq / prob->Hkv) * sizeof(float);
+    const int64_t units = (int64_t)prob->B * prob->Hkv;
+    if (L.part + (size_t)(units + AT_NW) * rec > HKV_NOALLOC_SCRATCH_BYTES)
         return HKV_ERR_WORKSPACE;
+    const int slots = (int)std::min<int64_t>(L.part_slots, (HKV_NOALLOC_SCRATCH_BYTES - L.part) / rec);
     const cudaStream_t st = (cudaStream_t)stream;
     if ((int64_t)prob->B * prob->Hkv == 0)
         return status ? (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) == cudaSuccess ? HKV_OK : HKV_ERR_CUDA)
@@ -893,7 +908,8 @@ extern "C" hkv_status hkv_cascade_decode_noalloc(const hkv_problem *prob, const 
     if ((s = noalloc_scratch(&scratch)) != HKV_OK)
         return s;
     char *base = static_cast<char *>(scratch);
-    Params P = base_params(prob, L, base);
+    Params P = base_params(prob, L, base, dense, sparse, condensed);
+    P.part_slots = slots;
     P.dense = tier_p(dense);
     P.sparse = tier_p(sparse);
     P.cond = tier_p(condensed);
@@ -905,7 +921,7 @@ extern "C" hkv_status hkv_cascade_decode_noalloc(const hkv_problem *prob, const 
     P.lse = lse;
     // the status word, the ticket and exit counters and the per-unit tile
     // counters must start at zero; the previous call may have left them set
-    if (cudaMemsetAsync(base, 0, L.tile_max, st) != cudaSuccess)
+    if (cudaMemsetAsync(base, 0, L.urange, st) != cudaSuccess)
         return HKV_ERR_CUDA;
     if ((s = dispatch<RunAttn>(prob, P, st, false)) != HKV_OK)
         return s;

@@ -128,6 +128,20 @@ __device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parity, uint
     }
 }
 
+// Wait at most wait_ns for the phase of `bar` with the given parity, whatever
+// the status word says (used to let copies already started land before a CTA
+// exits after a timeout).
+__device__ __noinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, uint64_t wait_ns)
+{
+    const uint64_t t0 = global_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity))
+            return true;
+        if ((it & 15u) == 0 && global_ns() - t0 > wait_ns)
+            return false;
+    }
+}
+
 // Wait for the phase of `bar` with the given parity to complete (bounded).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, const Ctl &c)
 {

@@ -7,13 +7,12 @@
 // Summary of that paper.
 //
 // Two kinds of kernels:
-//  - streaming kernels (scoring, attention): one producer warp feeds S_NCW
-//    consumer warps, each through its own S_SPW-slot shared-memory ring. The
-//    producer claims tiles (runs of stages) for each warp from a global ticket
-//    counter and issues the stage copies (1-D TMA bulk copies for contiguous
-//    rows, 16-byte cp.async for gathered rows); a stage descriptor travels with
-//    the data through the slot's mbarrier. Consumers never synchronise with
-//    each other, so tiles of different warps overlap freely.
+//  - streaming kernels (scoring, attention): every warp runs its own copy
+//    pipeline over a contiguous share of the kernel's work (a static, balanced
+//    partition: no tickets, no producer warp). It keeps several stages in
+//    flight in its own ring of shared-memory slots, armed and filled by the
+//    warp itself: 1-D TMA bulk copies for contiguous rows, 16-byte cp.async for
+//    gathered rows, completion on one mbarrier per slot.
 //  - per-unit kernels (selection, compaction, calibration, layout): one CTA of
 //    SEL_THREADS threads per (sequence, KV head).
 // No tensor cores: a one-query decode is a GEMV (about 4 flop per byte), bound
@@ -24,15 +23,17 @@
 
 namespace hkv {
 
-constexpr int S_NCW = 8;                  // consumer warps of a streaming CTA
-constexpr int S_SPW = 2;                  // ring slots per consumer warp
-constexpr int S_SLOT = 8192;              // bytes per slot
-constexpr int S_THREADS = (S_NCW + 1) * 32;
-constexpr int S_PROD = S_NCW;             // warp index of the producer
-constexpr int SCORE_TILE_STAGES = 4;      // stages per scoring tile
-constexpr int ATTN_TILE_STAGES = 8;       // stages per attention tile
+constexpr int SC_SLOT = 4096;             // scoring: bytes per stage (K rows)
+// scoring: warps per CTA and ring slots per warp (192 KB of slots per CTA);
+// eight query heads per group keep 64 more registers of queries per lane, so
+// they run half the warps with twice the slots
+__host__ __device__ constexpr int sc_nw(int G) { return G >= 8 ? 8 : 16; }
+__host__ __device__ constexpr int sc_stages(int G) { return G >= 8 ? 6 : 3; }
+constexpr int AT_NW = 8;                  // attention: warps per CTA
+constexpr int AT_SLOT = 8192;             // attention: bytes per stage (K rows, then as many V rows)
+constexpr int AT_STAGES = 3;              // attention: ring slots per warp
 constexpr int SC_FLOATS = 256;            // per-warp logits of one attention stage
-constexpr int TTOK_CAP = 256;             // tokens of one attention tile (any geometry)
+constexpr int PREFIX_CAP = 2048;          // attention: units whose token prefix fits in shared memory
 constexpr int SEL_THREADS = 512;          // per-unit kernels
 constexpr float LOG2E = 1.4426950408889634f;
 
@@ -61,18 +62,16 @@ struct Params {
     float *out, *lse, *m_out, *logZ_out, *P_out;
     char *k_out, *v_out;
     // workspace
-    uint32_t *ctl;        // [0] status, [1] ticket, [2] exit count
-    uint32_t *attn_done;  // [units] finished attention tiles
-    float *tile_max;      // [units * score_tiles]
-    float *tile_min;      // [units * score_tiles] smallest finite score of the tile
-    float *part;          // [units * attn_tiles * part_stride] attention tile records
-    // tiling
-    int32_t score_tiles, attn_tiles;  // per unit
-    int32_t score_rows;               // rows per scoring tile
-    int32_t attn_toks;                // tokens per attention tile
-    int32_t have_range;               // tile_max / tile_min hold the units' score range
-    int32_t do_select, do_compact;    // per-unit kernel: which steps to run
-    int32_t withhold;                 // fault injection: the producer never arms a slot
+    uint32_t *ctl;        // [0] status word
+    uint32_t *urange;     // [units][2] score range of each unit as order keys (step only, else nullptr)
+    uint32_t *attn_cnt;   // [units] attention records finished
+    float *part;          // [part_slots * part_stride] attention records
+    int32_t part_slots;   // record slots (streaming warps of the attention grid + units)
+    int32_t attn_prefix;  // attention partition over actual tokens (units <= PREFIX_CAP), else over capacity
+    int32_t attn_span;    // capacity partition: token positions per unit (W cap + min(bmax, n cap) + C cap)
+    int32_t have_range;   // per-unit kernel: urange holds the units' score ranges
+    int32_t do_select, do_compact;  // per-unit kernel: which steps to run
+    int32_t withhold;     // fault injection: streaming warps never arm their stages
     uint64_t wait_ns;
 };
 
@@ -127,9 +126,20 @@ __device__ __forceinline__ int unit_budget(const Params &P, int u, int n, const 
     return k;
 }
 
-// Floats of one attention tile record (o[G][D], m[G], l[G]), padded to a
-// multiple of 4.
+// Floats of one attention record (o[G][D], m[G], l[G]), padded to a multiple of 4.
 __host__ __device__ constexpr int part_stride(int D, int G) { return (G * (D + 2) + 3) / 4 * 4; }
+
+// Order-preserving 32-bit keys of floats (larger float, larger key), so that
+// atomicMax on keys takes the maximum of floats. Key 0 means "none".
+__device__ __forceinline__ uint32_t ord_key(float x)
+{
+    const uint32_t b = __float_as_uint(x);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float ord_val(uint32_t k)
+{
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
 
 // Compile-time geometry of a (element size, head dim, group size) instance.
 // A K row is read by LPR lanes, each taking CPL 16-byte chunks (chunk l % LPR
@@ -144,20 +154,18 @@ struct Geo {
     static constexpr int VEC = 16 / ES;                   // elements per 16-byte chunk
     static constexpr int NP = CPL * VEC / 2;              // float2 pairs per lane per row
     static constexpr int ITB = 32 * 16 * CPL;             // bytes of one warp iteration
-    static constexpr int SITERS = S_SLOT / ITB;           // iterations per scoring stage
-    static constexpr int AITERS = (S_SLOT / 2) / ITB;     // iterations over an attention stage's keys
+    static constexpr int SITERS = SC_SLOT / ITB;          // iterations per scoring stage
+    static constexpr int AITERS = (AT_SLOT / 2) / ITB;    // iterations over an attention stage's keys
     static constexpr int NB0 = LPR / G;
-    static constexpr int NB = NB0 < AITERS ? NB0 : AITERS;  // iterations reduced together
+    static constexpr int NB0S = NB0 < SITERS ? NB0 : SITERS;
+    static constexpr int NB = NB0S < AITERS ? NB0S : AITERS;  // iterations reduced together
     static constexpr int NV = NB * G;                     // partial sums per lane before reduction
     static constexpr int REP = LPR / NV;                  // lanes holding the same sum afterwards
-    static constexpr int SROWS = S_SLOT / ROWB;           // rows per scoring stage
-    static constexpr int ATOK = (S_SLOT / 2) / ROWB;      // tokens per attention stage
+    static constexpr int SROWS = SC_SLOT / ROWB;          // rows per scoring stage
+    static constexpr int ATOK = (AT_SLOT / 2) / ROWB;     // tokens per attention stage
     static constexpr int DPL = D / 32;                    // PV: head-dim elements per lane
-    static constexpr int QB = G * D * ES;                 // bytes of the group's queries
     static_assert(G >= 1 && G <= LPR, "group size must not exceed lanes per row");
-    static_assert(ATOK * G <= SC_FLOATS && ATOK <= 32, "attention stage");
-    static_assert(ATOK * ATTN_TILE_STAGES <= TTOK_CAP, "attention tile");
-    static_assert(QB % 16 == 0, "query buffer");
+    static_assert(ATOK * G <= SC_FLOATS && ATOK <= 32 && SROWS <= 32, "stage sizes");
     static_assert(SITERS % NB == 0 && AITERS % NB == 0 && LPR % NV == 0, "iteration batches");
 };
 
@@ -165,54 +173,76 @@ struct Geo {
 // Streaming engine
 // =============================================================================
 
-enum StageKind : int32_t { STG_END = 0, STG_SCORE = 1, STG_ATTN = 2 };
+enum : int32_t { SD_FIRST = 1, SD_LAST = 2, SD_GATHER = 4, SD_ARMED = 8 };
 
 struct StageDesc {
-    int32_t kind, unit, start, count;  // rows (scoring) or tokens (attention) [start, start + count)
-    int32_t tile, last, total, first;  // tile id; last / first stage of the tile; attention: tokens of the unit
+    int32_t unit, start, count, flags;  // rows (scoring) or unit-local tokens (attention) [start, start + count)
 };
 
-struct ProdState {  // producer's view of one consumer warp
-    int32_t tile, unit, next, nst, base, limit, ended, ntile;
-    int32_t W, k, total, pad;
-    uint32_t issued;
+template <int NW, int SLOT, int NS>
+struct __align__(128) Ring {
+    static constexpr int kNW = NW, kNS = NS;
+    unsigned char slot[NW][NS][SLOT];
+    uint64_t full[NW][NS];
+    StageDesc desc[NW][NS];
 };
 
-template <int ES, int D, int G>
-struct __align__(128) SSmem {
-    unsigned char slot[S_NCW][S_SPW][S_SLOT];
-    unsigned char qbuf[S_NCW][2][G * D * ES];  // the tile's queries, double-buffered per warp
-    float sc[S_NCW][SC_FLOATS];
-    int32_t tidx[S_NCW][TTOK_CAP];             // producer: sparse rows of each warp's attention tile
-    StageDesc desc[S_NCW][S_SPW];
-    uint64_t full[S_NCW][S_SPW];
-    uint64_t empty[S_NCW][S_SPW];
-    ProdState ps[S_NCW];
-    const char *ksrc[32], *vsrc[32];           // producer scratch: rows of one attention stage
-    int32_t ticket_bc;
-};
-
-template <class SM>
-__device__ __forceinline__ void stream_init(SM &sm)
+template <class R>
+__device__ __forceinline__ void ring_init(R &r)
 {
     if (threadIdx.x == 0) {
-        for (int w = 0; w < S_NCW; ++w)
-            for (int j = 0; j < S_SPW; ++j) {
-                mbar_init(&sm.full[w][j], 1);
-                mbar_init(&sm.empty[w][j], 1);
-            }
-        for (int w = 0; w < S_NCW; ++w) {
-            ProdState &s = sm.ps[w];
-            s.tile = -1;
-            s.next = s.nst = 0;
-            s.ended = 0;
-            s.issued = 0;
-            s.ntile = 0;
-            s.unit = -1;
-        }
+        for (int w = 0; w < R::kNW; ++w)
+            for (int j = 0; j < R::kNS; ++j)
+                mbar_init(&r.full[w][j], 1);
         mbar_fence_init();
     }
     __syncthreads();
+}
+
+// The warp's pipeline. Job supplies (all lanes call each, warp-uniformly):
+//   bool next(StageDesc &d)                  -- the warp's next stage, or false
+//   void issue(const StageDesc &d, int j)    -- record d in slot j, arm it and start its copies
+//   void consume(const StageDesc &d, const unsigned char *slot)
+// Up to NS stages are in flight. If a wait runs out (status word set), the
+// warp stops consuming, waits (bounded) for the copies it started, and returns.
+template <class Job, class R>
+__device__ void warp_pipeline(Job &job, R &ring, const Ctl &c)
+{
+    constexpr int NS = Job::NS;
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    uint32_t issued = 0, consumed = 0;
+    StageDesc d;
+    while (issued < (uint32_t)NS && job.next(d)) {
+        job.issue(d, (int)issued);
+        ++issued;
+    }
+    bool ok = true;
+    while (consumed < issued) {
+        const int j = (int)(consumed % NS);
+        if (!mbar_wait(&ring.full[w][j], (consumed / NS) & 1u, c)) {
+            ok = false;
+            break;
+        }
+        const StageDesc cd = ring.desc[w][j];
+        job.consume(cd, ring.slot[w][j]);
+        __syncwarp();
+        ++consumed;
+        if (job.next(d)) {
+            if (lane == 0)
+                fence_proxy_async_smem();  // this warp's reads of the slot before the copies that refill it
+            job.issue(d, j);
+            ++issued;
+        }
+    }
+    if (!ok) {
+        // the copies already started must land before the CTA may exit
+        for (uint32_t i = consumed; i < issued; ++i) {
+            const int j = (int)(i % NS);
+            if (ring.desc[w][j].flags & SD_ARMED)
+                mbar_wait_bounded(&ring.full[w][j], (i / NS) & 1u, c.wait_ns);
+        }
+    }
+    __syncwarp();
 }
 
 // ---- warp butterfly over the LPR lanes of a row: NV partial sums per lane ->
@@ -254,19 +284,26 @@ __device__ __forceinline__ void unpack16(const uint4 &w, float2 *kv)
     }
 }
 
-// The lane's slice of the group's G queries (chunks l % LPR and l % LPR + LPR
-// of each row), from the warp's shared query buffer.
+// The lane's slice of the group's G queries of unit u (chunks l % LPR and
+// l % LPR + LPR of each row), read from global memory (small, L2-resident).
 template <int ES, int D, int G>
-__device__ __forceinline__ void load_q_smem(const unsigned char *qb, int lane, float2 (&qv)[G][Geo<ES, D, G>::NP])
+__device__ __forceinline__ void load_q(const Params &P, int u, int lane, float2 (&qv)[G][Geo<ES, D, G>::NP])
 {
     using Gm = Geo<ES, D, G>;
+    const int b = u / P.Hkv, h = u % P.Hkv;
+    const char *qb = P.q + (int64_t)(b * P.Hq + h * G) * D * ES;
     const int c0 = lane % Gm::LPR;
+    uint4 w[G][Gm::CPL];
 #pragma unroll
     for (int g = 0; g < G; ++g)
 #pragma unroll
         for (int cc = 0; cc < Gm::CPL; ++cc)
-            unpack16<ES>(*reinterpret_cast<const uint4 *>(qb + g * Gm::ROWB + (c0 + cc * Gm::LPR) * 16),
-                         &qv[g][cc * (Gm::VEC / 2)]);
+            w[g][cc] = __ldg(reinterpret_cast<const uint4 *>(qb + g * Gm::ROWB + (c0 + cc * Gm::LPR) * 16));
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int cc = 0; cc < Gm::CPL; ++cc)
+            unpack16<ES>(w[g][cc], &qv[g][cc * (Gm::VEC / 2)]);
 }
 
 // One batch of NB warp iterations over staged rows: per-lane partial dot
@@ -300,344 +337,159 @@ __device__ __forceinline__ float qk_batch(const unsigned char *stage, int it0, i
     return v[0];
 }
 
-// Is the producer's next slot of warp w free?
-template <class SM>
-__device__ __forceinline__ bool slot_free(SM &sm, int w)
+// Warp g of NW warps over a line of T positions takes [T g / NW, T (g+1) / NW).
+__device__ __forceinline__ int64_t share_begin(int64_t g, int64_t NW, int64_t T) { return g * T / NW; }
+
+// The warp whose share holds position t (0 <= t < T): the last g with
+// share_begin(g) <= t, which is never an empty share.
+__device__ __forceinline__ int64_t share_owner(int64_t t, int64_t NW, int64_t T)
 {
-    const uint32_t i = sm.ps[w].issued;
-    return mbar_test(&sm.empty[w][i % S_SPW], ((i / S_SPW) & 1u) ^ 1u);
+    return ((t + 1) * NW + T - 1) / T - 1;
 }
 
-// Producer loop shared by both streaming kernels (all 32 lanes of the producer
-// warp run it together). Tile is a policy type:
-//   setup(P, sm, w, tile, c)           -- fill sm.ps[w] for a claimed tile
-//   issue(P, sm, w, slot, c, policy)   -- arm the slot's barrier and copy a stage
-// Returns when every consumer warp has been sent an END stage.
-template <class Tile, class SM>
-__device__ void producer_loop(const Params &P, SM &sm, const Ctl &c, int n_tiles, uint64_t policy)
-{
-    const int lane = threadIdx.x & 31;
-    int rr = 0, ended = 0;
-    bool exhausted = false;
-    uint64_t idle_since = 0;
-    while (ended < S_NCW) {
-        bool want = false;
-        if (lane < S_NCW && !sm.ps[lane].ended)
-            want = slot_free(sm, lane);
-        const unsigned mask = __ballot_sync(0xffffffffu, want);
-        if (mask == 0) {
-            // every ring is full: wait, bounded, for a consumer to free a slot
-            if (idle_since == 0)
-                idle_since = global_ns();
-            else if (global_ns() - idle_since > c.wait_ns || timed_out(c)) {
-                if (lane == 0)
-                    raise_flag(c, HKV_DEV_TIMEOUT);
-                break;
+// ---- scoring ([TS 2.B] max-pooled attention logits; [TS 2.A] Tier 2) --------
+//
+// Work line: the sparse tier's capacity rows of all units, unit-major; a warp
+// scores the rows of its share that lie below the unit's length. In hkv_step
+// each warp also folds the range of the scores it wrote into its units'
+// range words (atomic max of order keys), which the selection starts from.
+
+template <int ES, int D, int G>
+struct ScoreJob {
+    using Gm = Geo<ES, D, G>;
+    static constexpr int NS = sc_stages(G), NW = sc_nw(G);
+    using RingT = Ring<NW, SC_SLOT, NS>;
+
+    const Params &P;
+    const Ctl &c;
+    RingT &ring;
+    uint64_t policy;
+    int w, lane;
+    // generator: the share's next row is row j of unit u; `left` rows remain
+    int u, j;
+    int64_t left;
+    int gu = -1, gn = 0, last_unit = -1;
+    const char *kbase = nullptr;  // K rows of unit gu (the unit of the stage last returned)
+    // consumer
+    float2 qv[G][Gm::NP];
+    float tmax = -INFINITY, tmin = INFINITY;
+
+    __device__ ScoreJob(const Params &P_, const Ctl &c_, RingT &ring_, int64_t r0, int64_t r1)
+        : P(P_), c(c_), ring(ring_), policy(evict_first_policy()), w(threadIdx.x >> 5), lane(threadIdx.x & 31)
+    {
+        const int cap = max(P.sparse.cap, 1);
+        u = (int)(r0 / cap);
+        j = (int)(r0 - (int64_t)u * cap);
+        left = r1 - r0;
+    }
+
+    __device__ __forceinline__ bool next(StageDesc &d)
+    {
+        while (left > 0) {
+            if (u != gu) {  // length and K rows of a new unit
+                gu = u;
+                gn = tier_len(P.sparse, u, c);
+                const int b = u / P.Hkv, h = u % P.Hkv;
+                kbase = P.sparse.k + ((int64_t)b * P.sparse.sb + (int64_t)h * P.sparse.sh) * ES;
             }
-            __nanosleep(64);
-            continue;
-        }
-        idle_since = 0;
-        const unsigned hi = mask & ~((1u << rr) - 1u);
-        const int w = (hi ? __ffs(hi) : __ffs(mask)) - 1;
-        rr = (w + 1) % S_NCW;
-        ProdState &s = sm.ps[w];
-        if (s.tile < 0 || s.next >= s.nst) {
-            // the warp needs a new tile
-            int t = n_tiles;
-            if (!exhausted) {
-                if (lane == 0)
-                    sm.ticket_bc = (int)atomicAdd(P.ctl + 1, 1u);
-                __syncwarp();
-                t = sm.ticket_bc;
-                __syncwarp();
-            }
-            if (t >= n_tiles) {
-                exhausted = true;
-                const uint32_t i = s.issued;
-                const int j = i % S_SPW;
-                if (lane == 0) {
-                    sm.desc[w][j].kind = STG_END;
-                    mbar_arrive(&sm.full[w][j]);
-                    s.issued = i + 1;
-                    s.ended = 1;
-                }
-                __syncwarp();
-                ++ended;
+            const int seg = (int)min(left, (int64_t)(P.sparse.cap - j));  // rows of unit u left in the share
+            const int vend = min(j + seg, gn);
+            if (j >= vend) {
+                left -= seg;
+                ++u;
+                j = 0;
                 continue;
             }
-            Tile::setup(P, sm, w, t, c);
-            __syncwarp();
-            if (s.nst == 0)
-                continue;  // nothing to stream for this tile
-        }
-        const uint32_t i = s.issued;
-        const int j = i % S_SPW;
-        Tile::issue(P, sm, w, j, c, policy);
-        __syncwarp();
-        if (lane == 0) {
-            s.issued = i + 1;
-            s.next += 1;
-        }
-        __syncwarp();
-    }
-    // Before the CTA can exit, every copy this producer started must have
-    // landed: wait (bounded) for the last phases it armed.
-    if (lane < S_NCW) {
-        const uint32_t iss = sm.ps[lane].issued;
-        for (uint32_t i = iss > S_SPW ? iss - S_SPW : 0; i < iss; ++i)
-            mbar_wait(&sm.full[lane][i % S_SPW], (i / S_SPW) & 1u, c);
-    }
-    __syncwarp();
-}
-
-// ---- scoring tiles ([TS 2.B] max-pooled attention logits; [TS 2.A] Tier 2) ----
-
-template <int ES, int D, int G>
-struct ScoreTile {
-    using Gm = Geo<ES, D, G>;
-    using SM = SSmem<ES, D, G>;
-
-    __device__ static void setup(const Params &P, SM &sm, int w, int t, const Ctl &c)
-    {
-        const int lane = threadIdx.x & 31;
-        const int u = t / P.score_tiles, ct = t % P.score_tiles;
-        const int n = tier_len(P.sparse, u, c);
-        const int r0 = ct * P.score_rows, r1 = min(n, r0 + P.score_rows);
-        ProdState &s = sm.ps[w];
-        if (lane == 0) {
-            s.tile = t;
-            s.unit = u;
-            s.base = r0;
-            s.limit = r1;
-            s.next = 0;
-            s.nst = r1 > r0 ? (r1 - r0 + Gm::SROWS - 1) / Gm::SROWS : 0;
-            if (s.nst == 0) {  // an empty tile still reports its (empty) score range
-                P.tile_max[t] = -INFINITY;
-                P.tile_min[t] = INFINITY;
-            }
-        }
-    }
-
-    __device__ static void issue(const Params &P, SM &sm, int w, int j, const Ctl &c, uint64_t policy)
-    {
-        const int lane = threadIdx.x & 31;
-        const ProdState &s = sm.ps[w];
-        const int rs = s.base + s.next * Gm::SROWS;
-        const int nr = min(Gm::SROWS, s.limit - rs);
-        const int b = s.unit / P.Hkv, h = s.unit % P.Hkv;
-        const TierP &T = P.sparse;
-        const char *kbase = T.k + ((int64_t)b * T.sb + (int64_t)h * T.sh) * ES;
-        const bool first = s.next == 0;
-        const uint32_t qbytes = first ? (uint32_t)Gm::QB : 0u;
-        unsigned char *qdst = sm.qbuf[w][s.ntile & 1];
-        if (lane == 0) {
-            StageDesc &d = sm.desc[w][j];
-            d.kind = STG_SCORE;
-            d.unit = s.unit;
-            d.start = rs;
-            d.count = nr;
-            d.tile = s.tile;
-            d.last = s.next == s.nst - 1;
-            d.first = first;
-            d.total = 0;
-            if (!P.withhold) {
-                mbar_arrive_expect_tx(&sm.full[w][j], (uint32_t)(nr * Gm::ROWB) + qbytes);
-                if (first)
-                    bulk_g2s(qdst, P.q + (int64_t)(b * P.Hq + h * G) * D * ES, Gm::QB, &sm.full[w][j], policy);
-                if (T.st == D)
-                    bulk_g2s(sm.slot[w][j], kbase + (int64_t)rs * T.st * ES, nr * Gm::ROWB, &sm.full[w][j],
-                             policy);
-            }
-        }
-        if (T.st != D && !P.withhold) {
-            __syncwarp();
-            for (int r = lane; r < nr; r += 32)
-                bulk_g2s(sm.slot[w][j] + r * Gm::ROWB, kbase + (int64_t)(rs + r) * T.st * ES, Gm::ROWB,
-                         &sm.full[w][j], policy);
-        }
-        if (lane == 0 && first)
-            sm.ps[w].ntile += 1;
-    }
-};
-
-// Consumer side of a scoring stage: z_j = scale * max_g q_g . k_j.
-template <int ES, int D, int G>
-__device__ __forceinline__ void score_stage(const Params &P, const unsigned char *stage, const StageDesc &d,
-                                            const float2 (&qv)[G][Geo<ES, D, G>::NP], float &tmax, float &tmin)
-{
-    using Gm = Geo<ES, D, G>;
-    const int lane = threadIdx.x & 31;
-    const int vi = (lane % Gm::LPR) / Gm::REP;
-    const bool writer = (lane % Gm::REP) == 0 && (vi % G) == 0;
-    float *zu = P.z + (int64_t)d.unit * P.z_stride + d.start;
-    for (int it0 = 0; it0 < Gm::SITERS && it0 * Gm::RPW < d.count; it0 += Gm::NB) {
-        float v = qk_batch<ES, D, G>(stage, it0, lane, qv);
-#pragma unroll
-        for (int o = 1; o < G; o <<= 1)
-            v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o * Gm::REP));
-        const int row = (it0 + vi / G) * Gm::RPW + lane / Gm::LPR;
-        if (writer && row < d.count) {
-            const float zz = v * P.scale;
-            zu[row] = zz;
-            tmax = fmaxf(tmax, zz);
-            if (zz != -INFINITY)
-                tmin = fminf(tmin, zz);
-        }
-    }
-}
-
-// ---- attention tiles ([TS 2.A] dense ++ selected sparse ++ condensed;
-// [TS 2.C] Sparse Loading: selected rows are read through the indices) --------
-
-template <int ES, int D, int G>
-struct AttnTile {
-    using Gm = Geo<ES, D, G>;
-    using SM = SSmem<ES, D, G>;
-
-    __device__ static void setup(const Params &P, SM &sm, int w, int t, const Ctl &c)
-    {
-        const int lane = threadIdx.x & 31;
-        const int u = t / P.attn_tiles, a = t % P.attn_tiles;
-        ProdState &s = sm.ps[w];
-        int W = s.W, k = s.k, total = s.total;
-        if (u != s.unit) {  // lengths of a new unit (every lane loads the same words)
-            const int n = tier_len(P.sparse, u, c);
-            W = tier_len(P.dense, u, c);
-            k = unit_budget(P, u, n, c);
-            total = W + k + tier_len(P.cond, u, c);
-        }
-        const int t0 = a * P.attn_toks, t1 = min(total, t0 + P.attn_toks);
-        // sparse rows of the tile, loaded with all loads in flight and checked
-        const int s0 = max(t0, W), s1 = min(t1, W + k);
-        if (s1 > s0) {
-            const int32_t *idx_row =
-                P.layout == HKV_LAYOUT_FLAT_SUM ? P.idx + __ldcg(P.offsets + u) : P.idx + (int64_t)u * P.bmax;
-            const int n_sparse = tier_len(P.sparse, u, c);
-            constexpr int PF = TTOK_CAP / 32;
-            int jv[PF];
-#pragma unroll
-            for (int i = 0; i < PF; ++i) {
-                const int tt = s0 + lane + 32 * i;
-                jv[i] = tt < s1 ? __ldcg(idx_row + (tt - W)) : 0;
-            }
-#pragma unroll
-            for (int i = 0; i < PF; ++i) {
-                const int tt = s0 + lane + 32 * i;
-                if (tt < s1) {
-                    int jj = jv[i];
-                    if (jj < 0 || jj >= n_sparse) {
-                        raise_flag(c, HKV_DEV_BAD_INDEX);
-                        jj = 0;
-                    }
-                    sm.tidx[w][tt - t0] = jj;
-                }
-            }
-        }
-        __syncwarp();
-        if (lane == 0) {
-            s.tile = t;
-            s.unit = u;
-            s.W = W;
-            s.k = k;
-            s.total = total;
-            s.base = t0;
-            s.limit = max(t0, t1);
-            s.next = 0;
-            // an empty tile still sends one (empty) stage so that it is counted
-            s.nst = t1 > t0 ? (t1 - t0 + Gm::ATOK - 1) / Gm::ATOK : 1;
-        }
-    }
-
-    __device__ static void issue(const Params &P, SM &sm, int w, int j, const Ctl &c, uint64_t policy)
-    {
-        const int lane = threadIdx.x & 31;
-        const ProdState &s = sm.ps[w];
-        const int ts = s.base + s.next * Gm::ATOK;
-        const int nt = max(0, min(Gm::ATOK, s.limit - ts));
-        const int b = s.unit / P.Hkv, h = s.unit % P.Hkv;
-        const int W = s.W, k = s.k;
-        const bool first = s.next == 0;
-        unsigned char *dst = sm.slot[w][j];
-        unsigned char *qdst = sm.qbuf[w][s.ntile & 1];
-        const char *qsrc = P.q + (int64_t)(b * P.Hq + h * G) * D * ES;
-        // contiguous dense or condensed run: two bulk copies
-        const bool in_dense = ts + nt <= W && P.dense.st == D;
-        const bool in_cond = ts >= W + k && P.cond.st == D;
-        if (lane == 0) {
-            StageDesc &d = sm.desc[w][j];
-            d.kind = STG_ATTN;
-            d.unit = s.unit;
-            d.start = ts;
-            d.count = nt;
-            d.tile = s.tile;
-            d.last = s.next == s.nst - 1;
-            d.first = first;
-            d.total = s.total;
-        }
-        if (!P.withhold) {
-            if (nt == 0 || in_dense || in_cond) {
-                if (lane == 0) {
-                    const uint32_t bytes = (uint32_t)(2 * nt * Gm::ROWB) + (first ? (uint32_t)Gm::QB : 0u);
-                    mbar_arrive_expect_tx(&sm.full[w][j], bytes);
-                    if (first)
-                        bulk_g2s(qdst, qsrc, Gm::QB, &sm.full[w][j], policy);
-                    if (nt > 0) {
-                        const TierP &T = in_dense ? P.dense : P.cond;
-                        const int64_t r0 = in_dense ? ts : ts - W - k;
-                        const int64_t off = ((int64_t)b * T.sb + (int64_t)h * T.sh + r0 * T.st) * ES;
-                        bulk_g2s(dst, T.k + off, nt * Gm::ROWB, &sm.full[w][j], policy);
-                        bulk_g2s(dst + S_SLOT / 2, T.v + off, nt * Gm::ROWB, &sm.full[w][j], policy);
-                    }
-                }
+            const int cnt = min(Gm::SROWS, vend - j);
+            const bool last = j + cnt >= vend;
+            d.unit = u;
+            d.start = j;
+            d.count = cnt;
+            d.flags = (u != last_unit ? SD_FIRST : 0) | (last ? SD_LAST : 0);
+            last_unit = u;
+            if (last) {
+                left -= seg;
+                ++u;
+                j = 0;
             } else {
-                // gathered rows: 16-byte cp.async by the whole warp
-                if (lane < nt) {
-                    const int t = ts + lane;
-                    const char *kb, *vb;
-                    int64_t off;
-                    if (t < W) {
-                        kb = P.dense.k;
-                        vb = P.dense.v;
-                        off = (int64_t)b * P.dense.sb + (int64_t)h * P.dense.sh + (int64_t)t * P.dense.st;
-                    } else if (t < W + k) {
-                        kb = P.sparse.k;
-                        vb = P.sparse.v;
-                        off = (int64_t)b * P.sparse.sb + (int64_t)h * P.sparse.sh +
-                              (int64_t)sm.tidx[w][t - s.base] * P.sparse.st;
-                    } else {
-                        kb = P.cond.k;
-                        vb = P.cond.v;
-                        off = (int64_t)b * P.cond.sb + (int64_t)h * P.cond.sh + (int64_t)(t - W - k) * P.cond.st;
-                    }
-                    sm.ksrc[lane] = kb + off * ES;
-                    sm.vsrc[lane] = vb + off * ES;
-                }
-                __syncwarp();
-                constexpr int CH = Gm::ROWB / 16;
-                static_assert(32 % CH == 0, "row chunks");
-                constexpr int RPI = 32 / CH;  // rows per warp instruction
-                const int cc = lane % CH, r0 = lane / CH;
-                for (int r = r0; r < nt; r += RPI) {
-                    cp_async16(dst + r * Gm::ROWB + cc * 16, sm.ksrc[r] + cc * 16);
-                    cp_async16(dst + S_SLOT / 2 + r * Gm::ROWB + cc * 16, sm.vsrc[r] + cc * 16);
-                }
-                if (first)
-                    for (int i = lane; i < Gm::QB / 16; i += 32)
-                        cp_async16(qdst + i * 16, qsrc + i * 16);
-                cp_async_arrive(&sm.full[w][j]);
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&sm.full[w][j]);
+                left -= cnt;
+                j += cnt;
+            }
+            return true;
+        }
+        return false;
+    }
+
+    __device__ __forceinline__ void issue(const StageDesc &d, int slot)
+    {
+        const TierP &T = P.sparse;
+        const char *src = kbase + (int64_t)d.start * T.st * ES;
+        unsigned char *dst = ring.slot[w][slot];
+        uint64_t *bar = &ring.full[w][slot];
+        const bool arm = !P.withhold;
+        if (lane == 0) {
+            ring.desc[w][slot] = StageDesc{d.unit, d.start, d.count, d.flags | (arm ? SD_ARMED : 0)};
+            if (arm) {
+                mbar_arrive_expect_tx(bar, (uint32_t)(d.count * Gm::ROWB));
+                if (T.st == D)
+                    bulk_g2s(dst, src, d.count * Gm::ROWB, bar, policy);
             }
         }
-        if (lane == 0 && first)
-            sm.ps[w].ntile += 1;
+        if (arm && T.st != D) {
+            __syncwarp();
+            if (lane < d.count)
+                bulk_g2s(dst + lane * Gm::ROWB, src + (int64_t)lane * T.st * ES, Gm::ROWB, bar, policy);
+        }
+        __syncwarp();
+    }
+
+    __device__ __forceinline__ void consume(const StageDesc &d, const unsigned char *stage)
+    {
+        if (d.flags & SD_FIRST) {
+            load_q<ES, D, G>(P, d.unit, lane, qv);
+            tmax = -INFINITY;
+            tmin = INFINITY;
+        }
+        const int vi = (lane % Gm::LPR) / Gm::REP;
+        const bool writer = (lane % Gm::REP) == 0 && (vi % G) == 0;
+        float *zu = P.z + (int64_t)d.unit * P.z_stride + d.start;
+        for (int it0 = 0; it0 < Gm::SITERS && it0 * Gm::RPW < d.count; it0 += Gm::NB) {
+            float v = qk_batch<ES, D, G>(stage, it0, lane, qv);
+#pragma unroll
+            for (int o = 1; o < G; o <<= 1)
+                v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o * Gm::REP));
+            const int row = (it0 + vi / G) * Gm::RPW + lane / Gm::LPR;
+            if (writer && row < d.count) {
+                const float zz = v * P.scale;
+                zu[row] = zz;
+                tmax = fmaxf(tmax, zz);
+                if (zz != -INFINITY)
+                    tmin = fminf(tmin, zz);
+            }
+        }
+        if ((d.flags & SD_LAST) && P.urange != nullptr) {
+            const float mx = warp_max(tmax);
+            const float mn = -warp_max(-tmin);
+            if (lane == 0) {
+                atomicMax(P.urange + 2 * d.unit, ord_key(mx));
+                if (mn != INFINITY)
+                    atomicMax(P.urange + 2 * d.unit + 1, ~ord_key(mn));
+            }
+        }
     }
 };
 
-// Online-softmax state of one warp over the tokens of its current attention
-// tile, kept in the log2 domain: logits are scale * log2(e) * q . k.
+// ---- attention ([TS 2.A] dense ++ selected sparse ++ condensed; [TS 2.C]
+// Sparse Loading: selected rows are read through the indices) ----------------
+//
+// Work line: the tokens of all units, unit-major, unit u holding
+// W_u + k_u + C_u tokens (attn_prefix: the actual counts, prefix-summed per
+// CTA in shared memory) or attn_span positions (capacity partition, for very
+// many units; positions past the unit's tokens are skipped). Each warp keeps an
+// online-softmax state over its share within one unit and writes it as a
+// record into slot (warp + unit), which is unique; the warp that completes a
+// unit's records merges them in a fixed order.
+
 template <int D, int G>
 struct AttnState {
     static constexpr int NPV = D / 64;  // float2 pairs of the lane's head-dim slice (D / 32 elements)
@@ -685,7 +537,7 @@ __device__ __forceinline__ void attn_stage(const Params &P, const unsigned char 
         const float pr = (m_new == -INFINITY || lane >= nt) ? 0.0f : ex2(s_ - m_new);
         if (lane < nt)
             sc[lane * G + g] = pr;
-        st.l[g] = st.l[g] * alpha[g] + pr;  // per-lane partial, summed at the tile's end
+        st.l[g] = st.l[g] * alpha[g] + pr;  // per-lane partial, summed at the segment's end
         st.m[g] = m_new;
     }
     __syncwarp();
@@ -697,7 +549,7 @@ __device__ __forceinline__ void attn_stage(const Params &P, const unsigned char 
             st.o[g][e].x *= alpha[g];
             st.o[g][e].y *= alpha[g];
         }
-    const unsigned char *vbase = stage + S_SLOT / 2 + lane * Gm::DPL * ES;
+    const unsigned char *vbase = stage + AT_SLOT / 2 + lane * Gm::DPL * ES;
 #pragma unroll 2
     for (int r = 0; r < nt; ++r) {
         float2 vv[NPV];
@@ -742,16 +594,17 @@ __device__ __forceinline__ void attn_stage(const Params &P, const unsigned char 
     __syncwarp();
 }
 
-// The unit's output from its attention tile records (fixed tile order), by one
+// Output of unit u from its records in slots [s0, s1] (fixed order), by one
 // warp: lane l owns head-dim elements l*DPL .. l*DPL + DPL - 1 of every head.
+// Records with m = -inf (no tokens) are skipped; no tokens at all gives
+// out = 0 and lse = -inf.
 template <int D, int G>
-__device__ void merge_unit_warp(const Params &P, int u, int ntiles)
+__device__ __noinline__ void merge_records(const Params &P, int u, int s0, int s1)
 {
     constexpr int DPL = D / 32;
     constexpr int RS = part_stride(D, G);
     const int lane = threadIdx.x & 31;
     const int b = u / P.Hkv, h = u % P.Hkv;
-    const float *rec = P.part + (int64_t)u * P.attn_tiles * RS;
     float M[G], L[G], O[G][DPL];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
@@ -762,12 +615,12 @@ __device__ void merge_unit_warp(const Params &P, int u, int ntiles)
             O[g][e] = 0.f;
     }
     constexpr int RB = 4;  // records loaded together
-    for (int t0 = 0; t0 < ntiles; t0 += RB) {
+    for (int t0 = s0; t0 <= s1; t0 += RB) {
         float mt[RB][G], lt[RB][G], ot[RB][G][DPL];
 #pragma unroll
         for (int r = 0; r < RB; ++r) {
-            const bool ok = t0 + r < ntiles;
-            const float *pr = rec + (int64_t)(t0 + r) * RS;
+            const bool ok = t0 + r <= s1;
+            const float *pr = P.part + (int64_t)(t0 + r) * RS;
 #pragma unroll
             for (int g = 0; g < G; ++g) {
                 mt[r][g] = ok ? __ldcg(pr + g * (D + 2) + D) : -INFINITY;
@@ -806,104 +659,316 @@ __device__ void merge_unit_warp(const Params &P, int u, int ntiles)
     }
 }
 
-// Write the warp's tile record, count the tile, and merge the unit if it was
-// its last tile.
+// out = 0, lse = -inf for a unit with no tokens (one warp).
 template <int D, int G>
-__device__ void finish_attn_tile(const Params &P, const StageDesc &d, AttnState<D, G> &st, bool had_tokens)
+__device__ void write_empty_unit(const Params &P, int u)
 {
-    constexpr int NPV = AttnState<D, G>::NPV;
-    constexpr int RS = part_stride(D, G);
     const int lane = threadIdx.x & 31;
-    const int u = d.unit, a = d.tile % P.attn_tiles;
-    float lsum[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-        lsum[g] = warp_sum(st.l[g]);
-    if (had_tokens) {
-        float *rec = P.part + ((int64_t)u * P.attn_tiles + a) * RS;
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-#pragma unroll
-            for (int e = 0; e < NPV; ++e)
-                *reinterpret_cast<float2 *>(rec + g * (D + 2) + lane * 2 * NPV + 2 * e) = st.o[g][e];
-            if (lane == 0) {
-                rec[g * (D + 2) + D] = st.m[g];
-                rec[g * (D + 2) + D + 1] = lsum[g];
-            }
-        }
-    }
-    __syncwarp();
-    int last = 0;
-    if (lane == 0) {
-        __threadfence();
-        const uint32_t prev = atomicAdd(P.attn_done + u, 1u);
-        last = prev == (uint32_t)P.attn_tiles - 1;
-    }
-    last = __shfl_sync(0xffffffffu, last, 0);
-    if (last) {
-        __threadfence();
-        merge_unit_warp<D, G>(P, u, (d.total + P.attn_toks - 1) / P.attn_toks);
-        if (lane == 0)
-            P.attn_done[u] = 0;
-    }
+    const int b = u / P.Hkv, h = u % P.Hkv;
+    for (int i = lane; i < G * D; i += 32)
+        P.out[((int64_t)b * P.Hq + h * G) * D + i] = 0.0f;
+    if (lane < G && P.lse != nullptr)
+        P.lse[(int64_t)b * P.Hq + h * G + lane] = -INFINITY;
 }
 
-// Consumer loop of a streaming kernel: ATTN selects the attention stages
-// (else scoring stages), so each kernel carries only its own consumer state.
-template <int ES, int D, int G, bool ATTN>
-__device__ void consumer_loop(const Params &P, SSmem<ES, D, G> &sm, const Ctl &c)
-{
+template <int ES, int D, int G>
+struct AttnSmem {
+    Ring<AT_NW, AT_SLOT, AT_STAGES> ring;
+    float sc[AT_NW][SC_FLOATS];
+    int64_t pre[PREFIX_CAP + 1];  // attn_prefix: token start of each unit
+};
+
+template <int ES, int D, int G>
+struct AttnJob {
     using Gm = Geo<ES, D, G>;
-    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    static constexpr int NS = AT_STAGES, NW = AT_NW;
+    using SM = AttnSmem<ES, D, G>;
+
+    const Params &P;
+    const Ctl &c;
+    SM &sm;
+    uint64_t policy;
+    int w, lane;
+    int64_t NWt, T, g;  // streaming warps, tokens on the line, this warp's index
+    // generator
+    int64_t t, t_end;
+    int gu = -1, gW = 0, gk = 0, gtot = 0, last_unit = -1;
+    int64_t gS = 0, gspan = 0;
+    const int32_t *gidx = nullptr;
+    int gn = 0;
+    // the lane's sparse index for the next stage, loaded one stage ahead
+    int pf_j = 0, pf_unit = -1, pf_start = -1;
+    // consumer
     float2 qv[G][Gm::NP];
-    float tmax = -INFINITY, tmin = INFINITY;
     AttnState<D, G> st;
-    if constexpr (ATTN)
+    bool had = false;
+
+    __device__ AttnJob(const Params &P_, const Ctl &c_, SM &sm_, int64_t NWt_, int64_t T_, int64_t g_)
+        : P(P_), c(c_), sm(sm_), policy(evict_first_policy()), w(threadIdx.x >> 5), lane(threadIdx.x & 31),
+          NWt(NWt_), T(T_), g(g_)
+    {
+        t = share_begin(g, NWt, T);
+        t_end = share_begin(g + 1, NWt, T);
         st.reset();
-    bool had_tokens = false;
-    uint32_t ntile = 0;
-    for (uint32_t i = 0;; ++i) {
-        const int j = i % S_SPW;
-        if (!mbar_wait(&sm.full[w][j], (i / S_SPW) & 1u, c))
-            break;
-        const StageDesc d = sm.desc[w][j];
-        if (d.kind == STG_END)
-            break;
-        if (d.first) {
-            load_q_smem<ES, D, G>(sm.qbuf[w][ntile & 1], lane, qv);
-            ++ntile;
-        }
-        const unsigned char *stage = sm.slot[w][j];
-        if constexpr (!ATTN) {
-            score_stage<ES, D, G>(P, stage, d, qv, tmax, tmin);
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&sm.empty[w][j]);
-            if (d.last) {
-                tmax = warp_max(tmax);
-                tmin = -warp_max(-tmin);
-                if (lane == 0) {
-                    P.tile_max[d.tile] = tmax;
-                    P.tile_min[d.tile] = tmin;
+    }
+
+    __device__ __forceinline__ int64_t unit_start(int u) const { return P.attn_prefix ? sm.pre[u] : (int64_t)u * P.attn_span; }
+
+    // Records of unit u occupy slots [first warp + u, last warp + u].
+    __device__ __forceinline__ void record_slots(int u, int *s0, int *s1) const
+    {
+        const int64_t a = unit_start(u), e = unit_start(u + 1);
+        *s0 = (int)(share_owner(a, NWt, T) + u);
+        *s1 = (int)(share_owner(e - 1, NWt, T) + u);
+    }
+
+    __device__ __forceinline__ void enter_unit(int u)
+    {
+        gu = u;
+        gS = unit_start(u);
+        gspan = unit_start(u + 1) - gS;
+        gW = tier_len(P.dense, u, c);
+        gn = tier_len(P.sparse, u, c);
+        gk = unit_budget(P, u, gn, c);
+        gtot = gW + gk + tier_len(P.cond, u, c);
+        if (gk > 0)
+            gidx = P.layout == HKV_LAYOUT_FLAT_SUM ? P.idx + __ldcg(P.offsets + u) : P.idx + (int64_t)u * P.bmax;
+    }
+
+    __device__ __forceinline__ bool next(StageDesc &d)
+    {
+        while (t < t_end) {
+            if (gu < 0 || t >= gS + gspan) {
+                int u = gu + 1;
+                if (gu < 0) {  // first unit of the share: binary search
+                    int lo = 0, hi = P.units - 1;
+                    while (lo < hi) {
+                        const int mid = (lo + hi + 1) >> 1;
+                        if (unit_start(mid) <= t)
+                            lo = mid;
+                        else
+                            hi = mid - 1;
+                    }
+                    u = lo;
                 }
-                tmax = -INFINITY;
-                tmin = INFINITY;
+                while (u + 1 < P.units && unit_start(u + 1) <= t)
+                    ++u;
+                enter_unit(u);
             }
-        } else {
-            if (d.count > 0) {
-                attn_stage<ES, D, G>(P, stage, d.count, sm.sc[w], qv, st);
-                had_tokens = true;
+            const int a = (int)(t - gS);
+            const int seg_end = (int)(min(t_end - gS, gspan));
+            const int vend = min(seg_end, gtot);
+            if (a >= vend) {
+                // capacity partition: the share holds only unused positions of
+                // this unit; one empty stage still counts the warp's record
+                const bool first = gu != last_unit;
+                t = gS + seg_end;
+                if (!first)
+                    continue;
+                d = StageDesc{gu, a, 0, SD_FIRST | SD_LAST};
+                last_unit = gu;
+                return true;
+            }
+            const int cnt = min(Gm::ATOK, vend - a);
+            const bool last = a + cnt >= vend;
+            const bool contiguous = (a + cnt <= gW && P.dense.st == D) || (a >= gW + gk && P.cond.st == D);
+            d = StageDesc{gu, a, cnt,
+                          (gu != last_unit ? SD_FIRST : 0) | (last ? SD_LAST : 0) | (contiguous ? 0 : SD_GATHER)};
+            last_unit = gu;
+            t = last ? gS + seg_end : t + cnt;
+            return true;
+        }
+        return false;
+    }
+
+    __device__ __forceinline__ void issue(const StageDesc &d, int j)
+    {
+        const int u = d.unit;
+        const int b = u / P.Hkv, h = u % P.Hkv;
+        unsigned char *dst = sm.ring.slot[w][j];
+        uint64_t *bar = &sm.ring.full[w][j];
+        const bool arm = !P.withhold;
+        if (lane == 0)
+            sm.ring.desc[w][j] = StageDesc{d.unit, d.start, d.count, d.flags | (arm ? SD_ARMED : 0)};
+        if (!arm) {
+            __syncwarp();
+            return;
+        }
+        if (!(d.flags & SD_GATHER)) {
+            if (lane == 0) {
+                mbar_arrive_expect_tx(bar, (uint32_t)(2 * d.count * Gm::ROWB));
+                if (d.count > 0) {
+                    const bool dn = d.start < gW;
+                    const TierP &Tt = dn ? P.dense : P.cond;
+                    const int64_t r0 = dn ? d.start : d.start - gW - gk;
+                    const int64_t off = ((int64_t)b * Tt.sb + (int64_t)h * Tt.sh + r0 * Tt.st) * ES;
+                    bulk_g2s(dst, Tt.k + off, d.count * Gm::ROWB, bar, policy);
+                    bulk_g2s(dst + AT_SLOT / 2, Tt.v + off, d.count * Gm::ROWB, bar, policy);
+                }
             }
             __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&sm.empty[w][j]);
-            if (d.last) {
-                finish_attn_tile<D, G>(P, d, st, had_tokens);
-                st.reset();
-                had_tokens = false;
+            prefetch_index(d);
+            return;
+        }
+        // gathered rows: lane r finds the source of token d.start + r
+        const char *ks = nullptr, *vs = nullptr;
+        if (lane < d.count) {
+            const int tt = d.start + lane;
+            int64_t off;
+            if (tt < gW) {
+                ks = P.dense.k;
+                vs = P.dense.v;
+                off = (int64_t)b * P.dense.sb + (int64_t)h * P.dense.sh + (int64_t)tt * P.dense.st;
+            } else if (tt < gW + gk) {
+                int jj = (pf_unit == u && pf_start == d.start) ? pf_j : __ldcg(gidx + (tt - gW));
+                if (jj < 0 || jj >= gn) {
+                    raise_flag(c, HKV_DEV_BAD_INDEX);
+                    jj = 0;
+                }
+                ks = P.sparse.k;
+                vs = P.sparse.v;
+                off = (int64_t)b * P.sparse.sb + (int64_t)h * P.sparse.sh + (int64_t)jj * P.sparse.st;
+            } else {
+                ks = P.cond.k;
+                vs = P.cond.v;
+                off = (int64_t)b * P.cond.sb + (int64_t)h * P.cond.sh + (int64_t)(tt - gW - gk) * P.cond.st;
             }
+            ks += off * ES;
+            vs += off * ES;
+        }
+        constexpr int CH = Gm::ROWB / 16;  // 16-byte chunks of a row
+        static_assert(32 % CH == 0 || CH % 32 == 0, "row chunks");
+        if constexpr (CH <= 32) {
+            constexpr int RPI = 32 / CH;  // rows per warp instruction
+            const int cc = lane % CH, rr = lane / CH;
+            for (int r0 = 0; r0 < d.count; r0 += RPI) {
+                const int r = r0 + rr;
+                const char *k_ = reinterpret_cast<const char *>(
+                    (uintptr_t)__shfl_sync(0xffffffffu, (unsigned long long)(uintptr_t)ks, r & 31));
+                const char *v_ = reinterpret_cast<const char *>(
+                    (uintptr_t)__shfl_sync(0xffffffffu, (unsigned long long)(uintptr_t)vs, r & 31));
+                if (r < d.count) {
+                    cp_async16(dst + r * Gm::ROWB + cc * 16, k_ + cc * 16);
+                    cp_async16(dst + AT_SLOT / 2 + r * Gm::ROWB + cc * 16, v_ + cc * 16);
+                }
+            }
+        }
+        cp_async_arrive(bar);
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(bar);
+        prefetch_index(d);
+    }
+
+    // Start loading the lane's sparse index of the stage after d (same unit),
+    // to be used when that stage is issued.
+    __device__ __forceinline__ void prefetch_index(const StageDesc &d)
+    {
+        const int ns = d.start + d.count;
+        const int tt = ns + lane;
+        pf_unit = -1;
+        if (!(d.flags & SD_LAST) && ns < gW + gk && ns + Gm::ATOK > gW) {
+            pf_unit = d.unit;
+            pf_start = ns;
+            if (tt >= gW && tt < gW + gk)
+                pf_j = __ldcg(gidx + (tt - gW));
         }
     }
+
+    __device__ __forceinline__ void consume(const StageDesc &d, const unsigned char *stage)
+    {
+        if (d.flags & SD_FIRST) {
+            load_q<ES, D, G>(P, d.unit, lane, qv);
+            st.reset();
+            had = false;
+        }
+        if (d.count > 0) {
+            attn_stage<ES, D, G>(P, stage, d.count, sm.sc[w], qv, st);
+            had = true;
+        }
+        if (d.flags & SD_LAST)
+            finish(d.unit);
+    }
+
+    // Write the warp's record for unit u, count it, and merge the unit if the
+    // record was its last.
+    __device__ __forceinline__ void finish(int u)
+    {
+        constexpr int NPV = AttnState<D, G>::NPV;
+        constexpr int RS = part_stride(D, G);
+        float lsum[G];
+#pragma unroll
+        for (int gg = 0; gg < G; ++gg)
+            lsum[gg] = warp_sum(st.l[gg]);
+        float *rec = P.part + (g + u) * RS;
+#pragma unroll
+        for (int gg = 0; gg < G; ++gg) {
+#pragma unroll
+            for (int e = 0; e < NPV; ++e)
+                *reinterpret_cast<float2 *>(rec + gg * (D + 2) + lane * 2 * NPV + 2 * e) = st.o[gg][e];
+            if (lane == 0) {
+                rec[gg * (D + 2) + D] = had ? st.m[gg] : -INFINITY;
+                rec[gg * (D + 2) + D + 1] = lsum[gg];
+            }
+        }
+        int s0, s1;
+        record_slots(u, &s0, &s1);
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+            __threadfence();
+            const uint32_t prev = atomicAdd(P.attn_cnt + u, 1u);
+            last = prev == (uint32_t)(s1 - s0);
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {
+            __threadfence();
+            merge_records<D, G>(P, u, s0, s1);
+            if (lane == 0)
+                P.attn_cnt[u] = 0;
+        }
+        __syncwarp();
+    }
+};
+
+// Attention prologue of a CTA: token starts of all units (attn_prefix), and
+// out = 0 / lse = -inf for this CTA's share of units without tokens. Returns
+// the tokens on the line.
+template <int ES, int D, int G>
+__device__ int64_t attn_prologue(const Params &P, AttnSmem<ES, D, G> &sm, const Ctl &c, unsigned long long *red)
+{
+    const int w = threadIdx.x >> 5;
+    int64_t T;
+    if (P.attn_prefix) {
+        unsigned long long carry = 0;
+        for (int base = 0; base < P.units; base += AT_NW * 32) {
+            const int u = base + threadIdx.x;
+            int tot = 0;
+            if (u < P.units) {
+                const int n = tier_len(P.sparse, u, c);
+                tot = tier_len(P.dense, u, c) + unit_budget(P, u, n, c) + tier_len(P.cond, u, c);
+            }
+            unsigned long long sum;
+            const unsigned long long ex = block_exclusive_scan<AT_NW * 32>((unsigned long long)tot, red, &sum);
+            if (u < P.units)
+                sm.pre[u] = (int64_t)(carry + ex);
+            carry += sum;
+        }
+        if (threadIdx.x == 0)
+            sm.pre[P.units] = (int64_t)carry;
+        __syncthreads();
+        T = (int64_t)carry;
+        // units without tokens get no record: their output is written here
+        for (int u = blockIdx.x * AT_NW + w; u < P.units; u += gridDim.x * AT_NW)
+            if (sm.pre[u + 1] == sm.pre[u])
+                write_empty_unit<D, G>(P, u);
+    } else {
+        T = (int64_t)P.units * P.attn_span;
+        if (T == 0)
+            for (int u = blockIdx.x * AT_NW + w; u < P.units; u += gridDim.x * AT_NW)
+                write_empty_unit<D, G>(P, u);
+    }
+    return T;
 }
 
 // =============================================================================

@@ -226,11 +226,12 @@ hkv_status hkv_step(const hkv_problem *prob, const void *q, const hkv_tier *dens
  * the same arguments minus ws/ws_bytes, and allocates nothing (no cudaMalloc,
  * no cudaFree, no allocating library routine): its scratch is a fixed device
  * array of HKV_NOALLOC_SCRATCH_BYTES bytes inside the library.
- * - Size limit: the scratch is the front of the layout hkv_workspace_size
- *   describes (status and counter words, per-tile score ranges, attention
- *   tile records): about 2.6 MB for bf16, D = 128, G = 4, 64 units of up to
- *   2368 attended tokens. A problem that needs more than the array holds is
- *   refused with HKV_ERR_WORKSPACE before anything is launched; use
+ * - Size limit: the scratch holds a few counter words per unit and one
+ *   attention record of 4*G*(D+2) bytes per streaming warp and per unit
+ *   (2.6 MB for bf16, D = 128, G = 4, 64 units on a 148-SM B200). When the
+ *   array cannot hold records for a full grid, fewer CTAs run; a problem with
+ *   too many units for even one CTA (about 2000 units at G = 4, D = 128) is
+ *   refused with HKV_ERR_WORKSPACE before anything is launched: use
  *   hkv_cascade_decode with a workspace for those.
  * - Set-up: the first call on each device looks up the array's device address
  *   and sets the kernel's shared-memory attribute. Make that first call outside

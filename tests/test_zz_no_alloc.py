@@ -54,8 +54,8 @@ def test_noalloc_decode_matches_workspace_decode_on_consecutive_calls():
 
 def test_noalloc_refuses_problems_beyond_its_array():
     """Refused on the host before anything touches a device (runs without a GPU)."""
-    prob = hkv.Problem(B=64, Hq=32, Hkv=8, D=128, dtype=torch.bfloat16, p=0.9, bmin=32, bmax=4096)
-    cap = 32448
+    prob = hkv.Problem(B=512, Hq=32, Hkv=8, D=128, dtype=torch.bfloat16, p=0.9, bmin=32, bmax=256)
+    cap = 4096
 
     def tier(cap_, addr):
         return hkv._Tier(addr, addr + 0x1000000, 8 * 128 * cap_, 128 * cap_, 128, cap_, 0x2000)
