@@ -27,8 +27,10 @@ namespace hkv {
 
 // Trace slots (builds with -DHKV_TRACE only): per unit u of the per-unit
 // kernel, TR_SEL + 8u + i: 0 start, 1 sweep 1 done, 2 sweep 2 done, 3 cut
-// found, 4 range known, 5 compacted.
-[[maybe_unused]] constexpr int TR_SEL = 250000;
+// found, 4 range known, 5 compacted, 6 scores staged; per streaming warp g,
+// TR_SW + 4g (scoring) or TR_AW + 4g (attention) + i: 0 pipeline start,
+// 1 first stage landed, 2 pipeline done, 3 kernel entry (attention).
+[[maybe_unused]] constexpr int TR_SEL = 250000, TR_SW = 0, TR_AW = 20000;
 
 // =============================================================================
 // Kernels
@@ -50,7 +52,8 @@ __global__ void __launch_bounds__(sc_nw(G) * 32, 1) k_score_stream(const __grid_
     const int64_t NW = (int64_t)gridDim.x * Job::NW;
     const int64_t g = (int64_t)blockIdx.x * Job::NW + (threadIdx.x >> 5);
     Job job(P, c, ring, share_begin(g, NW, R), share_begin(g + 1, NW, R));
-    warp_pipeline(job, ring, c);
+    HKV_TRACE_WARP(TR_SW + 4 * (int)g);
+    warp_pipeline(job, ring, c, TR_SW + 4 * (int)g);
 }
 
 // S5 ([TS 2.A] cascade decode over the three tiers; [TS 2.C] Sparse Loading):
@@ -66,13 +69,15 @@ __global__ void __launch_bounds__(AT_NW * 32, 1) k_attn_stream(const __grid_cons
     ring_init(sm.ring);
     allow_dependents();
     wait_prior_grid();
+    HKV_TRACE_WARP(TR_AW + 4 * (blockIdx.x * AT_NW + (threadIdx.x >> 5)) + 3);
     const int64_t T = attn_prologue<ES, D, G>(P, sm, c, red);
     // every warp that takes part gets a non-empty share
     const int64_t NW = min((int64_t)gridDim.x * AT_NW, T);
     const int64_t g = (int64_t)blockIdx.x * AT_NW + (threadIdx.x >> 5);
     if (g < NW) {
         AttnJob<ES, D, G> job(P, c, sm, NW, T, g);
-        warp_pipeline(job, sm.ring, c);
+        HKV_TRACE_WARP(TR_AW + 4 * (int)g);
+        warp_pipeline(job, sm.ring, c, TR_AW + 4 * (int)g);
     }
 }
 
@@ -134,7 +139,8 @@ __global__ void __launch_bounds__(NT) k_unit(const __grid_constant__ Params P)
     wait_prior_grid();
     HKV_TRACE_AT(TR_SEL + 8 * u);
     const int n = tier_len(P.sparse, u, c);
-    const float *zu = P.z + (int64_t)u * P.z_stride;
+    const float *zu = stage_scores(P.z + (int64_t)u * P.z_stride, n, sm);
+    HKV_TRACE_AT(TR_SEL + 8 * u + 6);
     int k, n_tie;
     uint32_t key;
     if (P.do_select) {
@@ -208,7 +214,7 @@ __global__ void __launch_bounds__(NT) k_calibrate(const __grid_constant__ Params
     const Ctl c = make_ctl(P);
     const int u = blockIdx.x;
     const int n = tier_len(P.sparse, u, c);
-    const float *zu = P.z + (int64_t)u * P.z_stride;
+    const float *zu = stage_scores(P.z + (int64_t)u * P.z_stride, n, sm);
     float m, zlo;
     unit_range(zu, n, &m, &zlo, sm);
     const float bl2 = unit_beta(P, u, c) * LOG2E;

@@ -23,12 +23,12 @@
 
 namespace hkv {
 
-constexpr int SC_SLOT = 4096;             // scoring: bytes per stage (K rows)
+constexpr int SC_SLOT = 8192;             // scoring: bytes per stage (K rows)
 // scoring: warps per CTA and ring slots per warp (192 KB of slots per CTA);
-// eight query heads per group keep 64 more registers of queries per lane, so
-// they run half the warps with twice the slots
-__host__ __device__ constexpr int sc_nw(int G) { return G >= 8 ? 8 : 16; }
-__host__ __device__ constexpr int sc_stages(int G) { return G >= 8 ? 6 : 3; }
+// eight query heads per group keep twice the query registers per lane, so
+// they run fewer warps with more slots each
+__host__ __device__ constexpr int sc_nw(int G) { return G >= 8 ? 8 : 12; }
+__host__ __device__ constexpr int sc_stages(int G) { return G >= 8 ? 3 : 2; }
 constexpr int AT_NW = 8;                  // attention: warps per CTA
 constexpr int AT_SLOT = 8192;             // attention: bytes per stage (K rows, then as many V rows)
 constexpr int AT_STAGES = 3;              // attention: ring slots per warp
@@ -165,7 +165,7 @@ struct Geo {
     static constexpr int ATOK = (AT_SLOT / 2) / ROWB;     // tokens per attention stage
     static constexpr int DPL = D / 32;                    // PV: head-dim elements per lane
     static_assert(G >= 1 && G <= LPR, "group size must not exceed lanes per row");
-    static_assert(ATOK * G <= SC_FLOATS && ATOK <= 32 && SROWS <= 32, "stage sizes");
+    static_assert(ATOK * G <= SC_FLOATS && ATOK <= 32, "stage sizes");
     static_assert(SITERS % NB == 0 && AITERS % NB == 0 && LPR % NV == 0, "iteration batches");
 };
 
@@ -174,6 +174,10 @@ struct Geo {
 // =============================================================================
 
 enum : int32_t { SD_FIRST = 1, SD_LAST = 2, SD_GATHER = 4, SD_ARMED = 8 };
+
+// Trace builds (-DHKV_TRACE): per warp trace slot base s (4 slots), the issue
+// and landing times of its first 12 stages at TRACE_STAGES + 8 s + 2 i (+1).
+[[maybe_unused]] constexpr int TRACE_STAGES = 40000;
 
 struct StageDesc {
     int32_t unit, start, count, flags;  // rows (scoring) or unit-local tokens (attention) [start, start + count)
@@ -206,13 +210,15 @@ __device__ __forceinline__ void ring_init(R &r)
 // Up to NS stages are in flight. If a wait runs out (status word set), the
 // warp stops consuming, waits (bounded) for the copies it started, and returns.
 template <class Job, class R>
-__device__ void warp_pipeline(Job &job, R &ring, const Ctl &c)
+__device__ void warp_pipeline(Job &job, R &ring, const Ctl &c, int tslot = -1)
 {
     constexpr int NS = Job::NS;
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint32_t issued = 0, consumed = 0;
     StageDesc d;
     while (issued < (uint32_t)NS && job.next(d)) {
+        if (issued < 12)
+            HKV_TRACE_WARP(tslot < 0 ? -1 : TRACE_STAGES + tslot * 8 + 2 * (int)issued);
         job.issue(d, (int)issued);
         ++issued;
     }
@@ -223,6 +229,10 @@ __device__ void warp_pipeline(Job &job, R &ring, const Ctl &c)
             ok = false;
             break;
         }
+        if (consumed == 0)
+            HKV_TRACE_WARP(tslot < 0 ? -1 : tslot + 1);
+        if (consumed < 12)
+            HKV_TRACE_WARP(tslot < 0 ? -1 : TRACE_STAGES + tslot * 8 + 2 * (int)consumed + 1);
         const StageDesc cd = ring.desc[w][j];
         job.consume(cd, ring.slot[w][j]);
         __syncwarp();
@@ -230,6 +240,8 @@ __device__ void warp_pipeline(Job &job, R &ring, const Ctl &c)
         if (job.next(d)) {
             if (lane == 0)
                 fence_proxy_async_smem();  // this warp's reads of the slot before the copies that refill it
+            if (issued < 12)
+                HKV_TRACE_WARP(tslot < 0 ? -1 : TRACE_STAGES + tslot * 8 + 2 * (int)issued);
             job.issue(d, j);
             ++issued;
         }
@@ -243,6 +255,7 @@ __device__ void warp_pipeline(Job &job, R &ring, const Ctl &c)
         }
     }
     __syncwarp();
+    HKV_TRACE_WARP(tslot < 0 ? -1 : tslot + 2);
 }
 
 // ---- warp butterfly over the LPR lanes of a row: NV partial sums per lane ->
@@ -437,8 +450,8 @@ struct ScoreJob {
         }
         if (arm && T.st != D) {
             __syncwarp();
-            if (lane < d.count)
-                bulk_g2s(dst + lane * Gm::ROWB, src + (int64_t)lane * T.st * ES, Gm::ROWB, bar, policy);
+            for (int r = lane; r < d.count; r += 32)
+                bulk_g2s(dst + r * Gm::ROWB, src + (int64_t)r * T.st * ES, Gm::ROWB, bar, policy);
         }
         __syncwarp();
     }
@@ -453,19 +466,33 @@ struct ScoreJob {
         const int vi = (lane % Gm::LPR) / Gm::REP;
         const bool writer = (lane % Gm::REP) == 0 && (vi % G) == 0;
         float *zu = P.z + (int64_t)d.unit * P.z_stride + d.start;
-        for (int it0 = 0; it0 < Gm::SITERS && it0 * Gm::RPW < d.count; it0 += Gm::NB) {
-            float v = qk_batch<ES, D, G>(stage, it0, lane, qv);
+        const auto emit = [&](float v, int it0, bool check) {
 #pragma unroll
             for (int o = 1; o < G; o <<= 1)
                 v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o * Gm::REP));
             const int row = (it0 + vi / G) * Gm::RPW + lane / Gm::LPR;
-            if (writer && row < d.count) {
+            if (writer && (!check || row < d.count)) {
                 const float zz = v * P.scale;
                 zu[row] = zz;
                 tmax = fmaxf(tmax, zz);
                 if (zz != -INFINITY)
                     tmin = fminf(tmin, zz);
             }
+        };
+        if (d.count == Gm::SROWS) {
+            // a full stage: every batch unrolled, so that the loads and products
+            // of one batch overlap the reductions of the previous one
+            constexpr int NBAT = Gm::SITERS / Gm::NB;
+            float v[NBAT];
+#pragma unroll
+            for (int b = 0; b < NBAT; ++b)
+                v[b] = qk_batch<ES, D, G>(stage, b * Gm::NB, lane, qv);
+#pragma unroll
+            for (int b = 0; b < NBAT; ++b)
+                emit(v[b], b * Gm::NB, false);
+        } else {
+            for (int it0 = 0; it0 < Gm::SITERS && it0 * Gm::RPW < d.count; it0 += Gm::NB)
+                emit(qk_batch<ES, D, G>(stage, it0, lane, qv), it0, true);
         }
         if ((d.flags & SD_LAST) && P.urange != nullptr) {
             const float mx = warp_max(tmax);
@@ -519,11 +546,25 @@ __device__ __forceinline__ void attn_stage(const Params &P, const unsigned char 
     const bool writer = (lane % Gm::REP) == 0;
     const float scale2 = P.scale * LOG2E;
     // logits of the stage's tokens for all G query heads
-    for (int it0 = 0; it0 < Gm::AITERS && it0 * Gm::RPW < nt; it0 += Gm::NB) {
-        const float v = qk_batch<ES, D, G>(stage, it0, lane, qv);
-        const int row = (it0 + vi / G) * Gm::RPW + lane / Gm::LPR;
-        if (writer && row < nt)
-            sc[row * G + (vi % G)] = v * scale2;
+    if (nt == Gm::ATOK) {
+        constexpr int NBAT = Gm::AITERS / Gm::NB;
+        float v[NBAT];
+#pragma unroll
+        for (int b = 0; b < NBAT; ++b)
+            v[b] = qk_batch<ES, D, G>(stage, b * Gm::NB, lane, qv);
+#pragma unroll
+        for (int b = 0; b < NBAT; ++b) {
+            const int row = (b * Gm::NB + vi / G) * Gm::RPW + lane / Gm::LPR;
+            if (writer)
+                sc[row * G + (vi % G)] = v[b] * scale2;
+        }
+    } else {
+        for (int it0 = 0; it0 < Gm::AITERS && it0 * Gm::RPW < nt; it0 += Gm::NB) {
+            const float v = qk_batch<ES, D, G>(stage, it0, lane, qv);
+            const int row = (it0 + vi / G) * Gm::RPW + lane / Gm::LPR;
+            if (writer && row < nt)
+                sc[row * G + (vi % G)] = v * scale2;
+        }
     }
     __syncwarp();
     // online softmax: lane r owns token r of the stage (ATOK <= 32)
@@ -810,7 +851,8 @@ struct AttnJob {
             prefetch_index(d);
             return;
         }
-        // gathered rows: lane r finds the source of token d.start + r
+        // gathered rows: lane r copies the K and V rows of token d.start + r,
+        // one bulk copy each, after lane 0 has armed the slot for all of them
         const char *ks = nullptr, *vs = nullptr;
         if (lane < d.count) {
             const int tt = d.start + lane;
@@ -836,27 +878,14 @@ struct AttnJob {
             ks += off * ES;
             vs += off * ES;
         }
-        constexpr int CH = Gm::ROWB / 16;  // 16-byte chunks of a row
-        static_assert(32 % CH == 0 || CH % 32 == 0, "row chunks");
-        if constexpr (CH <= 32) {
-            constexpr int RPI = 32 / CH;  // rows per warp instruction
-            const int cc = lane % CH, rr = lane / CH;
-            for (int r0 = 0; r0 < d.count; r0 += RPI) {
-                const int r = r0 + rr;
-                const char *k_ = reinterpret_cast<const char *>(
-                    (uintptr_t)__shfl_sync(0xffffffffu, (unsigned long long)(uintptr_t)ks, r & 31));
-                const char *v_ = reinterpret_cast<const char *>(
-                    (uintptr_t)__shfl_sync(0xffffffffu, (unsigned long long)(uintptr_t)vs, r & 31));
-                if (r < d.count) {
-                    cp_async16(dst + r * Gm::ROWB + cc * 16, k_ + cc * 16);
-                    cp_async16(dst + AT_SLOT / 2 + r * Gm::ROWB + cc * 16, v_ + cc * 16);
-                }
-            }
-        }
-        cp_async_arrive(bar);
-        __syncwarp();
         if (lane == 0)
-            mbar_arrive(bar);
+            mbar_arrive_expect_tx(bar, (uint32_t)(2 * d.count * Gm::ROWB));
+        __syncwarp();
+        if (lane < d.count) {
+            bulk_g2s(dst + lane * Gm::ROWB, ks, Gm::ROWB, bar, policy);
+            bulk_g2s(dst + AT_SLOT / 2 + lane * Gm::ROWB, vs, Gm::ROWB, bar, policy);
+        }
+        __syncwarp();
         prefetch_index(d);
     }
 
@@ -977,50 +1006,38 @@ __device__ int64_t attn_prologue(const Params &P, AttnSmem<ES, D, G> &sm, const 
 
 constexpr int NT = SEL_THREADS;
 
-// Scores of one unit read from L2 in batches (32 per thread in flight).
-// f(z, j, valid) is called by every thread the same number of times.
+// Scores of one unit, from shared memory (staged) or global memory, in batches
+// of Q quads per thread with all loads in flight. Thread t takes quads
+// t, t + NT, ... of each batch, whatever the source or its alignment, so sums
+// taken in call order are identical on every path. f(z, j, valid) is called
+// by every thread the same number of times.
 template <typename F>
 __device__ __forceinline__ void sweep_scores(const float *zu, int n, F &&f)
 {
-    constexpr int BATCH = 32;
+    constexpr int Q = 8;
     const bool vec = (((uintptr_t)zu) & 15) == 0;
-    if (vec) {
-        const int n4 = n >> 2;
-        const float4 *z4 = reinterpret_cast<const float4 *>(zu);
-        for (int base = 0; base < n4; base += NT * (BATCH / 4)) {
-            float4 v[BATCH / 4];
+    const int nq = (n + 3) >> 2;
+    for (int base = 0; base < nq; base += NT * Q) {
+        float4 v[Q];
 #pragma unroll
-            for (int i = 0; i < BATCH / 4; ++i) {
-                const int q4 = base + i * NT + threadIdx.x;
-                v[i] = q4 < n4 ? __ldcg(z4 + q4) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-#pragma unroll
-            for (int i = 0; i < BATCH / 4; ++i) {
-                const int q4 = base + i * NT + threadIdx.x;
-                const bool ok = q4 < n4;
-                f(v[i].x, 4 * q4, ok);
-                f(v[i].y, 4 * q4 + 1, ok);
-                f(v[i].z, 4 * q4 + 2, ok);
-                f(v[i].w, 4 * q4 + 3, ok);
+        for (int i = 0; i < Q; ++i) {
+            const int j = 4 * (base + i * NT + (int)threadIdx.x);
+            if (vec && j + 4 <= n) {
+                v[i] = *reinterpret_cast<const float4 *>(zu + j);
+            } else {
+                v[i].x = j < n ? zu[j] : 0.f;
+                v[i].y = j + 1 < n ? zu[j + 1] : 0.f;
+                v[i].z = j + 2 < n ? zu[j + 2] : 0.f;
+                v[i].w = j + 3 < n ? zu[j + 3] : 0.f;
             }
         }
-        for (int base = n4 * 4; base < n; base += NT) {
-            const int j = base + threadIdx.x;
-            f(j < n ? __ldcg(zu + j) : 0.f, j, j < n);
-        }
-    } else {
-        for (int base = 0; base < n; base += NT * BATCH) {
-            float v[BATCH];
 #pragma unroll
-            for (int i = 0; i < BATCH; ++i) {
-                const int j = base + i * NT + threadIdx.x;
-                v[i] = j < n ? __ldcg(zu + j) : 0.f;
-            }
-#pragma unroll
-            for (int i = 0; i < BATCH; ++i) {
-                const int j = base + i * NT + threadIdx.x;
-                f(v[i], j, j < n);
-            }
+        for (int i = 0; i < Q; ++i) {
+            const int j = 4 * (base + i * NT + (int)threadIdx.x);
+            f(v[i].x, j, j < n);
+            f(v[i].y, j + 1, j + 1 < n);
+            f(v[i].z, j + 2, j + 2 < n);
+            f(v[i].w, j + 3, j + 3 < n);
         }
     }
 }
@@ -1029,7 +1046,10 @@ __device__ __forceinline__ void sweep_scores(const float *zu, int n, F &&f)
 constexpr int SBINS = 2048;
 constexpr int CAND_CAP = 4096;
 
+constexpr int ZSTAGE = 24576;  // scores of a unit staged in shared memory (units up to this length)
+
 struct __align__(16) USmem {  // shared memory of the per-unit kernels
+    float zs[ZSTAGE];
     uint32_t cnt[SBINS];
     uint32_t mlo[SBINS];  // bin mass, low 32 bits (fixed point)
     uint32_t mhi[SBINS];  // bin mass, high 32 bits
@@ -1092,6 +1112,39 @@ __device__ void unit_range(const float *zu, int n, float *m, float *zlo, USmem &
     });
     *m = block_max<NT>(mx, sm.redf);
     *zlo = -block_max<NT>(-mn, sm.redf);
+}
+
+// Copy a unit's n <= ZSTAGE scores into shared memory (all loads in flight)
+// and return the staged copy; longer units stay in global memory.
+__device__ const float *stage_scores(const float *zu, int n, USmem &sm)
+{
+    if (n > ZSTAGE)
+        return zu;
+    const bool vec = (((uintptr_t)zu) & 15) == 0;
+    if (vec) {
+        constexpr int PER = ZSTAGE / 4 / NT;
+        float4 v[PER];
+        const int n4 = n >> 2;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int q = i * NT + threadIdx.x;
+            if (q < n4)
+                v[i] = __ldcg(reinterpret_cast<const float4 *>(zu) + q);
+        }
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            const int q = i * NT + threadIdx.x;
+            if (q < n4)
+                reinterpret_cast<float4 *>(sm.zs)[q] = v[i];
+        }
+        for (int j = n4 * 4 + threadIdx.x; j < n; j += NT)
+            sm.zs[j] = __ldcg(zu + j);
+    } else {
+        for (int j = threadIdx.x; j < n; j += NT)
+            sm.zs[j] = __ldcg(zu + j);
+    }
+    __syncthreads();
+    return sm.zs;
 }
 
 // First bin whose cumulative count (by_mass = false) or mass reaches target
@@ -1457,7 +1510,7 @@ __device__ void compact_unit(const float *zu, int n, uint32_t cut_key, int n_tie
             if (vec && j0 + E <= n) {
 #pragma unroll
                 for (int e = 0; e < E; e += 4) {
-                    const float4 v = __ldcg(reinterpret_cast<const float4 *>(zu + j0 + e));
+                    const float4 v = *reinterpret_cast<const float4 *>(zu + j0 + e);
                     zz[e] = v.x;
                     zz[e + 1] = v.y;
                     zz[e + 2] = v.z;
@@ -1466,7 +1519,7 @@ __device__ void compact_unit(const float *zu, int n, uint32_t cut_key, int n_tie
             } else {
 #pragma unroll
                 for (int e = 0; e < E; ++e)
-                    zz[e] = (j0 + e < n) ? __ldcg(zu + j0 + e) : 0.f;
+                    zz[e] = (j0 + e < n) ? zu[j0 + e] : 0.f;
             }
             uint32_t lt_bits = 0, eq_bits = 0;
 #pragma unroll
