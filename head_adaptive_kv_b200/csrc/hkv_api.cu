@@ -26,8 +26,10 @@
 namespace hkv {
 
 // Trace slots (builds with -DHKV_TRACE only): per unit u of the per-unit
-// kernel, TR_SEL + 8u + i: 0 start, 1 sweep 1 done, 2 sweep 2 done, 3 cut
-// found, 4 range known, 5 compacted, 6 scores staged; per streaming warp g,
+// kernel, TR_SEL + 16u + i: 0 start, 1 sweep 1 done, 2 sweep 2 done, 3 cut
+// found, 4 range known, 5 compacted, 6 scores staged, 7 rank bin found,
+// 8 mass through it summed, 9 count bin found, 10 bin sorted, 11 results
+// written; per streaming warp g,
 // TR_SW + 4g (scoring) or TR_AW + 4g (attention) + i: 0 pipeline start,
 // 1 first stage landed, 2 pipeline done, 3 kernel entry (attention).
 [[maybe_unused]] constexpr int TR_SEL = 250000, TR_SW = 0, TR_AW = 20000;
@@ -121,26 +123,10 @@ __device__ __forceinline__ void write_offsets(const Params &P, int u, int64_t of
     }
 }
 
-// S2-S4 per unit, one CTA per (sequence, KV head).
-//  do_select  ([TS 2.B] calibration, [Abstract]/[TS 2.A] Top-p budget with the
-//             hard limits): writes sel_len, cut, m, logZ. With have_range the
-//             unit's score range comes from the scorer's tile records.
-//  do_compact ([TS 2.C] Flatten Index): writes the unit's indices in score
-//             order from the cut -- PAD_MAX rows, or FLAT_SUM (standalone) --
-//             and, standalone, the Rewrite Cache copy when k_out is given.
-template <int ES>
-__global__ void __launch_bounds__(NT) k_unit(const __grid_constant__ Params P)
+// S2-S4 of unit u, scores at zu (in shared memory when ZS).
+template <int ES, bool ZS>
+__device__ __forceinline__ void unit_work(const Params &P, USmem &sm, const Ctl &c, int u, int n, const float *zu)
 {
-    extern __shared__ __align__(128) unsigned char smem_raw[];
-    USmem &sm = *reinterpret_cast<USmem *>(smem_raw);
-    const Ctl c = make_ctl(P);
-    const int u = blockIdx.x;
-    allow_dependents();
-    wait_prior_grid();
-    HKV_TRACE_AT(TR_SEL + 8 * u);
-    const int n = tier_len(P.sparse, u, c);
-    const float *zu = stage_scores(P.z + (int64_t)u * P.z_stride, n, sm);
-    HKV_TRACE_AT(TR_SEL + 8 * u + 6);
     int k, n_tie;
     uint32_t key;
     if (P.do_select) {
@@ -160,11 +146,11 @@ __global__ void __launch_bounds__(NT) k_unit(const __grid_constant__ Params P)
             zlo = sm.redf[1];
             __syncthreads();
         } else {
-            unit_range(zu, n, &m, &zlo, sm);
+            unit_range<ZS>(zu, n, &m, &zlo, sm);
         }
-        HKV_TRACE_AT(TR_SEL + 8 * u + 4);
-        const Selection s = select_unit(zu, n, m, zlo, unit_beta(P, u, c), unit_p(P, u, c), P.bmin, P.bmax, sm,
-                                        TR_SEL + 8 * u);
+        HKV_TRACE_AT(TR_SEL + 16 * u + 4);
+        const Selection s = select_unit<ZS>(zu, n, m, zlo, unit_beta(P, u, c), unit_p(P, u, c), P.bmin, P.bmax,
+                                            sm, TR_SEL + 16 * u);
         k = s.k;
         key = s.key;
         n_tie = s.cut.n_tie;
@@ -177,6 +163,7 @@ __global__ void __launch_bounds__(NT) k_unit(const __grid_constant__ Params P)
             if (P.logZ_out)
                 P.logZ_out[u] = n > 0 ? (float)log(s.Z) : -INFINITY;
         }
+        HKV_TRACE_AT(TR_SEL + 16 * u + 11);
     } else {
         k = __ldcg(P.sel_len + u);
         const hkv_cut ct = P.cut[u];
@@ -196,30 +183,54 @@ __global__ void __launch_bounds__(NT) k_unit(const __grid_constant__ Params P)
         write_offsets(P, u, off);
     }
     int32_t *row = P.idx + off;
-    compact_unit(zu, n, key, n_tie, k, row, flat ? k : P.bmax, sm.red);
-    HKV_TRACE_AT(TR_SEL + 8 * u + 5);
+    compact_unit<ZS>(zu, n, key, n_tie, k, row, flat ? k : P.bmax, sm.red);
+    HKV_TRACE_AT(TR_SEL + 16 * u + 5);
     if (P.k_out != nullptr && !P.do_select) {
         __syncthreads();
         rewrite_rows(P, u, row, k, off, ES, c, n);
     }
 }
 
-// S2 standalone ([TS 2.B]): m, logZ and optionally the calibrated
-// probabilities of each unit. Z is summed exactly as the selection sums it,
-// so m and logZ match hkv_step's bit for bit.
-__global__ void __launch_bounds__(NT) k_calibrate(const __grid_constant__ Params P)
+// S2-S4 per unit, one CTA per (sequence, KV head). Units of up to ZSTAGE
+// tokens work on a copy of their scores in shared memory.
+//  do_select  ([TS 2.B] calibration, [Abstract]/[TS 2.A] Top-p budget with the
+//             hard limits): writes sel_len, cut, m, logZ. With have_range the
+//             unit's score range comes from the scorer's range words.
+//  do_compact ([TS 2.C] Flatten Index): writes the unit's indices in score
+//             order from the cut -- PAD_MAX rows, or FLAT_SUM (standalone) --
+//             and, standalone, the Rewrite Cache copy when k_out is given.
+template <int ES>
+__global__ void __launch_bounds__(NT) k_unit(const __grid_constant__ Params P)
 {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     USmem &sm = *reinterpret_cast<USmem *>(smem_raw);
     const Ctl c = make_ctl(P);
     const int u = blockIdx.x;
+    allow_dependents();
+    wait_prior_grid();
+    HKV_TRACE_AT(TR_SEL + 16 * u);
     const int n = tier_len(P.sparse, u, c);
-    const float *zu = stage_scores(P.z + (int64_t)u * P.z_stride, n, sm);
+    const float *zg = P.z + (int64_t)u * P.z_stride;
+    const bool staged = stage_scores(zg, n, sm);
+    HKV_TRACE_AT(TR_SEL + 16 * u + 6);
+    if (staged)
+        unit_work<ES, true>(P, sm, c, u, n, sm.zs);
+    else
+        unit_work<ES, false>(P, sm, c, u, n, zg);
+}
+
+// S2 standalone ([TS 2.B]) for unit u: m, logZ and optionally the calibrated
+// probabilities. Z is summed exactly as the selection sums it, so m and logZ
+// match hkv_step's bit for bit.
+template <bool ZS>
+__device__ __forceinline__ void calibrate_unit(const Params &P, USmem &sm, const Ctl &c, int u, int n,
+                                               const float *zu)
+{
     float m, zlo;
-    unit_range(zu, n, &m, &zlo, sm);
+    unit_range<ZS>(zu, n, &m, &zlo, sm);
     const float bl2 = unit_beta(P, u, c) * LOG2E;
     double part = 0.0;
-    sweep_scores(zu, n, [&](float z, int, bool valid) {
+    sweep_scores<ZS>(zu, n, [&](float z, int, bool valid) {
         if (valid)
             part += (double)wcal(z, m, bl2);
     });
@@ -227,7 +238,7 @@ __global__ void __launch_bounds__(NT) k_calibrate(const __grid_constant__ Params
     if (P.P_out != nullptr && n > 0) {
         const float inv = (float)(1.0 / Z);
         float *Pu = P.P_out + (int64_t)u * P.z_stride;
-        sweep_scores(zu, n, [&](float z, int j, bool valid) {
+        sweep_scores<ZS>(zu, n, [&](float z, int j, bool valid) {
             if (valid)
                 Pu[j] = wcal(z, m, bl2) * inv;
         });
@@ -236,6 +247,20 @@ __global__ void __launch_bounds__(NT) k_calibrate(const __grid_constant__ Params
         P.m_out[u] = m;
         P.logZ_out[u] = n > 0 ? (float)log(Z) : -INFINITY;
     }
+}
+
+__global__ void __launch_bounds__(NT) k_calibrate(const __grid_constant__ Params P)
+{
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    USmem &sm = *reinterpret_cast<USmem *>(smem_raw);
+    const Ctl c = make_ctl(P);
+    const int u = blockIdx.x;
+    const int n = tier_len(P.sparse, u, c);
+    const float *zg = P.z + (int64_t)u * P.z_stride;
+    if (stage_scores(zg, n, sm))
+        calibrate_unit<true>(P, sm, c, u, n, sm.zs);
+    else
+        calibrate_unit<false>(P, sm, c, u, n, zg);
 }
 
 // FLAT_SUM rows and Rewrite Cache copies after the step's PAD_MAX compaction

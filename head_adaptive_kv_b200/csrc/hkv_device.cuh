@@ -201,6 +201,40 @@ __device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol
 // reads anything this grid writes.
 __device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// ---- shared-memory accesses with an explicit state space ----------------------
+// (functions that receive shared memory through a reference cannot always
+// prove it is shared, and would otherwise use slower generic accesses)
+
+__device__ __forceinline__ void sred_add(uint32_t *p, uint32_t v)
+{
+    asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(smem_addr(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ void sred_add(unsigned long long *p, unsigned long long v)
+{
+    asm volatile("red.shared.add.u64 [%0], %1;" ::"r"(smem_addr(p)), "l"(v) : "memory");
+}
+__device__ __forceinline__ int satom_add(int *p, int v)
+{
+    int old;
+    asm volatile("atom.shared.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(smem_addr(p)), "r"(v) : "memory");
+    return old;
+}
+__device__ __forceinline__ float4 lds4(const float *p)
+{
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "r"(smem_addr(p))
+                 : "memory");
+    return v;
+}
+__device__ __forceinline__ float lds1(const float *p)
+{
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(smem_addr(p)) : "memory");
+    return v;
+}
+
 // ---- arithmetic -------------------------------------------------------------
 
 // Two bf16 packed in a 32-bit word widened to two floats (exact).

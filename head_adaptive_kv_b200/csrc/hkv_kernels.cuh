@@ -33,6 +33,7 @@ constexpr int AT_NW = 8;                  // attention: warps per CTA
 constexpr int AT_SLOT = 8192;             // attention: bytes per stage (K rows, then as many V rows)
 constexpr int AT_STAGES = 3;              // attention: ring slots per warp
 constexpr int SC_FLOATS = 256;            // per-warp logits of one attention stage
+constexpr bool ATTN_UNROLL_QK = true;     // attention: unroll the logit batches of a full stage
 constexpr int PREFIX_CAP = 2048;          // attention: units whose token prefix fits in shared memory
 constexpr int SEL_THREADS = 512;          // per-unit kernels
 constexpr float LOG2E = 1.4426950408889634f;
@@ -546,7 +547,7 @@ __device__ __forceinline__ void attn_stage(const Params &P, const unsigned char 
     const bool writer = (lane % Gm::REP) == 0;
     const float scale2 = P.scale * LOG2E;
     // logits of the stage's tokens for all G query heads
-    if (nt == Gm::ATOK) {
+    if (ATTN_UNROLL_QK && nt == Gm::ATOK) {
         constexpr int NBAT = Gm::AITERS / Gm::NB;
         float v[NBAT];
 #pragma unroll
@@ -1006,16 +1007,16 @@ __device__ int64_t attn_prologue(const Params &P, AttnSmem<ES, D, G> &sm, const 
 
 constexpr int NT = SEL_THREADS;
 
-// Scores of one unit, from shared memory (staged) or global memory, in batches
-// of Q quads per thread with all loads in flight. Thread t takes quads
-// t, t + NT, ... of each batch, whatever the source or its alignment, so sums
-// taken in call order are identical on every path. f(z, j, valid) is called
-// by every thread the same number of times.
-template <typename F>
+// Scores of one unit, from shared memory (ZS: staged there by stage_scores)
+// or global memory, in batches of Q quads per thread with all loads in
+// flight. Thread t takes quads t, t + NT, ... of each batch, whatever the
+// source or its alignment, so sums taken in call order are identical on every
+// path. f(z, j, valid) is called by every thread the same number of times.
+template <bool ZS, typename F>
 __device__ __forceinline__ void sweep_scores(const float *zu, int n, F &&f)
 {
     constexpr int Q = 8;
-    const bool vec = (((uintptr_t)zu) & 15) == 0;
+    const bool vec = ZS || (((uintptr_t)zu) & 15) == 0;
     const int nq = (n + 3) >> 2;
     for (int base = 0; base < nq; base += NT * Q) {
         float4 v[Q];
@@ -1023,12 +1024,12 @@ __device__ __forceinline__ void sweep_scores(const float *zu, int n, F &&f)
         for (int i = 0; i < Q; ++i) {
             const int j = 4 * (base + i * NT + (int)threadIdx.x);
             if (vec && j + 4 <= n) {
-                v[i] = *reinterpret_cast<const float4 *>(zu + j);
+                v[i] = ZS ? lds4(zu + j) : __ldcg(reinterpret_cast<const float4 *>(zu + j));
             } else {
-                v[i].x = j < n ? zu[j] : 0.f;
-                v[i].y = j + 1 < n ? zu[j + 1] : 0.f;
-                v[i].z = j + 2 < n ? zu[j + 2] : 0.f;
-                v[i].w = j + 3 < n ? zu[j + 3] : 0.f;
+                v[i].x = j < n ? (ZS ? lds1(zu + j) : __ldcg(zu + j)) : 0.f;
+                v[i].y = j + 1 < n ? (ZS ? lds1(zu + j + 1) : __ldcg(zu + j + 1)) : 0.f;
+                v[i].z = j + 2 < n ? (ZS ? lds1(zu + j + 2) : __ldcg(zu + j + 2)) : 0.f;
+                v[i].w = j + 3 < n ? (ZS ? lds1(zu + j + 3) : __ldcg(zu + j + 3)) : 0.f;
             }
         }
 #pragma unroll
@@ -1051,8 +1052,7 @@ constexpr int ZSTAGE = 24576;  // scores of a unit staged in shared memory (unit
 struct __align__(16) USmem {  // shared memory of the per-unit kernels
     float zs[ZSTAGE];
     uint32_t cnt[SBINS];
-    uint32_t mlo[SBINS];  // bin mass, low 32 bits (fixed point)
-    uint32_t mhi[SBINS];  // bin mass, high 32 bits
+    unsigned long long mass[SBINS];  // bin mass (fixed point)
     unsigned long long cand[CAND_CAP];  // (order key << 32) | token index
     unsigned long long red[NT / 32];
     double redd[NT / 32];
@@ -1060,17 +1060,6 @@ struct __align__(16) USmem {  // shared memory of the per-unit kernels
     int32_t bc[8];
     unsigned long long bcl[4];
 };
-
-// Exact 64-bit add into a (lo, hi) pair of 32-bit shared words: the carry out
-// of the low word goes to the high word, so the sum is order-independent.
-__device__ __forceinline__ void add_split(uint32_t *lo, uint32_t *hi, unsigned long long v)
-{
-    const uint32_t l = (uint32_t)v;
-    const uint32_t old = atomicAdd(lo, l);
-    const uint32_t h = (uint32_t)(v >> 32) + ((uint32_t)(old + l) < old ? 1u : 0u);
-    if (h)
-        atomicAdd(hi, h);
-}
 
 struct BinFn {
     float m, s;
@@ -1100,10 +1089,11 @@ struct Selection {
 };
 
 // Largest and smallest finite score of a unit.
+template <bool ZS>
 __device__ void unit_range(const float *zu, int n, float *m, float *zlo, USmem &sm)
 {
     float mx = -INFINITY, mn = INFINITY;
-    sweep_scores(zu, n, [&](float z, int, bool valid) {
+    sweep_scores<ZS>(zu, n, [&](float z, int, bool valid) {
         if (!valid)
             return;
         mx = fmaxf(mx, z);
@@ -1114,12 +1104,12 @@ __device__ void unit_range(const float *zu, int n, float *m, float *zlo, USmem &
     *zlo = -block_max<NT>(-mn, sm.redf);
 }
 
-// Copy a unit's n <= ZSTAGE scores into shared memory (all loads in flight)
-// and return the staged copy; longer units stay in global memory.
-__device__ const float *stage_scores(const float *zu, int n, USmem &sm)
+// Copy a unit's n <= ZSTAGE scores into shared memory (all loads in flight);
+// longer units stay in global memory. Returns whether they were staged.
+__device__ bool stage_scores(const float *zu, int n, USmem &sm)
 {
     if (n > ZSTAGE)
-        return zu;
+        return false;
     const bool vec = (((uintptr_t)zu) & 15) == 0;
     if (vec) {
         constexpr int PER = ZSTAGE / 4 / NT;
@@ -1144,7 +1134,7 @@ __device__ const float *stage_scores(const float *zu, int n, USmem &sm)
             sm.zs[j] = __ldcg(zu + j);
     }
     __syncthreads();
-    return sm.zs;
+    return true;
 }
 
 // First bin whose cumulative count (by_mass = false) or mass reaches target
@@ -1217,24 +1207,34 @@ __device__ void sort_candidates(unsigned long long *cand, int P)
     }
 }
 
-__device__ __forceinline__ void gather_token(float z, int j, USmem &sm)
+// Append (key, index) of the lanes with `hit` to sm.cand (one shared atomic
+// per warp). All lanes of the warp call it together.
+__device__ __forceinline__ void gather_warp(bool hit, float z, int j, USmem &sm)
 {
-    const int pos = atomicAdd(&sm.bc[1], 1);
-    if (pos < CAND_CAP)
-        sm.cand[pos] = ((unsigned long long)score_key(z) << 32) | (uint32_t)j;
+    const unsigned mask = __ballot_sync(0xffffffffu, hit);
+    if (mask == 0)
+        return;
+    const int lane = threadIdx.x & 31, leader = __ffs(mask) - 1;
+    int base = 0;
+    if (lane == leader)
+        base = satom_add(&sm.bc[1], __popc(mask));
+    base = __shfl_sync(0xffffffffu, base, leader);
+    if (hit) {
+        const int pos = base + __popc(mask & ((1u << lane) - 1u));
+        if (pos < CAND_CAP)
+            sm.cand[pos] = ((unsigned long long)score_key(z) << 32) | (uint32_t)j;
+    }
 }
 
 // Collect the (key, index) of the tokens of bin `bin` into sm.cand (call only
 // when the bin holds at most CAND_CAP tokens).
+template <bool ZS>
 __device__ void gather_bin(const float *zu, int n, const BinFn &bins, int bin, USmem &sm)
 {
     if (threadIdx.x == 0)
         sm.bc[1] = 0;
     __syncthreads();
-    sweep_scores(zu, n, [&](float z, int j, bool valid) {
-        if (valid && bins(z) == bin)
-            gather_token(z, j, sm);
-    });
+    sweep_scores<ZS>(zu, n, [&](float z, int j, bool valid) { gather_warp(valid && bins(z) == bin, z, j, sm); });
     __syncthreads();
 }
 
@@ -1284,6 +1284,7 @@ __device__ int sort_and_locate(int cnt_in, bool by_mass, unsigned long long targ
 // fallback of sort_and_locate for bins above CAND_CAP tokens). Returns the cut
 // key; *above gets the bin's tokens with a smaller key (higher score) and
 // *above_mass their mass (mass targets only).
+template <bool ZS>
 __device__ uint32_t descend_bin(const float *zu, int n, const BinFn &bins, int bin, bool by_mass,
                                 unsigned long long target, float m, float bl2, USmem &sm,
                                 unsigned long long *above, unsigned long long *above_mass)
@@ -1305,16 +1306,16 @@ __device__ uint32_t descend_bin(const float *zu, int n, const BinFn &bins, int b
             dmass[i] = 0;
         }
         __syncthreads();
-        sweep_scores(zu, n, [&](float z, int, bool valid) {
+        sweep_scores<ZS>(zu, n, [&](float z, int, bool valid) {
             if (!valid || bins(z) != bin)
                 return;
             const uint32_t key = score_key(z);
             if (pshift < 32 && (key >> pshift) != prefix)
                 return;
             const uint32_t d = (key >> shift) & (uint32_t)(nb - 1);
-            atomicAdd(&dcnt[d], 1u);
+            sred_add(&dcnt[d], 1u);
             if (by_mass)
-                atomicAdd(&dmass[d], wfix(z, m, bl2));
+                sred_add(&dmass[d], wfix(z, m, bl2));
         });
         __syncthreads();
         unsigned long long bc_, bm_;
@@ -1344,6 +1345,7 @@ __device__ uint32_t descend_bin(const float *zu, int n, const BinFn &bins, int b
 // sorting its tokens by (key, index); a bin too large to sort falls back to an
 // exact radix descent over its keys.
 // =============================================================================
+template <bool ZS>
 __device__ Selection select_unit(const float *zu, int n, float m, float zlo, float beta, float p, int bmin, int bmax,
                                  USmem &sm, int tb = -1)
 {
@@ -1352,18 +1354,17 @@ __device__ Selection select_unit(const float *zu, int n, float m, float zlo, flo
     const BinFn bins = make_bins(m, zlo);
     for (int i = threadIdx.x; i < SBINS; i += NT) {
         sm.cnt[i] = 0;
-        sm.mlo[i] = 0;
-        sm.mhi[i] = 0;
+        sm.mass[i] = 0;
     }
     __syncthreads();
-    const auto mass = [&](int b) { return ((unsigned long long)sm.mhi[b] << 32) + sm.mlo[b]; };
+    const auto mass = [&](int b) { return sm.mass[b]; };
     // sweep 1: bin counts and the normaliser
     double zsum = 0.0;
-    sweep_scores(zu, n, [&](float z, int, bool valid) {
+    sweep_scores<ZS>(zu, n, [&](float z, int, bool valid) {
         if (!valid)
             return;
         zsum += (double)wcal(z, m, bl2);
-        atomicAdd(&sm.cnt[bins(z)], 1u);
+        sred_add(&sm.cnt[bins(z)], 1u);
     });
     r.Z = block_sum_f64<NT>(zsum, sm.redd);
     HKV_TRACE_AT(tb < 0 ? -1 : tb + 1);
@@ -1374,6 +1375,7 @@ __device__ Selection select_unit(const float *zu, int n, float m, float zlo, flo
     unsigned long long hb_c = 0, hb_m = 0;
     const int b_hi = n > 0 ? find_crossing(sm.cnt, mass, SBINS, false, (unsigned long long)r_hi, &hb_c, &hb_m, sm)
                            : 0;
+    HKV_TRACE_AT(tb < 0 ? -1 : tb + 7);
     const int cnt_hi = n > 0 ? (int)sm.cnt[b_hi] : 0;
     const bool gather_hi = n > 0 && cnt_hi <= CAND_CAP;
     const bool need_mass = n > 0 && p > 0.0f && p < 1.0f;
@@ -1381,12 +1383,12 @@ __device__ Selection select_unit(const float *zu, int n, float m, float zlo, flo
         sm.bc[1] = 0;
     __syncthreads();
     if (need_mass || gather_hi) {
-        sweep_scores(zu, n, [&](float z, int j, bool valid) {
+        sweep_scores<ZS>(zu, n, [&](float z, int j, bool valid) {
             const int bz = valid ? bins(z) : SBINS;
             if (need_mass && bz <= b_hi)
-                add_split(&sm.mlo[bz], &sm.mhi[bz], wfix(z, m, bl2));
-            if (gather_hi && bz == b_hi)
-                gather_token(z, j, sm);
+                sred_add(&sm.mass[bz], wfix(z, m, bl2));  // integer sum: exact in any order
+            if (gather_hi)
+                gather_warp(bz == b_hi, z, j, sm);
         });
         __syncthreads();
     }
@@ -1412,13 +1414,14 @@ __device__ Selection select_unit(const float *zu, int n, float m, float zlo, flo
         for (int i = threadIdx.x; i <= b_hi; i += NT)
             part += mass(i);
         const unsigned long long through = block_sum_u64<NT>(part, sm.red);
+        HKV_TRACE_AT(tb < 0 ? -1 : tb + 8);
         if (through >= T) {
             unsigned long long mb_c, mb_m;
             const int b_m = find_crossing(sm.cnt, mass, SBINS, true, T, &mb_c, &mb_m, sm);
             const int cnt_in = (int)sm.cnt[b_m];
             if (cnt_in <= CAND_CAP) {
                 if (gathered != b_m) {
-                    gather_bin(zu, n, bins, b_m, sm);
+                    gather_bin<ZS>(zu, n, bins, b_m, sm);
                     gathered = b_m;
                 }
                 const int pos = sort_and_locate(cnt_in, true, T, mb_m, m, bl2, sm);
@@ -1429,7 +1432,7 @@ __device__ Selection select_unit(const float *zu, int n, float m, float zlo, flo
                 cut_before = mb_c;
             } else {
                 unsigned long long ab, am;
-                const uint32_t key = descend_bin(zu, n, bins, b_m, true, T - mb_m, m, bl2, sm, &ab, &am);
+                const uint32_t key = descend_bin<ZS>(zu, n, bins, b_m, true, T - mb_m, m, bl2, sm, &ab, &am);
                 gathered = -1;
                 const unsigned long long w_at = wfix(key_score(key), m, bl2);
                 const unsigned long long need = T - mb_m - am;
@@ -1457,16 +1460,18 @@ __device__ Selection select_unit(const float *zu, int n, float m, float zlo, flo
         sorted_cut = false;
         unsigned long long kb_c, kb_m;
         const int b_k = find_crossing(sm.cnt, mass, SBINS, false, (unsigned long long)k, &kb_c, &kb_m, sm);
+        HKV_TRACE_AT(tb < 0 ? -1 : tb + 9);
         const int cnt_in = (int)sm.cnt[b_k];
         if (cnt_in <= CAND_CAP) {
             if (gathered != b_k)
-                gather_bin(zu, n, bins, b_k, sm);
+                gather_bin<ZS>(zu, n, bins, b_k, sm);
             cut_pos = sort_and_locate(cnt_in, false, (unsigned long long)k - kb_c, 0, m, bl2, sm);
+            HKV_TRACE_AT(tb < 0 ? -1 : tb + 10);
             sorted_cut = true;
             cut_before = kb_c;
         } else {
             unsigned long long ab, am;
-            r.key = descend_bin(zu, n, bins, b_k, false, (unsigned long long)k - kb_c, m, bl2, sm, &ab, &am);
+            r.key = descend_bin<ZS>(zu, n, bins, b_k, false, (unsigned long long)k - kb_c, m, bl2, sm, &ab, &am);
             r.cut.n_above = (int32_t)(kb_c + ab);
         }
     }
@@ -1497,6 +1502,7 @@ __device__ Selection select_unit(const float *zu, int n, float m, float zlo, flo
 // key == cut key into row[0, k); PAD_MAX rows are padded with -1 to `pad`.
 // Each thread takes E consecutive tokens of a chunk (loaded together).
 // =============================================================================
+template <bool ZS>
 __device__ void compact_unit(const float *zu, int n, uint32_t cut_key, int n_tie, int k, int32_t *row, int pad,
                              unsigned long long *red)
 {
@@ -1510,7 +1516,7 @@ __device__ void compact_unit(const float *zu, int n, uint32_t cut_key, int n_tie
             if (vec && j0 + E <= n) {
 #pragma unroll
                 for (int e = 0; e < E; e += 4) {
-                    const float4 v = *reinterpret_cast<const float4 *>(zu + j0 + e);
+                    const float4 v = ZS ? lds4(zu + j0 + e) : __ldcg(reinterpret_cast<const float4 *>(zu + j0 + e));
                     zz[e] = v.x;
                     zz[e + 1] = v.y;
                     zz[e + 2] = v.z;
@@ -1519,7 +1525,7 @@ __device__ void compact_unit(const float *zu, int n, uint32_t cut_key, int n_tie
             } else {
 #pragma unroll
                 for (int e = 0; e < E; ++e)
-                    zz[e] = (j0 + e < n) ? zu[j0 + e] : 0.f;
+                    zz[e] = (j0 + e < n) ? (ZS ? lds1(zu + j0 + e) : __ldcg(zu + j0 + e)) : 0.f;
             }
             uint32_t lt_bits = 0, eq_bits = 0;
 #pragma unroll
