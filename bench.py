@@ -118,14 +118,24 @@ def whole_job_value(units_per_rank: int, units_per_step: int, world: int, second
 # ---- algorithmic bytes --------------------------------------------------------------
 
 
+def logit_floats(G: int) -> int:
+    """Floats of one token's per-head logit record (G logits padded to 16 bytes)."""
+    return (G + 3) // 4 * 4
+
+
 def step_bytes(wl, sparse_len, dense_len, cond_len, sel_len) -> int:
-    """Bytes the method must move in one step: every sparse key is scored once;
-    dense, selected and condensed K and V rows are attended once; plus q, the
+    """Bytes one step must move in this design: every sparse key is read once
+    and scored (its max-pooled score and its per-head logits written); dense
+    and condensed K and V rows are attended; a selected sparse token's V row
+    and logit record are read back (its K row is not read again); plus q, the
     outputs and the compacted rows."""
     e = 2 if wl.dtype == torch.bfloat16 else 4
     D = wl.D
-    scored = int(np.sum(sparse_len)) * D * e
-    attended = int(np.sum(dense_len) + np.sum(cond_len) + np.sum(sel_len)) * 2 * D * e
+    lb = logit_floats(wl.G) * 4
+    n = int(np.sum(sparse_len))
+    k = int(np.sum(sel_len))
+    scored = n * (D * e + 4 + lb)
+    attended = int(np.sum(dense_len) + np.sum(cond_len)) * 2 * D * e + k * (D * e + lb)
     q = wl.B * wl.Hq * D * e
     out = wl.B * wl.Hq * (D + 1) * 4
     idx = wl.units * wl.bmax * 4 + wl.units * 4

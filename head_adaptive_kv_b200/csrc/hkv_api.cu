@@ -59,7 +59,8 @@ __global__ void __launch_bounds__(sc_nw(G) * 32, 1) k_score_stream(const __grid_
 }
 
 // S5 ([TS 2.A] cascade decode over the three tiers; [TS 2.C] Sparse Loading):
-// persistent streaming attention over the tokens of all units.
+// persistent streaming attention over line A (dense and condensed tokens)
+// and line B (selected sparse tokens); writes one record per warp and unit.
 template <int ES, int D, int G>
 __global__ void __launch_bounds__(AT_NW * 32, 1) k_attn_stream(const __grid_constant__ Params P)
 {
@@ -72,15 +73,24 @@ __global__ void __launch_bounds__(AT_NW * 32, 1) k_attn_stream(const __grid_cons
     allow_dependents();
     wait_prior_grid();
     HKV_TRACE_WARP(TR_AW + 4 * (blockIdx.x * AT_NW + (threadIdx.x >> 5)) + 3);
-    const int64_t T = attn_prologue<ES, D, G>(P, sm, c, red);
-    // every warp that takes part gets a non-empty share
-    const int64_t NW = min((int64_t)gridDim.x * AT_NW, T);
+    AttnLine A, B;
+    attn_prologue<ES, D, G>(P, sm, c, red, &A, &B);
     const int64_t g = (int64_t)blockIdx.x * AT_NW + (threadIdx.x >> 5);
-    if (g < NW) {
-        AttnJob<ES, D, G> job(P, c, sm, NW, T, g);
-        HKV_TRACE_WARP(TR_AW + 4 * (int)g);
-        warp_pipeline(job, sm.ring, c, TR_AW + 4 * (int)g);
-    }
+    AttnJob<ES, D, G> job(P, c, sm, A, B, g);
+    HKV_TRACE_WARP(TR_AW + 4 * (int)g);
+    warp_pipeline(job, sm.ring, c, TR_AW + 4 * (int)g);
+}
+
+// S5 merge: out and lse of each (unit, query head) from the unit's records on
+// both attention lines, in slot order (one warp per query head).
+template <int D, int G>
+__global__ void __launch_bounds__(G * 32) k_merge(const __grid_constant__ Params P)
+{
+    allow_dependents();
+    wait_prior_grid();
+    const int u = blockIdx.x;
+    const int4 r = __ldcg(reinterpret_cast<const int4 *>(P.rec_range) + u);
+    merge_head<D, G>(P, u, threadIdx.x >> 5, r.x, r.y, r.z, r.w);
 }
 
 // Rewrite Cache ([TS 2.C]): copy the k selected K/V rows of unit u, listed in
@@ -183,7 +193,7 @@ __device__ __forceinline__ void unit_work(const Params &P, USmem &sm, const Ctl 
         write_offsets(P, u, off);
     }
     int32_t *row = P.idx + off;
-    compact_unit<ZS>(zu, n, key, n_tie, k, row, flat ? k : P.bmax, sm.red);
+    compact_unit<ZS>(zu, n, key, n_tie, k, row, flat ? k : P.bmax, sm.red, TR_SEL + 16 * u);
     HKV_TRACE_AT(TR_SEL + 16 * u + 5);
     if (P.k_out != nullptr && !P.do_select) {
         __syncthreads();
@@ -295,7 +305,7 @@ std::atomic<uint64_t> g_wait_ns{1000000000ull};
 std::atomic<int32_t> g_withhold{0};
 
 struct WsLayout {
-    size_t ctl, attn_cnt, urange, part, idxbuf, zbuf, total;
+    size_t ctl, urange, rec_range, part, idxbuf, zbuf, logits, total;
     int64_t z_stride;
     int part_slots;
 };
@@ -374,7 +384,7 @@ static WsLayout layout_of(const hkv_problem *p, const hkv_tier *dense, const hkv
     const int64_t units = (int64_t)p->B * p->Hkv;
     const int G = p->Hq / p->Hkv;
     const int ncap = sparse ? sparse->cap : 0;
-    L.part_slots = (int)(stream_ctas() * (int64_t)AT_NW + units);
+    L.part_slots = (int)(2 * (stream_ctas() * (int64_t)AT_NW + units));
     L.z_stride = (int64_t)align_up((size_t)std::max(ncap, 1), 4);
     size_t o = 0;
     auto take = [&](size_t bytes) {
@@ -382,13 +392,14 @@ static WsLayout layout_of(const hkv_problem *p, const hkv_tier *dense, const hkv
         o = align_up(o + bytes, 256);
         return at;
     };
-    // what must start at zero comes first: status word, counters, range words
+    // what must start at zero comes first: status word, range words
     L.ctl = take(256);
-    L.attn_cnt = take(units * 4);
     L.urange = take(units * 8);
+    L.rec_range = take(units * 16);
     L.part = take((size_t)L.part_slots * part_stride(p->D, G) * 4);
     L.idxbuf = take(units * (size_t)std::max(p->bmax, 1) * 4);
     L.zbuf = take((size_t)units * L.z_stride * 4);
+    L.logits = take((size_t)units * ncap * logit_floats(G) * 4);
     L.total = o;
     return L;
 }
@@ -414,12 +425,13 @@ static Params base_params(const hkv_problem *p, const WsLayout &L, char *ws, con
     P.wait_ns = g_wait_ns.load();
     P.withhold = g_withhold.load();
     P.ctl = reinterpret_cast<uint32_t *>(ws + L.ctl);
-    P.attn_cnt = reinterpret_cast<uint32_t *>(ws + L.attn_cnt);
+    P.rec_range = reinterpret_cast<int32_t *>(ws + L.rec_range);
     P.part = reinterpret_cast<float *>(ws + L.part);
     P.part_slots = L.part_slots;
     P.attn_prefix = P.units <= PREFIX_CAP;
-    const int ncap = sparse ? sparse->cap : 0;
-    P.attn_span = (dense ? dense->cap : 0) + std::min(p->bmax, ncap) + (cond ? cond->cap : 0);
+    (void)dense;
+    (void)sparse;
+    (void)cond;
     return P;
 }
 
@@ -554,12 +566,18 @@ struct RunScore {
 
 template <int ES, int D, int G>
 struct RunAttn {
+    // attention then merge
     static hkv_status run(const Params &P, cudaStream_t s, bool pdl)
     {
-        // the records hold (CTAs x warps + units) slots
-        const int max_ctas = (P.part_slots - P.units) / AT_NW;
-        return launch_stream(k_attn_stream<ES, D, G>, AT_NW * 32, sizeof(AttnSmem<ES, D, G>), max_ctas, s, P,
-                             pdl);
+        // the records hold 2 x (CTAs x warps + units) slots
+        const int max_ctas = (P.part_slots / 2 - P.units) / AT_NW;
+        if (max_ctas < 1)
+            return HKV_ERR_WORKSPACE;
+        hkv_status st = launch_stream(k_attn_stream<ES, D, G>, AT_NW * 32, sizeof(AttnSmem<ES, D, G>), max_ctas, s,
+                                      P, pdl);
+        if (st != HKV_OK)
+            return st;
+        return launch(k_merge<D, G>, P.units, G * 32, 0, s, P, true);
     }
 };
 
@@ -831,6 +849,7 @@ hkv_status hkv_step(const hkv_problem *prob, const void *q, const hkv_tier *dens
     P.logZ_out = o->logZ;
     P.k_out = static_cast<char *>(o->k_out);
     P.v_out = static_cast<char *>(o->v_out);
+    P.logit = reinterpret_cast<float *>(wsb + L.logits);  // scorer -> attention of the selected tokens
     P.layout = HKV_LAYOUT_PAD_MAX;  // the three kernels work on PAD_MAX rows
     // 1. scores, and the score range of each unit
     const bool scored = sparse->cap > 0;
@@ -921,14 +940,14 @@ extern "C" hkv_status hkv_cascade_decode_noalloc(const hkv_problem *prob, const 
         if (prob->layout == HKV_LAYOUT_FLAT_SUM && offsets == nullptr)
             return HKV_ERR_INVALID_ARG;
     }
-    // The attention uses the front of the workspace layout: the status and
-    // counter words, the range words and the records. It needs at least the
-    // records of one CTA (a record per warp and per unit); when the array
-    // holds fewer than a full grid needs, fewer CTAs run.
+    // The attention uses the front of the workspace layout: the status word,
+    // the range words, the record slots of each unit and the records. It needs
+    // at least the records of one CTA (two per warp and per unit); when the
+    // array holds fewer than a full grid needs, fewer CTAs run.
     const WsLayout L = layout_of(prob, dense, sparse, condensed);
     const size_t rec = (size_t)part_stride(prob->D, prob->Hq / prob->Hkv) * sizeof(float);
     const int64_t units = (int64_t)prob->B * prob->Hkv;
-    if (L.part + (size_t)(units + AT_NW) * rec > HKV_NOALLOC_SCRATCH_BYTES)
+    if (L.part + 2 * (size_t)(units + AT_NW) * rec > HKV_NOALLOC_SCRATCH_BYTES)
         return HKV_ERR_WORKSPACE;
     const int slots = (int)std::min<int64_t>(L.part_slots, (HKV_NOALLOC_SCRATCH_BYTES - L.part) / rec);
     const cudaStream_t st = (cudaStream_t)stream;
@@ -950,9 +969,8 @@ extern "C" hkv_status hkv_cascade_decode_noalloc(const hkv_problem *prob, const 
     P.sel_len = const_cast<int32_t *>(sel_len);
     P.out = out;
     P.lse = lse;
-    // the status word, the ticket and exit counters and the per-unit tile
-    // counters must start at zero; the previous call may have left them set
-    if (cudaMemsetAsync(base, 0, L.urange, st) != cudaSuccess)
+    // the status word must start at zero; the previous call may have left it set
+    if (cudaMemsetAsync(base, 0, sizeof(uint32_t), st) != cudaSuccess)
         return HKV_ERR_CUDA;
     if ((s = dispatch<RunAttn>(prob, P, st, false)) != HKV_OK)
         return s;

@@ -11,8 +11,8 @@
 //    pipeline over a contiguous share of the kernel's work (a static, balanced
 //    partition: no tickets, no producer warp). It keeps several stages in
 //    flight in its own ring of shared-memory slots, armed and filled by the
-//    warp itself: 1-D TMA bulk copies for contiguous rows, 16-byte cp.async for
-//    gathered rows, completion on one mbarrier per slot.
+//    warp itself with 1-D TMA bulk copies (one per contiguous run, or one per
+//    gathered row), completion on one mbarrier per slot.
 //  - per-unit kernels (selection, compaction, calibration, layout): one CTA of
 //    SEL_THREADS threads per (sequence, KV head).
 // No tensor cores: a one-query decode is a GEMV (about 4 flop per byte), bound
@@ -34,7 +34,7 @@ constexpr int AT_SLOT = 8192;             // attention: bytes per stage (K rows,
 constexpr int AT_STAGES = 3;              // attention: ring slots per warp
 constexpr int SC_FLOATS = 256;            // per-warp logits of one attention stage
 constexpr bool ATTN_UNROLL_QK = true;     // attention: unroll the logit batches of a full stage
-constexpr int PREFIX_CAP = 2048;          // attention: units whose token prefix fits in shared memory
+constexpr int PREFIX_CAP = 1024;          // attention: units whose token prefixes fit in shared memory
 constexpr int SEL_THREADS = 512;          // per-unit kernels
 constexpr float LOG2E = 1.4426950408889634f;
 
@@ -62,14 +62,17 @@ struct Params {
     int32_t *offsets;
     float *out, *lse, *m_out, *logZ_out, *P_out;
     char *k_out, *v_out;
+    // per-head logits scale * q_g . k_j of every sparse token, written by the
+    // scorer and read back by the attention for the selected tokens (hkv_step
+    // only, else nullptr): token j of unit u at logit + (u cap + j) * LG
+    float *logit;
     // workspace
     uint32_t *ctl;        // [0] status word
     uint32_t *urange;     // [units][2] score range of each unit as order keys (step only, else nullptr)
-    uint32_t *attn_cnt;   // [units] attention records finished
+    int32_t *rec_range;   // [units][4] first and last record slot of each unit on attention lines A and B
     float *part;          // [part_slots * part_stride] attention records
-    int32_t part_slots;   // record slots (streaming warps of the attention grid + units)
+    int32_t part_slots;   // record slots: 2 x (streaming warps of the attention grid + units)
     int32_t attn_prefix;  // attention partition over actual tokens (units <= PREFIX_CAP), else over capacity
-    int32_t attn_span;    // capacity partition: token positions per unit (W cap + min(bmax, n cap) + C cap)
     int32_t have_range;   // per-unit kernel: urange holds the units' score ranges
     int32_t do_select, do_compact;  // per-unit kernel: which steps to run
     int32_t withhold;     // fault injection: streaming warps never arm their stages
@@ -130,6 +133,9 @@ __device__ __forceinline__ int unit_budget(const Params &P, int u, int n, const 
 // Floats of one attention record (o[G][D], m[G], l[G]), padded to a multiple of 4.
 __host__ __device__ constexpr int part_stride(int D, int G) { return (G * (D + 2) + 3) / 4 * 4; }
 
+// Floats of one token's logit record (G logits, padded to 16 bytes).
+__host__ __device__ constexpr int logit_floats(int G) { return (G + 3) / 4 * 4; }
+
 // Order-preserving 32-bit keys of floats (larger float, larger key), so that
 // atomicMax on keys takes the maximum of floats. Key 0 means "none".
 __device__ __forceinline__ uint32_t ord_key(float x)
@@ -167,6 +173,7 @@ struct Geo {
     static constexpr int DPL = D / 32;                    // PV: head-dim elements per lane
     static_assert(G >= 1 && G <= LPR, "group size must not exceed lanes per row");
     static_assert(ATOK * G <= SC_FLOATS && ATOK <= 32, "stage sizes");
+    static_assert(ATOK * logit_floats(G) * 4 <= AT_SLOT / 2, "logit records of a stage");
     static_assert(SITERS % NB == 0 && AITERS % NB == 0 && LPR % NV == 0, "iteration batches");
 };
 
@@ -174,7 +181,7 @@ struct Geo {
 // Streaming engine
 // =============================================================================
 
-enum : int32_t { SD_FIRST = 1, SD_LAST = 2, SD_GATHER = 4, SD_ARMED = 8 };
+enum : int32_t { SD_FIRST = 1, SD_LAST = 2, SD_GATHER = 4, SD_ARMED = 8, SD_LOGIT = 16, SD_LINEB = 32 };
 
 // Trace builds (-DHKV_TRACE): per warp trace slot base s (4 slots), the issue
 // and landing times of its first 12 stages at TRACE_STAGES + 8 s + 2 i (+1).
@@ -467,11 +474,16 @@ struct ScoreJob {
         const int vi = (lane % Gm::LPR) / Gm::REP;
         const bool writer = (lane % Gm::REP) == 0 && (vi % G) == 0;
         float *zu = P.z + (int64_t)d.unit * P.z_stride + d.start;
+        float *lg = P.logit == nullptr
+                        ? nullptr
+                        : P.logit + ((int64_t)d.unit * P.sparse.cap + d.start) * logit_floats(G) + vi % G;
         const auto emit = [&](float v, int it0, bool check) {
+            const int row = (it0 + vi / G) * Gm::RPW + lane / Gm::LPR;
+            if (lg != nullptr && (lane % Gm::REP) == 0 && (!check || row < d.count))
+                lg[row * logit_floats(G)] = v * P.scale;
 #pragma unroll
             for (int o = 1; o < G; o <<= 1)
                 v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o * Gm::REP));
-            const int row = (it0 + vi / G) * Gm::RPW + lane / Gm::LPR;
             if (writer && (!check || row < d.count)) {
                 const float zz = v * P.scale;
                 zu[row] = zz;
@@ -510,13 +522,17 @@ struct ScoreJob {
 // ---- attention ([TS 2.A] dense ++ selected sparse ++ condensed; [TS 2.C]
 // Sparse Loading: selected rows are read through the indices) ----------------
 //
-// Work line: the tokens of all units, unit-major, unit u holding
-// W_u + k_u + C_u tokens (attn_prefix: the actual counts, prefix-summed per
-// CTA in shared memory) or attn_span positions (capacity partition, for very
-// many units; positions past the unit's tokens are skipped). Each warp keeps an
-// online-softmax state over its share within one unit and writes it as a
-// record into slot (warp + unit), which is unique; the warp that completes a
-// unit's records merges them in a fixed order.
+// Two work lines, each split evenly over all warps of the grid:
+//   line A: the dense and condensed tokens of all units (W_u + C_u per unit;
+//           contiguous rows, full q.k and softmax-weighted V);
+//   line B: the selected sparse tokens of all units (k_u per unit; gathered
+//           rows, with the scorer's logits when hkv_step provides them).
+// A line's units are laid end to end (attn_prefix: actual counts, prefix-summed
+// per CTA in shared memory; else capacities, positions past a unit's tokens
+// skipped), and warp g takes an equal share of it. The online-softmax state
+// of a warp over its part of one unit becomes a record in slot
+// line_base + g + u (unique); k_merge combines a unit's records afterwards in
+// a fixed order.
 
 template <int D, int G>
 struct AttnState {
@@ -536,9 +552,12 @@ struct AttnState {
     }
 };
 
+// One attention stage: K rows at stage[0, AT_SLOT/2) (or, from_logits, the
+// tokens' logit records there), V rows at stage[AT_SLOT/2, AT_SLOT).
 template <int ES, int D, int G>
 __device__ __forceinline__ void attn_stage(const Params &P, const unsigned char *stage, int nt, float *sc,
-                                           const float2 (&qv)[G][Geo<ES, D, G>::NP], AttnState<D, G> &st)
+                                           const float2 (&qv)[G][Geo<ES, D, G>::NP], AttnState<D, G> &st,
+                                           bool from_logits)
 {
     using Gm = Geo<ES, D, G>;
     constexpr int NPV = AttnState<D, G>::NPV;
@@ -547,7 +566,15 @@ __device__ __forceinline__ void attn_stage(const Params &P, const unsigned char 
     const bool writer = (lane % Gm::REP) == 0;
     const float scale2 = P.scale * LOG2E;
     // logits of the stage's tokens for all G query heads
-    if (ATTN_UNROLL_QK && nt == Gm::ATOK) {
+    if (from_logits) {
+        // the scorer's logits: lane r < nt converts token r's record
+        if (lane < nt) {
+            const float *lr = reinterpret_cast<const float *>(stage) + lane * logit_floats(G);
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+                sc[lane * G + g] = lr[g] * LOG2E;
+        }
+    } else if (ATTN_UNROLL_QK && nt == Gm::ATOK) {
         constexpr int NBAT = Gm::AITERS / Gm::NB;
         float v[NBAT];
 #pragma unroll
@@ -636,88 +663,84 @@ __device__ __forceinline__ void attn_stage(const Params &P, const unsigned char 
     __syncwarp();
 }
 
-// Output of unit u from its records in slots [s0, s1] (fixed order), by one
-// warp: lane l owns head-dim elements l*DPL .. l*DPL + DPL - 1 of every head.
-// Records with m = -inf (no tokens) are skipped; no tokens at all gives
-// out = 0 and lse = -inf.
+// Record layout (part_stride floats): o[G][D] (unnormalised, log2 domain
+// weights), then m[G], then l[G]. m = -inf marks a record without tokens.
+
+// Output of head g of unit u from the records in slots [a0, a1] and [b0, b1]
+// (fixed order), by one warp: lane l owns head-dim elements l*DPL ..
+// l*DPL + DPL - 1. No tokens at all gives out = 0 and lse = -inf.
 template <int D, int G>
-__device__ __noinline__ void merge_records(const Params &P, int u, int s0, int s1)
+__device__ void merge_head(const Params &P, int u, int g, int a0, int a1, int b0, int b1)
 {
     constexpr int DPL = D / 32;
     constexpr int RS = part_stride(D, G);
     const int lane = threadIdx.x & 31;
-    const int b = u / P.Hkv, h = u % P.Hkv;
-    float M[G], L[G], O[G][DPL];
+    float M = -INFINITY, L = 0.f, O[DPL];
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-        M[g] = -INFINITY;
-        L[g] = 0.f;
-#pragma unroll
-        for (int e = 0; e < DPL; ++e)
-            O[g][e] = 0.f;
-    }
-    constexpr int RB = 4;  // records loaded together
-    for (int t0 = s0; t0 <= s1; t0 += RB) {
-        float mt[RB][G], lt[RB][G], ot[RB][G][DPL];
+    for (int e = 0; e < DPL; ++e)
+        O[e] = 0.f;
+    constexpr int RB = 8;  // records loaded together
+    const int na = a1 >= a0 ? a1 - a0 + 1 : 0, nb = b1 >= b0 ? b1 - b0 + 1 : 0;
+    for (int t0 = 0; t0 < na + nb; t0 += RB) {
+        float mt[RB], lt[RB], ot[RB][DPL];
 #pragma unroll
         for (int r = 0; r < RB; ++r) {
-            const bool ok = t0 + r <= s1;
-            const float *pr = P.part + (int64_t)(t0 + r) * RS;
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                mt[r][g] = ok ? __ldcg(pr + g * (D + 2) + D) : -INFINITY;
-                lt[r][g] = ok ? __ldcg(pr + g * (D + 2) + D + 1) : 0.f;
+            const int t = t0 + r;
+            const bool ok = t < na + nb;
+            const int slot = t < na ? a0 + t : b0 + (t - na);
+            const float *pr = P.part + (int64_t)(ok ? slot : 0) * RS;
+            mt[r] = ok ? __ldcg(pr + G * D + g) : -INFINITY;
+            lt[r] = ok ? __ldcg(pr + G * D + G + g) : 0.f;
+            if constexpr (DPL == 4) {
+                const float4 v = ok ? __ldcg(reinterpret_cast<const float4 *>(pr + g * D + lane * 4))
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+                ot[r][0] = v.x;
+                ot[r][1] = v.y;
+                ot[r][2] = v.z;
+                ot[r][3] = v.w;
+            } else {
 #pragma unroll
                 for (int e = 0; e < DPL; ++e)
-                    ot[r][g][e] = ok ? __ldcg(pr + g * (D + 2) + lane * DPL + e) : 0.f;
+                    ot[r][e] = ok ? __ldcg(pr + g * D + lane * DPL + e) : 0.f;
             }
         }
 #pragma unroll
-        for (int r = 0; r < RB; ++r)
+        for (int r = 0; r < RB; ++r) {
+            if (mt[r] == -INFINITY)
+                continue;
+            const float Mn = fmaxf(M, mt[r]);
+            const float a = (M == -INFINITY) ? 0.0f : ex2(M - Mn);
+            const float f = ex2(mt[r] - Mn);
+            L = L * a + lt[r] * f;
 #pragma unroll
-            for (int g = 0; g < G; ++g) {
-                if (mt[r][g] == -INFINITY)
-                    continue;
-                const float Mn = fmaxf(M[g], mt[r][g]);
-                const float a = (M[g] == -INFINITY) ? 0.0f : ex2(M[g] - Mn);
-                const float f = ex2(mt[r][g] - Mn);
-                L[g] = L[g] * a + lt[r][g] * f;
-#pragma unroll
-                for (int e = 0; e < DPL; ++e)
-                    O[g][e] = O[g][e] * a + ot[r][g][e] * f;
-                M[g] = Mn;
-            }
+            for (int e = 0; e < DPL; ++e)
+                O[e] = O[e] * a + ot[r][e] * f;
+            M = Mn;
+        }
     }
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-        const int hq = h * G + g;
-        float *orow = P.out + ((int64_t)b * P.Hq + hq) * D + lane * DPL;
-#pragma unroll
-        for (int e = 0; e < DPL; ++e)
-            orow[e] = (M[g] == -INFINITY) ? 0.0f : O[g][e] / L[g];
-        if (lane == 0 && P.lse != nullptr)
-            P.lse[(int64_t)b * P.Hq + hq] =
-                (M[g] == -INFINITY) ? -INFINITY : (M[g] + log2f(L[g])) * 0.6931471805599453f;
-    }
-}
-
-// out = 0, lse = -inf for a unit with no tokens (one warp).
-template <int D, int G>
-__device__ void write_empty_unit(const Params &P, int u)
-{
-    const int lane = threadIdx.x & 31;
     const int b = u / P.Hkv, h = u % P.Hkv;
-    for (int i = lane; i < G * D; i += 32)
-        P.out[((int64_t)b * P.Hq + h * G) * D + i] = 0.0f;
-    if (lane < G && P.lse != nullptr)
-        P.lse[(int64_t)b * P.Hq + h * G + lane] = -INFINITY;
+    const int hq = h * G + g;
+    float *orow = P.out + ((int64_t)b * P.Hq + hq) * D + lane * DPL;
+#pragma unroll
+    for (int e = 0; e < DPL; ++e)
+        orow[e] = (M == -INFINITY) ? 0.0f : O[e] / L;
+    if (lane == 0 && P.lse != nullptr)
+        P.lse[(int64_t)b * P.Hq + hq] = (M == -INFINITY) ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
 }
 
 template <int ES, int D, int G>
 struct AttnSmem {
     Ring<AT_NW, AT_SLOT, AT_STAGES> ring;
     float sc[AT_NW][SC_FLOATS];
-    int64_t pre[PREFIX_CAP + 1];  // attn_prefix: token start of each unit
+    int64_t pre[2][PREFIX_CAP + 1];  // attn_prefix: start of each unit on line A and on line B
+};
+
+// A line of the attention work: the units' spans laid end to end and the
+// share of it that this warp takes.
+struct AttnLine {
+    int64_t T;       // positions on the line
+    int64_t NW;      // warps with a share (min(streaming warps, T)): every share is non-empty
+    int64_t base;    // first record slot of the line
 };
 
 template <int ES, int D, int G>
@@ -731,9 +754,11 @@ struct AttnJob {
     SM &sm;
     uint64_t policy;
     int w, lane;
-    int64_t NWt, T, g;  // streaming warps, tokens on the line, this warp's index
+    AttnLine ln[2];
+    int64_t g;  // this warp's index among the streaming warps
     // generator
-    int64_t t, t_end;
+    int line = 0;
+    int64_t t = 0, t_end = 0;
     int gu = -1, gW = 0, gk = 0, gtot = 0, last_unit = -1;
     int64_t gS = 0, gspan = 0;
     const int32_t *gidx = nullptr;
@@ -744,24 +769,37 @@ struct AttnJob {
     float2 qv[G][Gm::NP];
     AttnState<D, G> st;
     bool had = false;
+    int q_unit = -1;
 
-    __device__ AttnJob(const Params &P_, const Ctl &c_, SM &sm_, int64_t NWt_, int64_t T_, int64_t g_)
-        : P(P_), c(c_), sm(sm_), policy(evict_first_policy()), w(threadIdx.x >> 5), lane(threadIdx.x & 31),
-          NWt(NWt_), T(T_), g(g_)
+    __device__ AttnJob(const Params &P_, const Ctl &c_, SM &sm_, const AttnLine &A, const AttnLine &B, int64_t g_)
+        : P(P_), c(c_), sm(sm_), policy(evict_first_policy()), w(threadIdx.x >> 5), lane(threadIdx.x & 31), g(g_)
     {
-        t = share_begin(g, NWt, T);
-        t_end = share_begin(g + 1, NWt, T);
+        ln[0] = A;
+        ln[1] = B;
+        start_line(0);
         st.reset();
     }
 
-    __device__ __forceinline__ int64_t unit_start(int u) const { return P.attn_prefix ? sm.pre[u] : (int64_t)u * P.attn_span; }
-
-    // Records of unit u occupy slots [first warp + u, last warp + u].
-    __device__ __forceinline__ void record_slots(int u, int *s0, int *s1) const
+    __device__ __forceinline__ void start_line(int l)
     {
-        const int64_t a = unit_start(u), e = unit_start(u + 1);
-        *s0 = (int)(share_owner(a, NWt, T) + u);
-        *s1 = (int)(share_owner(e - 1, NWt, T) + u);
+        line = l;
+        gu = -1;
+        last_unit = -1;
+        if (g < ln[l].NW) {
+            t = share_begin(g, ln[l].NW, ln[l].T);
+            t_end = share_begin(g + 1, ln[l].NW, ln[l].T);
+        } else {
+            t = t_end = 0;
+        }
+    }
+
+    // Start of unit u on the current line.
+    __device__ __forceinline__ int64_t unit_start(int u) const
+    {
+        if (P.attn_prefix)
+            return sm.pre[line][u];
+        const int span = line == 0 ? P.dense.cap + P.cond.cap : min(P.bmax, P.sparse.cap);
+        return (int64_t)u * span;
     }
 
     __device__ __forceinline__ void enter_unit(int u)
@@ -772,14 +810,24 @@ struct AttnJob {
         gW = tier_len(P.dense, u, c);
         gn = tier_len(P.sparse, u, c);
         gk = unit_budget(P, u, gn, c);
-        gtot = gW + gk + tier_len(P.cond, u, c);
-        if (gk > 0)
+        // tokens of the unit on this line: dense ++ condensed (A) or the selection (B)
+        gtot = line == 0 ? gW + tier_len(P.cond, u, c) : gk;
+        if (line == 1 && gk > 0)
             gidx = P.layout == HKV_LAYOUT_FLAT_SUM ? P.idx + __ldcg(P.offsets + u) : P.idx + (int64_t)u * P.bmax;
     }
 
+    // Stages never cross a unit or a tier. Line A positions a < W are dense
+    // rows, the rest condensed rows a - W; line B positions are selection
+    // entries.
     __device__ __forceinline__ bool next(StageDesc &d)
     {
-        while (t < t_end) {
+        for (;;) {
+            if (t >= t_end) {
+                if (line == 1)
+                    return false;
+                start_line(1);
+                continue;
+            }
             if (gu < 0 || t >= gS + gspan) {
                 int u = gu + 1;
                 if (gu < 0) {  // first unit of the share: binary search
@@ -800,27 +848,51 @@ struct AttnJob {
             const int a = (int)(t - gS);
             const int seg_end = (int)(min(t_end - gS, gspan));
             const int vend = min(seg_end, gtot);
+            const int lflag = line ? SD_LINEB : 0;
             if (a >= vend) {
                 // capacity partition: the share holds only unused positions of
-                // this unit; one empty stage still counts the warp's record
+                // this unit; one empty stage still writes the warp's record
                 const bool first = gu != last_unit;
                 t = gS + seg_end;
                 if (!first)
                     continue;
-                d = StageDesc{gu, a, 0, SD_FIRST | SD_LAST};
+                d = StageDesc{gu, a, 0, SD_FIRST | SD_LAST | lflag};
                 last_unit = gu;
                 return true;
             }
-            const int cnt = min(Gm::ATOK, vend - a);
+            int cnt, flags;
+            if (line == 0) {
+                const int tier_end = a < gW ? gW : vend;
+                cnt = min(Gm::ATOK, min(vend, tier_end) - a);
+                const bool contiguous = a < gW ? P.dense.st == D : P.cond.st == D;
+                flags = contiguous ? 0 : SD_GATHER;
+            } else {
+                cnt = min(Gm::ATOK, vend - a);
+                flags = P.logit != nullptr ? SD_LOGIT : SD_GATHER;
+            }
             const bool last = a + cnt >= vend;
-            const bool contiguous = (a + cnt <= gW && P.dense.st == D) || (a >= gW + gk && P.cond.st == D);
-            d = StageDesc{gu, a, cnt,
-                          (gu != last_unit ? SD_FIRST : 0) | (last ? SD_LAST : 0) | (contiguous ? 0 : SD_GATHER)};
+            d = StageDesc{gu, a, cnt, flags | lflag | (gu != last_unit ? SD_FIRST : 0) | (last ? SD_LAST : 0)};
             last_unit = gu;
             t = last ? gS + seg_end : t + cnt;
             return true;
         }
-        return false;
+    }
+
+    // Source rows of line position a of the current unit (lane-level).
+    __device__ __forceinline__ int64_t row_offset(const TierP &T_, int b, int h, int64_t r) const
+    {
+        return ((int64_t)b * T_.sb + (int64_t)h * T_.sh + r * T_.st) * ES;
+    }
+
+    __device__ __forceinline__ int sparse_row(const StageDesc &d) const
+    {
+        const int e = d.start + lane;  // selection entry
+        int jj = (pf_unit == d.unit && pf_start == d.start) ? pf_j : __ldcg(gidx + e);
+        if (jj < 0 || jj >= gn) {
+            raise_flag(c, HKV_DEV_BAD_INDEX);
+            jj = 0;
+        }
+        return jj;
     }
 
     __device__ __forceinline__ void issue(const StageDesc &d, int j)
@@ -836,169 +908,181 @@ struct AttnJob {
             __syncwarp();
             return;
         }
-        if (!(d.flags & SD_GATHER)) {
+        const bool lineb = (d.flags & SD_LINEB) != 0;
+        if (!lineb && !(d.flags & SD_GATHER)) {
+            // contiguous dense or condensed rows: two bulk copies
             if (lane == 0) {
                 mbar_arrive_expect_tx(bar, (uint32_t)(2 * d.count * Gm::ROWB));
                 if (d.count > 0) {
                     const bool dn = d.start < gW;
                     const TierP &Tt = dn ? P.dense : P.cond;
-                    const int64_t r0 = dn ? d.start : d.start - gW - gk;
-                    const int64_t off = ((int64_t)b * Tt.sb + (int64_t)h * Tt.sh + r0 * Tt.st) * ES;
+                    const int64_t off = row_offset(Tt, b, h, dn ? d.start : d.start - gW);
                     bulk_g2s(dst, Tt.k + off, d.count * Gm::ROWB, bar, policy);
                     bulk_g2s(dst + AT_SLOT / 2, Tt.v + off, d.count * Gm::ROWB, bar, policy);
                 }
             }
             __syncwarp();
-            prefetch_index(d);
             return;
         }
-        // gathered rows: lane r copies the K and V rows of token d.start + r,
-        // one bulk copy each, after lane 0 has armed the slot for all of them
+        // one row per lane: K (or the logit record) and V, one bulk copy each,
+        // after lane 0 has armed the slot for all of them
+        constexpr int LB = logit_floats(G) * 4;
+        const bool from_logits = (d.flags & SD_LOGIT) != 0;
         const char *ks = nullptr, *vs = nullptr;
         if (lane < d.count) {
-            const int tt = d.start + lane;
             int64_t off;
-            if (tt < gW) {
-                ks = P.dense.k;
-                vs = P.dense.v;
-                off = (int64_t)b * P.dense.sb + (int64_t)h * P.dense.sh + (int64_t)tt * P.dense.st;
-            } else if (tt < gW + gk) {
-                int jj = (pf_unit == u && pf_start == d.start) ? pf_j : __ldcg(gidx + (tt - gW));
-                if (jj < 0 || jj >= gn) {
-                    raise_flag(c, HKV_DEV_BAD_INDEX);
-                    jj = 0;
-                }
-                ks = P.sparse.k;
-                vs = P.sparse.v;
-                off = (int64_t)b * P.sparse.sb + (int64_t)h * P.sparse.sh + (int64_t)jj * P.sparse.st;
+            if (lineb) {
+                const int jj = sparse_row(d);
+                off = row_offset(P.sparse, b, h, jj);
+                ks = from_logits ? reinterpret_cast<const char *>(P.logit + ((int64_t)u * P.sparse.cap + jj) *
+                                                                               logit_floats(G))
+                                 : P.sparse.k + off;
+                vs = P.sparse.v + off;
             } else {
-                ks = P.cond.k;
-                vs = P.cond.v;
-                off = (int64_t)b * P.cond.sb + (int64_t)h * P.cond.sh + (int64_t)(tt - gW - gk) * P.cond.st;
+                const int a = d.start + lane;
+                const bool dn = a < gW;
+                const TierP &Tt = dn ? P.dense : P.cond;
+                off = row_offset(Tt, b, h, dn ? a : a - gW);
+                ks = Tt.k + off;
+                vs = Tt.v + off;
             }
-            ks += off * ES;
-            vs += off * ES;
         }
+        const uint32_t kb = from_logits ? (uint32_t)LB : (uint32_t)Gm::ROWB;
         if (lane == 0)
-            mbar_arrive_expect_tx(bar, (uint32_t)(2 * d.count * Gm::ROWB));
+            mbar_arrive_expect_tx(bar, (uint32_t)d.count * (kb + Gm::ROWB));
         __syncwarp();
         if (lane < d.count) {
-            bulk_g2s(dst + lane * Gm::ROWB, ks, Gm::ROWB, bar, policy);
+            bulk_g2s(dst + lane * kb, ks, kb, bar, policy);
             bulk_g2s(dst + AT_SLOT / 2 + lane * Gm::ROWB, vs, Gm::ROWB, bar, policy);
         }
         __syncwarp();
-        prefetch_index(d);
+        if (lineb)
+            prefetch_index(d);
     }
 
-    // Start loading the lane's sparse index of the stage after d (same unit),
-    // to be used when that stage is issued.
+    // Start loading the lane's selection entry of the stage after d (same
+    // unit), to be used when that stage is issued.
     __device__ __forceinline__ void prefetch_index(const StageDesc &d)
     {
         const int ns = d.start + d.count;
-        const int tt = ns + lane;
         pf_unit = -1;
-        if (!(d.flags & SD_LAST) && ns < gW + gk && ns + Gm::ATOK > gW) {
+        if (!(d.flags & SD_LAST) && ns < gk) {
             pf_unit = d.unit;
             pf_start = ns;
-            if (tt >= gW && tt < gW + gk)
-                pf_j = __ldcg(gidx + (tt - gW));
+            if (ns + lane < gk)
+                pf_j = __ldcg(gidx + ns + lane);
         }
     }
 
     __device__ __forceinline__ void consume(const StageDesc &d, const unsigned char *stage)
     {
         if (d.flags & SD_FIRST) {
-            load_q<ES, D, G>(P, d.unit, lane, qv);
             st.reset();
             had = false;
         }
         if (d.count > 0) {
-            attn_stage<ES, D, G>(P, stage, d.count, sm.sc[w], qv, st);
+            if (!(d.flags & SD_LOGIT) && d.unit != q_unit) {
+                load_q<ES, D, G>(P, d.unit, lane, qv);
+                q_unit = d.unit;
+            }
+            attn_stage<ES, D, G>(P, stage, d.count, sm.sc[w], qv, st, (d.flags & SD_LOGIT) != 0);
             had = true;
         }
         if (d.flags & SD_LAST)
-            finish(d.unit);
+            finish(d);
     }
 
-    // Write the warp's record for unit u, count it, and merge the unit if the
-    // record was its last.
-    __device__ __forceinline__ void finish(int u)
+    // Write the warp's record for its part of unit d.unit on d's line.
+    __device__ __forceinline__ void finish(const StageDesc &d)
     {
         constexpr int NPV = AttnState<D, G>::NPV;
         constexpr int RS = part_stride(D, G);
-        float lsum[G];
-#pragma unroll
-        for (int gg = 0; gg < G; ++gg)
-            lsum[gg] = warp_sum(st.l[gg]);
-        float *rec = P.part + (g + u) * RS;
+        const int l = (d.flags & SD_LINEB) ? 1 : 0;
+        float *rec = P.part + (ln[l].base + g + d.unit) * RS;
 #pragma unroll
         for (int gg = 0; gg < G; ++gg) {
+            const float lsum = warp_sum(st.l[gg]);
 #pragma unroll
             for (int e = 0; e < NPV; ++e)
-                *reinterpret_cast<float2 *>(rec + gg * (D + 2) + lane * 2 * NPV + 2 * e) = st.o[gg][e];
+                *reinterpret_cast<float2 *>(rec + gg * D + lane * 2 * NPV + 2 * e) = st.o[gg][e];
             if (lane == 0) {
-                rec[gg * (D + 2) + D] = had ? st.m[gg] : -INFINITY;
-                rec[gg * (D + 2) + D + 1] = lsum[gg];
+                rec[G * D + gg] = had ? st.m[gg] : -INFINITY;
+                rec[G * D + G + gg] = lsum;
             }
-        }
-        int s0, s1;
-        record_slots(u, &s0, &s1);
-        __syncwarp();
-        int last = 0;
-        if (lane == 0) {
-            __threadfence();
-            const uint32_t prev = atomicAdd(P.attn_cnt + u, 1u);
-            last = prev == (uint32_t)(s1 - s0);
-        }
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (last) {
-            __threadfence();
-            merge_records<D, G>(P, u, s0, s1);
-            if (lane == 0)
-                P.attn_cnt[u] = 0;
         }
         __syncwarp();
     }
 };
 
-// Attention prologue of a CTA: token starts of all units (attn_prefix), and
-// out = 0 / lse = -inf for this CTA's share of units without tokens. Returns
-// the tokens on the line.
+// Attention prologue of a CTA: the two lines and, with attn_prefix, the start
+// of every unit on each; CTA 0 also writes every unit's record slots
+// (rec_range[u] = first and last slot on line A, then on line B; first > last
+// when empty) for k_merge.
 template <int ES, int D, int G>
-__device__ int64_t attn_prologue(const Params &P, AttnSmem<ES, D, G> &sm, const Ctl &c, unsigned long long *red)
+__device__ void attn_prologue(const Params &P, AttnSmem<ES, D, G> &sm, const Ctl &c, unsigned long long *red,
+                              AttnLine *A, AttnLine *B)
 {
-    const int w = threadIdx.x >> 5;
-    int64_t T;
+    constexpr int NTA = AT_NW * 32;
+    const int64_t NWt = (int64_t)gridDim.x * AT_NW;
+    int64_t TA, TB;
     if (P.attn_prefix) {
-        unsigned long long carry = 0;
-        for (int base = 0; base < P.units; base += AT_NW * 32) {
+        unsigned long long ca = 0, cb = 0;
+        for (int base = 0; base < P.units; base += NTA) {
             const int u = base + threadIdx.x;
-            int tot = 0;
+            unsigned long long ta = 0, tb = 0;
             if (u < P.units) {
                 const int n = tier_len(P.sparse, u, c);
-                tot = tier_len(P.dense, u, c) + unit_budget(P, u, n, c) + tier_len(P.cond, u, c);
+                ta = (unsigned long long)(tier_len(P.dense, u, c) + tier_len(P.cond, u, c));
+                tb = (unsigned long long)unit_budget(P, u, n, c);
             }
+            // both prefixes in one scan (each sum stays below 2^32)
             unsigned long long sum;
-            const unsigned long long ex = block_exclusive_scan<AT_NW * 32>((unsigned long long)tot, red, &sum);
-            if (u < P.units)
-                sm.pre[u] = (int64_t)(carry + ex);
-            carry += sum;
+            const unsigned long long ex = block_exclusive_scan<NTA>((tb << 32) | ta, red, &sum);
+            if (u < P.units) {
+                sm.pre[0][u] = (int64_t)(ca + (ex & 0xffffffffull));
+                sm.pre[1][u] = (int64_t)(cb + (ex >> 32));
+            }
+            ca += sum & 0xffffffffull;
+            cb += sum >> 32;
         }
-        if (threadIdx.x == 0)
-            sm.pre[P.units] = (int64_t)carry;
+        if (threadIdx.x == 0) {
+            sm.pre[0][P.units] = (int64_t)ca;
+            sm.pre[1][P.units] = (int64_t)cb;
+        }
         __syncthreads();
-        T = (int64_t)carry;
-        // units without tokens get no record: their output is written here
-        for (int u = blockIdx.x * AT_NW + w; u < P.units; u += gridDim.x * AT_NW)
-            if (sm.pre[u + 1] == sm.pre[u])
-                write_empty_unit<D, G>(P, u);
+        TA = (int64_t)ca;
+        TB = (int64_t)cb;
     } else {
-        T = (int64_t)P.units * P.attn_span;
-        if (T == 0)
-            for (int u = blockIdx.x * AT_NW + w; u < P.units; u += gridDim.x * AT_NW)
-                write_empty_unit<D, G>(P, u);
+        TA = (int64_t)P.units * (P.dense.cap + P.cond.cap);
+        TB = (int64_t)P.units * min(P.bmax, P.sparse.cap);
     }
-    return T;
+    *A = AttnLine{TA, min(NWt, TA), 0};
+    *B = AttnLine{TB, min(NWt, TB), NWt + P.units};
+    if (blockIdx.x == 0) {
+        for (int u = threadIdx.x; u < P.units; u += NTA) {
+            int r[4];
+            for (int l = 0; l < 2; ++l) {
+                const AttnLine &L = l ? *B : *A;
+                int64_t s0, s1;
+                if (P.attn_prefix) {
+                    s0 = sm.pre[l][u];
+                    s1 = sm.pre[l][u + 1];
+                } else {
+                    const int64_t span = l ? min(P.bmax, P.sparse.cap) : P.dense.cap + P.cond.cap;
+                    s0 = (int64_t)u * span;
+                    s1 = s0 + span;
+                }
+                if (s1 > s0) {
+                    r[2 * l] = (int)(L.base + share_owner(s0, L.NW, L.T) + u);
+                    r[2 * l + 1] = (int)(L.base + share_owner(s1 - 1, L.NW, L.T) + u);
+                } else {
+                    r[2 * l] = 1;
+                    r[2 * l + 1] = 0;
+                }
+            }
+            *reinterpret_cast<int4 *>(P.rec_range + 4 * u) = make_int4(r[0], r[1], r[2], r[3]);
+        }
+    }
 }
 
 // =============================================================================
@@ -1006,6 +1090,7 @@ __device__ int64_t attn_prologue(const Params &P, AttnSmem<ES, D, G> &sm, const 
 // =============================================================================
 
 constexpr int NT = SEL_THREADS;
+constexpr int SWEEP_Q = 8;  // quads per thread per batch of a score sweep
 
 // Scores of one unit, from shared memory (ZS: staged there by stage_scores)
 // or global memory, in batches of Q quads per thread with all loads in
@@ -1015,7 +1100,33 @@ constexpr int NT = SEL_THREADS;
 template <bool ZS, typename F>
 __device__ __forceinline__ void sweep_scores(const float *zu, int n, F &&f)
 {
-    constexpr int Q = 8;
+    if constexpr (ZS) {
+        // staged scores: shared-memory latency is short, so a rolled loop (a
+        // single copy of f's code) beats unrolling; these kernels run their
+        // code once per unit and are bound by instruction fetch otherwise
+        const int nq = (n + 3) >> 2;
+        for (int base = 0; base < nq; base += NT * SWEEP_Q) {
+#pragma unroll 1
+            for (int i = 0; i < SWEEP_Q; ++i) {
+                const int j = 4 * (base + i * NT + (int)threadIdx.x);
+                float4 v;
+                if (j + 4 <= n) {
+                    v = lds4(zu + j);
+                } else {
+                    v.x = j < n ? lds1(zu + j) : 0.f;
+                    v.y = j + 1 < n ? lds1(zu + j + 1) : 0.f;
+                    v.z = j + 2 < n ? lds1(zu + j + 2) : 0.f;
+                    v.w = j + 3 < n ? lds1(zu + j + 3) : 0.f;
+                }
+                f(v.x, j, j < n);
+                f(v.y, j + 1, j + 1 < n);
+                f(v.z, j + 2, j + 2 < n);
+                f(v.w, j + 3, j + 3 < n);
+            }
+        }
+        return;
+    }
+    constexpr int Q = SWEEP_Q;
     const bool vec = ZS || (((uintptr_t)zu) & 15) == 0;
     const int nq = (n + 3) >> 2;
     for (int base = 0; base < nq; base += NT * Q) {
@@ -1044,6 +1155,7 @@ __device__ __forceinline__ void sweep_scores(const float *zu, int n, F &&f)
 }
 
 // Select: linear score bins, then an exact sort of the candidates of one bin.
+
 constexpr int SBINS = 2048;
 constexpr int CAND_CAP = 4096;
 
@@ -1500,62 +1612,61 @@ __device__ Selection select_unit(const float *zu, int n, float m, float zlo, flo
 // S4 Index Regularization of one unit, whole CTA ([TS 2.C] Flatten Index):
 // order-preserving compaction of {key < cut key} + the first n_tie tokens with
 // key == cut key into row[0, k); PAD_MAX rows are padded with -1 to `pad`.
-// Each thread takes E consecutive tokens of a chunk (loaded together).
+// Warp w owns the w-th of NT/32 contiguous segments of the unit's tokens and
+// walks it 32 tokens at a time (lane = token): pass 1 counts the selected and
+// tied tokens with ballots, a block scan turns the counts into each warp's
+// starting position and tie rank, and pass 2 writes the indices. Rolled loops
+// keep the code small: the kernel runs it once per unit.
 // =============================================================================
 template <bool ZS>
-__device__ void compact_unit(const float *zu, int n, uint32_t cut_key, int n_tie, int k, int32_t *row, int pad,
-                             unsigned long long *red)
+__device__ __forceinline__ float zload(const float *zu, int j)
 {
-    constexpr int E = 16;
-    unsigned long long lt_carry = 0, eq_carry = 0;
-    const bool vec = (((uintptr_t)zu) & 15) == 0;
+    return ZS ? lds1(zu + j) : __ldcg(zu + j);
+}
+
+template <bool ZS>
+__device__ void compact_unit(const float *zu, int n, uint32_t cut_key, int n_tie, int k, int32_t *row, int pad,
+                             unsigned long long *red, int tb = -1)
+{
+    constexpr int NW = NT / 32;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     if (k > 0) {
-        for (int base = 0; base < n; base += NT * E) {
-            const int j0 = base + threadIdx.x * E;
-            float zz[E];
-            if (vec && j0 + E <= n) {
-#pragma unroll
-                for (int e = 0; e < E; e += 4) {
-                    const float4 v = ZS ? lds4(zu + j0 + e) : __ldcg(reinterpret_cast<const float4 *>(zu + j0 + e));
-                    zz[e] = v.x;
-                    zz[e + 1] = v.y;
-                    zz[e + 2] = v.z;
-                    zz[e + 3] = v.w;
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < E; ++e)
-                    zz[e] = (j0 + e < n) ? (ZS ? lds1(zu + j0 + e) : __ldcg(zu + j0 + e)) : 0.f;
-            }
-            uint32_t lt_bits = 0, eq_bits = 0;
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-                const uint32_t key = score_key(zz[e]);
-                const bool valid = j0 + e < n;
-                lt_bits |= (valid && key < cut_key) ? (1u << e) : 0u;
-                eq_bits |= (valid && key == cut_key) ? (1u << e) : 0u;
-            }
-            const uint32_t nlt = __popc(lt_bits), neq = __popc(eq_bits);
-            unsigned long long tot;
-            const unsigned long long ex =
-                block_exclusive_scan<NT>(((unsigned long long)neq << 32) | nlt, red, &tot);
-            const unsigned long long eq_before = eq_carry + (ex >> 32);
-            const unsigned long long lt_before = lt_carry + (ex & 0xffffffffull);
-            unsigned long long pos = lt_before + min(eq_before, (unsigned long long)n_tie);
-            unsigned long long eq_rank = eq_before;
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-                bool take = (lt_bits >> e) & 1u;
-                if ((eq_bits >> e) & 1u) {
-                    take = eq_rank < (unsigned long long)n_tie;
-                    ++eq_rank;
-                }
-                if (take && pos < (unsigned long long)k)  // a caller's inconsistent cut stays in the row
-                    row[pos++] = j0 + e;
-            }
-            lt_carry += tot & 0xffffffffull;
-            eq_carry += tot >> 32;
+        const int seg = ((n + NW - 1) / NW + 31) / 32 * 32;  // tokens per warp, a multiple of 32
+        const int j0 = w * seg, j1 = min(n, j0 + seg);
+        // pass 1: the warp's selected (key < cut) and tied (key == cut) tokens
+        uint32_t nlt = 0, neq = 0;
+#pragma unroll 1
+        for (int j = j0 + lane; j - lane < j1; j += 32) {
+            const bool valid = j < j1;
+            const uint32_t key = valid ? score_key(zload<ZS>(zu, j)) : 0xffffffffu;
+            nlt += __popc(__ballot_sync(0xffffffffu, valid && key < cut_key));
+            neq += __popc(__ballot_sync(0xffffffffu, valid && key == cut_key));
         }
+        unsigned long long tot;
+        const unsigned long long mine = lane == 0 ? (((unsigned long long)neq << 32) | nlt) : 0ull;
+        const unsigned long long ex = block_exclusive_scan<NT>(mine, red, &tot);
+        // every lane needs its warp's prefix: lane 0 holds it
+        uint32_t lt_before = (uint32_t)__shfl_sync(0xffffffffu, (unsigned int)(ex & 0xffffffffull), 0);
+        uint32_t eq_before = (uint32_t)__shfl_sync(0xffffffffu, (unsigned int)(ex >> 32), 0);
+        HKV_TRACE_AT(tb < 0 ? -1 : tb + 12);
+        // pass 2: positions of the taken tokens, in index order
+        const unsigned lower = (1u << lane) - 1u;
+#pragma unroll 1
+        for (int j = j0 + lane; j - lane < j1; j += 32) {
+            const bool valid = j < j1;
+            const uint32_t key = valid ? score_key(zload<ZS>(zu, j)) : 0xffffffffu;
+            const unsigned mlt = __ballot_sync(0xffffffffu, valid && key < cut_key);
+            const unsigned meq = __ballot_sync(0xffffffffu, valid && key == cut_key);
+            const uint32_t eq_rank = eq_before + __popc(meq & lower);
+            const uint32_t eq_taken_before = min(eq_rank, (uint32_t)n_tie);
+            const bool take = ((mlt >> lane) & 1u) || (((meq >> lane) & 1u) && eq_rank < (uint32_t)n_tie);
+            const uint32_t pos = lt_before + __popc(mlt & lower) + eq_taken_before;
+            if (take && pos < (uint32_t)k)  // a caller's inconsistent cut stays in the row
+                row[pos] = j;
+            lt_before += __popc(mlt);
+            eq_before += __popc(meq);
+        }
+        HKV_TRACE_AT(tb < 0 ? -1 : tb + 13);
     }
     for (int i = k + threadIdx.x; i < pad; i += NT)
         row[i] = -1;

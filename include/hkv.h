@@ -183,8 +183,9 @@ hkv_status hkv_compact(const hkv_problem *prob, const float *z, int64_t z_stride
 
 /* S5 Cascade decode attention ([TS 2.A] three tiers; [Abstract]): for each
  * query head, softmax attention (scale * q.k) over dense[0, len) ++
- * sparse[idx_0 .. idx_{k-1}] ++ condensed[0, len), split across CTAs and merged
- * by online softmax. out: device [B, Hq, D] fp32; lse: device [B, Hq] fp32 or
+ * sparse[idx_0 .. idx_{k-1}] ++ condensed[0, len), split across all warps of a
+ * persistent grid (dense and condensed tokens on one work line, the selected
+ * tokens on another) and merged by online softmax in a second kernel. out: device [B, Hq, D] fp32; lse: device [B, Hq] fp32 or
  * NULL. idx/offsets in prob->layout with k = sel_len[u]. An empty token list
  * gives out = 0, lse = -inf. Any tier may be NULL (empty). ws: workspace of
  * hkv_workspace_size bytes, zeroed once by hkv_workspace_init. */
@@ -226,20 +227,20 @@ hkv_status hkv_step(const hkv_problem *prob, const void *q, const hkv_tier *dens
  * the same arguments minus ws/ws_bytes, and allocates nothing (no cudaMalloc,
  * no cudaFree, no allocating library routine): its scratch is a fixed device
  * array of HKV_NOALLOC_SCRATCH_BYTES bytes inside the library.
- * - Size limit: the scratch holds a few counter words per unit and one
- *   attention record of 4*G*(D+2) bytes per streaming warp and per unit
- *   (2.6 MB for bf16, D = 128, G = 4, 64 units on a 148-SM B200). When the
- *   array cannot hold records for a full grid, fewer CTAs run; a problem with
- *   too many units for even one CTA (about 2000 units at G = 4, D = 128) is
- *   refused with HKV_ERR_WORKSPACE before anything is launched: use
- *   hkv_cascade_decode with a workspace for those.
+ * - Size limit: the scratch holds a status word, a few words per unit and
+ *   two attention records of 4*G*(D+2) bytes per streaming warp and per unit
+ *   (5.2 MB for a full 148-SM grid at bf16, D = 128, G = 4, 64 units). When the
+ *   array cannot hold the records of a full grid, fewer CTAs run (117 CTAs in
+ *   that example); a problem with too many units for even one CTA (about 1000
+ *   units at G = 4, D = 128) is refused with HKV_ERR_WORKSPACE before anything
+ *   is launched: use hkv_cascade_decode with a workspace for those.
  * - Set-up: the first call on each device looks up the array's device address
  *   and sets the kernel's shared-memory attribute. Make that first call outside
  *   any stream capture.
  * - Sharing: every call on a device uses the same array, which keeps the last
- *   call's contents. Each call zeroes the words that must start at zero (status
- *   and counters) on `stream` before its kernel runs; the tile records are
- *   always written before they are read. Calls that overlap on the GPU (other
+ *   call's contents. Each call zeroes the one word that must start at zero
+ *   (the status word) on `stream` before its kernels run; everything else is
+ *   written before it is read. Calls that overlap on the GPU (other
  *   streams, other host threads) race on the array and give undefined results:
  *   serialise them.
  * - status: device pointer to one uint32 or NULL; when given it receives this

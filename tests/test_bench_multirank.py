@@ -59,6 +59,8 @@ def test_step_bytes_counts_scored_and_attended_rows():
     wl = WORKLOADS[2]
     U = wl.units
     b = bench.step_bytes(wl, np.full(U, 16064), np.full(U, 256), np.full(U, 64), np.full(U, 2048))
-    scored = U * 16064 * 128 * 2
-    attended = U * (256 + 64 + 2048) * 2 * 128 * 2
+    # keys read once with a 4-byte score and a 16-byte logit record written per key
+    scored = U * 16064 * (128 * 2 + 4 + 16)
+    # dense and condensed K and V; selected tokens: V row and logit record
+    attended = U * (256 + 64) * 2 * 128 * 2 + U * 2048 * (128 * 2 + 16)
     assert b - scored - attended == wl.B * wl.Hq * 128 * 2 + wl.B * wl.Hq * 129 * 4 + U * 2048 * 4 + U * 4

@@ -62,7 +62,10 @@ def test_step_small(name):
 
 @pytest.mark.parametrize("name", sorted(CASES))
 def test_step_equals_stage_chain(name):
-    """The fused kernel and the five separate calls give bit-identical results."""
+    """hkv_step and the five separate calls give bit-identical scores,
+    selections, index rows, m and logZ. The attention outputs agree to a few
+    ulp: hkv_step reuses the scorer's per-head logits for the selected tokens,
+    while hkv_cascade_decode recomputes them from K."""
     wl = CASES[name]
     x = H.inputs(wl)
     prob, out, ws = H.run_step(wl, x)
@@ -90,8 +93,8 @@ def test_step_equals_stage_chain(name):
     assert torch.equal(sel, out.sel_len)
     assert torch.equal(cut, out.cut)
     assert torch.equal(idx, out.idx)
-    assert torch.equal(o, out.out)
-    assert torch.equal(lse, out.lse)
+    torch.testing.assert_close(o, out.out, atol=1e-5, rtol=1e-5)
+    torch.testing.assert_close(lse, out.lse, atol=1e-5, rtol=1e-5)
     assert torch.equal(m, out.m)
     assert torch.equal(lz, out.logZ)
 
