@@ -159,20 +159,34 @@ __device__ __forceinline__ void unit_work(const Params &P, USmem &sm, const Ctl 
             unit_range<ZS>(zu, n, &m, &zlo, sm);
         }
         HKV_TRACE_AT(TR_SEL + 16 * u + 4);
-        const Selection s = select_unit<ZS>(zu, n, m, zlo, unit_beta(P, u, c), unit_p(P, u, c), P.bmin, P.bmax,
-                                            sm, TR_SEL + 16 * u);
+        const float beta = unit_beta(P, u, c), pu = unit_p(P, u, c);
+        const auto publish = [&](const Selection &s) {
+            if (threadIdx.x == 0) {
+                P.sel_len[u] = s.k;
+                if (P.cut)
+                    P.cut[u] = s.cut;
+                if (P.m_out)
+                    P.m_out[u] = m;
+                if (P.logZ_out)
+                    P.logZ_out[u] = n > 0 ? (float)log(s.Z) : -INFINITY;
+            }
+        };
+        if constexpr (ZS) {
+            // selection and PAD_MAX compaction in one go (hkv_step)
+            Selection s;
+            if (P.do_compact &&
+                select_compact_fast(zu, n, m, zlo, beta, pu, P.bmin, P.bmax, sm, s, P.idx + (int64_t)u * P.bmax,
+                                    P.bmax, TR_SEL + 16 * u)) {
+                publish(s);
+                HKV_TRACE_AT(TR_SEL + 16 * u + 5);
+                return;
+            }
+        }
+        const Selection s = select_unit<ZS>(zu, n, m, zlo, beta, pu, P.bmin, P.bmax, sm, TR_SEL + 16 * u);
         k = s.k;
         key = s.key;
         n_tie = s.cut.n_tie;
-        if (threadIdx.x == 0) {
-            P.sel_len[u] = k;
-            if (P.cut)
-                P.cut[u] = s.cut;
-            if (P.m_out)
-                P.m_out[u] = m;
-            if (P.logZ_out)
-                P.logZ_out[u] = n > 0 ? (float)log(s.Z) : -INFINITY;
-        }
+        publish(s);
         HKV_TRACE_AT(TR_SEL + 16 * u + 11);
     } else {
         k = __ldcg(P.sel_len + u);

@@ -1157,7 +1157,8 @@ __device__ __forceinline__ void sweep_scores(const float *zu, int n, F &&f)
 // Select: linear score bins, then an exact sort of the candidates of one bin.
 
 constexpr int SBINS = 2048;
-constexpr int CAND_CAP = 4096;
+constexpr int CAND_CAP = 6144;
+constexpr int BIN_CAP = 2048;  // tokens of one bin sorted by the staged fast path
 
 constexpr int ZSTAGE = 24576;  // scores of a unit staged in shared memory (units up to this length)
 
@@ -1166,6 +1167,8 @@ struct __align__(16) USmem {  // shared memory of the per-unit kernels
     uint32_t cnt[SBINS];
     unsigned long long mass[SBINS];  // bin mass (fixed point)
     unsigned long long cand[CAND_CAP];  // (order key << 32) | token index
+    unsigned long long binbuf[BIN_CAP];  // the tokens of one bin, sorted (staged fast path)
+    uint32_t bits[ZSTAGE / 32];          // selected tokens (staged fast path)
     unsigned long long red[NT / 32];
     double redd[NT / 32];
     float redf[NT / 32];
@@ -1353,24 +1356,26 @@ __device__ void gather_bin(const float *zu, int n, const BinFn &bins, int bin, U
 // Sort the cnt_in gathered tokens of a bin by (key, index) and locate the cut:
 // by_mass, the first token at which the cumulative mass (from mass_before)
 // reaches `target`; else the token of rank `target` (1-based, within the bin).
-// Returns its position in the sorted bin (left in sm.cand).
+// Returns its position in the sorted bin (left in buf, default sm.cand).
 __device__ int sort_and_locate(int cnt_in, bool by_mass, unsigned long long target, unsigned long long mass_before,
-                               float m, float bl2, USmem &sm)
+                               float m, float bl2, USmem &sm, unsigned long long *buf = nullptr)
 {
+    if (buf == nullptr)
+        buf = sm.cand;
     int P = 1;
     while (P < cnt_in)
         P <<= 1;
     for (int i = cnt_in + threadIdx.x; i < P; i += NT)
-        sm.cand[i] = ~0ull;
+        buf[i] = ~0ull;
     __syncthreads();
-    sort_candidates(sm.cand, P);
+    sort_candidates(buf, P);
     if (!by_mass)
         return (int)target - 1;
     const int per = (cnt_in + NT - 1) / NT;
     const int lo = threadIdx.x * per, hi = min(cnt_in, lo + per);
     unsigned long long mine = 0;
     for (int i = lo; i < hi; ++i)
-        mine += wfix(key_score((uint32_t)(sm.cand[i] >> 32)), m, bl2);
+        mine += wfix(key_score((uint32_t)(buf[i] >> 32)), m, bl2);
     unsigned long long tot;
     const unsigned long long ex = block_exclusive_scan<NT>(mine, sm.red, &tot) + mass_before;
     if (threadIdx.x == 0)
@@ -1379,7 +1384,7 @@ __device__ int sort_and_locate(int cnt_in, bool by_mass, unsigned long long targ
     if (ex < target && target <= ex + mine) {
         unsigned long long acc = ex;
         for (int i = lo; i < hi; ++i) {
-            acc += wfix(key_score((uint32_t)(sm.cand[i] >> 32)), m, bl2);
+            acc += wfix(key_score((uint32_t)(buf[i] >> 32)), m, bl2);
             if (acc >= target) {
                 sm.bc[2] = i;
                 break;
@@ -1606,6 +1611,204 @@ __device__ Selection select_unit(const float *zu, int n, float m, float zlo, flo
     __syncthreads();
     HKV_TRACE_AT(tb < 0 ? -1 : tb + 3);
     return r;
+}
+
+// =============================================================================
+// S2-S4 fused for a unit whose scores are staged in shared memory (hkv_step):
+// the same budget and cut as select_unit followed by compact_unit, with fewer
+// passes over the unit. After the count histogram (sweep 1, which also sums
+// Z exactly as select_unit does), one sweep gathers every token of the bins up
+// to the one holding rank min(n, bmax) -- a superset of any selection -- and
+// the rest works on that short list: bin masses, the crossing bin sorted on
+// its own, and a bitmap of the selected tokens expanded in index order.
+// Returns false, having written nothing, when the list or a bin outgrows its
+// buffer; the caller then takes select_unit and compact_unit.
+// =============================================================================
+
+// Copy the listed candidates of bin b into sm.binbuf (positions from a block
+// scan of per-thread counts, no shared counter); returns their number, or -1
+// when the bin holds more than BIN_CAP tokens.
+__device__ int load_sorted_bin(int b, int ncand, const BinFn &bins, USmem &sm)
+{
+    const int cb = (int)sm.cnt[b];
+    if (cb > BIN_CAP)
+        return -1;
+    const auto hit = [&](int i) { return bins(key_score((uint32_t)(sm.cand[i] >> 32))) == b; };
+    unsigned long long mine = 0;
+    for (int i = threadIdx.x; i < ncand; i += NT)
+        mine += hit(i) ? 1u : 0u;
+    unsigned long long tot;
+    int at = (int)block_exclusive_scan<NT>(mine, sm.red, &tot);
+    for (int i = threadIdx.x; i < ncand; i += NT)
+        if (hit(i))
+            sm.binbuf[at++] = sm.cand[i];
+    __syncthreads();
+    return cb;
+}
+
+// Append the (key, index) of every staged token with bin <= b_hi to sm.cand,
+// at positions from a block scan of per-thread counts (no shared counter):
+// one sweep counts, the second writes. Returns the number listed.
+__device__ int list_candidates(const float *zs, int n, const BinFn &bins, int b_hi, USmem &sm)
+{
+    unsigned long long mine = 0;
+    sweep_scores<true>(zs, n, [&](float z, int, bool valid) { mine += (valid && bins(z) <= b_hi) ? 1u : 0u; });
+    unsigned long long tot;
+    int at = (int)block_exclusive_scan<NT>(mine, sm.red, &tot);
+    sweep_scores<true>(zs, n, [&](float z, int j, bool valid) {
+        if (valid && bins(z) <= b_hi)
+            sm.cand[at++] = ((unsigned long long)score_key(z) << 32) | (uint32_t)j;
+    });
+    __syncthreads();
+    return (int)tot;
+}
+
+__device__ bool select_compact_fast(const float *zs, int n, float m, float zlo, float beta, float p, int bmin,
+                                    int bmax, USmem &sm, Selection &r, int32_t *row, int pad, int tb)
+{
+    const float bl2 = beta * LOG2E;
+    const BinFn bins = make_bins(m, zlo);
+    r = Selection{};
+    for (int i = threadIdx.x; i < SBINS; i += NT) {
+        sm.cnt[i] = 0;
+        sm.mass[i] = 0;
+    }
+    __syncthreads();
+    const auto mass = [&](int b) { return sm.mass[b]; };
+    // sweep 1: bin counts and the normaliser
+    double zsum = 0.0;
+    sweep_scores<true>(zs, n, [&](float z, int, bool valid) {
+        if (!valid)
+            return;
+        zsum += (double)wcal(z, m, bl2);
+        sred_add(&sm.cnt[bins(z)], 1u);
+    });
+    r.Z = block_sum_f64<NT>(zsum, sm.redd);
+    HKV_TRACE_AT(tb < 0 ? -1 : tb + 1);
+    int k = 0, kstar = 0;
+    uint32_t cut_key = 0u;
+    int n_above = 0;
+    int tie0 = 0;  // first tie in sm.binbuf
+    if (n > 0) {
+        const int r_hi = min(n, max(bmax, 1));
+        unsigned long long hb_c, hb_m;
+        const int b_hi = find_crossing(sm.cnt, mass, SBINS, false, (unsigned long long)r_hi, &hb_c, &hb_m, sm);
+        const int ncand = (int)hb_c + (int)sm.cnt[b_hi];
+        if (ncand > CAND_CAP)
+            return false;
+        // sweeps 2 and 3: the tokens of bins 0 .. b_hi
+        list_candidates(zs, n, bins, b_hi, sm);
+        HKV_TRACE_AT(tb < 0 ? -1 : tb + 2);
+        // Top-p budget from the listed tokens' bin masses
+        kstar = -1;
+        bool mass_cut = false;
+        int pos = -1;
+        unsigned long long before_c = 0;
+        if (p >= 1.0f) {
+            kstar = n;
+        } else if (p <= 0.0f) {
+            kstar = 0;
+        } else {
+            for (int i = threadIdx.x; i < ncand; i += NT) {
+                const float z = key_score((uint32_t)(sm.cand[i] >> 32));
+                sred_add(&sm.mass[bins(z)], wfix(z, m, bl2));
+            }
+            __syncthreads();
+            const double t = ceil((double)p * r.Z * 1099511627776.0);
+            const unsigned long long T = t < 1.0 ? 1ull : (unsigned long long)t;
+            unsigned long long part = 0;
+            for (int i = threadIdx.x; i <= b_hi; i += NT)
+                part += sm.mass[i];
+            const unsigned long long through = block_sum_u64<NT>(part, sm.red);
+            if (through >= T) {
+                unsigned long long mb_c, mb_m;
+                const int b_m = find_crossing(sm.cnt, mass, SBINS, true, T, &mb_c, &mb_m, sm);
+                const int cb = load_sorted_bin(b_m, ncand, bins, sm);
+                if (cb < 0)
+                    return false;
+                pos = sort_and_locate(cb, true, T, mb_m, m, bl2, sm, sm.binbuf);
+                kstar = (int)mb_c + pos + 1;
+                before_c = mb_c;
+                mass_cut = true;
+            }
+        }
+        k = kstar < 0 ? bmax : min(kstar, bmax);
+        k = min(max(k, bmin), n);
+        HKV_TRACE_AT(tb < 0 ? -1 : tb + 8);
+        if (k > 0) {
+            if (!(mass_cut && k == kstar)) {
+                // the clamp decides: the token of rank k
+                unsigned long long kb_c, kb_m;
+                const int b_k = find_crossing(sm.cnt, mass, SBINS, false, (unsigned long long)k, &kb_c, &kb_m, sm);
+                const int cb = load_sorted_bin(b_k, ncand, bins, sm);
+                if (cb < 0)
+                    return false;
+                pos = sort_and_locate(cb, false, (unsigned long long)k - kb_c, 0, m, bl2, sm, sm.binbuf);
+                before_c = kb_c;
+            }
+            cut_key = (uint32_t)(sm.binbuf[pos] >> 32);
+            if (threadIdx.x == 0) {
+                int first = pos;
+                while (first > 0 && (uint32_t)(sm.binbuf[first - 1] >> 32) == cut_key)
+                    --first;
+                sm.bc[4] = first;
+            }
+            __syncthreads();
+            tie0 = sm.bc[4];
+            n_above = (int)before_c + tie0;
+            HKV_TRACE_AT(tb < 0 ? -1 : tb + 3);
+            // bitmap of the selection: listed tokens above the cut, and the
+            // first n_tie ties (consecutive in binbuf, by index)
+            const int nwords = (n + 31) >> 5;
+            for (int i = threadIdx.x; i < nwords; i += NT)
+                sm.bits[i] = 0u;
+            __syncthreads();
+            for (int i = threadIdx.x; i < ncand; i += NT) {
+                const unsigned long long e = sm.cand[i];
+                if ((uint32_t)(e >> 32) < cut_key) {
+                    const uint32_t j = (uint32_t)e;
+                    atomicOr(&sm.bits[j >> 5], 1u << (j & 31));
+                }
+            }
+            const int n_tie = k - n_above;
+            for (int i = threadIdx.x; i < n_tie; i += NT) {
+                const uint32_t j = (uint32_t)sm.binbuf[tie0 + i];
+                atomicOr(&sm.bits[j >> 5], 1u << (j & 31));
+            }
+            __syncthreads();
+            // expansion in index order: thread t takes a contiguous run of words
+            const int wpt = (nwords + NT - 1) / NT;
+            const int w0 = threadIdx.x * wpt, w1 = min(nwords, w0 + wpt);
+            unsigned long long cntw = 0;
+            for (int i = w0; i < w1; ++i)
+                cntw += __popc(sm.bits[i]);
+            unsigned long long tot;
+            int at = (int)block_exclusive_scan<NT>(cntw, sm.red, &tot);
+            for (int i = w0; i < w1; ++i) {
+                uint32_t b = sm.bits[i];
+                while (b) {
+                    const int bit = __ffs(b) - 1;
+                    if (at < k)
+                        row[at] = i * 32 + bit;
+                    ++at;
+                    b &= b - 1u;
+                }
+            }
+        }
+    }
+    for (int i = k + threadIdx.x; i < pad; i += NT)
+        row[i] = -1;
+    r.k = k;
+    r.kstar = kstar;
+    r.key = cut_key;
+    r.cut.z_cut = key_score(cut_key);
+    r.cut.n_above = n_above;
+    r.cut.n_tie = k - n_above;
+    r.cut.kstar = kstar;
+    if (k == 0)
+        r.cut = hkv_cut{0.0f, 0, 0, kstar};
+    __syncthreads();
+    return true;
 }
 
 // =============================================================================
