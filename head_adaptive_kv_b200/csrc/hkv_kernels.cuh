@@ -924,19 +924,49 @@ struct AttnJob {
             __syncwarp();
             return;
         }
-        // one row per lane: K (or the logit record) and V, one bulk copy each,
-        // after lane 0 has armed the slot for all of them
         constexpr int LB = logit_floats(G) * 4;
         const bool from_logits = (d.flags & SD_LOGIT) != 0;
+        if (from_logits) {
+            // selected tokens with the scorer's logits: V rows and logit records
+            // in 16-byte cp.async chunks spread over the warp (random rows
+            // stream faster this way than as one bulk copy per row)
+            const char *vs = nullptr, *ls = nullptr;
+            if (lane < d.count) {
+                const int jj = sparse_row(d);
+                vs = P.sparse.v + row_offset(P.sparse, b, h, jj);
+                ls = reinterpret_cast<const char *>(P.logit + ((int64_t)u * P.sparse.cap + jj) * logit_floats(G));
+            }
+            constexpr int CH = Gm::ROWB / 16;  // chunks of a V row
+            static_assert(CH <= 32 && 32 % CH == 0, "row chunks");
+            constexpr int RPI = 32 / CH;       // rows per warp instruction
+            const int cc = lane % CH, rr = lane / CH;
+            for (int r0 = 0; r0 < d.count; r0 += RPI) {
+                const int r = r0 + rr;
+                const char *v_ = reinterpret_cast<const char *>(
+                    (uintptr_t)__shfl_sync(0xffffffffu, (unsigned long long)(uintptr_t)vs, r & 31));
+                if (r < d.count)
+                    cp_async16(dst + AT_SLOT / 2 + r * Gm::ROWB + cc * 16, v_ + cc * 16);
+            }
+            if (lane < d.count)
+#pragma unroll
+                for (int i = 0; i < LB / 16; ++i)
+                    cp_async16(dst + lane * LB + i * 16, ls + i * 16);
+            cp_async_arrive(bar);
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar);
+            prefetch_index(d);
+            return;
+        }
+        // one row per lane: K and V, one bulk copy each, after lane 0 has armed
+        // the slot for all of them
         const char *ks = nullptr, *vs = nullptr;
         if (lane < d.count) {
             int64_t off;
             if (lineb) {
                 const int jj = sparse_row(d);
                 off = row_offset(P.sparse, b, h, jj);
-                ks = from_logits ? reinterpret_cast<const char *>(P.logit + ((int64_t)u * P.sparse.cap + jj) *
-                                                                               logit_floats(G))
-                                 : P.sparse.k + off;
+                ks = P.sparse.k + off;
                 vs = P.sparse.v + off;
             } else {
                 const int a = d.start + lane;
@@ -947,7 +977,7 @@ struct AttnJob {
                 vs = Tt.v + off;
             }
         }
-        const uint32_t kb = from_logits ? (uint32_t)LB : (uint32_t)Gm::ROWB;
+        const uint32_t kb = (uint32_t)Gm::ROWB;
         if (lane == 0)
             mbar_arrive_expect_tx(bar, (uint32_t)d.count * (kb + Gm::ROWB));
         __syncwarp();
