@@ -71,10 +71,12 @@ __global__ void __launch_bounds__(AT_NW * 32, 1) k_attn_stream(const __grid_cons
     const Ctl c = make_ctl(P);
     ring_init(sm.ring);
     allow_dependents();
+    AttnLens lens;
+    attn_read_lengths(P, c, lens);  // inputs only: overlaps the previous kernel's tail
     wait_prior_grid();
     HKV_TRACE_WARP(TR_AW + 4 * (blockIdx.x * AT_NW + (threadIdx.x >> 5)) + 3);
     AttnLine A, B;
-    attn_prologue<ES, D, G>(P, sm, c, red, &A, &B);
+    attn_prologue<ES, D, G>(P, sm, c, red, lens, &A, &B);
     const int64_t g = (int64_t)blockIdx.x * AT_NW + (threadIdx.x >> 5);
     AttnJob<ES, D, G> job(P, c, sm, A, B, g);
     HKV_TRACE_WARP(TR_AW + 4 * (int)g);
@@ -134,8 +136,11 @@ __device__ __forceinline__ void write_offsets(const Params &P, int u, int64_t of
 }
 
 // S2-S4 of unit u, scores at zu (in shared memory when ZS).
+// zg_stage (ZS only): the unit's scores are still in global memory there and
+// the fast path stages them during its first sweep.
 template <int ES, bool ZS>
-__device__ __forceinline__ void unit_work(const Params &P, USmem &sm, const Ctl &c, int u, int n, const float *zu)
+__device__ __forceinline__ void unit_work(const Params &P, USmem &sm, const Ctl &c, int u, int n, const float *zu,
+                                          const float *zg_stage = nullptr)
 {
     int k, n_tie;
     uint32_t key;
@@ -176,7 +181,7 @@ __device__ __forceinline__ void unit_work(const Params &P, USmem &sm, const Ctl 
             Selection s;
             if (P.do_compact &&
                 select_compact_fast(zu, n, m, zlo, beta, pu, P.bmin, P.bmax, sm, s, P.idx + (int64_t)u * P.bmax,
-                                    P.bmax, TR_SEL + 16 * u)) {
+                                    P.bmax, TR_SEL + 16 * u, zg_stage)) {
                 publish(s);
                 HKV_TRACE_AT(TR_SEL + 16 * u + 5);
                 return;
@@ -235,6 +240,11 @@ __global__ void __launch_bounds__(NT) k_unit(const __grid_constant__ Params P)
     HKV_TRACE_AT(TR_SEL + 16 * u);
     const int n = tier_len(P.sparse, u, c);
     const float *zg = P.z + (int64_t)u * P.z_stride;
+    if (P.have_range && P.do_select && P.do_compact && n <= ZSTAGE) {
+        // hkv_step: the range is known, so the first sweep stages the scores
+        unit_work<ES, true>(P, sm, c, u, n, sm.zs, zg);
+        return;
+    }
     const bool staged = stage_scores(zg, n, sm);
     HKV_TRACE_AT(TR_SEL + 16 * u + 6);
     if (staged)
@@ -442,10 +452,11 @@ static Params base_params(const hkv_problem *p, const WsLayout &L, char *ws, con
     P.rec_range = reinterpret_cast<int32_t *>(ws + L.rec_range);
     P.part = reinterpret_cast<float *>(ws + L.part);
     P.part_slots = L.part_slots;
-    P.attn_prefix = P.units <= PREFIX_CAP;
-    (void)dense;
-    (void)sparse;
-    (void)cond;
+    // lines laid out by actual counts when the counts fit shared memory and
+    // every line position fits 31 bits
+    const int64_t span = (int64_t)(dense ? dense->cap : 0) + std::min(p->bmax, sparse ? sparse->cap : 0) +
+                         (cond ? cond->cap : 0);
+    P.attn_prefix = P.units <= PREFIX_CAP && (int64_t)P.units * span < (1ll << 31);
     return P;
 }
 

@@ -72,7 +72,7 @@ struct Params {
     int32_t *rec_range;   // [units][4] first and last record slot of each unit on attention lines A and B
     float *part;          // [part_slots * part_stride] attention records
     int32_t part_slots;   // record slots: 2 x (streaming warps of the attention grid + units)
-    int32_t attn_prefix;  // attention partition over actual tokens (units <= PREFIX_CAP), else over capacity
+    int32_t attn_prefix;  // attention partition over actual tokens (units <= PREFIX_CAP, lines < 2^31), else over capacity
     int32_t have_range;   // per-unit kernel: urange holds the units' score ranges
     int32_t do_select, do_compact;  // per-unit kernel: which steps to run
     int32_t withhold;     // fault injection: streaming warps never arm their stages
@@ -732,7 +732,10 @@ template <int ES, int D, int G>
 struct AttnSmem {
     Ring<AT_NW, AT_SLOT, AT_STAGES> ring;
     float sc[AT_NW][SC_FLOATS];
-    int64_t pre[2][PREFIX_CAP + 1];  // attn_prefix: start of each unit on line A and on line B
+    // attn_prefix (every line shorter than 2^31): start of each unit on line A
+    // and on line B, and each unit's dense, sparse, selected and condensed counts
+    int32_t pre[2][PREFIX_CAP + 1];
+    int32_t uW[PREFIX_CAP], uN[PREFIX_CAP], uK[PREFIX_CAP], uC[PREFIX_CAP];
 };
 
 // A line of the attention work: the units' spans laid end to end and the
@@ -807,11 +810,20 @@ struct AttnJob {
         gu = u;
         gS = unit_start(u);
         gspan = unit_start(u + 1) - gS;
-        gW = tier_len(P.dense, u, c);
-        gn = tier_len(P.sparse, u, c);
-        gk = unit_budget(P, u, gn, c);
+        int C;
+        if (P.attn_prefix) {  // counts the prologue checked and kept
+            gW = sm.uW[u];
+            gn = sm.uN[u];
+            gk = sm.uK[u];
+            C = sm.uC[u];
+        } else {
+            gW = tier_len(P.dense, u, c);
+            gn = tier_len(P.sparse, u, c);
+            gk = unit_budget(P, u, gn, c);
+            C = tier_len(P.cond, u, c);
+        }
         // tokens of the unit on this line: dense ++ condensed (A) or the selection (B)
-        gtot = line == 0 ? gW + tier_len(P.cond, u, c) : gk;
+        gtot = line == 0 ? gW + C : gk;
         if (line == 1 && gk > 0)
             gidx = P.layout == HKV_LAYOUT_FLAT_SUM ? P.idx + __ldcg(P.offsets + u) : P.idx + (int64_t)u * P.bmax;
     }
@@ -1044,40 +1056,66 @@ struct AttnJob {
     }
 };
 
-// Attention prologue of a CTA: the two lines and, with attn_prefix, the start
-// of every unit on each; CTA 0 also writes every unit's record slots
-// (rec_range[u] = first and last slot on line A, then on line B; first > last
-// when empty) for k_merge.
+// Attention prologue, part 1 (before the wait for the previous kernel): each
+// thread reads the input lengths of its units (attn_prefix).
+constexpr int AT_UPT = PREFIX_CAP / (AT_NW * 32);  // units per thread
+struct AttnLens {
+    int W[AT_UPT], N[AT_UPT], C[AT_UPT];
+};
+
+__device__ __forceinline__ void attn_read_lengths(const Params &P, const Ctl &c, AttnLens &L)
+{
+    if (!P.attn_prefix)
+        return;
+#pragma unroll
+    for (int i = 0; i < AT_UPT; ++i) {
+        const int u = i * AT_NW * 32 + threadIdx.x;
+        const bool ok = u < P.units;
+        L.W[i] = ok ? tier_len(P.dense, u, c) : 0;
+        L.N[i] = ok ? tier_len(P.sparse, u, c) : 0;
+        L.C[i] = ok ? tier_len(P.cond, u, c) : 0;
+    }
+}
+
+// Part 2 (after the wait): the budgets, the two lines and, with attn_prefix,
+// each unit's start on each line and its counts in shared memory; CTA 0 also
+// writes every unit's record slots (rec_range[u] = first and last slot on line
+// A, then on line B; first > last when empty) for k_merge.
 template <int ES, int D, int G>
 __device__ void attn_prologue(const Params &P, AttnSmem<ES, D, G> &sm, const Ctl &c, unsigned long long *red,
-                              AttnLine *A, AttnLine *B)
+                              const AttnLens &Ln, AttnLine *A, AttnLine *B)
 {
     constexpr int NTA = AT_NW * 32;
     const int64_t NWt = (int64_t)gridDim.x * AT_NW;
     int64_t TA, TB;
     if (P.attn_prefix) {
         unsigned long long ca = 0, cb = 0;
-        for (int base = 0; base < P.units; base += NTA) {
-            const int u = base + threadIdx.x;
+#pragma unroll
+        for (int i = 0; i < AT_UPT; ++i) {
+            const int u = i * NTA + threadIdx.x;
             unsigned long long ta = 0, tb = 0;
             if (u < P.units) {
-                const int n = tier_len(P.sparse, u, c);
-                ta = (unsigned long long)(tier_len(P.dense, u, c) + tier_len(P.cond, u, c));
-                tb = (unsigned long long)unit_budget(P, u, n, c);
+                const int k = unit_budget(P, u, Ln.N[i], c);
+                sm.uW[u] = Ln.W[i];
+                sm.uN[u] = Ln.N[i];
+                sm.uK[u] = k;
+                sm.uC[u] = Ln.C[i];
+                ta = (unsigned long long)(Ln.W[i] + Ln.C[i]);
+                tb = (unsigned long long)k;
             }
-            // both prefixes in one scan (each sum stays below 2^32)
+            // both prefixes in one scan (each line is shorter than 2^31)
             unsigned long long sum;
             const unsigned long long ex = block_exclusive_scan<NTA>((tb << 32) | ta, red, &sum);
             if (u < P.units) {
-                sm.pre[0][u] = (int64_t)(ca + (ex & 0xffffffffull));
-                sm.pre[1][u] = (int64_t)(cb + (ex >> 32));
+                sm.pre[0][u] = (int32_t)(ca + (ex & 0xffffffffull));
+                sm.pre[1][u] = (int32_t)(cb + (ex >> 32));
             }
             ca += sum & 0xffffffffull;
             cb += sum >> 32;
         }
         if (threadIdx.x == 0) {
-            sm.pre[0][P.units] = (int64_t)ca;
-            sm.pre[1][P.units] = (int64_t)cb;
+            sm.pre[0][P.units] = (int32_t)ca;
+            sm.pre[1][P.units] = (int32_t)cb;
         }
         __syncthreads();
         TA = (int64_t)ca;
@@ -1280,6 +1318,41 @@ __device__ bool stage_scores(const float *zu, int n, USmem &sm)
     }
     __syncthreads();
     return true;
+}
+
+// A sweep over a unit's scores in global memory that also stages them in
+// shared memory: thread t takes the same quads in the same order as
+// sweep_scores<true>, so sums taken in call order match it bit for bit.
+template <typename F>
+__device__ __forceinline__ void sweep_stage(const float *zg, float *zs, int n, F &&f)
+{
+    const bool vec = (((uintptr_t)zg) & 15) == 0;
+    const int nq = (n + 3) >> 2;
+    for (int base = 0; base < nq; base += NT * SWEEP_Q) {
+        float4 v[SWEEP_Q];
+#pragma unroll
+        for (int i = 0; i < SWEEP_Q; ++i) {
+            const int j = 4 * (base + i * NT + (int)threadIdx.x);
+            if (vec && j + 4 <= n) {
+                v[i] = __ldcg(reinterpret_cast<const float4 *>(zg + j));
+            } else {
+                v[i].x = j < n ? __ldcg(zg + j) : 0.f;
+                v[i].y = j + 1 < n ? __ldcg(zg + j + 1) : 0.f;
+                v[i].z = j + 2 < n ? __ldcg(zg + j + 2) : 0.f;
+                v[i].w = j + 3 < n ? __ldcg(zg + j + 3) : 0.f;
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < SWEEP_Q; ++i) {
+            const int j = 4 * (base + i * NT + (int)threadIdx.x);
+            if (j < n)
+                reinterpret_cast<float4 *>(zs)[j >> 2] = v[i];  // j < n <= ZSTAGE, j a multiple of 4
+            f(v[i].x, j, j < n);
+            f(v[i].y, j + 1, j + 1 < n);
+            f(v[i].z, j + 2, j + 2 < n);
+            f(v[i].w, j + 3, j + 3 < n);
+        }
+    }
 }
 
 // First bin whose cumulative count (by_mass = false) or mass reaches target
@@ -1694,7 +1767,8 @@ __device__ int list_candidates(const float *zs, int n, const BinFn &bins, int b_
 }
 
 __device__ bool select_compact_fast(const float *zs, int n, float m, float zlo, float beta, float p, int bmin,
-                                    int bmax, USmem &sm, Selection &r, int32_t *row, int pad, int tb)
+                                    int bmax, USmem &sm, Selection &r, int32_t *row, int pad, int tb,
+                                    const float *zg = nullptr)
 {
     const float bl2 = beta * LOG2E;
     const BinFn bins = make_bins(m, zlo);
@@ -1705,14 +1779,19 @@ __device__ bool select_compact_fast(const float *zs, int n, float m, float zlo, 
     }
     __syncthreads();
     const auto mass = [&](int b) { return sm.mass[b]; };
-    // sweep 1: bin counts and the normaliser
+    // sweep 1: bin counts and the normaliser (staging the scores when they
+    // still are in global memory at zg)
     double zsum = 0.0;
-    sweep_scores<true>(zs, n, [&](float z, int, bool valid) {
+    const auto count = [&](float z, int, bool valid) {
         if (!valid)
             return;
         zsum += (double)wcal(z, m, bl2);
         sred_add(&sm.cnt[bins(z)], 1u);
-    });
+    };
+    if (zg != nullptr)
+        sweep_stage(zg, sm.zs, n, count);
+    else
+        sweep_scores<true>(zs, n, count);
     r.Z = block_sum_f64<NT>(zsum, sm.redd);
     HKV_TRACE_AT(tb < 0 ? -1 : tb + 1);
     int k = 0, kstar = 0;
