@@ -281,6 +281,16 @@ def cpu_baseline(wl, hs, min_seconds=10.0):
             "sample": f"{reps} whole step(s) of {wl.name} ({wl.units} units), {dt:.1f} s"}
 
 
+def config_of(wl, world: int) -> dict:
+    """The workload named in every line (both arms)."""
+    return {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "D": wl.D,
+            "ctx": wl.w_cap + wl.c_cap + wl.n_cap, "dense": wl.w_cap, "condensed": wl.c_cap,
+            "sparse": wl.n_cap, "p": wl.p, "clamp": [wl.bmin, wl.bmax], "layout": "pad_max",
+            "l2": f"inputs larger than L2 ({wl.units * wl.n_cap * wl.D * 2 / 1e6:.0f} MB of sparse "
+                  f"keys per set), {NSETS} distinct sets rotated",
+            "parallelism": f"replicas x{world}", "timing": "CUDA graph replay per step"}
+
+
 # ---- our arm ----------------------------------------------------------------------------
 
 
@@ -426,12 +436,7 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded Gaussian decode states with planted heavy hitters)",
-            "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "D": wl.D,
-                       "ctx": wl.w_cap + wl.c_cap + wl.n_cap, "dense": wl.w_cap, "condensed": wl.c_cap,
-                       "sparse": wl.n_cap, "p": wl.p, "clamp": [wl.bmin, wl.bmax], "layout": "pad_max",
-                       "l2": f"inputs larger than L2 ({wl.units * wl.n_cap * wl.D * 2 / 1e6:.0f} MB of sparse "
-                             f"keys per set), {NSETS} distinct sets rotated",
-                       "parallelism": f"replicas x{world}", "timing": "CUDA graph replay per step"},
+            "config": config_of(wl, world),
             "kv_gbs": round(bytes_per_step * world / (region_ms_max / args.steps / 1e3) / 1e9, 1),
             "frac_of_8tbs": round(bytes_per_step / (ms / 1e3) / 1e9 / NORTH_STAR_HBM_GBS, 4),
             "roofline": roofline,
@@ -474,10 +479,10 @@ def run_reference(args):
     value = args.steps * per_step / wl.units / dt
     sample = f"{per_step} of {wl.units} units of {wl.name} per step"
     line = {
-        "metric": METRIC, "value": round(value, 4), "unit": "steps/s", "n_gpus": 0, "steps": args.steps,
+        "metric": METRIC, "value": round(value, 4), "unit": "steps/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(1e3 / value, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name}, "impl": "reference",
+        "config": config_of(wl, world), "impl": "reference",
         "cpu_baseline": {"value": round(value, 4), "unit": "steps/s", "cores": oracle.num_threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

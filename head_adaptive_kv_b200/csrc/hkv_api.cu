@@ -55,7 +55,8 @@ __global__ void __launch_bounds__(sc_nw(G) * 32, 1) k_score_stream(const __grid_
     const int64_t g = (int64_t)blockIdx.x * Job::NW + (threadIdx.x >> 5);
     Job job(P, c, ring, share_begin(g, NW, R), share_begin(g + 1, NW, R));
     HKV_TRACE_WARP(TR_SW + 4 * (int)g);
-    warp_pipeline(job, ring, c, TR_SW + 4 * (int)g);
+    if (!job.run_single_unit())
+        warp_pipeline(job, ring, c, TR_SW + 4 * (int)g);
 }
 
 // S5 ([TS 2.A] cascade decode over the three tiers; [TS 2.C] Sparse Loading):

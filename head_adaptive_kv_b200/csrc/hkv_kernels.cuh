@@ -441,6 +441,74 @@ struct ScoreJob {
         return false;
     }
 
+    // Copies of a stage (no descriptor record).
+    __device__ __forceinline__ void copy_stage(const StageDesc &d, int slot)
+    {
+        const TierP &T = P.sparse;
+        const char *src = kbase + (int64_t)d.start * T.st * ES;
+        unsigned char *dst = ring.slot[w][slot];
+        uint64_t *bar = &ring.full[w][slot];
+        if (lane == 0) {
+            mbar_arrive_expect_tx(bar, (uint32_t)(d.count * Gm::ROWB));
+            if (T.st == D)
+                bulk_g2s(dst, src, d.count * Gm::ROWB, bar, policy);
+        }
+        if (T.st != D) {
+            __syncwarp();
+            for (int r = lane; r < d.count; r += 32)
+                bulk_g2s(dst + r * Gm::ROWB, src + (int64_t)r * T.st * ES, Gm::ROWB, bar, policy);
+        }
+        __syncwarp();
+    }
+
+    // A share inside one unit whose rows are all present (the common case):
+    // the stages follow from their number alone, so the warp runs this short
+    // loop instead of warp_pipeline's general generator. Returns false when
+    // the share does not qualify.
+    __device__ __forceinline__ bool run_single_unit()
+    {
+        if (left <= 0 || P.withhold)
+            return false;
+        const int cap = P.sparse.cap;
+        if ((int64_t)j + left > cap)
+            return false;
+        const int n = tier_len(P.sparse, u, c);
+        if (j + (int)left > n)
+            return false;
+        gu = u;
+        gn = n;
+        {
+            const int b = u / P.Hkv, h = u % P.Hkv;
+            kbase = P.sparse.k + ((int64_t)b * P.sparse.sb + (int64_t)h * P.sparse.sh) * ES;
+        }
+        const int j0 = j, rows = (int)left;
+        const int nst = (rows + Gm::SROWS - 1) / Gm::SROWS;
+        const auto stage = [&](int sidx) {
+            const int st0 = j0 + sidx * Gm::SROWS;
+            return StageDesc{u, st0, min(Gm::SROWS, j0 + rows - st0),
+                             (sidx == 0 ? SD_FIRST : 0) | (sidx == nst - 1 ? SD_LAST : 0)};
+        };
+        for (int sidx = 0; sidx < NS && sidx < nst; ++sidx)
+            copy_stage(stage(sidx), sidx);
+        for (int sidx = 0; sidx < nst; ++sidx) {
+            const int slot = sidx % NS;
+            if (!mbar_wait(&ring.full[w][slot], (sidx / NS) & 1u, c)) {
+                // let the copies already started land before returning
+                for (int i = sidx; i < nst && i < sidx + NS; ++i)
+                    mbar_wait_bounded(&ring.full[w][i % NS], (i / NS) & 1u, c.wait_ns);
+                return true;
+            }
+            consume(stage(sidx), ring.slot[w][slot]);
+            __syncwarp();
+            if (sidx + NS < nst) {
+                if (lane == 0)
+                    fence_proxy_async_smem();
+                copy_stage(stage(sidx + NS), slot);
+            }
+        }
+        return true;
+    }
+
     __device__ __forceinline__ void issue(const StageDesc &d, int slot)
     {
         const TierP &T = P.sparse;
@@ -1766,6 +1834,74 @@ __device__ int list_candidates(const float *zs, int n, const BinFn &bins, int b_
     return (int)tot;
 }
 
+// One-sweep version of list_candidates: warp w walks its contiguous segment
+// of the staged scores four tokens per lane at a time and appends its hits to
+// its own region of sm.cand (CAND_CAP / warps entries, no atomics); the regions
+// are then closed up into one list. Returns the number listed, or -1 (and
+// nothing usable in sm.cand) when a region overflows.
+__device__ int list_candidates_warp(const float *zs, int n, const BinFn &bins, int b_hi, USmem &sm)
+{
+    constexpr int NW = NT / 32, REG = CAND_CAP / NW;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int seg = ((n + NW - 1) / NW + 127) / 128 * 128;
+    const int j0 = min(n, w * seg), j1 = min(n, j0 + seg);
+    unsigned long long *reg = sm.cand + w * REG;
+    const unsigned lower = (1u << lane) - 1u;
+    int cnt = 0;
+#pragma unroll 1
+    for (int jb = j0; jb < j1; jb += 128) {
+        const int j = jb + 4 * lane;
+        float a[4];
+        if (j + 4 <= j1) {
+            const float4 v = lds4(zs + j);
+            a[0] = v.x;
+            a[1] = v.y;
+            a[2] = v.z;
+            a[3] = v.w;
+        } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                a[e] = j + e < j1 ? lds1(zs + j + e) : 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const bool hit = j + e < j1 && bins(a[e]) <= b_hi;
+            const unsigned m = __ballot_sync(0xffffffffu, hit);
+            const int at = cnt + __popc(m & lower);
+            if (hit && at < REG)
+                reg[at] = ((unsigned long long)score_key(a[e]) << 32) | (uint32_t)(j + e);
+            cnt += __popc(m);
+        }
+    }
+    unsigned long long tot;
+    const unsigned long long before = block_exclusive_scan<NT>(lane == 0 ? (unsigned long long)cnt : 0ull, sm.red, &tot);
+    if (lane == 0)
+        sm.bc[6] = 0;
+    __syncthreads();
+    if (lane == 0 && cnt > REG)
+        sm.bc[6] = 1;
+    __syncthreads();
+    if (sm.bc[6] != 0) {
+        __syncthreads();
+        return -1;
+    }
+    // close up: every warp moves its region down to its place in the list; a
+    // destination can overlap any earlier region, so all reads come first
+    const int dst = (int)__shfl_sync(0xffffffffu, (unsigned long long)before, 0);
+    constexpr int PER = (REG + 31) / 32;
+    unsigned long long v[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+        v[i] = lane + 32 * i < cnt ? reg[lane + 32 * i] : 0ull;
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+        if (lane + 32 * i < cnt)
+            sm.cand[dst + lane + 32 * i] = v[i];
+    __syncthreads();
+    return (int)tot;
+}
+
 __device__ bool select_compact_fast(const float *zs, int n, float m, float zlo, float beta, float p, int bmin,
                                     int bmax, USmem &sm, Selection &r, int32_t *row, int pad, int tb,
                                     const float *zg = nullptr)
@@ -1805,8 +1941,10 @@ __device__ bool select_compact_fast(const float *zs, int n, float m, float zlo, 
         const int ncand = (int)hb_c + (int)sm.cnt[b_hi];
         if (ncand > CAND_CAP)
             return false;
-        // sweeps 2 and 3: the tokens of bins 0 .. b_hi
-        list_candidates(zs, n, bins, b_hi, sm);
+        // the tokens of bins 0 .. b_hi: one sweep, or two when a warp's share
+        // of them outgrows its region
+        if (list_candidates_warp(zs, n, bins, b_hi, sm) < 0)
+            list_candidates(zs, n, bins, b_hi, sm);
         HKV_TRACE_AT(tb < 0 ? -1 : tb + 2);
         // Top-p budget from the listed tokens' bin masses
         kstar = -1;
