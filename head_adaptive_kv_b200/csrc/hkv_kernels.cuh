@@ -1160,6 +1160,8 @@ __device__ void attn_prologue(const Params &P, AttnSmem<ES, D, G> &sm, const Ctl
         unsigned long long ca = 0, cb = 0;
 #pragma unroll
         for (int i = 0; i < AT_UPT; ++i) {
+            if (i * NTA >= P.units)
+                break;  // uniform over the CTA
             const int u = i * NTA + threadIdx.x;
             unsigned long long ta = 0, tb = 0;
             if (u < P.units) {
