@@ -877,18 +877,20 @@ hkv_status hkv_step(const hkv_problem *prob, const void *q, const hkv_tier *dens
     P.v_out = static_cast<char *>(o->v_out);
     P.logit = reinterpret_cast<float *>(wsb + L.logits);  // scorer -> attention of the selected tokens
     P.layout = HKV_LAYOUT_PAD_MAX;  // the three kernels work on PAD_MAX rows
-    // 1. scores, and the score range of each unit
+    // 1. scores, and the score range of each unit (a programmatic dependent of
+    // whatever ran before on the stream: it waits for that kernel before its
+    // first global access)
     const bool scored = sparse->cap > 0;
     Params S = P;
     S.urange = reinterpret_cast<uint32_t *>(wsb + L.urange);
-    if (scored && (s = dispatch<RunScore>(prob, S, st, false)) != HKV_OK)
+    if (scored && (s = dispatch<RunScore>(prob, S, st, true)) != HKV_OK)
         return s;
     // 2. calibration, Top-p budget, cut and compaction, per unit
     Params U = S;
     U.have_range = scored;
     U.do_select = 1;
     U.do_compact = 1;
-    if ((s = launch_unit(prob, U, st, scored)) != HKV_OK)
+    if ((s = launch_unit(prob, U, st, true)) != HKV_OK)
         return s;
     // 3. attention over the three tiers and the merge of each unit
     if ((s = dispatch<RunAttn>(prob, P, st, true)) != HKV_OK)
