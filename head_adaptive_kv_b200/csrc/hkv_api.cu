@@ -877,13 +877,13 @@ hkv_status hkv_step(const hkv_problem *prob, const void *q, const hkv_tier *dens
     P.v_out = static_cast<char *>(o->v_out);
     P.logit = reinterpret_cast<float *>(wsb + L.logits);  // scorer -> attention of the selected tokens
     P.layout = HKV_LAYOUT_PAD_MAX;  // the three kernels work on PAD_MAX rows
-    // 1. scores, and the score range of each unit (a programmatic dependent of
-    // whatever ran before on the stream: it waits for that kernel before its
-    // first global access)
+    // 1. scores, and the score range of each unit (launched in stream order:
+    // as a programmatic dependent of the previous step its CTAs would sit on
+    // SMs the previous attention is leaving, which measured slower)
     const bool scored = sparse->cap > 0;
     Params S = P;
     S.urange = reinterpret_cast<uint32_t *>(wsb + L.urange);
-    if (scored && (s = dispatch<RunScore>(prob, S, st, true)) != HKV_OK)
+    if (scored && (s = dispatch<RunScore>(prob, S, st, false)) != HKV_OK)
         return s;
     // 2. calibration, Top-p budget, cut and compaction, per unit
     Params U = S;

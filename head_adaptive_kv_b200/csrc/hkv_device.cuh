@@ -45,9 +45,18 @@ __device__ unsigned long long hkv_trace_buf[HKV_TRACE_SLOTS];  // one translatio
         if ((cond) && hkv_slot_ >= 0 && hkv_slot_ < HKV_TRACE_SLOTS)               \
             hkv_trace_buf[hkv_slot_] = global_ns();                                \
     } while (0)
+#define HKV_TRACE_VAL(slot, v)                                                     \
+    do {                                                                           \
+        const int hkv_slot_ = (slot);                                              \
+        if (threadIdx.x == 0 && hkv_slot_ >= 0 && hkv_slot_ < HKV_TRACE_SLOTS)     \
+            hkv_trace_buf[hkv_slot_] = (unsigned long long)(v);                    \
+    } while (0)
 #else
 #define HKV_TRACE_IF(cond, slot) \
     do {                         \
+    } while (0)
+#define HKV_TRACE_VAL(slot, v) \
+    do {                       \
     } while (0)
 #endif
 #define HKV_TRACE_AT(slot) HKV_TRACE_IF(threadIdx.x == 0, slot)

@@ -1478,6 +1478,25 @@ __device__ int find_crossing(const uint32_t *cnt, MassFn mass, int nbins, bool b
 // Bitonic sort of cand[0, P) ascending (P a power of two).
 __device__ void sort_candidates(unsigned long long *cand, int P)
 {
+    if (P <= 32) {
+        // one warp, in registers
+        if (threadIdx.x < 32) {
+            const int lane = threadIdx.x;
+            unsigned long long x = lane < P ? cand[lane] : ~0ull;
+#pragma unroll 1
+            for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll 1
+                for (int j = k >> 1; j > 0; j >>= 1) {
+                    const unsigned long long y = __shfl_xor_sync(0xffffffffu, x, j);
+                    const bool take_min = ((lane & j) == 0) == ((lane & k) == 0);
+                    x = take_min ? (x < y ? x : y) : (x < y ? y : x);
+                }
+            if (lane < P)
+                cand[lane] = x;
+        }
+        __syncthreads();
+        return;
+    }
     for (int k = 2; k <= P; k <<= 1) {
         for (int j = k >> 1; j > 0; j >>= 1) {
             for (int i = threadIdx.x; i < P / 2; i += NT) {
@@ -1798,23 +1817,34 @@ __device__ Selection select_unit(const float *zu, int n, float m, float zlo, flo
 // buffer; the caller then takes select_unit and compact_unit.
 // =============================================================================
 
-// Copy the listed candidates of bin b into sm.binbuf (positions from a block
-// scan of per-thread counts, no shared counter); returns their number, or -1
-// when the bin holds more than BIN_CAP tokens.
+// Copy the listed candidates of bin b into sm.binbuf (one pass, one shared
+// atomic per warp and step: the order does not matter, the bin is sorted
+// next); returns their number, or -1 when the bin holds more than BIN_CAP
+// tokens.
 __device__ int load_sorted_bin(int b, int ncand, const BinFn &bins, USmem &sm)
 {
     const int cb = (int)sm.cnt[b];
     if (cb > BIN_CAP)
         return -1;
-    const auto hit = [&](int i) { return bins(key_score((uint32_t)(sm.cand[i] >> 32))) == b; };
-    unsigned long long mine = 0;
-    for (int i = threadIdx.x; i < ncand; i += NT)
-        mine += hit(i) ? 1u : 0u;
-    unsigned long long tot;
-    int at = (int)block_exclusive_scan<NT>(mine, sm.red, &tot);
-    for (int i = threadIdx.x; i < ncand; i += NT)
-        if (hit(i))
-            sm.binbuf[at++] = sm.cand[i];
+    if (threadIdx.x == 0)
+        sm.bc[3] = 0;
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+    for (int base = 0; base < ncand; base += NT) {
+        const int i = base + threadIdx.x;
+        const unsigned long long e = i < ncand ? sm.cand[i] : 0ull;
+        const bool hit = i < ncand && bins(key_score((uint32_t)(e >> 32))) == b;
+        const unsigned mask = __ballot_sync(0xffffffffu, hit);
+        if (mask != 0) {
+            const int leader = __ffs(mask) - 1;
+            int at = 0;
+            if (lane == leader)
+                at = satom_add(&sm.bc[3], __popc(mask));
+            at = __shfl_sync(0xffffffffu, at, leader);
+            if (hit)
+                sm.binbuf[at + __popc(mask & ((1u << lane) - 1u))] = e;
+        }
+    }
     __syncthreads();
     return cb;
 }
@@ -1989,10 +2019,14 @@ __device__ bool select_compact_fast(const float *zs, int n, float m, float zlo, 
                 // the clamp decides: the token of rank k
                 unsigned long long kb_c, kb_m;
                 const int b_k = find_crossing(sm.cnt, mass, SBINS, false, (unsigned long long)k, &kb_c, &kb_m, sm);
+                HKV_TRACE_AT(tb < 0 ? -1 : tb + 9);
                 const int cb = load_sorted_bin(b_k, ncand, bins, sm);
+                HKV_TRACE_AT(tb < 0 ? -1 : tb + 10);
+                HKV_TRACE_VAL(tb < 0 ? -1 : tb + 15, cb);
                 if (cb < 0)
                     return false;
                 pos = sort_and_locate(cb, false, (unsigned long long)k - kb_c, 0, m, bl2, sm, sm.binbuf);
+                HKV_TRACE_AT(tb < 0 ? -1 : tb + 14);
                 before_c = kb_c;
             }
             cut_key = (uint32_t)(sm.binbuf[pos] >> 32);
