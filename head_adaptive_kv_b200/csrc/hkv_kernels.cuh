@@ -747,7 +747,7 @@ __device__ void merge_head(const Params &P, int u, int g, int a0, int a1, int b0
 #pragma unroll
     for (int e = 0; e < DPL; ++e)
         O[e] = 0.f;
-    constexpr int RB = 8;  // records loaded together
+    constexpr int RB = 16;  // records loaded together
     const int na = a1 >= a0 ? a1 - a0 + 1 : 0, nb = b1 >= b0 ? b1 - b0 + 1 : 0;
     for (int t0 = 0; t0 < na + nb; t0 += RB) {
         float mt[RB], lt[RB], ot[RB][DPL];

@@ -196,18 +196,21 @@ hkv_status hkv_cascade_decode(const hkv_problem *prob, const void *q,
                               float *out, float *lse, void *ws, size_t ws_bytes,
                               hkv_stream_t stream);
 
-/* S1..S5 in one call ([TS 2.A] pipeline steps 2 and 3 plus decoding): three
- * kernels on `stream`, the second and third launched as programmatic
- * dependents of the one before. (1) A persistent streaming kernel scores every
- * sparse token (the same kernel as hkv_score) and records each scoring tile's
- * score range; (2) one CTA per unit calibrates, takes the Top-p budget and the
- * cut, and compacts the unit's indices into PAD_MAX rows; (3) a persistent
- * streaming kernel runs the split attention tiles (the same kernel as
- * hkv_cascade_decode), reading the selected rows through the indices
- * ([TS 2.C] Sparse Loading); the last tile of a unit merges it. A FLAT_SUM
- * layout or k_out/v_out (the Rewrite Cache copy) adds a fourth kernel. The
- * results equal those of the five separate calls bit for bit. ws as for
- * hkv_cascade_decode. */
+/* S1..S5 in one call ([TS 2.A] pipeline steps 2 and 3 plus decoding): four
+ * kernels on `stream`, all but the first launched as programmatic dependents
+ * of the one before. (1) A persistent streaming kernel scores every sparse
+ * token (the same kernel as hkv_score), also writing each token's per-head
+ * logits and each unit's score range into the workspace; (2) one CTA per unit
+ * calibrates, takes the Top-p budget and the cut, and compacts the unit's
+ * indices into PAD_MAX rows; (3) a persistent streaming kernel attends over
+ * the dense and condensed tokens and over the selected tokens, whose rows it
+ * reads through the indices ([TS 2.C] Sparse Loading) together with the
+ * scorer's logits (so their K rows are not read again); (4) a merge kernel
+ * combines each unit's partial softmax records. A FLAT_SUM layout or
+ * k_out/v_out (the Rewrite Cache copy) adds a fifth kernel. Scores, budgets,
+ * cuts, index rows, m and logZ equal those of the separate calls bit for bit;
+ * out and lse agree to a few ulp (hkv_cascade_decode recomputes the logits
+ * from K). ws as for hkv_cascade_decode. */
 hkv_status hkv_step(const hkv_problem *prob, const void *q, const hkv_tier *dense,
                     const hkv_tier *sparse, const hkv_tier *condensed,
                     const hkv_step_out *out, void *ws, size_t ws_bytes,
