@@ -18,6 +18,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -49,11 +50,16 @@ def peaks():
 
 
 def csrc_hash() -> str:
+    """Hash of the kernel sources with comments and blank space removed, so a
+    profile stays attached to its kernels across comment-only edits."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "head_adaptive_kv_b200", "csrc")
     for f in sorted(os.listdir(d)):
-        with open(os.path.join(d, f), "rb") as fh:
-            h.update(f.encode() + fh.read())
+        with open(os.path.join(d, f), encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(f.encode() + " ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 
@@ -149,6 +155,18 @@ def score_bytes_of(wl, sparse_len) -> int:
     e = 2 if wl.dtype == torch.bfloat16 else 4
     n = int(np.sum(sparse_len))
     return n * wl.D * e + wl.B * wl.Hq * wl.D * e + n * 4
+
+
+# Sparse-tier room kept free while the append is timed (above the launches
+# kernel_ms makes: one, 64 captured, 3 + up to 20 replays of 64).
+APPEND_ROOM = 2048
+
+
+def append_bytes(wl) -> int:
+    """Algorithmic bytes of one append that rolls the window: per unit the new
+    K and V rows read, the oldest window rows read, written to the sparse tier,
+    and the new rows written in their place."""
+    return wl.units * 8 * wl.D * (2 if wl.dtype == torch.bfloat16 else 4)
 
 
 def kernel_ms(launch_round, launches_per_round: int, stream, args) -> float:
@@ -391,6 +409,22 @@ def run_ours(args):
                                                     out.out, ws, lse=out.lse) for x, prob, tiers, out in sets],
                         NSETS, stream, args)
     attn_ms = max_over_ranks(attn_ms, dist, device)
+    # KV append with the dense-window roll, timed on copies of one decode state
+    # whose sparse tiers keep room for every append of the timing (so each
+    # launch moves a full window row into the sparse tier)
+    x0, prob0 = sets[0][0], sets[0][1]
+    room = APPEND_ROOM
+    a_dense = hkv.Tier(x0.dense.k.clone(), x0.dense.v.clone(), x0.dense.len.clone())
+    a_sparse = hkv.Tier(x0.sparse.k.clone(), x0.sparse.v.clone(),
+                        torch.clamp(x0.sparse.len - room, min=0).to(torch.int32))
+    a_head = torch.zeros(wl.units, dtype=torch.int32, device=device)
+    a_new = torch.randn(2, wl.B, wl.Hkv, wl.D, device=device).to(wl.dtype)
+    append_ms = kernel_ms(lambda: hkv.append(prob0, a_new[0], a_new[1], a_dense, a_head, a_sparse, ws), 1,
+                          stream, args)
+    append_ms = max_over_ranks(append_ms, dist, device)
+    grew = int((a_sparse.len - torch.clamp(x0.sparse.len - room, min=0)).min().item())
+    assert 0 < grew < room, "append timing ran out of sparse room"
+    del a_dense, a_sparse
     assert ws.status() == 0, "device status word set during the kernel timing"
     score_bytes = float(np.mean([score_bytes_of(wl, x.sparse.len.cpu().numpy()) for x, *_ in sets]))
     achieved_gbs = score_bytes / (score_ms / 1e3) / 1e9
@@ -402,7 +436,9 @@ def run_ours(args):
                 "launch_us": round(score_ms * 1e3, 2)}
     kernels = {"step_us": round(launch_ms_max * 1e3, 2), "step_gbs": round(step_gbs, 1),
                "score_us": round(score_ms * 1e3, 2), "attn_us": round(attn_ms * 1e3, 2),
-               "select_compact_us_remainder": round((launch_ms_max - score_ms - attn_ms) * 1e3, 2)}
+               "select_compact_us_remainder": round((launch_ms_max - score_ms - attn_ms) * 1e3, 2),
+               "append_us": round(append_ms * 1e3, 2),
+               "append_bytes": int(append_bytes(wl))}
 
     # end to end through the public API: per step, copy the step's query and the
     # per-unit lengths from pinned host memory, run, and read the outputs back

@@ -6,15 +6,18 @@
 // paper ("Cascade Cache Hierarchy", "Logits Calibration Mechanism",
 // "System-Aware Index Regularization").
 //
-// One decode step (hkv_step) is three kernels on the caller's stream, the last
-// two launched as programmatic dependents so that their launch and prologue
+// One decode step (hkv_step) is four kernels on the caller's stream, the last
+// three launched as programmatic dependents so that their launch and prologue
 // overlap the previous kernel's tail:
 //   1. k_score_stream -- S1: every sparse-tier key scored once (streaming);
 //   2. k_unit         -- S2-S4: per unit, calibration + Top-p budget + cut,
 //                        then the order-preserving compaction of the indices;
 //   3. k_attn_stream  -- S5: attention over dense ++ selected ++ condensed,
-//                        per-tile online softmax, the last tile merges the unit.
-// FLAT_SUM layouts and the Rewrite Cache copy add k_flatten.
+//                        one online-softmax record per warp and unit part;
+//   4. k_merge        -- S5: each unit's records combined per query head.
+// FLAT_SUM layouts and the Rewrite Cache copy add k_flatten. hkv_append
+// (k_append, at the end of this file) adds each step's new token to the dense
+// window and moves the displaced one into the sparse tier.
 #include <algorithm>
 #include <atomic>
 #include <cmath>
@@ -1005,5 +1008,152 @@ extern "C" hkv_status hkv_cascade_decode_noalloc(const hkv_problem *prob, const 
     if (status != nullptr &&
         cudaMemcpyAsync(status, base, sizeof(uint32_t), cudaMemcpyDeviceToDevice, st) != cudaSuccess)
         return HKV_ERR_CUDA;
+    return HKV_OK;
+}
+
+// =============================================================================
+// KV append with the dense-window roll ([TS 2.A] pipeline step 1)
+//
+// The newest token enters the dense window of each unit. The window is a ring
+// of cap slots: while it has room the token takes slot len; once it is full
+// the token replaces the oldest one, at slot head, and head advances. The
+// token that leaves the window is appended to the sparse tier (so the sparse
+// tier stays in age order), or dropped and reported when that tier is full.
+// With no window (cap 0) the new token goes straight to the sparse tier.
+// =============================================================================
+
+namespace hkv {
+
+struct AppendP {
+    const char *k_new, *v_new;  // [units, D] rows of row_bytes
+    char *dk, *dv, *sk, *sv;    // tier storage, written in place
+    int64_t dsb, dsh, dst, ssb, ssh, sst;  // byte strides
+    int32_t wcap, ncap;
+    int32_t *dlen, *slen, *head, *dropped;
+    int32_t Hkv, units, chunks;  // chunks: 16-byte pieces of one row
+    uint32_t *status;
+};
+
+constexpr int APPEND_WARPS = 8;
+
+// One warp per unit. Lane l moves the 16-byte pieces l, l+32, ... of the K row
+// followed by the V row; each piece is read and rewritten by the same lane, so
+// the old window row is in registers before its slot is overwritten.
+__global__ void __launch_bounds__(APPEND_WARPS * 32) k_append(const __grid_constant__ AppendP A)
+{
+    const int u = blockIdx.x * APPEND_WARPS + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (u >= A.units)
+        return;
+    const int b = u / A.Hkv, h = u - b * A.Hkv;
+    const int W = A.wcap > 0 ? __ldcg(A.dlen + u) : 0;
+    const int n = A.ncap > 0 ? __ldcg(A.slen + u) : 0;
+    const int hd = A.wcap > 0 ? __ldcg(A.head + u) : 0;
+    const bool bad_len = W < 0 || W > A.wcap || n < 0 || n > A.ncap;
+    const bool bad_head = A.wcap > 0 && (hd < 0 || hd >= A.wcap);
+    if (bad_len || bad_head) {
+        // a corrupt unit is left as it is
+        if (lane == 0) {
+            atomicOr(A.status, (bad_len ? HKV_DEV_LEN_CLAMPED : 0u) | (bad_head ? HKV_DEV_BAD_INDEX : 0u));
+            if (A.dropped)
+                A.dropped[u] = 0;
+        }
+        return;
+    }
+    const bool room = W < A.wcap;            // the window takes the token without a roll
+    const bool age_out = !room;              // a token leaves the window (or bypasses it)
+    const bool keep = age_out && n < A.ncap; // ... and finds room in the sparse tier
+    const int dslot = room ? W : hd;
+    char *drow[2], *srow[2];
+    const char *nrow[2] = {A.k_new + (int64_t)u * A.chunks * 16, A.v_new + (int64_t)u * A.chunks * 16};
+    const int64_t doff = (int64_t)b * A.dsb + (int64_t)h * A.dsh + (int64_t)dslot * A.dst;
+    const int64_t soff = (int64_t)b * A.ssb + (int64_t)h * A.ssh + (int64_t)n * A.sst;
+    drow[0] = A.dk + doff;
+    drow[1] = A.dv + doff;
+    srow[0] = A.sk + soff;
+    srow[1] = A.sv + soff;
+    for (int c = lane; c < 2 * A.chunks; c += 32) {
+        const int kv = c >= A.chunks, off = (c - kv * A.chunks) * 16;
+        const uint4 fresh = __ldg(reinterpret_cast<const uint4 *>(nrow[kv] + off));
+        if (A.wcap > 0) {
+            uint4 *slot = reinterpret_cast<uint4 *>(drow[kv] + off);
+            if (keep)
+                *reinterpret_cast<uint4 *>(srow[kv] + off) = *slot;  // the oldest row moves on
+            *slot = fresh;
+        } else if (keep) {
+            *reinterpret_cast<uint4 *>(srow[kv] + off) = fresh;
+        }
+    }
+    if (lane == 0) {
+        if (room)
+            A.dlen[u] = W + 1;
+        else if (A.wcap > 0)
+            A.head[u] = hd + 1 == A.wcap ? 0 : hd + 1;
+        if (keep)
+            A.slen[u] = n + 1;
+        if (age_out && !keep)
+            atomicOr(A.status, HKV_DEV_SPARSE_FULL);
+        if (A.dropped)
+            A.dropped[u] = age_out && !keep;
+    }
+}
+
+}  // namespace hkv
+
+extern "C" hkv_status hkv_append(const hkv_problem *prob, const void *k_new, const void *v_new,
+                                 const hkv_tier *dense, int32_t *dense_head, const hkv_tier *sparse,
+                                 int32_t *dropped, void *ws, size_t ws_bytes, hkv_stream_t stream)
+{
+    hkv_status s = check_problem(prob);
+    if (s != HKV_OK)
+        return s;
+    if ((s = check_tier(dense, prob, true)) != HKV_OK || (s = check_tier(sparse, prob, true)) != HKV_OK)
+        return s;
+    if (ws == nullptr || !aligned(ws, 256) || ws_bytes < 256)
+        return HKV_ERR_WORKSPACE;
+    if (k_new == nullptr || v_new == nullptr || !aligned(k_new, 16) || !aligned(v_new, 16))
+        return HKV_ERR_INVALID_ARG;
+    const int wcap = dense ? dense->cap : 0, ncap = sparse ? sparse->cap : 0;
+    if (wcap > 0 && (dense_head == nullptr || !aligned(dense_head, 4)))
+        return HKV_ERR_INVALID_ARG;
+    if (dropped != nullptr && !aligned(dropped, 4))
+        return HKV_ERR_INVALID_ARG;
+    const int64_t units = (int64_t)prob->B * prob->Hkv;
+    if (units == 0)
+        return HKV_OK;
+    const int es = es_of(prob->dtype);
+    AppendP A{};
+    A.k_new = static_cast<const char *>(k_new);
+    A.v_new = static_cast<const char *>(v_new);
+    if (wcap > 0) {
+        A.dk = static_cast<char *>(const_cast<void *>(dense->k));
+        A.dv = static_cast<char *>(const_cast<void *>(dense->v));
+        A.dsb = dense->stride_b * es;
+        A.dsh = dense->stride_h * es;
+        A.dst = dense->stride_t * es;
+        A.dlen = const_cast<int32_t *>(dense->len);
+        A.head = dense_head;
+    }
+    if (ncap > 0) {
+        A.sk = static_cast<char *>(const_cast<void *>(sparse->k));
+        A.sv = static_cast<char *>(const_cast<void *>(sparse->v));
+        A.ssb = sparse->stride_b * es;
+        A.ssh = sparse->stride_h * es;
+        A.sst = sparse->stride_t * es;
+        A.slen = const_cast<int32_t *>(sparse->len);
+    }
+    A.wcap = wcap;
+    A.ncap = ncap;
+    A.dropped = dropped;
+    A.Hkv = prob->Hkv;
+    A.units = (int32_t)units;
+    A.chunks = prob->D * es / 16;
+    A.status = static_cast<uint32_t *>(ws);
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)((units + APPEND_WARPS - 1) / APPEND_WARPS));
+    cfg.blockDim = dim3(APPEND_WARPS * 32);
+    cfg.stream = (cudaStream_t)stream;
+    if (cudaLaunchKernelEx(&cfg, k_append, A) != cudaSuccess)
+        return HKV_ERR_CUDA;
+    g_launches.fetch_add(1);
     return HKV_OK;
 }

@@ -21,6 +21,7 @@ PAD_MAX, FLAT_SUM = 0, 1
 STATUS = {0: "HKV_OK", 1: "HKV_ERR_INVALID_ARG", 2: "HKV_ERR_UNSUPPORTED", 3: "HKV_ERR_CUDA",
           4: "HKV_ERR_TIMEOUT", 5: "HKV_ERR_DEVICE", 6: "HKV_ERR_WORKSPACE"}
 DEV_LEN_CLAMPED, DEV_TIMEOUT, DEV_BAD_TEMP, DEV_BAD_INDEX, DEV_BAD_P = 0x1, 0x2, 0x4, 0x8, 0x10
+DEV_SPARSE_FULL = 0x20
 
 
 class HkvError(RuntimeError):
@@ -67,6 +68,7 @@ def _load():
         "hkv_cascade_decode": [P, P, P, P, P, P, P, P, P, P, P, sz, P],
         "hkv_step": [P, P, P, P, P, P, P, sz, P],
         "hkv_cascade_decode_noalloc": [P, P, P, P, P, P, P, P, P, P, P, P],
+        "hkv_append": [P, P, P, P, P, P, P, P, sz, P],
         "hkv_get_status": [P, C.POINTER(C.c_uint32), P],
         "hkv_set_wait_limit_ns": [C.c_uint64],
         "hkv_debug_withhold_publish": [i32],
@@ -290,6 +292,22 @@ def cascade_decode_noalloc(prob: Problem, q: torch.Tensor, dense: Optional[Tier]
     _check(lib.hkv_cascade_decode_noalloc(C.byref(prob.c()), _ptr(q), _tref(dense), _tref(sparse), _ptr(idx),
                                           _ptr(offsets), _ptr(sel_len), _tref(condensed), _ptr(out), _ptr(lse),
                                           _ptr(status), _stream(stream)), "hkv_cascade_decode_noalloc")
+
+
+def append(prob: Problem, k_new: torch.Tensor, v_new: torch.Tensor, dense: Optional[Tier],
+           head: Optional[torch.Tensor], sparse: Optional[Tier], ws: Workspace,
+           dropped: Optional[torch.Tensor] = None, stream=None):
+    """KV append with the dense-window roll, in place on the tiers' K, V and
+    lengths and on head (int32 [B*Hkv]). k_new, v_new: [B, Hkv, D] contiguous.
+    dropped: optional int32 [B*Hkv], 1 where a token left the window while the
+    sparse tier was full."""
+    for t in (k_new, v_new):
+        if not t.is_contiguous() or t.dtype != prob.dtype:
+            raise ValueError("k_new and v_new must be contiguous [B, Hkv, D] of the problem's dtype")
+    if head is not None and head.dtype != torch.int32:
+        raise TypeError("head must be int32")
+    _check(lib.hkv_append(C.byref(prob.c()), _ptr(k_new), _ptr(v_new), _tref(dense), _ptr(head),
+                          _tref(sparse), _ptr(dropped), ws.ptr, ws.nbytes, _stream(stream)), "hkv_append")
 
 
 def set_wait_limit_ns(ns: int):

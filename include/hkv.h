@@ -76,6 +76,8 @@ typedef enum {
 #define HKV_DEV_BAD_TEMP     0x4u  /* a negative or NaN inverse temperature; 1 used */
 #define HKV_DEV_BAD_INDEX    0x8u  /* an index or budget outside its range; row 0 / a clamp used */
 #define HKV_DEV_BAD_P        0x10u /* a NaN per-unit p; p = 1 used */
+#define HKV_DEV_SPARSE_FULL  0x20u /* hkv_append: a token left the dense window while the
+                                      sparse tier was full, and was dropped */
 
 /* One cache tier ([TS 2.A]: dense recent window, sparse tier, condensed slots). */
 typedef struct {
@@ -215,6 +217,41 @@ hkv_status hkv_step(const hkv_problem *prob, const void *q, const hkv_tier *dens
                     const hkv_tier *sparse, const hkv_tier *condensed,
                     const hkv_step_out *out, void *ws, size_t ws_bytes,
                     hkv_stream_t stream);
+
+/* KV append with the dense-window roll ([TS 2.A] Cascade Cache Hierarchy,
+ * pipeline step 1: the new token joins the dense window of recent tokens, and
+ * the token that leaves the window moves to the sparse tier). One kernel, one
+ * warp per unit. Per unit u = b*Hkv + h, with W = dense->len[u],
+ * n = sparse->len[u], and the window a ring of Wc = dense->cap slots whose
+ * oldest token sits at slot dense_head[u]:
+ *   - W < Wc: the new row goes to dense slot W; dense->len[u] = W + 1.
+ *   - W == Wc > 0: the row at slot dense_head[u] leaves the window and the new
+ *     row takes its slot; dense_head[u] = (dense_head[u] + 1) mod Wc.
+ *   - Wc == 0 (dense NULL or empty): the new row itself leaves at once.
+ *   - a row that leaves goes to sparse slot n and sparse->len[u] = n + 1; if
+ *     n == sparse->cap it is dropped, dropped[u] = 1 and the status word gets
+ *     HKV_DEV_SPARSE_FULL.
+ * Rows are copied bit for bit, K and V alike. The sparse tier thus holds the
+ * aged-out tokens in age order, which is the token order every other call of
+ * this library scores, selects and compacts in. Start a window with len 0 and
+ * head 0; a window filled some other way must set head to its oldest slot.
+ * - k_new, v_new: device [B, Hkv, D] contiguous, 16-byte aligned, element type
+ *   of prob->dtype; must not overlap the tiers.
+ * - dense, sparse: tiers as elsewhere (either may be NULL or empty); THIS CALL
+ *   WRITES through their k, v and len pointers (declared const in hkv_tier for
+ *   the calls that only read them). Both need v.
+ * - dense_head: device int32 [B*Hkv], read and written; required when the
+ *   dense tier has slots, else may be NULL.
+ * - dropped: device int32 [B*Hkv] or NULL; receives 0 or 1 per unit.
+ * - Only prob's B, Hkv, D and dtype are used (the rest must still validate).
+ * - A unit whose lengths are outside [0, cap] or whose head is outside
+ *   [0, Wc) is left untouched and sets HKV_DEV_LEN_CLAMPED or
+ *   HKV_DEV_BAD_INDEX.
+ * - ws: any workspace of at least 256 bytes (256-byte aligned, zeroed once);
+ *   only its status word is used, so the step's workspace serves. */
+hkv_status hkv_append(const hkv_problem *prob, const void *k_new, const void *v_new,
+                      const hkv_tier *dense, int32_t *dense_head, const hkv_tier *sparse,
+                      int32_t *dropped, void *ws, size_t ws_bytes, hkv_stream_t stream);
 
 /* Capacity, in bytes, of the device scratch array behind
  * hkv_cascade_decode_noalloc (one array per GPU that loads the library, held

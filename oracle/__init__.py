@@ -234,3 +234,53 @@ def step(q: np.ndarray, dense: Optional[Tier], sparse: Tier, condensed: Optional
 
 def num_threads() -> int:
     return int(lib().hkvo_num_threads())
+
+
+# ---- KV append with the dense-window roll ----------------------------------------------
+#
+# [TS 2.A] Cascade Cache Hierarchy, pipeline step (1): the new token enters the
+# dense window of recent tokens; once the window is full, its oldest token
+# ages out into the sparse tier. Reading taken: the window is a ring of W_cap
+# slots per unit (attention does not depend on the order of its tokens), its
+# oldest slot is head[u]; an aged-out token is appended at the end of the
+# sparse tier (so sparse order is age order); when the sparse tier is full
+# the aged-out token is dropped and reported (forming condensed slots is not
+# part of this step).
+
+
+def append(k_new: np.ndarray, v_new: np.ndarray, dense: Tier, head: np.ndarray, sparse: Tier):
+    """One append per unit, in place on copies: returns (dense, head, sparse,
+    dropped) with dropped[u] = 1 where an aged-out token found the sparse tier
+    full. k_new, v_new: [B, Hkv, D]. All arrays keep their dtypes."""
+    B, H, D = k_new.shape
+    dk, dv = dense.k.copy(), dense.v.copy()
+    sk, sv = sparse.k.copy(), sparse.v.copy()
+    dlen = np.array(dense.len, dtype=np.int32).copy()
+    slen = np.array(sparse.len, dtype=np.int32).copy()
+    hd = np.array(head, dtype=np.int32).copy()
+    wcap, ncap = dk.shape[2], sk.shape[2]
+    dropped = np.zeros(B * H, dtype=np.int32)
+    for b in range(B):
+        for h in range(H):
+            u = b * H + h
+            if dlen[u] < wcap:  # the window still has room
+                dk[b, h, dlen[u]] = k_new[b, h]
+                dv[b, h, dlen[u]] = v_new[b, h]
+                dlen[u] += 1
+                continue
+            # full window (or none): the oldest token ages out first
+            if wcap > 0:
+                old_k, old_v = dk[b, h, hd[u]].copy(), dv[b, h, hd[u]].copy()
+            else:
+                old_k, old_v = k_new[b, h], v_new[b, h]
+            if slen[u] < ncap:
+                sk[b, h, slen[u]] = old_k
+                sv[b, h, slen[u]] = old_v
+                slen[u] += 1
+            else:
+                dropped[u] = 1
+            if wcap > 0:
+                dk[b, h, hd[u]] = k_new[b, h]
+                dv[b, h, hd[u]] = v_new[b, h]
+                hd[u] = (hd[u] + 1) % wcap
+    return Tier(dk, dv, dlen), hd, Tier(sk, sv, slen), dropped

@@ -408,4 +408,71 @@ def pin_attention_empty_and_golden():
         assert abs(lse[0, 0] - case["lse"]) < 1e-6
 
 
+# ---- KV append (TS 2.A pipeline step 1) -----------------------------------------------
+
+
+def pin_append_matches_list_model():
+    """A run of appends against a plain Python model: per unit, a list of the
+    window's tokens in arrival order (a token leaving the window goes to the
+    end of the sparse list), compared as multisets of rows for the window
+    (its slot order is the ring's) and in order for the sparse tier."""
+    rng = np.random.default_rng(11)
+    B, H, D, wcap, ncap = 2, 3, 8, 4, 6
+    dense = oracle.Tier(np.zeros((B, H, wcap, D), np.float32), np.zeros((B, H, wcap, D), np.float32),
+                        np.array([0, 2, 4, 4, 1, 3], np.int32))
+    sparse = oracle.Tier(np.zeros((B, H, ncap, D), np.float32), np.zeros((B, H, ncap, D), np.float32),
+                         np.array([0, 5, 0, 6, 2, 1], np.int32))
+    # give the pre-filled slots distinct contents
+    dense.k[...] = rng.standard_normal(dense.k.shape).astype(np.float32)
+    dense.v[...] = rng.standard_normal(dense.v.shape).astype(np.float32)
+    sparse.k[...] = rng.standard_normal(sparse.k.shape).astype(np.float32)
+    sparse.v[...] = rng.standard_normal(sparse.v.shape).astype(np.float32)
+    head = np.zeros(B * H, np.int32)
+    # the model: window list (oldest first) and sparse list
+    win = [[(dense.k[u // H, u % H, i].copy(), dense.v[u // H, u % H, i].copy()) for i in range(dense.len[u])]
+           for u in range(B * H)]
+    sp = [[(sparse.k[u // H, u % H, i].copy(), sparse.v[u // H, u % H, i].copy()) for i in range(sparse.len[u])]
+          for u in range(B * H)]
+    drops = 0
+    for step in range(9):
+        kn = rng.standard_normal((B, H, D)).astype(np.float32)
+        vn = rng.standard_normal((B, H, D)).astype(np.float32)
+        dense, head, sparse, dropped = oracle.append(kn, vn, dense, head, sparse)
+        for u in range(B * H):
+            win[u].append((kn[u // H, u % H], vn[u // H, u % H]))
+            dropped_now = 0
+            if len(win[u]) > wcap:
+                old = win[u].pop(0)
+                if len(sp[u]) < ncap:
+                    sp[u].append(old)
+                else:
+                    dropped_now = 1
+            drops += dropped_now
+            assert dropped[u] == dropped_now, (step, u)
+            assert dense.len[u] == len(win[u]) and sparse.len[u] == len(sp[u])
+            rows = sorted(tuple(dense.k[u // H, u % H, i]) for i in range(dense.len[u]))
+            assert rows == sorted(tuple(k) for k, _ in win[u]), (step, u)
+            vrows = sorted(tuple(dense.v[u // H, u % H, i]) for i in range(dense.len[u]))
+            assert vrows == sorted(tuple(v) for _, v in win[u]), (step, u)
+            # the ring's head slot holds the oldest token once the window is full
+            if dense.len[u] == wcap:
+                assert np.array_equal(dense.k[u // H, u % H, head[u]], win[u][0][0])
+            for i, (k, v) in enumerate(sp[u]):
+                assert np.array_equal(sparse.k[u // H, u % H, i], k) and np.array_equal(sparse.v[u // H, u % H, i], v)
+    assert drops > 0  # the run reaches full sparse tiers
+
+
+def pin_append_without_window_goes_to_sparse():
+    """W_cap = 0: every new token goes straight to the end of the sparse tier."""
+    B, H, D = 1, 2, 4
+    dense = oracle.Tier(np.zeros((B, H, 0, D), np.float32), np.zeros((B, H, 0, D), np.float32),
+                        np.zeros(B * H, np.int32))
+    sparse = oracle.Tier(np.zeros((B, H, 3, D), np.float32), np.zeros((B, H, 3, D), np.float32),
+                         np.array([1, 3], np.int32))
+    kn = np.arange(B * H * D, dtype=np.float32).reshape(B, H, D)
+    d2, hd, s2, dropped = oracle.append(kn, -kn, dense, np.zeros(B * H, np.int32), sparse)
+    assert list(s2.len) == [2, 3] and list(dropped) == [0, 1]
+    assert np.array_equal(s2.k[0, 0, 1], kn[0, 0]) and np.array_equal(s2.v[0, 0, 1], -kn[0, 0])
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

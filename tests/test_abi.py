@@ -28,7 +28,7 @@ def declared_symbols():
 
 def test_every_declared_symbol_is_exported(hk):
     names = declared_symbols()
-    assert len(names) == 14, names
+    assert len(names) == 15, names
     for n in names:
         assert hasattr(hk.lib, n), n
     nm = os.popen(f"nm -D --defined-only {hk.LIB_PATH}").read()
@@ -106,3 +106,26 @@ def test_valid_call_without_gpu_fails_cleanly(hk):
     s = _tier(hk, 1000)
     code = hk.lib.hkv_score(C.byref(prob.c()), 0x1000, C.byref(s), 0x40000, 1000, 0x100000, 1 << 30, None)
     assert code == 3  # HKV_ERR_CUDA, not a crash
+
+
+def test_append_validates_on_the_host(hk):
+    """hkv_append refuses bad arguments before launching anything."""
+    prob = _prob(hk)
+    d, s = _tier(hk, 64), _tier(hk, 1000, addr=0x40000000)
+    ws, kn, vn, head = C.c_void_p(0x500000), C.c_void_p(0x600000), C.c_void_p(0x700000), C.c_void_p(0x800000)
+
+    def call(kn=kn, vn=vn, dense=d, head=head, sparse=s, ws=ws, ws_bytes=256):
+        return hk.STATUS[hk.lib.hkv_append(C.byref(prob.c()), kn, vn, dense and C.byref(dense), head,
+                                           sparse and C.byref(sparse), None, ws, ws_bytes, None)]
+
+    assert call(head=None) == "HKV_ERR_INVALID_ARG"            # a window needs its head
+    assert call(kn=C.c_void_p(0x600008)) == "HKV_ERR_INVALID_ARG"  # new rows 16-byte aligned
+    assert call(vn=None) == "HKV_ERR_INVALID_ARG"
+    assert call(ws_bytes=128) == "HKV_ERR_WORKSPACE"
+    assert call(ws=C.c_void_p(0x500010)) == "HKV_ERR_WORKSPACE"
+    assert call(ws=None) == "HKV_ERR_WORKSPACE"
+    bad = _tier(hk, 64)
+    bad.stride_t = 100                                         # 200-byte rows: not 16-byte multiples
+    assert call(dense=bad) == "HKV_ERR_INVALID_ARG"
+    assert hk.STATUS[hk.lib.hkv_append(C.byref(_prob(hk, D=96).c()), kn, vn, C.byref(d), head, C.byref(s),
+                                       None, ws, 256, None)] == "HKV_ERR_UNSUPPORTED"

@@ -76,3 +76,37 @@ def test_mutant_is_caught(name, src_text, tmp_path, monkeypatch):
             caught.append((pin.__name__, type(e).__name__))
             break
     assert caught, f"mutant {name} passed every pin"
+
+
+# ---- the numpy append (TS 2.A pipeline step 1): planted mistakes in copies of it ----
+
+APPEND_MUTANTS = {
+    "head_not_advanced": ("hd[u] = (hd[u] + 1) % wcap", "hd[u] = hd[u] % wcap"),
+    "newest_ages_out": ("old_k, old_v = dk[b, h, hd[u]].copy(), dv[b, h, hd[u]].copy()",
+                        "old_k, old_v = k_new[b, h], v_new[b, h]"),
+    "sparse_full_one_early": ("if slen[u] < ncap:", "if slen[u] < ncap - 1:"),
+    "window_never_fills": ("if dlen[u] < wcap:", "if dlen[u] < wcap - 1:"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(APPEND_MUTANTS))
+def test_append_mutant_is_caught(name, monkeypatch):
+    import inspect
+    import textwrap
+
+    import oracle
+    from tests import pins
+
+    src = textwrap.dedent(inspect.getsource(oracle.append))
+    old, new = APPEND_MUTANTS[name]
+    assert old in src, name
+    ns = dict(vars(oracle))
+    exec(compile(src.replace(old, new), "<mutant>", "exec"), ns)
+    monkeypatch.setattr(oracle, "append", ns["append"])
+    failed = False
+    for pin in (pins.pin_append_matches_list_model, pins.pin_append_without_window_goes_to_sparse):
+        try:
+            pin()
+        except Exception:
+            failed = True
+    assert failed, f"mutant {name} passed every append pin"
