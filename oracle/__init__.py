@@ -4,9 +4,11 @@ TEST INFRASTRUCTURE ONLY. Only ``tests/``, ``__graft_entry__.smoke()`` and the
 benchmark's CPU-baseline leg import this package. The CUDA library and its
 Python binding never import it; the two implementations share no code.
 
-The arithmetic lives in ``hkv_oracle.c`` (plain C, IEEE double); this module
-only marshals arrays. bf16 tensors travel as their raw 16-bit patterns
-(``numpy.uint16``); fp32 tensors as ``numpy.float32``.
+The arithmetic of S1-S5 lives in ``hkv_oracle.c`` (plain C, IEEE double) and
+this module only marshals arrays for it; the KV append and the fitted
+temperature, further down, are plain numpy (float64 for the arithmetic).
+bf16 tensors travel as their raw 16-bit patterns (``numpy.uint16``); fp32
+tensors as ``numpy.float32``.
 """
 from __future__ import annotations
 
@@ -284,3 +286,92 @@ def append(k_new: np.ndarray, v_new: np.ndarray, dense: Tier, head: np.ndarray, 
                 dv[b, h, hd[u]] = v_new[b, h]
                 hd[u] = (hd[u] + 1) % wcap
     return Tier(dk, dv, dlen), hd, Tier(sk, sv, slen), dropped
+
+
+# ---- Fitted temperature: group-averaged raw-attention entropy and the beta that meets it ----
+#
+# [TS 2.B] Logits Calibration maps an importance metric onto a softmax
+# distribution "by adjusting the temperature"; [TS 3] says the mapping goes
+# onto the raw attention distribution; [TS 2.A] Tier 2 sets each head's budget
+# from its attention entropy. Reading taken: the target of unit u is the mean,
+# over the G query heads of its group, of the entropy (natural log) of each
+# head's raw attention softmax(scale q_g . k_j) over the unit's sparse tokens;
+# the fitted inverse temperature is the beta in [0, FIT_BETA_MAX] at which the
+# calibrated distribution softmax(beta z) of the unit's metric z has that
+# entropy. The entropy of softmax(beta z) does not increase with beta (its
+# derivative is -beta Var(z)), so the root is unique wherever z is not
+# constant. Degenerate units (n <= 1, or every score equal) get beta = 1.
+
+FIT_BETA_MAX = 64.0
+
+
+def _f64(a: np.ndarray) -> np.ndarray:
+    """Exact float64 values of bf16 bit patterns (uint16) or float32 arrays."""
+    if a.dtype == np.uint16:
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)
+
+
+def softmax_entropy(x: np.ndarray) -> float:
+    """Entropy (nats) of softmax(x) for a 1-D float64 array, 0 log 0 = 0."""
+    x = np.asarray(x, np.float64)
+    if x.size == 0:
+        return 0.0
+    w = np.exp(x - x.max())
+    P = w / w.sum()
+    nz = P > 0
+    return float(-(P[nz] * np.log(P[nz])).sum())
+
+
+def attention_entropy(q: np.ndarray, sparse: Tier, scale: float) -> np.ndarray:
+    """Per unit: mean over the group's query heads of the entropy of their raw
+    attention over the sparse tier. q: [B, Hq, D]. Returns float64 [B*Hkv]
+    (0 for an empty unit)."""
+    B, Hq, D = q.shape
+    Hkv = sparse.k.shape[1]
+    G = Hq // Hkv
+    qf = _f64(q)
+    kf = _f64(sparse.k)
+    out = np.zeros(B * Hkv, np.float64)
+    for b in range(B):
+        for h in range(Hkv):
+            u = b * Hkv + h
+            n = int(sparse.len[u])
+            if n == 0:
+                continue
+            logits = scale * (qf[b, h * G:(h + 1) * G] @ kf[b, h, :n].T)  # [G, n]
+            out[u] = np.mean([softmax_entropy(logits[g]) for g in range(G)])
+    return out
+
+
+def fit_temperature(z: np.ndarray, length: np.ndarray, h_target: np.ndarray,
+                    beta_max: float = FIT_BETA_MAX) -> np.ndarray:
+    """Per unit the beta in [0, beta_max] with entropy(softmax(beta z)) equal
+    to h_target[u], by bisection in float64 on the monotone entropy. A target
+    at or above ln n gives 0; one below the entropy at beta_max gives beta_max.
+    z: [units, >= n] scores. Returns float64 [units]."""
+    units = len(length)
+    beta = np.ones(units, np.float64)
+    for u in range(units):
+        n = int(length[u])
+        zu = _f64(np.asarray(z[u, :n]))
+        if n <= 1 or zu.max() == zu.min():
+            continue
+        t = float(h_target[u])
+        if t >= np.log(n):
+            beta[u] = 0.0
+            continue
+        if softmax_entropy(beta_max * zu) >= t:
+            beta[u] = beta_max
+            continue
+        lo, hi = 0.0, beta_max  # entropy(lo) > t > entropy(hi)
+        for _ in range(200):
+            mid = 0.5 * (lo + hi)
+            if mid <= lo or mid >= hi:
+                break
+            if softmax_entropy(mid * zu) > t:
+                lo = mid
+            else:
+                hi = mid
+        beta[u] = 0.5 * (lo + hi)
+    return beta

@@ -475,4 +475,119 @@ def pin_append_without_window_goes_to_sparse():
     assert np.array_equal(s2.k[0, 0, 1], kn[0, 0]) and np.array_equal(s2.v[0, 0, 1], -kn[0, 0])
 
 
+# ---- Fitted temperature (TS 2.B, TS 3, TS 2.A Tier 2 "attention entropy") ----------------
+
+
+def _entropy_ref(x):
+    """Entropy of softmax(x) by library routines (scipy), not the oracle's code."""
+    import scipy.special as sps
+    import scipy.stats as sst
+
+    return float(sst.entropy(sps.softmax(np.asarray(x, np.float64))))
+
+
+def pin_attention_entropy_matches_scipy():
+    """Group-averaged raw-attention entropy against torch float64 logits and
+    scipy's softmax and entropy, on bf16 (exact widening by torch) and fp32
+    inputs with GQA groups and ragged lengths."""
+    import torch
+
+    rng = np.random.default_rng(21)
+    # the last case has logits spread over hundreds (exp overflows without the max shift)
+    for dt, spread in ((torch.bfloat16, 2.0), (torch.float32, 2.0), (torch.float32, 400.0)):
+        B, Hkv, G, D, cap = 2, 2, 4, 16, 40
+        q = torch.as_tensor(rng.standard_normal((B, Hkv * G, D)), dtype=torch.float32).to(dt)
+        k = torch.as_tensor(rng.standard_normal((B, Hkv, cap, D)) * spread, dtype=torch.float32).to(dt)
+        ln = np.array([40, 17, 1, 0], np.int32)
+        scale = 0.3
+        def host(x):
+            return x.view(torch.int16).numpy().view(np.uint16) if x.dtype == torch.bfloat16 else x.numpy()
+
+        t = oracle.Tier(host(k), host(k), ln)
+        got = oracle.attention_entropy(host(q), t, scale)
+        qd, kd = q.double(), k.double()
+        for u in range(B * Hkv):
+            b, h = divmod(u, Hkv)
+            n = int(ln[u])
+            if n == 0:
+                assert got[u] == 0.0
+                continue
+            lg = scale * torch.einsum("gd,nd->gn", qd[b, h * G:(h + 1) * G], kd[b, h, :n]).numpy()
+            want = np.mean([_entropy_ref(lg[g]) for g in range(G)])
+            assert abs(got[u] - want) <= 1e-12 * max(1.0, want), (dt, u, got[u], want)
+
+
+def pin_attention_entropy_of_equal_keys_is_log_n():
+    """Keys all equal: every head attends uniformly, so the entropy is ln n."""
+    B, Hkv, G, D, n = 1, 1, 2, 8, 37
+    q = np.random.default_rng(3).standard_normal((B, Hkv * G, D)).astype(np.float32)
+    k = np.tile(np.linspace(-1, 1, D, dtype=np.float32), (B, Hkv, n, 1))
+    got = oracle.attention_entropy(q, oracle.Tier(k, k, np.array([n], np.int32)), 1.0)
+    assert abs(got[0] - np.log(n)) < 1e-12
+
+
+def pin_fit_identical_heads_gives_one():
+    """A group of identical query heads: the max-pooled logits are each head's
+    raw logits, so the temperature that matches their entropy is 1."""
+    rng = np.random.default_rng(5)
+    B, Hkv, G, D, cap = 1, 2, 4, 32, 300
+    q1 = rng.standard_normal((B, Hkv, 1, D)).astype(np.float32)
+    q = np.repeat(q1, G, axis=2).reshape(B, Hkv * G, D)
+    k = (rng.standard_normal((B, Hkv, cap, D)) * 1.5).astype(np.float32)
+    ln = np.array([300, 123], np.int32)
+    t = oracle.Tier(k, k, ln)
+    scale = 1.0 / np.sqrt(D)
+    z = np.einsum("bhd,bhnd->bhn", q1[:, :, 0].astype(np.float64), k.astype(np.float64)).reshape(B * Hkv, cap)
+    beta = oracle.fit_temperature(scale * z, ln, oracle.attention_entropy(q, t, scale))
+    assert np.all(np.abs(beta - 1.0) < 1e-9), beta
+
+
+def pin_fit_two_tokens_closed_form():
+    """Two tokens a gap d apart: softmax(beta z) is Bernoulli(1/(1+e^(-beta d))),
+    whose entropy is the binary entropy; the fit inverts it."""
+    for d, b0 in ((1.0, 0.5), (3.0, 2.25), (0.2, 9.0), (5.0, 0.01)):
+        pr = 1.0 / (1.0 + np.exp(-b0 * d))
+        h = -(pr * np.log(pr) + (1 - pr) * np.log(1 - pr))
+        beta = oracle.fit_temperature(np.array([[0.0, d]]), np.array([2]), np.array([h]))
+        assert abs(beta[0] - b0) < 1e-9 * max(1.0, b0), (d, b0, beta)
+
+
+def pin_fit_matches_brentq():
+    """Random metrics and reachable targets: the same root as scipy's brentq on
+    scipy's entropy of scipy's softmax."""
+    from scipy.optimize import brentq
+
+    rng = np.random.default_rng(9)
+    units, cap = 6, 500
+    z = (rng.standard_normal((units, cap)) * rng.uniform(0.2, 3.0, (units, 1))).astype(np.float32)
+    ln = np.array([500, 2, 77, 300, 499, 10], np.int32)
+    tgt = np.array([rng.uniform(0.05, 0.95) * np.log(n) for n in ln])
+    beta = oracle.fit_temperature(z, ln, tgt)
+    for u in range(units):
+        zu = z[u, :ln[u]].astype(np.float64)
+        f = lambda b: _entropy_ref(b * zu) - tgt[u]
+        if f(oracle.FIT_BETA_MAX) > 0:
+            assert beta[u] == oracle.FIT_BETA_MAX
+            continue
+        want = brentq(f, 0.0, oracle.FIT_BETA_MAX, xtol=1e-14, rtol=1e-14)
+        assert abs(beta[u] - want) < 1e-9 * max(1.0, want), (u, beta[u], want)
+
+
+def pin_fit_boundaries_and_order():
+    """Targets at or above ln n give 0; below the entropy at the largest beta
+    give that beta; n <= 1 and constant metrics give 1; a larger target never
+    gives a larger beta."""
+    z = np.array([[0.0, 1.0, 3.0, 3.0, -2.0], [1.0, 1.0, 1.0, 1.0, 1.0], [4.0, 0, 0, 0, 0]])
+    n = np.array([5, 5, 1])
+    b = oracle.fit_temperature(z, n, np.array([np.log(5) + 1e-3, 0.3, 0.0]))
+    assert list(b) == [0.0, 1.0, 1.0]
+    b = oracle.fit_temperature(z[:1], n[:1], np.array([1e-30]))
+    assert b[0] == oracle.FIT_BETA_MAX
+    ts = np.linspace(0.75, 1.55, 9)
+    bs = [oracle.fit_temperature(z[:1], n[:1], np.array([t]))[0] for t in ts]
+    assert all(x > y for x, y in zip(bs, bs[1:])), bs
+    # ties at the top: the entropy falls to ln 2, not 0, so a lower target is out of reach
+    assert oracle.fit_temperature(z[:1], n[:1], np.array([np.log(2) - 1e-6]))[0] == oracle.FIT_BETA_MAX
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

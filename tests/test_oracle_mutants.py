@@ -110,3 +110,43 @@ def test_append_mutant_is_caught(name, monkeypatch):
         except Exception:
             failed = True
     assert failed, f"mutant {name} passed every append pin"
+
+
+# ---- the numpy fitted temperature (TS 2.B, TS 3): planted mistakes in copies of it ----
+
+FIT_MUTANTS = {
+    "entropy_in_bits": ("softmax_entropy", "np.log(P[nz])", "np.log2(P[nz])"),
+    "entropy_sign": ("softmax_entropy", "-(P[nz] * np.log(P[nz])).sum()", "(P[nz] * np.log(P[nz])).sum()"),
+    "softmax_without_max": ("softmax_entropy", "w = np.exp(x - x.max())", "w = np.exp(x - x.min())"),
+    "max_over_heads": ("attention_entropy", "np.mean([softmax_entropy", "np.max([softmax_entropy"),
+    "wrong_group": ("attention_entropy", "qf[b, h * G:(h + 1) * G]", "qf[b, h:h + G]"),
+    "scale_dropped": ("attention_entropy", "logits = scale * (", "logits = ("),
+    "bisection_flipped": ("fit_temperature", "> t:\n                lo = mid", "< t:\n                lo = mid"),
+    "temperature_not_inverse": ("fit_temperature", "softmax_entropy(mid * zu)", "softmax_entropy(zu / mid)"),
+    "lower_bound_missing": ("fit_temperature", "if t >= np.log(n):", "if t > np.log(n) + 1.0:"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(FIT_MUTANTS))
+def test_fit_mutant_is_caught(name, monkeypatch):
+    import inspect
+    import textwrap
+
+    import oracle
+    from tests import pins
+
+    fn, old, new = FIT_MUTANTS[name]
+    src = textwrap.dedent(inspect.getsource(getattr(oracle, fn)))
+    assert old in src, name
+    ns = dict(vars(oracle))
+    exec(compile(src.replace(old, new), "<mutant>", "exec"), ns)
+    monkeypatch.setattr(oracle, fn, ns[fn])
+    failed = False
+    for pin in (pins.pin_attention_entropy_matches_scipy, pins.pin_attention_entropy_of_equal_keys_is_log_n,
+                pins.pin_fit_identical_heads_gives_one, pins.pin_fit_two_tokens_closed_form,
+                pins.pin_fit_matches_brentq, pins.pin_fit_boundaries_and_order):
+        try:
+            pin()
+        except Exception:
+            failed = True
+    assert failed, f"mutant {name} passed every fitted-temperature pin"
