@@ -409,6 +409,17 @@ def run_ours(args):
                                                     out.out, ws, lse=out.lse) for x, prob, tiers, out in sets],
                         NSETS, stream, args)
     attn_ms = max_over_ranks(attn_ms, dist, device)
+    # the step with the fitted temperature (beta per unit solved before the
+    # selection), same rotation of decode states
+    fit_outs = []
+    for x, prob, tiers, out in sets:
+        fo = hkv.StepOutputs.allocate(prob, tiers[1], device)
+        fo.beta_fit = torch.zeros(wl.units, device=device)
+        fit_outs.append(fo)
+    fitted_ms = kernel_ms(lambda: [hkv.step(prob, x.q, *tiers, fo, ws)
+                                   for (x, prob, tiers, out), fo in zip(sets, fit_outs)], NSETS, stream, args)
+    fitted_ms = max_over_ranks(fitted_ms, dist, device)
+    del fit_outs
     # KV append with the dense-window roll, timed on copies of one decode state
     # whose sparse tiers keep room for every append of the timing (so each
     # launch moves a full window row into the sparse tier)
@@ -438,6 +449,7 @@ def run_ours(args):
                "score_us": round(score_ms * 1e3, 2), "attn_us": round(attn_ms * 1e3, 2),
                "select_compact_us_remainder": round((launch_ms_max - score_ms - attn_ms) * 1e3, 2),
                "append_us": round(append_ms * 1e3, 2),
+               "fitted_step_us": round(fitted_ms * 1e3, 2),
                "append_bytes": int(append_bytes(wl))}
 
     # end to end through the public API: per step, copy the step's query and the

@@ -35,7 +35,9 @@ namespace hkv {
 // written; per streaming warp g,
 // TR_SW + 4g (scoring) or TR_AW + 4g (attention) + i: 0 pipeline start,
 // 1 first stage landed, 2 pipeline done, 3 kernel entry (attention).
-[[maybe_unused]] constexpr int TR_SEL = 250000, TR_SW = 0, TR_AW = 20000;
+// Per unit u of the fitting kernel, TR_FIT + 16u + i: 0 start, 1 entropy
+// done, 2 scores staged, 3 beta found; 4 holds the number of evaluations.
+[[maybe_unused]] constexpr int TR_SEL = 250000, TR_SW = 0, TR_AW = 20000, TR_FIT = 240000;
 
 // =============================================================================
 // Kernels
@@ -299,6 +301,44 @@ __global__ void __launch_bounds__(NT) k_calibrate(const __grid_constant__ Params
         calibrate_unit<true>(P, sm, c, u, n, sm.zs);
     else
         calibrate_unit<false>(P, sm, c, u, n, zg);
+}
+
+// Fitted temperature, one unit per CTA: the target entropy from the scorer's
+// per-head logit records (when P.logit is set; else P.h_target), then, when
+// P.beta_out is set, the inverse temperature that meets it on the unit's
+// scores P.z.
+template <int G>
+__global__ void __launch_bounds__(NT, 1) k_fit(const __grid_constant__ Params P)
+{
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    FSmem &sm = *reinterpret_cast<FSmem *>(smem_raw);
+    const Ctl c = make_ctl(P);
+    const int u = blockIdx.x;
+    allow_dependents();
+    wait_prior_grid();
+    const int n = tier_len(P.sparse, u, c);
+    HKV_TRACE_AT(TR_FIT + 16 * u);
+    float target;
+    if (P.logit != nullptr) {
+        target = unit_attention_entropy<G>(P.logit + (int64_t)u * P.sparse.cap * logit_floats(G), n, sm);
+        if (P.h_out != nullptr && threadIdx.x == 0)
+            P.h_out[u] = target;
+    } else {
+        target = __ldcg(P.h_target + u);
+    }
+    HKV_TRACE_AT(TR_FIT + 16 * u + 1);
+    if (P.beta_out == nullptr)
+        return;
+    const float *zg = P.z + (int64_t)u * P.z_stride;
+    const bool staged = stage_scores(zg, n, sm);
+    HKV_TRACE_AT(TR_FIT + 16 * u + 2);
+    int evals = 0;
+    const float beta = staged ? fit_unit<true>(sm.zs, n, target, sm, c, &evals)
+                              : fit_unit<false>(zg, n, target, sm, c, &evals);
+    HKV_TRACE_AT(TR_FIT + 16 * u + 3);
+    HKV_TRACE_VAL(TR_FIT + 16 * u + 4, evals);
+    if (threadIdx.x == 0)
+        P.beta_out[u] = beta;
 }
 
 // FLAT_SUM rows and Rewrite Cache copies after the step's PAD_MAX compaction
@@ -610,6 +650,14 @@ struct RunAttn {
     }
 };
 
+template <int ES, int D, int G>
+struct RunFit {
+    static hkv_status run(const Params &P, cudaStream_t s, bool pdl)
+    {
+        return launch(k_fit<G>, P.units, NT, sizeof(FSmem), s, P, pdl);
+    }
+};
+
 static hkv_status launch_unit(const hkv_problem *prob, const Params &P, cudaStream_t s, bool pdl)
 {
     if (prob->dtype == HKV_BF16)
@@ -860,6 +908,9 @@ hkv_status hkv_step(const hkv_problem *prob, const void *q, const hkv_tier *dens
         return HKV_ERR_INVALID_ARG;
     if (o->z && !aligned(o->z, 4))
         return HKV_ERR_INVALID_ARG;
+    if ((o->h_attn != nullptr && o->beta_fit == nullptr) || (o->beta_fit && !aligned(o->beta_fit, 4)) ||
+        (o->h_attn && !aligned(o->h_attn, 4)))
+        return HKV_ERR_INVALID_ARG;
     if (P.units == 0)
         return HKV_OK;
     char *wsb = static_cast<char *>(ws);
@@ -888,8 +939,19 @@ hkv_status hkv_step(const hkv_problem *prob, const void *q, const hkv_tier *dens
     S.urange = reinterpret_cast<uint32_t *>(wsb + L.urange);
     if (scored && (s = dispatch<RunScore>(prob, S, st, false)) != HKV_OK)
         return s;
-    // 2. calibration, Top-p budget, cut and compaction, per unit
+    // 1b. optionally the fitted inverse temperature of every unit, from the
+    // scorer's logit records and scores; the selection then uses it
     Params U = S;
+    if (o->beta_fit != nullptr) {
+        Params F = S;
+        F.urange = nullptr;
+        F.beta_out = o->beta_fit;
+        F.h_out = o->h_attn;
+        if ((s = dispatch<RunFit>(prob, F, st, scored)) != HKV_OK)
+            return s;
+        U.inv_temp = o->beta_fit;
+    }
+    // 2. calibration, Top-p budget, cut and compaction, per unit
     U.have_range = scored;
     U.do_select = 1;
     U.do_compact = 1;
@@ -904,6 +966,56 @@ hkv_status hkv_step(const hkv_problem *prob, const void *q, const hkv_tier *dens
     if (prob->dtype == HKV_BF16)
         return launch(k_flatten<2>, P.units, NT, 0, st, P, true);
     return launch(k_flatten<4>, P.units, NT, 0, st, P, true);
+}
+
+hkv_status hkv_attention_entropy(const hkv_problem *prob, const void *q, const hkv_tier *sparse, float *h, void *ws,
+                                 size_t ws_bytes, hkv_stream_t stream)
+{
+    WsLayout L;
+    Params P;
+    if (sparse == nullptr)
+        return HKV_ERR_INVALID_ARG;
+    hkv_status s = prologue(prob, nullptr, sparse, nullptr, false, ws, ws_bytes, &L, &P);
+    if (s != HKV_OK)
+        return s;
+    if (q == nullptr || !aligned(q, 16) || h == nullptr || !aligned(h, 4))
+        return HKV_ERR_INVALID_ARG;
+    if (P.units == 0)
+        return HKV_OK;
+    char *wsb = static_cast<char *>(ws);
+    const cudaStream_t st = (cudaStream_t)stream;
+    P.q = static_cast<const char *>(q);
+    P.z = reinterpret_cast<float *>(wsb + L.zbuf);
+    P.z_stride = L.z_stride;
+    P.logit = reinterpret_cast<float *>(wsb + L.logits);
+    const bool scored = sparse->cap > 0;
+    if (scored && (s = dispatch<RunScore>(prob, P, st, false)) != HKV_OK)
+        return s;
+    P.h_out = h;
+    return dispatch<RunFit>(prob, P, st, scored);
+}
+
+hkv_status hkv_fit_temperature(const hkv_problem *prob, const float *z, int64_t z_stride, const hkv_tier *sparse,
+                               const float *h_target, float *beta, void *ws, size_t ws_bytes, hkv_stream_t stream)
+{
+    WsLayout L;
+    Params P;
+    if (sparse == nullptr)
+        return HKV_ERR_INVALID_ARG;
+    hkv_status s = prologue(prob, nullptr, sparse, nullptr, false, ws, ws_bytes, &L, &P);
+    if (s != HKV_OK)
+        return s;
+    if (h_target == nullptr || !aligned(h_target, 4) || beta == nullptr || !aligned(beta, 4))
+        return HKV_ERR_INVALID_ARG;
+    if (sparse->cap > 0 && (z == nullptr || !aligned(z, 4) || z_stride < sparse->cap))
+        return HKV_ERR_INVALID_ARG;
+    if (P.units == 0)
+        return HKV_OK;
+    P.z = const_cast<float *>(z);
+    P.z_stride = z_stride;
+    P.h_target = h_target;
+    P.beta_out = beta;
+    return dispatch<RunFit>(prob, P, (cudaStream_t)stream, false);
 }
 
 }  // extern "C"
@@ -1063,24 +1175,21 @@ __global__ void __launch_bounds__(APPEND_WARPS * 32) k_append(const __grid_const
     const bool age_out = !room;              // a token leaves the window (or bypasses it)
     const bool keep = age_out && n < A.ncap; // ... and finds room in the sparse tier
     const int dslot = room ? W : hd;
-    char *drow[2], *srow[2];
-    const char *nrow[2] = {A.k_new + (int64_t)u * A.chunks * 16, A.v_new + (int64_t)u * A.chunks * 16};
+    const int64_t noff = (int64_t)u * A.chunks * 16;
     const int64_t doff = (int64_t)b * A.dsb + (int64_t)h * A.dsh + (int64_t)dslot * A.dst;
     const int64_t soff = (int64_t)b * A.ssb + (int64_t)h * A.ssh + (int64_t)n * A.sst;
-    drow[0] = A.dk + doff;
-    drow[1] = A.dv + doff;
-    srow[0] = A.sk + soff;
-    srow[1] = A.sv + soff;
     for (int c = lane; c < 2 * A.chunks; c += 32) {
-        const int kv = c >= A.chunks, off = (c - kv * A.chunks) * 16;
-        const uint4 fresh = __ldg(reinterpret_cast<const uint4 *>(nrow[kv] + off));
+        const bool isv = c >= A.chunks;
+        const int off = (c - (isv ? A.chunks : 0)) * 16;
+        const uint4 fresh = __ldg(reinterpret_cast<const uint4 *>((isv ? A.v_new : A.k_new) + noff + off));
+        uint4 *srow = reinterpret_cast<uint4 *>((isv ? A.sv : A.sk) + soff + off);
         if (A.wcap > 0) {
-            uint4 *slot = reinterpret_cast<uint4 *>(drow[kv] + off);
+            uint4 *slot = reinterpret_cast<uint4 *>((isv ? A.dv : A.dk) + doff + off);
             if (keep)
-                *reinterpret_cast<uint4 *>(srow[kv] + off) = *slot;  // the oldest row moves on
+                *srow = *slot;  // the oldest row moves on
             *slot = fresh;
         } else if (keep) {
-            *reinterpret_cast<uint4 *>(srow[kv] + off) = fresh;
+            *srow = fresh;
         }
     }
     if (lane == 0) {

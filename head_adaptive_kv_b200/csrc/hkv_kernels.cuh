@@ -76,6 +76,10 @@ struct Params {
     int32_t have_range;   // per-unit kernel: urange holds the units' score ranges
     int32_t do_select, do_compact;  // per-unit kernel: which steps to run
     int32_t withhold;     // fault injection: streaming warps never arm their stages
+    // fitted temperature: per-unit entropy target in (nullptr: from the logit
+    // records), target out, fitted inverse temperature out
+    const float *h_target;
+    float *h_out, *beta_out;
     uint64_t wait_ns;
 };
 
@@ -1342,8 +1346,8 @@ struct Selection {
 };
 
 // Largest and smallest finite score of a unit.
-template <bool ZS>
-__device__ void unit_range(const float *zu, int n, float *m, float *zlo, USmem &sm)
+template <bool ZS, class SM>
+__device__ void unit_range(const float *zu, int n, float *m, float *zlo, SM &sm)
 {
     float mx = -INFINITY, mn = INFINITY;
     sweep_scores<ZS>(zu, n, [&](float z, int, bool valid) {
@@ -1359,7 +1363,8 @@ __device__ void unit_range(const float *zu, int n, float *m, float *zlo, USmem &
 
 // Copy a unit's n <= ZSTAGE scores into shared memory (all loads in flight);
 // longer units stay in global memory. Returns whether they were staged.
-__device__ bool stage_scores(const float *zu, int n, USmem &sm)
+template <class SM>
+__device__ bool stage_scores(const float *zu, int n, SM &sm)
 {
     if (n > ZSTAGE)
         return false;
@@ -2156,6 +2161,278 @@ __device__ void compact_unit(const float *zu, int n, uint32_t cut_key, int n_tie
     }
     for (int i = k + threadIdx.x; i < pad; i += NT)
         row[i] = -1;
+}
+
+// =============================================================================
+// Fitted temperature ([TS 2.B] calibration by temperature, [TS 3] onto the raw
+// attention distribution, [TS 2.A] Tier 2 budgets from attention entropy)
+//
+// Per unit: the target entropy is the mean over the group's query heads of
+// the entropy of each head's raw attention softmax(scale q_g . k_j) over the
+// sparse tokens; the fitted inverse temperature beta in [0, FIT_BETA_MAX] is
+// the root of H(beta) = target, H(beta) the entropy of softmax(beta z). H does
+// not increase with beta (dH/dbeta = -beta Var(z)); the root is found by
+// Newton steps kept inside a shrinking bracket (bisection when a step leaves
+// it). Sums in double, exponentials on the SFU.
+// =============================================================================
+
+constexpr float FIT_BETA_MAX = 64.0f;
+
+struct __align__(16) FSmem {  // shared memory of the fitting kernel
+    float zs[ZSTAGE];
+    float redf[NT / 32];
+    float redv[8 * (NT / 32)];
+    double redd[16 * (NT / 32)];  // up to 2 G = 16 sums per thread
+};
+
+// Per-lane vectors summed (double) or maxed (float) over the CTA; every thread
+// gets the result. The sums run in a fixed order.
+template <int K>
+__device__ __forceinline__ void block_sum_vec(double (&v)[K], double *scratch)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int NW = NT / 32;
+#pragma unroll
+    for (int i = 0; i < K; ++i) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            v[i] += __shfl_xor_sync(0xffffffffu, v[i], o);
+        if (lane == 0)
+            scratch[i * NW + warp] = v[i];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < K; ++i) {
+        double r = 0.0;
+#pragma unroll
+        for (int w = 0; w < NW; ++w)
+            r += scratch[i * NW + w];
+        v[i] = r;
+    }
+    __syncthreads();
+}
+
+template <int K>
+__device__ __forceinline__ void block_max_vec(float (&v)[K], float *scratch)
+{
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int NW = NT / 32;
+#pragma unroll
+    for (int i = 0; i < K; ++i) {
+        v[i] = warp_max(v[i]);
+        if (lane == 0)
+            scratch[i * NW + warp] = v[i];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < K; ++i) {
+        float r = scratch[i * NW];
+#pragma unroll
+        for (int w = 1; w < NW; ++w)
+            r = fmaxf(r, scratch[i * NW + w]);
+        v[i] = r;
+    }
+    __syncthreads();
+}
+
+// The G per-head logits of one record (float4 loads; LG is a multiple of 4).
+template <int G>
+__device__ __forceinline__ void load_record(const float *p, float (&x)[G])
+{
+#pragma unroll
+    for (int c = 0; c < (G + 3) / 4; ++c) {
+        const float4 r = __ldcg(reinterpret_cast<const float4 *>(p) + c);
+        if (4 * c + 0 < G)
+            x[4 * c + 0] = r.x;
+        if (4 * c + 1 < G)
+            x[4 * c + 1] = r.y;
+        if (4 * c + 2 < G)
+            x[4 * c + 2] = r.z;
+        if (4 * c + 3 < G)
+            x[4 * c + 3] = r.w;
+    }
+}
+
+// Mean over the G heads of the entropy of softmax over a unit's n per-head
+// logit records (record j at rec + j * LG, head g at offset g), in one pass:
+// each thread keeps per head a running maximum m, Z = sum exp(l - m) and
+// S = sum exp(l - m) (l - m), rescaled when m grows (by batches of records,
+// all of a batch's loads in flight at once); the threads' triples are then
+// brought to the CTA's maximum and summed in double. H = ln Z - S / Z.
+template <int G>
+__device__ float unit_attention_entropy(const float *rec, int n, FSmem &sm)
+{
+    constexpr int LG = logit_floats(G);
+    constexpr int BATCH = G >= 8 ? 4 : 8;
+    if (n <= 0)
+        return 0.0f;
+    float m[G], Z[G], S[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        m[g] = -INFINITY;
+        Z[g] = 0.0f;
+        S[g] = 0.0f;
+    }
+#pragma unroll 1
+    for (int j0 = threadIdx.x; j0 < n; j0 += NT * BATCH) {
+        float x[BATCH][G];
+#pragma unroll
+        for (int b = 0; b < BATCH; ++b) {
+            const int j = j0 + b * NT;
+            if (j < n) {
+                load_record<G>(rec + (int64_t)j * LG, x[b]);
+            } else {
+#pragma unroll
+                for (int g = 0; g < G; ++g)
+                    x[b][g] = -INFINITY;
+            }
+        }
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            float bm = x[0][g];
+#pragma unroll
+            for (int b = 1; b < BATCH; ++b)
+                bm = fmaxf(bm, x[b][g]);
+            if (bm > m[g]) {  // rescale the running sums to the new maximum
+                if (Z[g] > 0.0f) {
+                    const float dm = m[g] - bm;
+                    const float r = ex2(dm * LOG2E);
+                    S[g] = r * (S[g] + Z[g] * dm);
+                    Z[g] *= r;
+                }
+                m[g] = bm;
+            }
+#pragma unroll
+            for (int b = 0; b < BATCH; ++b) {
+                const float d = x[b][g] - m[g];
+                const float e = d == 0.0f ? 1.0f : ex2(d * LOG2E);
+                if (e > 0.0f) {
+                    Z[g] += e;
+                    S[g] += e * d;
+                }
+            }
+        }
+    }
+    float M[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+        M[g] = m[g];
+    block_max_vec<G>(M, sm.redv);
+    double acc[2 * G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+        acc[2 * g] = 0.0;
+        acc[2 * g + 1] = 0.0;
+        if (Z[g] > 0.0f) {
+            const float dm = m[g] - M[g];
+            const float r = dm == 0.0f ? 1.0f : ex2(dm * LOG2E);
+            acc[2 * g] = (double)(Z[g] * r);
+            acc[2 * g + 1] = (double)r * ((double)S[g] + (double)Z[g] * (double)dm);
+        }
+    }
+    block_sum_vec<2 * G>(acc, sm.redd);
+    double h = 0.0;
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+        h += log(acc[2 * g]) - acc[2 * g + 1] / acc[2 * g];
+    return (float)(h / G);
+}
+
+// Entropy of softmax(beta z) over a unit and its derivative in beta. Thread t
+// takes the quads t, t + NT, ... of the scores and sums each of a quad's four
+// positions into its own fp32 accumulators (about n / (4 NT) terms each, so
+// their rounding stays near 1e-7 relative); the CTA sums in double.
+template <bool ZS>
+__device__ __forceinline__ void fit_eval(const float *zu, int n, float m, float beta, FSmem &sm, double *H,
+                                         double *dH)
+{
+    const float bl2 = beta * LOG2E;
+    const bool vec = ZS || (((uintptr_t)zu) & 15) == 0;
+    float a[4][3];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        a[i][0] = a[i][1] = a[i][2] = 0.0f;
+#pragma unroll 2
+    for (int j = 4 * (int)threadIdx.x; j < n; j += 4 * NT) {
+        float v[4];
+        if (vec && j + 4 <= n) {
+            const float4 t = ZS ? lds4(zu + j) : __ldcg(reinterpret_cast<const float4 *>(zu + j));
+            v[0] = t.x;
+            v[1] = t.y;
+            v[2] = t.z;
+            v[3] = t.w;
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                v[i] = j + i < n ? (ZS ? lds1(zu + j + i) : __ldcg(zu + j + i)) : -INFINITY;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float d = v[i] - m;
+            const float w = d == 0.0f ? 1.0f : ex2(d * bl2);
+            if (w > 0.0f) {
+                const float wd = w * d;
+                a[i][0] += w;
+                a[i][1] += wd;
+                a[i][2] = fmaf(wd, d, a[i][2]);
+            }
+        }
+    }
+    double acc[3];
+#pragma unroll
+    for (int k = 0; k < 3; ++k)
+        acc[k] = ((double)a[0][k] + (double)a[1][k]) + ((double)a[2][k] + (double)a[3][k]);
+    block_sum_vec<3>(acc, sm.redd);
+    const double mean = acc[1] / acc[0];
+    *H = log(acc[0]) - (double)beta * mean;
+    *dH = -(double)beta * (acc[2] / acc[0] - mean * mean);
+}
+
+// The fitted inverse temperature of one unit (see the section comment).
+template <bool ZS>
+__device__ float fit_unit(const float *zu, int n, float target, FSmem &sm, const Ctl &c, int *evals)
+{
+    float m, zlo;
+    unit_range<ZS>(zu, n, &m, &zlo, sm);
+    if (n <= 1 || !(m > zlo))
+        return 1.0f;  // every beta gives the same distribution
+    if (target != target) {
+        if (threadIdx.x == 0)
+            raise_flag(c, HKV_DEV_BAD_TEMP);
+        return 1.0f;
+    }
+    const double t = (double)target;
+    if (t >= log((double)n))
+        return 0.0f;
+    double H, dH;
+    fit_eval<ZS>(zu, n, m, FIT_BETA_MAX, sm, &H, &dH);
+    ++*evals;
+    if (H >= t)
+        return FIT_BETA_MAX;  // sharper than the metric can get
+    // H is known to a few 1e-7 relative (the sums' rounding), so the search
+    // stops at that level: H within 2e-6 of the target, a Newton step below
+    // 1e-6 of beta, or a bracket that narrow
+    float lo = 0.0f, hi = FIT_BETA_MAX, beta = 1.0f;
+#pragma unroll 1
+    for (int it = 0; it < 40; ++it) {
+        fit_eval<ZS>(zu, n, m, beta, sm, &H, &dH);
+        ++*evals;
+        if (fabs(H - t) <= 2e-6 * fmax(1.0, t))
+            break;
+        if (H > t)
+            lo = beta;
+        else
+            hi = beta;
+        if (hi - lo <= 1e-6f * hi)
+            break;
+        float next = dH < 0.0 ? (float)((double)beta - (H - t) / dH) : -1.0f;
+        if (!(next > lo && next < hi))
+            next = 0.5f * (lo + hi);
+        else if (fabsf(next - beta) <= 1e-6f * beta)
+            return next;
+        beta = next;
+    }
+    return beta;
 }
 
 }  // namespace hkv

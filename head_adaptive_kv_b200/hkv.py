@@ -50,7 +50,8 @@ class Cut(C.Structure):
 
 class _StepOut(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in
-                ("sel_len", "idx", "offsets", "out", "lse", "z", "cut", "m", "logZ", "k_out", "v_out")]
+                ("sel_len", "idx", "offsets", "out", "lse", "z", "cut", "m", "logZ", "k_out", "v_out",
+                 "beta_fit", "h_attn")]
 
 
 def _load():
@@ -69,6 +70,8 @@ def _load():
         "hkv_step": [P, P, P, P, P, P, P, sz, P],
         "hkv_cascade_decode_noalloc": [P, P, P, P, P, P, P, P, P, P, P, P],
         "hkv_append": [P, P, P, P, P, P, P, P, sz, P],
+        "hkv_attention_entropy": [P, P, P, P, P, sz, P],
+        "hkv_fit_temperature": [P, P, i64, P, P, P, P, sz, P],
         "hkv_get_status": [P, C.POINTER(C.c_uint32), P],
         "hkv_set_wait_limit_ns": [C.c_uint64],
         "hkv_debug_withhold_publish": [i32],
@@ -241,11 +244,13 @@ class StepOutputs:
     logZ: Optional[torch.Tensor] = None
     k_out: Optional[torch.Tensor] = None
     v_out: Optional[torch.Tensor] = None
+    beta_fit: Optional[torch.Tensor] = None
+    h_attn: Optional[torch.Tensor] = None
 
     def c(self) -> _StepOut:
         return _StepOut(*[None if t is None else t.data_ptr() for t in
                           (self.sel_len, self.idx, self.offsets, self.out, self.lse, self.z, self.cut,
-                           self.m, self.logZ, self.k_out, self.v_out)])
+                           self.m, self.logZ, self.k_out, self.v_out, self.beta_fit, self.h_attn)])
 
     @staticmethod
     def allocate(prob: Problem, sparse: Tier, device, with_z=False, with_cut=False, with_stats=False,
@@ -308,6 +313,20 @@ def append(prob: Problem, k_new: torch.Tensor, v_new: torch.Tensor, dense: Optio
         raise TypeError("head must be int32")
     _check(lib.hkv_append(C.byref(prob.c()), _ptr(k_new), _ptr(v_new), _tref(dense), _ptr(head),
                           _tref(sparse), _ptr(dropped), ws.ptr, ws.nbytes, _stream(stream)), "hkv_append")
+
+
+def attention_entropy(prob: Problem, q: torch.Tensor, sparse: Tier, h: torch.Tensor, ws: Workspace, stream=None):
+    """Per unit the group-averaged entropy of the raw attention over the sparse tier (h: fp32 [B*Hkv])."""
+    _check(lib.hkv_attention_entropy(C.byref(prob.c()), _ptr(q), C.byref(sparse.c()), _ptr(h), ws.ptr,
+                                     ws.nbytes, _stream(stream)), "hkv_attention_entropy")
+
+
+def fit_temperature(prob: Problem, z: torch.Tensor, sparse: Tier, h_target: torch.Tensor, beta: torch.Tensor,
+                    ws: Workspace, stream=None):
+    """Per unit the inverse temperature at which softmax(beta z) has entropy
+    h_target (z: fp32 [B*Hkv, >= cap]; h_target, beta: fp32 [B*Hkv])."""
+    _check(lib.hkv_fit_temperature(C.byref(prob.c()), _ptr(z), z.stride(0), C.byref(sparse.c()), _ptr(h_target),
+                                   _ptr(beta), ws.ptr, ws.nbytes, _stream(stream)), "hkv_fit_temperature")
 
 
 def set_wait_limit_ns(ns: int):

@@ -129,6 +129,12 @@ typedef struct {
     void *k_out, *v_out;      /* device Rewrite Cache rows in the idx layout:
                                  PAD_MAX [B*Hkv, bmax, D]; FLAT_SUM [B*Hkv*bmax, D] (optional,
                                  both or neither) */
+    float *beta_fit;          /* device [B*Hkv] (optional): when given, the step fits each
+                                 unit's inverse temperature as hkv_attention_entropy +
+                                 hkv_fit_temperature define it, writes it here and selects
+                                 with it in place of prob->inv_temp */
+    float *h_attn;            /* device [B*Hkv] (optional, only with beta_fit): the target
+                                 entropies the fit used */
 } hkv_step_out;
 
 /* Size in bytes of the workspace the calls below need for this problem and
@@ -252,6 +258,36 @@ hkv_status hkv_step(const hkv_problem *prob, const void *q, const hkv_tier *dens
 hkv_status hkv_append(const hkv_problem *prob, const void *k_new, const void *v_new,
                       const hkv_tier *dense, int32_t *dense_head, const hkv_tier *sparse,
                       int32_t *dropped, void *ws, size_t ws_bytes, hkv_stream_t stream);
+
+/* Fitted temperature, part 1 ([TS 2.A] Tier 2: budgets from attention
+ * entropy; [TS 3]: calibration onto the raw attention distribution): per unit
+ * the mean, over the G query heads of its group, of the entropy (natural log)
+ * of each head's raw attention softmax_j(scale * q_g . k_j) over the sparse
+ * tokens j < len[u]; 0 for an empty unit. Two kernels: the scorer (the same as
+ * hkv_score, here writing each token's per-head logits into the workspace)
+ * and one CTA per unit summing in double precision.
+ * q: device [B, Hq, D]; h: device [B*Hkv] fp32. */
+hkv_status hkv_attention_entropy(const hkv_problem *prob, const void *q, const hkv_tier *sparse,
+                                 float *h, void *ws, size_t ws_bytes, hkv_stream_t stream);
+
+/* Upper end of the fitted inverse temperature. */
+#define HKV_FIT_BETA_MAX 64.0f
+
+/* Fitted temperature, part 2 ([TS 2.B] calibration "by adjusting the
+ * temperature"): per unit the inverse temperature beta in [0, HKV_FIT_BETA_MAX]
+ * at which the calibrated distribution softmax(beta z) of the unit's metric
+ * z[u*z_stride + j], j < len[u], has entropy h_target[u]. That entropy does
+ * not increase with beta, so the root is unique when z is not constant; it is
+ * found by Newton steps inside a shrinking bracket, sums in double precision.
+ * A target at or above ln(len) gives 0, one below the entropy at
+ * HKV_FIT_BETA_MAX gives HKV_FIT_BETA_MAX, a unit with len <= 1 or constant
+ * scores gives 1, and a NaN target gives 1 and HKV_DEV_BAD_TEMP. z may be any
+ * metric (max-pooled logits from hkv_score, similarity scores, ...); the
+ * result can be passed as prob->inv_temp. One CTA per unit.
+ * z: device fp32, z_stride >= sparse->cap; h_target, beta: device [B*Hkv]. */
+hkv_status hkv_fit_temperature(const hkv_problem *prob, const float *z, int64_t z_stride,
+                               const hkv_tier *sparse, const float *h_target, float *beta,
+                               void *ws, size_t ws_bytes, hkv_stream_t stream);
 
 /* Capacity, in bytes, of the device scratch array behind
  * hkv_cascade_decode_noalloc (one array per GPU that loads the library, held

@@ -28,7 +28,7 @@ def declared_symbols():
 
 def test_every_declared_symbol_is_exported(hk):
     names = declared_symbols()
-    assert len(names) == 15, names
+    assert len(names) == 17, names
     for n in names:
         assert hasattr(hk.lib, n), n
     nm = os.popen(f"nm -D --defined-only {hk.LIB_PATH}").read()
@@ -129,3 +129,31 @@ def test_append_validates_on_the_host(hk):
     assert call(dense=bad) == "HKV_ERR_INVALID_ARG"
     assert hk.STATUS[hk.lib.hkv_append(C.byref(_prob(hk, D=96).c()), kn, vn, C.byref(d), head, C.byref(s),
                                        None, ws, 256, None)] == "HKV_ERR_UNSUPPORTED"
+
+
+def test_fit_entry_points_validate_on_the_host(hk):
+    """hkv_attention_entropy, hkv_fit_temperature and the step's fitted-temperature
+    outputs refuse bad arguments before launching anything."""
+    prob = _prob(hk)
+    s = _tier(hk, 1000, addr=0x40000000)
+    code, n = _ws_size(hk, prob, None, s, None)
+    assert code == 0
+    ws, q, z, h, b = (C.c_void_p(a) for a in (0x1000000, 0x600000, 0x700000, 0x800000, 0x900000))
+
+    def ent(q=q, h=h):
+        return hk.STATUS[hk.lib.hkv_attention_entropy(C.byref(prob.c()), q, C.byref(s), h, ws, n, None)]
+
+    def fit(z=z, zs=1000, h=h, b=b, nbytes=n):
+        return hk.STATUS[hk.lib.hkv_fit_temperature(C.byref(prob.c()), z, zs, C.byref(s), h, b, ws, nbytes, None)]
+
+    assert ent(h=None) == "HKV_ERR_INVALID_ARG"
+    assert ent(q=C.c_void_p(0x600004)) == "HKV_ERR_INVALID_ARG"
+    assert fit(h=None) == "HKV_ERR_INVALID_ARG"
+    assert fit(b=None) == "HKV_ERR_INVALID_ARG"
+    assert fit(zs=999) == "HKV_ERR_INVALID_ARG"        # z rows shorter than the tier's capacity
+    assert fit(z=None) == "HKV_ERR_INVALID_ARG"
+    assert fit(nbytes=n - 256) == "HKV_ERR_WORKSPACE"
+    # the step: h_attn without beta_fit is refused
+    o = hk._StepOut(sel_len=0x110000, idx=0x120000, out=0x130000, h_attn=0x140000)
+    st = hk.lib.hkv_step(C.byref(prob.c()), q, None, C.byref(s), None, C.byref(o), ws, n, None)
+    assert hk.STATUS[st] == "HKV_ERR_INVALID_ARG"
