@@ -303,42 +303,46 @@ __global__ void __launch_bounds__(NT) k_calibrate(const __grid_constant__ Params
         calibrate_unit<false>(P, sm, c, u, n, zg);
 }
 
-// Fitted temperature, one unit per CTA: the target entropy from the scorer's
-// per-head logit records (when P.logit is set; else P.h_target), then, when
-// P.beta_out is set, the inverse temperature that meets it on the unit's
-// scores P.z.
+// Fitted temperature, one cluster of FIT_CTAS CTAs per unit: the target
+// entropy from the scorer's per-head logit records (when P.logit is set; else
+// P.h_target), then, when P.beta_out is set, the inverse temperature that
+// meets it on the unit's scores P.z. The CTA of rank 0 writes the results.
 template <int G>
-__global__ void __launch_bounds__(NT, 1) k_fit(const __grid_constant__ Params P)
+__global__ void __cluster_dims__(FIT_CTAS, 1, 1) __launch_bounds__(NT, 1) k_fit(const __grid_constant__ Params P)
 {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     FSmem &sm = *reinterpret_cast<FSmem *>(smem_raw);
     const Ctl c = make_ctl(P);
-    const int u = blockIdx.x;
+    const int u = blockIdx.x / FIT_CTAS;
+    FitCluster cl;
     allow_dependents();
     wait_prior_grid();
     const int n = tier_len(P.sparse, u, c);
-    HKV_TRACE_AT(TR_FIT + 16 * u);
+    HKV_TRACE_IF(cl.rank == 0 && threadIdx.x == 0, TR_FIT + 16 * u);
     float target;
     if (P.logit != nullptr) {
-        target = unit_attention_entropy<G>(P.logit + (int64_t)u * P.sparse.cap * logit_floats(G), n, sm);
-        if (P.h_out != nullptr && threadIdx.x == 0)
+        target = unit_attention_entropy<G>(P.logit + (int64_t)u * P.sparse.cap * logit_floats(G), n, sm, cl);
+        if (P.h_out != nullptr && threadIdx.x == 0 && cl.rank == 0)
             P.h_out[u] = target;
     } else {
         target = __ldcg(P.h_target + u);
     }
-    HKV_TRACE_AT(TR_FIT + 16 * u + 1);
-    if (P.beta_out == nullptr)
-        return;
-    const float *zg = P.z + (int64_t)u * P.z_stride;
-    const bool staged = stage_scores(zg, n, sm);
-    HKV_TRACE_AT(TR_FIT + 16 * u + 2);
-    int evals = 0;
-    const float beta = staged ? fit_unit<true>(sm.zs, n, target, sm, c, &evals)
-                              : fit_unit<false>(zg, n, target, sm, c, &evals);
-    HKV_TRACE_AT(TR_FIT + 16 * u + 3);
-    HKV_TRACE_VAL(TR_FIT + 16 * u + 4, evals);
-    if (threadIdx.x == 0)
-        P.beta_out[u] = beta;
+    HKV_TRACE_IF(cl.rank == 0 && threadIdx.x == 0, TR_FIT + 16 * u + 1);
+    if (P.beta_out != nullptr) {
+        const float *zg = P.z + (int64_t)u * P.z_stride;
+        const bool staged = stage_scores(zg, n, sm);
+        HKV_TRACE_IF(cl.rank == 0 && threadIdx.x == 0, TR_FIT + 16 * u + 2);
+        int evals = 0;
+        const float beta = staged ? fit_unit<true>(sm.zs, n, target, sm, cl, c, &evals)
+                                  : fit_unit<false>(zg, n, target, sm, cl, c, &evals);
+        HKV_TRACE_IF(cl.rank == 0 && threadIdx.x == 0, TR_FIT + 16 * u + 3);
+        if (cl.rank == 0)
+            HKV_TRACE_VAL(TR_FIT + 16 * u + 4, evals);
+        if (threadIdx.x == 0 && cl.rank == 0)
+            P.beta_out[u] = beta;
+    }
+    // no CTA leaves while another may still read its shared memory
+    cooperative_groups::this_cluster().sync();
 }
 
 // FLAT_SUM rows and Rewrite Cache copies after the step's PAD_MAX compaction
@@ -654,7 +658,7 @@ template <int ES, int D, int G>
 struct RunFit {
     static hkv_status run(const Params &P, cudaStream_t s, bool pdl)
     {
-        return launch(k_fit<G>, P.units, NT, sizeof(FSmem), s, P, pdl);
+        return launch(k_fit<G>, P.units * FIT_CTAS, NT, sizeof(FSmem), s, P, pdl);  // clusters of FIT_CTAS
     }
 };
 

@@ -19,6 +19,9 @@
 // by HBM bandwidth.
 #pragma once
 
+#include <cfloat>
+#include <cooperative_groups.h>
+
 #include "hkv_device.cuh"
 
 namespace hkv {
@@ -2173,16 +2176,22 @@ __device__ void compact_unit(const float *zu, int n, uint32_t cut_key, int n_tie
 // the root of H(beta) = target, H(beta) the entropy of softmax(beta z). H does
 // not increase with beta (dH/dbeta = -beta Var(z)); the root is found by
 // Newton steps kept inside a shrinking bracket (bisection when a step leaves
-// it). Sums in double, exponentials on the SFU.
+// it). Each unit is worked by a cluster of FIT_CTAS CTAs (one per SM), each
+// taking an interleaved share of the tokens; their partial sums meet in
+// distributed shared memory, added in rank order, so every CTA of the cluster
+// sees the same values and takes the same branches.
 // =============================================================================
 
 constexpr float FIT_BETA_MAX = 64.0f;
+constexpr int FIT_CTAS = 2;
 
 struct __align__(16) FSmem {  // shared memory of the fitting kernel
     float zs[ZSTAGE];
     float redf[NT / 32];
     float redv[8 * (NT / 32)];
-    double redd[16 * (NT / 32)];  // up to 2 G = 16 sums per thread
+    double redd[16 * (NT / 32)];
+    double xd[2][16];  // cluster exchange, two buffers used in turn
+    float xf[2][8];
 };
 
 // Per-lane vectors summed (double) or maxed (float) over the CTA; every thread
@@ -2235,6 +2244,60 @@ __device__ __forceinline__ void block_max_vec(float (&v)[K], float *scratch)
     __syncthreads();
 }
 
+// The cluster's CTAs combine block-uniform vectors: sums in rank order, or
+// maxima. Exchanges alternate between two buffers, so one cluster barrier per
+// exchange suffices: a buffer is written again only after the next barrier,
+// which every CTA reaches after reading it.
+struct FitCluster {
+    int rank, phase;
+    __device__ FitCluster() : rank((int)cooperative_groups::this_cluster().block_rank()), phase(0) {}
+
+    template <int K>
+    __device__ __forceinline__ void sum(double (&v)[K], FSmem &sm)
+    {
+        auto cl = cooperative_groups::this_cluster();
+        double *mine = sm.xd[phase];
+        if (threadIdx.x == 0) {
+#pragma unroll
+            for (int i = 0; i < K; ++i)
+                mine[i] = v[i];
+        }
+        cl.sync();
+#pragma unroll
+        for (int i = 0; i < K; ++i) {
+            double r = 0.0;
+#pragma unroll
+            for (int c = 0; c < FIT_CTAS; ++c)
+                r += c == rank ? v[i] : cl.map_shared_rank(mine, c)[i];
+            v[i] = r;
+        }
+        phase ^= 1;
+    }
+
+    template <int K>
+    __device__ __forceinline__ void max(float (&v)[K], FSmem &sm)
+    {
+        auto cl = cooperative_groups::this_cluster();
+        float *mine = sm.xf[phase];
+        if (threadIdx.x == 0) {
+#pragma unroll
+            for (int i = 0; i < K; ++i)
+                mine[i] = v[i];
+        }
+        cl.sync();
+#pragma unroll
+        for (int c = 0; c < FIT_CTAS; ++c) {
+            if (c == rank)
+                continue;
+            const float *o = cl.map_shared_rank(mine, c);
+#pragma unroll
+            for (int i = 0; i < K; ++i)
+                v[i] = fmaxf(v[i], o[i]);
+        }
+        phase ^= 1;
+    }
+};
+
 // The G per-head logits of one record (float4 loads; LG is a multiple of 4).
 template <int G>
 __device__ __forceinline__ void load_record(const float *p, float (&x)[G])
@@ -2254,16 +2317,18 @@ __device__ __forceinline__ void load_record(const float *p, float (&x)[G])
 }
 
 // Mean over the G heads of the entropy of softmax over a unit's n per-head
-// logit records (record j at rec + j * LG, head g at offset g), in one pass:
-// each thread keeps per head a running maximum m, Z = sum exp(l - m) and
-// S = sum exp(l - m) (l - m), rescaled when m grows (by batches of records,
-// all of a batch's loads in flight at once); the threads' triples are then
-// brought to the CTA's maximum and summed in double. H = ln Z - S / Z.
+// logit records (record j at rec + j * LG, head g at offset g). The cluster's
+// CTA of rank r takes records r NT + t, r NT + t + FIT_CTAS NT, ... in thread
+// t. Each thread keeps per head a running maximum m, Z = sum exp(l - m) and
+// S = sum exp(l - m) (l - m), rescaled when m grows (per batch of records,
+// whose loads are all in flight at once); the triples are then brought to the
+// cluster's maximum and summed in double. H = ln Z - S / Z.
 template <int G>
-__device__ float unit_attention_entropy(const float *rec, int n, FSmem &sm)
+__device__ float unit_attention_entropy(const float *rec, int n, FSmem &sm, FitCluster &cl)
 {
     constexpr int LG = logit_floats(G);
     constexpr int BATCH = G >= 8 ? 4 : 8;
+    constexpr int STRIDE = FIT_CTAS * NT;
     if (n <= 0)
         return 0.0f;
     float m[G], Z[G], S[G];
@@ -2274,11 +2339,11 @@ __device__ float unit_attention_entropy(const float *rec, int n, FSmem &sm)
         S[g] = 0.0f;
     }
 #pragma unroll 1
-    for (int j0 = threadIdx.x; j0 < n; j0 += NT * BATCH) {
+    for (int j0 = cl.rank * NT + threadIdx.x; j0 < n; j0 += STRIDE * BATCH) {
         float x[BATCH][G];
 #pragma unroll
         for (int b = 0; b < BATCH; ++b) {
-            const int j = j0 + b * NT;
+            const int j = j0 + b * STRIDE;
             if (j < n) {
                 load_record<G>(rec + (int64_t)j * LG, x[b]);
             } else {
@@ -2304,12 +2369,11 @@ __device__ float unit_attention_entropy(const float *rec, int n, FSmem &sm)
             }
 #pragma unroll
             for (int b = 0; b < BATCH; ++b) {
-                const float d = x[b][g] - m[g];
-                const float e = d == 0.0f ? 1.0f : ex2(d * LOG2E);
-                if (e > 0.0f) {
-                    Z[g] += e;
-                    S[g] += e * d;
-                }
+                // -inf logits (and padding) weigh 0; the clamp keeps 0 * d finite
+                const float d = fmaxf(x[b][g] - m[g], -FLT_MAX);
+                const float e = ex2(d * LOG2E);
+                Z[g] += e;
+                S[g] = fmaf(e, d, S[g]);
             }
         }
     }
@@ -2318,6 +2382,7 @@ __device__ float unit_attention_entropy(const float *rec, int n, FSmem &sm)
     for (int g = 0; g < G; ++g)
         M[g] = m[g];
     block_max_vec<G>(M, sm.redv);
+    cl.max<G>(M, sm);
     double acc[2 * G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
@@ -2331,6 +2396,7 @@ __device__ float unit_attention_entropy(const float *rec, int n, FSmem &sm)
         }
     }
     block_sum_vec<2 * G>(acc, sm.redd);
+    cl.sum<2 * G>(acc, sm);
     double h = 0.0;
 #pragma unroll
     for (int g = 0; g < G; ++g)
@@ -2338,13 +2404,14 @@ __device__ float unit_attention_entropy(const float *rec, int n, FSmem &sm)
     return (float)(h / G);
 }
 
-// Entropy of softmax(beta z) over a unit and its derivative in beta. Thread t
-// takes the quads t, t + NT, ... of the scores and sums each of a quad's four
-// positions into its own fp32 accumulators (about n / (4 NT) terms each, so
-// their rounding stays near 1e-7 relative); the CTA sums in double.
+// Entropy of softmax(beta z) over a unit and its derivative in beta. The CTA of
+// rank r takes the quads r NT + t, r NT + t + FIT_CTAS NT, ... in thread t and
+// sums each of a quad's four positions into its own fp32 accumulators (a few
+// terms each, so their rounding stays near 1e-7 relative); CTA and cluster sum
+// in double.
 template <bool ZS>
-__device__ __forceinline__ void fit_eval(const float *zu, int n, float m, float beta, FSmem &sm, double *H,
-                                         double *dH)
+__device__ __forceinline__ void fit_eval(const float *zu, int n, float m, float beta, FSmem &sm, FitCluster &cl,
+                                         double *H, double *dH)
 {
     const float bl2 = beta * LOG2E;
     const bool vec = ZS || (((uintptr_t)zu) & 15) == 0;
@@ -2353,7 +2420,7 @@ __device__ __forceinline__ void fit_eval(const float *zu, int n, float m, float 
     for (int i = 0; i < 4; ++i)
         a[i][0] = a[i][1] = a[i][2] = 0.0f;
 #pragma unroll 2
-    for (int j = 4 * (int)threadIdx.x; j < n; j += 4 * NT) {
+    for (int j = 4 * (cl.rank * NT + (int)threadIdx.x); j < n; j += 4 * FIT_CTAS * NT) {
         float v[4];
         if (vec && j + 4 <= n) {
             const float4 t = ZS ? lds4(zu + j) : __ldcg(reinterpret_cast<const float4 *>(zu + j));
@@ -2368,14 +2435,13 @@ __device__ __forceinline__ void fit_eval(const float *zu, int n, float m, float 
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const float d = v[i] - m;
-            const float w = d == 0.0f ? 1.0f : ex2(d * bl2);
-            if (w > 0.0f) {
-                const float wd = w * d;
-                a[i][0] += w;
-                a[i][1] += wd;
-                a[i][2] = fmaf(wd, d, a[i][2]);
-            }
+            // -inf scores (and padding) weigh 0; the clamp keeps 0 * d finite
+            const float d = fmaxf(v[i] - m, -FLT_MAX);
+            const float w = ex2(d * bl2);
+            const float wd = w * d;
+            a[i][0] += w;
+            a[i][1] += wd;
+            a[i][2] = fmaf(wd, d, a[i][2]);
         }
     }
     double acc[3];
@@ -2383,39 +2449,41 @@ __device__ __forceinline__ void fit_eval(const float *zu, int n, float m, float 
     for (int k = 0; k < 3; ++k)
         acc[k] = ((double)a[0][k] + (double)a[1][k]) + ((double)a[2][k] + (double)a[3][k]);
     block_sum_vec<3>(acc, sm.redd);
+    cl.sum<3>(acc, sm);
     const double mean = acc[1] / acc[0];
     *H = log(acc[0]) - (double)beta * mean;
     *dH = -(double)beta * (acc[2] / acc[0] - mean * mean);
 }
 
-// The fitted inverse temperature of one unit (see the section comment).
+// The fitted inverse temperature of one unit (see the section comment). Every
+// CTA of the cluster calls it with the same arguments and returns the same
+// value.
 template <bool ZS>
-__device__ float fit_unit(const float *zu, int n, float target, FSmem &sm, const Ctl &c, int *evals)
+__device__ float fit_unit(const float *zu, int n, float target, FSmem &sm, FitCluster &cl, const Ctl &c, int *evals)
 {
     float m, zlo;
     unit_range<ZS>(zu, n, &m, &zlo, sm);
     if (n <= 1 || !(m > zlo))
         return 1.0f;  // every beta gives the same distribution
     if (target != target) {
-        if (threadIdx.x == 0)
+        if (threadIdx.x == 0 && cl.rank == 0)
             raise_flag(c, HKV_DEV_BAD_TEMP);
         return 1.0f;
     }
     const double t = (double)target;
     if (t >= log((double)n))
         return 0.0f;
-    double H, dH;
-    fit_eval<ZS>(zu, n, m, FIT_BETA_MAX, sm, &H, &dH);
-    ++*evals;
-    if (H >= t)
-        return FIT_BETA_MAX;  // sharper than the metric can get
     // H is known to a few 1e-7 relative (the sums' rounding), so the search
     // stops at that level: H within 2e-6 of the target, a Newton step below
-    // 1e-6 of beta, or a bracket that narrow
+    // 1e-6 of beta, or a bracket that narrow. Whether the target is reachable
+    // at all (H(FIT_BETA_MAX) < target) is checked only once the search heads
+    // above half of FIT_BETA_MAX.
     float lo = 0.0f, hi = FIT_BETA_MAX, beta = 1.0f;
+    bool top_checked = false;
+    double H, dH;
 #pragma unroll 1
     for (int it = 0; it < 40; ++it) {
-        fit_eval<ZS>(zu, n, m, beta, sm, &H, &dH);
+        fit_eval<ZS>(zu, n, m, beta, sm, cl, &H, &dH);
         ++*evals;
         if (fabs(H - t) <= 2e-6 * fmax(1.0, t))
             break;
@@ -2430,6 +2498,14 @@ __device__ float fit_unit(const float *zu, int n, float target, FSmem &sm, const
             next = 0.5f * (lo + hi);
         else if (fabsf(next - beta) <= 1e-6f * beta)
             return next;
+        if (!top_checked && next > 0.5f * FIT_BETA_MAX) {
+            top_checked = true;
+            double Ht, dHt;
+            fit_eval<ZS>(zu, n, m, FIT_BETA_MAX, sm, cl, &Ht, &dHt);
+            ++*evals;
+            if (Ht >= t)
+                return FIT_BETA_MAX;  // sharper than the metric can get
+        }
         beta = next;
     }
     return beta;
