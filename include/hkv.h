@@ -215,7 +215,10 @@ hkv_status hkv_cascade_decode(const hkv_problem *prob, const void *q,
  * reads through the indices ([TS 2.C] Sparse Loading) together with the
  * scorer's logits (so their K rows are not read again); (4) a merge kernel
  * combines each unit's partial softmax records. A FLAT_SUM layout or
- * k_out/v_out (the Rewrite Cache copy) adds a fifth kernel. Scores, budgets,
+ * k_out/v_out (the Rewrite Cache copy) adds a kernel at the end; out->beta_fit
+ * adds one between (1) and (2) that fits each unit's inverse temperature from
+ * the scorer's per-head logits and scores (hkv_attention_entropy and
+ * hkv_fit_temperature give the same bits), after which (2) selects with it. Scores, budgets,
  * cuts, index rows, m and logZ equal those of the separate calls bit for bit;
  * out and lse agree to a few ulp (hkv_cascade_decode recomputes the logits
  * from K). ws as for hkv_cascade_decode. */
