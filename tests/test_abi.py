@@ -157,3 +157,35 @@ def test_fit_entry_points_validate_on_the_host(hk):
     o = hk._StepOut(sel_len=0x110000, idx=0x120000, out=0x130000, h_attn=0x140000)
     st = hk.lib.hkv_step(C.byref(prob.c()), q, None, C.byref(s), None, C.byref(o), ws, n, None)
     assert hk.STATUS[st] == "HKV_ERR_INVALID_ARG"
+
+
+def test_struct_layouts_match_the_header(hk, tmp_path):
+    """The ctypes mirrors of the header's structs have the C compiler's field
+    names, order, offsets and sizes (gcc compiles a probe of the header)."""
+    import subprocess
+
+    mirrors = {"hkv_tier": hk._Tier, "hkv_problem": hk._Problem, "hkv_cut": hk.Cut, "hkv_step_out": hk._StepOut}
+    text = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", "hkv.h")).read(), flags=re.S)
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "hkv.h"', "int main(void) {"]
+    for cname, mirror in mirrors.items():
+        body = re.search(r"typedef struct \{([^{}]*)\}\s*" + cname + ";", text).group(1)
+        names = []
+        for decl in body.split(";"):
+            decl = decl.strip()
+            if decl:
+                names += [n.strip().lstrip("*") for n in re.sub(r"^[\w\s]+?(?=\*?\w+\s*(,|$))", "", decl).split(",")]
+        assert names == [f[0] for f in mirror._fields_], (cname, names)
+        lines.append(f'printf("{cname} size %zu\\n", sizeof({cname}));')
+        for n in names:
+            lines.append(f'printf("{cname} {n} %zu\\n", offsetof({cname}, {n}));')
+    lines += ["return 0; }"]
+    src = tmp_path / "probe.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "probe"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split("\n")
+    for line in filter(None, out):
+        cname, field, value = line.split()
+        mirror = mirrors[cname]
+        got = C.sizeof(mirror) if field == "size" else getattr(mirror, field).offset
+        assert got == int(value), (cname, field, got, value)
