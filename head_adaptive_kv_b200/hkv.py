@@ -315,8 +315,14 @@ def append(prob: Problem, k_new: torch.Tensor, v_new: torch.Tensor, dense: Optio
                           _tref(sparse), _ptr(dropped), ws.ptr, ws.nbytes, _stream(stream)), "hkv_append")
 
 
+def _f32_vector(t: torch.Tensor, n: int, what: str):
+    if t.dtype != torch.float32 or t.dim() != 1 or t.stride(0) != 1 or t.numel() < n:
+        raise ValueError(f"{what} must be a contiguous fp32 vector of at least {n} elements")
+
+
 def attention_entropy(prob: Problem, q: torch.Tensor, sparse: Tier, h: torch.Tensor, ws: Workspace, stream=None):
     """Per unit the group-averaged entropy of the raw attention over the sparse tier (h: fp32 [B*Hkv])."""
+    _f32_vector(h, prob.units, "h")
     _check(lib.hkv_attention_entropy(C.byref(prob.c()), _ptr(q), C.byref(sparse.c()), _ptr(h), ws.ptr,
                                      ws.nbytes, _stream(stream)), "hkv_attention_entropy")
 
@@ -325,6 +331,10 @@ def fit_temperature(prob: Problem, z: torch.Tensor, sparse: Tier, h_target: torc
                     ws: Workspace, stream=None):
     """Per unit the inverse temperature at which softmax(beta z) has entropy
     h_target (z: fp32 [B*Hkv, >= cap]; h_target, beta: fp32 [B*Hkv])."""
+    if z.dtype != torch.float32 or z.dim() != 2 or z.stride(1) != 1 or z.shape[1] < sparse.cap:
+        raise ValueError("z must be fp32 [B*Hkv, >= cap] with contiguous rows")
+    _f32_vector(h_target, prob.units, "h_target")
+    _f32_vector(beta, prob.units, "beta")
     _check(lib.hkv_fit_temperature(C.byref(prob.c()), _ptr(z), z.stride(0), C.byref(sparse.c()), _ptr(h_target),
                                    _ptr(beta), ws.ptr, ws.nbytes, _stream(stream)), "hkv_fit_temperature")
 

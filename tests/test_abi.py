@@ -189,3 +189,23 @@ def test_struct_layouts_match_the_header(hk, tmp_path):
         mirror = mirrors[cname]
         got = C.sizeof(mirror) if field == "size" else getattr(mirror, field).offset
         assert got == int(value), (cname, field, got, value)
+
+
+def test_binding_checks_fit_arguments_before_the_library(hk):
+    """The Python binding refuses ill-shaped fitted-temperature arguments
+    itself (CPU tensors suffice: nothing reaches the library)."""
+    prob = _prob(hk)
+    k = torch.zeros(2, 2, 16, 128, dtype=torch.bfloat16)
+    sparse = hk.Tier(k, k, torch.zeros(4, dtype=torch.int32))
+    ws = object()
+    good = torch.zeros(4, dtype=torch.float32)
+    with pytest.raises(ValueError):
+        hk.fit_temperature(prob, torch.zeros(4, 16, dtype=torch.float64), sparse, good, good, ws)
+    with pytest.raises(ValueError):
+        hk.fit_temperature(prob, torch.zeros(16, 4).t(), sparse, good, good, ws)   # rows not contiguous
+    with pytest.raises(ValueError):
+        hk.fit_temperature(prob, torch.zeros(4, 8), sparse, good, good, ws)        # rows shorter than cap
+    with pytest.raises(ValueError):
+        hk.fit_temperature(prob, torch.zeros(4, 16), sparse, good[:3], good, ws)   # too few targets
+    with pytest.raises(ValueError):
+        hk.attention_entropy(prob, torch.zeros(2, 8, 128), sparse, torch.zeros(4, dtype=torch.int32), ws)
