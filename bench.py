@@ -37,7 +37,7 @@ WORKLOAD_ID = 2
 NSETS = 3  # distinct decode states rotated so that no step re-reads the previous one from L2
 GRAPH_STEPS = 12  # steps per replayed CUDA graph (a multiple of NSETS)
 METRIC = "decode steps/sec and KV GB/s at 1 B200 (fraction of 8 TB/s HBM roofline)"
-NORTH_STAR_HBM_GBS = 8000.0
+NOMINAL_HBM_GBS = 8000.0  # nominal HBM3e bandwidth of the part (DGX figure)
 
 
 def peaks():
@@ -499,7 +499,7 @@ def run_ours(args):
             "data": "synthetic (seeded Gaussian decode states with planted heavy hitters)",
             "config": config_of(wl, world),
             "kv_gbs": round(bytes_per_step * world / (region_ms_max / args.steps / 1e3) / 1e9, 1),
-            "frac_of_8tbs": round(bytes_per_step / (ms / 1e3) / 1e9 / NORTH_STAR_HBM_GBS, 4),
+            "frac_of_8tbs": round(bytes_per_step / (ms / 1e3) / 1e9 / NOMINAL_HBM_GBS, 4),
             "roofline": roofline,
             "kernels": kernels,
             "cpu_baseline": base,
