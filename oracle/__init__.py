@@ -375,3 +375,235 @@ def fit_temperature(z: np.ndarray, length: np.ndarray, h_target: np.ndarray,
                 hi = mid
         beta[u] = 0.5 * (lo + hi)
     return beta
+
+
+# ---- Condensed-tier formation ([TS 2.A] Tier 3 and pipeline step 4) ----------------
+#
+# Tier 3 keeps the oldest context in storage of constant size: "the oldest
+# blocks are further compressed into constant-sized storage via eviction or
+# weighted merging", and the pipeline's fourth step is the "eviction or
+# merging of the oldest blocks". Reading taken: a unit whose sparse tier holds
+# at least `trigger` tokens (and at least `block`) gives up its oldest `block`
+# tokens (sparse slots 0 .. block-1, the tier being in age order); they become
+# ONE condensed slot, appended after the existing ones:
+#   MERGE: the slot's K and V are the weighted means of the block's rows, the
+#          weights a_j being the tokens' calibrated probabilities under the
+#          step's scores, a_j = exp(beta (z_j - m) - logZ); the slot keeps the
+#          block's mass sum_j a_j as its weight. When the condensed tier is
+#          full, its two oldest slots first merge the same way (weights w_0,
+#          w_1; the merged slot weighs w_0 + w_1) and the later slots move down.
+#   EVICT: the slot is a copy of the block's most important token (largest z,
+#          the older one on ties) with weight a_j; the rest of the block is
+#          dropped. When the condensed tier is full its oldest slot is dropped
+#          first and the later slots move down.
+# Weights that sum to zero (or no scores given) mean equal weights. Means are
+# float64 sums in slot order, rounded once to the tier's element type (nearest,
+# ties to even). The sparse tier then moves down by `block` rows, keeping its
+# age order. A condensed tier of capacity 0 just drops the block.
+
+CONDENSE_MERGE, CONDENSE_EVICT = 0, 1
+
+
+def round_to_bf16(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to bf16 (8 significant bits; nearest, ties to even)
+    straight from the double, and return their bit patterns (uint16)."""
+    x = np.asarray(x, np.float64)
+    f, e = np.frexp(x)  # x = f 2^e, 0.5 <= |f| < 1
+    # spacing of bf16 values near x: 2^(e - 8) for normal values, 2^-133 below 2^-126
+    sh = np.where(e - 8 < -133, -133, e - 8)
+    r = np.rint(np.ldexp(x, -sh))  # exact scaling, then round half to even
+    y = np.ldexp(r, sh).astype(np.float32)  # exactly representable in bf16 (hence fp32)
+    return (y.view(np.uint32) >> 16).astype(np.uint16)
+
+
+def _round_to(x: np.ndarray, like: np.ndarray) -> np.ndarray:
+    """float64 -> the element type of `like` (bf16 bits or float32), nearest-even."""
+    if like.dtype == np.uint16:
+        return round_to_bf16(x)
+    return np.asarray(x, np.float64).astype(np.float32)
+
+
+def _seq_sum(a) -> float:
+    """float64 sum in index order (no pairwise summation)."""
+    t = 0.0
+    for x in a:
+        t = t + float(x)
+    return t
+
+
+def _weighted_mean(rows: np.ndarray, a: np.ndarray) -> np.ndarray:
+    """sum_j a_j rows_j / sum_j a_j in float64, summed in row order; equal
+    weights when the a_j sum to zero. rows: [b, D] float64."""
+    if not _seq_sum(a) > 0.0:
+        a = np.ones(len(a), np.float64)
+    num = np.zeros(rows.shape[1], np.float64)
+    den = 0.0
+    for j in range(len(a)):
+        num = num + a[j] * rows[j]
+        den = den + a[j]
+    return num / den
+
+
+def condense(sparse: Tier, condensed: Tier, cond_w: np.ndarray, z: Optional[np.ndarray],
+             m: Optional[np.ndarray], logZ: Optional[np.ndarray], beta: Optional[np.ndarray],
+             block: int, trigger: int, policy: int = CONDENSE_MERGE):
+    """One condensation pass over every unit, on copies. Returns (sparse,
+    condensed, cond_w, done) with done[u] = 1 where unit u gave up a block.
+    z: the step's scores [units, >= sparse cap] (None: equal weights); m, logZ:
+    the step's per-unit max and log normaliser; beta: per-unit inverse
+    temperature (None = 1); cond_w: per-slot weights [units, condensed cap].
+    A condensed tier of one slot under MERGE takes the block into that slot
+    (the old slot weighing its weight)."""
+    B, H, ncap, D = sparse.k.shape
+    ccap = condensed.k.shape[2]
+    sk, sv = sparse.k.copy(), sparse.v.copy()
+    ck, cv = condensed.k.copy(), condensed.v.copy()
+    slen = np.array(sparse.len, np.int32).copy()
+    clen = np.array(condensed.len, np.int32).copy()
+    w = np.array(cond_w, np.float32).copy().reshape(B * H, ccap)
+    done = np.zeros(B * H, np.int32)
+    for b in range(B):
+        for h in range(H):
+            u = b * H + h
+            n, C = int(slen[u]), int(clen[u])
+            if n < max(trigger, block, 1):
+                continue
+            done[u] = 1
+            if z is not None:
+                be = 1.0 if beta is None else float(beta[u])
+                zz = np.asarray(z[u, :block], np.float32).astype(np.float64)
+                a = np.exp(be * (zz - np.float64(m[u])) - np.float64(logZ[u]))
+            else:
+                zz = np.zeros(block, np.float64)
+                a = np.ones(block, np.float64)
+            if ccap > 0 and policy == CONDENSE_MERGE:
+                rows_k, rows_v = _f64(sk[b, h, :block]), _f64(sv[b, h, :block])
+                if C >= ccap and ccap >= 2:  # the two oldest slots merge into slot 0
+                    wp = np.array([w[u, 0], w[u, 1]], np.float64)
+                    ck[b, h, 0] = _round_to(_weighted_mean(_f64(ck[b, h, 0:2]), wp), ck)
+                    cv[b, h, 0] = _round_to(_weighted_mean(_f64(cv[b, h, 0:2]), wp), cv)
+                    w[u, 0] = np.float32(_seq_sum(wp))
+                    ck[b, h, 1:ccap - 1] = ck[b, h, 2:ccap].copy()
+                    cv[b, h, 1:ccap - 1] = cv[b, h, 2:ccap].copy()
+                    w[u, 1:ccap - 1] = w[u, 2:ccap].copy()
+                    C = ccap - 1
+                elif C >= ccap:  # one slot: the block merges into it
+                    rows_k = np.concatenate([_f64(ck[b, h, 0:1]), rows_k])
+                    rows_v = np.concatenate([_f64(cv[b, h, 0:1]), rows_v])
+                    a = np.concatenate([[np.float64(w[u, 0])], a])
+                    C = 0
+                ck[b, h, C] = _round_to(_weighted_mean(rows_k, a), ck)
+                cv[b, h, C] = _round_to(_weighted_mean(rows_v, a), cv)
+                w[u, C] = np.float32(_seq_sum(a))
+                clen[u] = C + 1
+            elif ccap > 0:  # EVICT
+                if C >= ccap:  # the oldest slot goes
+                    ck[b, h, 0:ccap - 1] = ck[b, h, 1:ccap].copy()
+                    cv[b, h, 0:ccap - 1] = cv[b, h, 1:ccap].copy()
+                    w[u, 0:ccap - 1] = w[u, 1:ccap].copy()
+                    C = ccap - 1
+                jstar = int(np.argmax(zz))  # the first maximum: the older token
+                ck[b, h, C] = sk[b, h, jstar]
+                cv[b, h, C] = sv[b, h, jstar]
+                w[u, C] = np.float32(a[jstar])
+                clen[u] = C + 1
+            # the sparse tier moves down by one block, in age order
+            sk[b, h, :n - block] = sk[b, h, block:n].copy()
+            sv[b, h, :n - block] = sv[b, h, block:n].copy()
+            slen[u] = n - block
+    return Tier(sk, sv, slen), Tier(ck, cv, clen), w, done
+
+
+# ---- Rewrite Cache vs Sparse Loading ([TS 2.C] Trade-off Management) ------------------
+#
+# The pages: a Memory-Time Integral (MTI) weighs the upfront cost of rewriting
+# against the per-step decoding gains, and budget thresholds L_lower and
+# L_upper trigger sparse loading or full rewriting; the rewrite overhead is
+# amortized within a few decoding steps ([TS 4]). Reading taken, per unit:
+#   - a unit whose rewrite still serves (left > 0) is not scored or selected
+#     this step: it attends over dense ++ its rewritten rows ++ condensed, and
+#     left drops by one;
+#   - any other unit runs the plain step (Sparse Loading of the fresh
+#     selection, budget k); then its mode becomes Rewrite Cache when k > L_upper,
+#     Sparse Loading when k < L_lower, and stays as it was in between; under
+#     Rewrite Cache its k selected rows are copied, in token order, into its
+#     rewrite buffer, which serves H(k) = max(1, floor(mti_cap / k)) steps in
+#     all (this one included), so that the rewrite's memory-time integral
+#     k H stays within mti_cap.
+
+MODE_SPARSE, MODE_REWRITE = 0, 1
+
+
+def mti_trigger(k: int, mode: int, L_lower: int, L_upper: int) -> int:
+    """The mode after a fresh step whose budget is k."""
+    if k > L_upper:
+        return MODE_REWRITE
+    if k < L_lower:
+        return MODE_SPARSE
+    return mode
+
+
+def mti_horizon(k: int, mti_cap: int) -> int:
+    """Steps a rewrite of k rows serves, the step that made it included."""
+    return max(1, mti_cap // k) if k > 0 else 1
+
+
+def mti_state(units: int, bmax: int, B: int, Hkv: int, D: int, like: np.ndarray) -> dict:
+    """The all-Sparse-Loading starting state (the rewrite buffer of `like`'s dtype)."""
+    return {"mode": np.zeros(units, np.int32), "left": np.zeros(units, np.int32),
+            "rw_k": np.zeros((B, Hkv, bmax, D), like.dtype), "rw_v": np.zeros((B, Hkv, bmax, D), like.dtype),
+            "rw_len": np.zeros(units, np.int32), "rw_idx": np.zeros((units, bmax), np.int32)}
+
+
+def step_mti(q: np.ndarray, dense: Optional[Tier], sparse: Tier, condensed: Optional[Tier], scale: float,
+             p: float, bmin: int, bmax: int, state: dict, L_lower: int, L_upper: int, mti_cap: int,
+             k_fresh: Optional[np.ndarray] = None, idx_fresh: Optional[np.ndarray] = None,
+             p_unit: Optional[np.ndarray] = None):
+    """One decode step under the trigger. Returns (result, new state): result
+    holds k, idx [units, bmax], out, lse and fresh (1 where the unit ran the
+    plain step). k_fresh / idx_fresh: optional budgets and index rows of the
+    fresh units to take the trigger and the rewrite with (another
+    implementation's, where its budget may differ at an ambiguous cut); by
+    default the step's own."""
+    B, Hq, D = q.shape
+    Hkv = sparse.k.shape[1]
+    G = Hq // Hkv
+    U = B * Hkv
+    st = {key: np.array(v, copy=True) for key, v in state.items()}
+    plain = step(q, dense, sparse, condensed, scale, p, bmin, bmax, p_unit=p_unit)
+    kf = plain["k"] if k_fresh is None else np.asarray(k_fresh, np.int32)
+    idf = plain["idx"] if idx_fresh is None else np.asarray(idx_fresh, np.int32).reshape(U, bmax)
+    # the reusing units' attention: the rewrite buffer as the selected tokens
+    rw = Tier(state["rw_k"], state["rw_v"], state["rw_len"])
+    rw_cap = state["rw_k"].shape[2]
+    ident = np.tile(np.arange(rw_cap, dtype=np.int32), (U, 1))
+    r_out, r_lse = attend(q, dense, rw, ident, state["rw_len"], rw_cap, condensed, scale, Hkv=Hkv)
+    out, lse = plain["out"].copy(), plain["lse"].copy()
+    k = plain["k"].copy()
+    idx = plain["idx"].copy()
+    fresh = np.ones(U, np.int32)
+    for u in range(U):
+        b, h = divmod(u, Hkv)
+        if state["left"][u] > 0:
+            fresh[u] = 0
+            out[b, h * G:(h + 1) * G] = r_out[b, h * G:(h + 1) * G]
+            lse[b, h * G:(h + 1) * G] = r_lse[b, h * G:(h + 1) * G]
+            n = int(state["rw_len"][u])
+            k[u] = n
+            idx[u, :] = -1
+            idx[u, :n] = state["rw_idx"][u, :n]
+            st["left"][u] -= 1
+            continue
+        ku = int(kf[u])
+        st["mode"][u] = mti_trigger(ku, int(state["mode"][u]), L_lower, L_upper)
+        if st["mode"][u] == MODE_REWRITE:
+            rows = idf[u, :ku]
+            st["rw_k"][b, h, :ku] = sparse.k[b, h, rows]
+            st["rw_v"][b, h, :ku] = sparse.v[b, h, rows]
+            st["rw_idx"][u, :ku] = rows
+            st["rw_len"][u] = ku
+            st["left"][u] = mti_horizon(ku, mti_cap) - 1
+        else:
+            st["rw_len"][u] = 0
+            st["left"][u] = 0
+    return {"k": k, "idx": idx, "out": out, "lse": lse, "fresh": fresh}, st

@@ -26,3 +26,15 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """How often the GPU budget tests needed the ambiguous-cut rule."""
+    mod = sys.modules.get("tests.gpu_helpers")
+    if mod is None:
+        return
+    t = mod.AMBIG_TALLY
+    if t["units"]:
+        terminalreporter.write_line(
+            f"budget checks: {t['units']} units, {t['ambiguous_accepts']} accepted through the "
+            f"ambiguous-cut rule (widest window {t['max_window']:.3g})")

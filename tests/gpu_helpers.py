@@ -14,10 +14,44 @@ from head_adaptive_kv_b200 import hkv
 from head_adaptive_kv_b200.workloads import TierTensors, Workload, make_inputs, to_host_bits
 
 # Attention outputs: fp32 accumulation from bf16/fp32 inputs against the fp64
-# oracle, elementwise |a - b| <= ATOL + RTOL |b|.
+# oracle. Every element must be within ATOL = 2e-3 (the maximum absolute error
+# the target allows); RTOL = 1e-2 is its maximum relative error, which an
+# element within ATOL of a reference above 0.2 meets anyway, so ATOL alone is
+# asserted (the stricter of the two readings).
 ATOL, RTOL = 2e-3, 1e-2
-# Ambiguous cut: the oracle's prefix mass is this close to p on either side of k*.
-AMBIG = 1e-5
+# Ambiguous cut: the oracle's prefix mass lies within a unit's window of p on
+# either side of k*. The window follows from the error of the GPU weight
+# w = ex2((z - m) beta log2 e): ex2.approx is within 2^-22 relative, and the
+# exponent, rounded three times in fp32, is off by at most 3 2^-24 |x|
+# (x = (z - m) beta log2 e), which moves w by ln 2 times that. Summed over a
+# unit, the weights' error is at most Z (2^-22 + 3 2^-24 ln 2 E_P|x|), E_P the
+# calibrated mean. The GPU compares the exact integer sum of 40-bit fixed-point
+# weights with ceil(p Z 2^40), Z a double sum of the same weights, so its test
+# C_k >= p can differ from the exact one only within
+#     2 (2^-22 + 3 2^-24 ln 2 E_P|x|) + (k + 1) 2^-40
+# of p; window() takes 1.5 times that (second-order terms, the oracle's own
+# fp64 sums) and never less than AMBIG_FLOOR.
+AMBIG_FLOOR = 1e-6
+# Units checked by selection_ok / budgets_match, how many of them were accepted
+# through the ambiguous-cut rule, and the widest window used (reported at the
+# end of the session).
+AMBIG_TALLY = {"units": 0, "ambiguous_accepts": 0, "max_window": 0.0}
+
+
+def window(z_row: np.ndarray, n: int, beta: float, k: int) -> float:
+    """The ambiguous-cut window of one unit (see above)."""
+    z = np.asarray(z_row[:n], np.float32).astype(np.float64)
+    if n == 0:
+        return AMBIG_FLOOR
+    x = beta * math.log2(math.e) * (z.max() - z)
+    P = sps.softmax(beta * z)
+    ex = float(np.sum(P * x))
+    w = 1.5 * (2 * (2.0 ** -22 + 3 * 2.0 ** -24 * math.log(2) * ex) + (k + 1) * 2.0 ** -40)
+    w = max(w, AMBIG_FLOOR)
+    AMBIG_TALLY["max_window"] = max(AMBIG_TALLY["max_window"], w)
+    return w
+
+
 # End to end a token may flip only if its calibrated probability is this close
 # to the probability of the oracle's last selected token.
 P_FLIP = 1e-6
@@ -67,9 +101,13 @@ def selection_ok(z_ref: np.ndarray, n: int, k_gpu: int, idx_gpu: np.ndarray, p: 
     r = oracle.topp(z_ref[None, :n].astype(np.float32), np.array([n], np.int32), p, bmin, bmax,
                     np.array([beta], np.float32))
     k_ref = int(r["k"][0])
-    amb = (abs(r["c_before"][0] - p) < AMBIG) or (abs(r["c_at"][0] - p) < AMBIG)
-    if k_gpu != k_ref and not (amb and abs(k_gpu - k_ref) <= 1):
-        return False, f"k {k_gpu} vs oracle {k_ref} (not an ambiguous cut)"
+    win = window(z_ref, n, beta, k_ref)
+    amb = (abs(r["c_before"][0] - p) < win) or (abs(r["c_at"][0] - p) < win)
+    AMBIG_TALLY["units"] += 1
+    if k_gpu != k_ref:
+        if not (amb and abs(k_gpu - k_ref) <= 1):
+            return False, f"k {k_gpu} vs oracle {k_ref} (not an ambiguous cut)"
+        AMBIG_TALLY["ambiguous_accepts"] += 1
     if n == 0:
         return True, ""
     P = sps.softmax(beta * z)
@@ -90,13 +128,35 @@ def selection_ok(z_ref: np.ndarray, n: int, k_gpu: int, idx_gpu: np.ndarray, p: 
     return True, f"{len(diff)} flipped at the cut"
 
 
+def budgets_match(k_gpu: np.ndarray, r: dict, p, z: np.ndarray, ln: np.ndarray, beta=None) -> tuple:
+    """Budgets equal to the oracle's (topp result r on scores z, lengths ln)
+    except at an ambiguous cut, where they may differ by one. p and beta:
+    scalars or per-unit arrays (beta None = 1)."""
+    pu = np.broadcast_to(np.asarray(p, np.float64), k_gpu.shape)
+    be = np.broadcast_to(np.asarray(1.0 if beta is None else beta, np.float64), k_gpu.shape)
+    bad = []
+    for u in range(len(k_gpu)):
+        AMBIG_TALLY["units"] += 1
+        if int(k_gpu[u]) == int(r["k"][u]):
+            continue
+        win = window(z[u], int(ln[u]), float(be[u]), int(r["k"][u]))
+        amb = abs(r["c_before"][u] - pu[u]) < win or abs(r["c_at"][u] - pu[u]) < win
+        if amb and abs(int(k_gpu[u]) - int(r["k"][u])) <= 1:
+            AMBIG_TALLY["ambiguous_accepts"] += 1
+        else:
+            bad.append((u, int(k_gpu[u]), int(r["k"][u])))
+    return not bad, bad
+
+
 def attn_close(out, ref):
+    """Elementwise |out - ref| <= ATOL on finite references, and -inf exactly
+    where the reference is -inf. Returns (ok, max abs error)."""
     out = np.asarray(out, np.float64)
     ref = np.asarray(ref, np.float64)
     fin = np.isfinite(ref)
     same_inf = np.array_equal(np.isneginf(out), np.isneginf(ref))
     err = np.abs(out[fin] - ref[fin])
-    ok = same_inf and bool(np.all(err <= ATOL + RTOL * np.abs(ref[fin])))
+    ok = same_inf and bool(np.all(err <= ATOL))
     return ok, (float(err.max()) if err.size else 0.0)
 
 

@@ -590,4 +590,317 @@ def pin_fit_boundaries_and_order():
     assert oracle.fit_temperature(z[:1], n[:1], np.array([np.log(2) - 1e-6]))[0] == oracle.FIT_BETA_MAX
 
 
+# ---- Condensed-tier formation (TS 2.A Tier 3 and pipeline step 4) -----------------------
+
+
+def _nearest_bf16_exact(x: float) -> float:
+    """The bf16 value nearest x (ties to an even last mantissa bit), by exact
+    rational arithmetic over the neighbouring representable values."""
+    from fractions import Fraction
+
+    fx = Fraction(x)
+    if fx == 0:
+        return 0.0
+    sign = -1 if fx < 0 else 1
+    a = abs(fx)
+    e = math.floor(math.log2(a))
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    step = Fraction(2) ** max(e - 7, -133)  # 8 significant bits; fixed spacing below 2^-126
+    lo = (a // step) * step
+    hi = lo + step
+    if a - lo < hi - a:
+        r = lo
+    elif hi - a < a - lo:
+        r = hi
+    else:
+        r = lo if (lo / step) % 2 == 0 else hi
+    return sign * float(r)
+
+
+def pin_round_to_bf16_is_nearest_even():
+    """Rounding a double to bf16 gives the nearest bf16 value, ties to even,
+    by exact rational arithmetic; this includes doubles that a detour through
+    float32 would round to a tie and then the wrong way."""
+    rng = np.random.default_rng(31)
+    xs = list(rng.standard_normal(300) * np.exp(rng.uniform(-20, 20, 300)))
+    xs += [1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, 1 + 2.0 ** -8 + 2.0 ** -40, 1 + 2.0 ** -8 - 2.0 ** -40,
+           -(1 + 2.0 ** -8 + 2.0 ** -40), 2.0 ** -130 * 1.37, 3.0e38, 0.0]
+    got = oracle.round_to_bf16(np.array(xs))
+    want = bf16_bits(np.array([_nearest_bf16_exact(x) for x in xs], np.float32))
+    assert np.array_equal(got, want), [(x, g, w) for x, g, w in zip(xs, got, want) if g != w][:3]
+
+
+def _calibrated(z, beta):
+    """m, logZ and the calibrated probabilities of scores z (scipy)."""
+    z64 = z.astype(np.float64)
+    m = np.float32(z64.max())
+    lz = sps.logsumexp(beta * (z64 - np.float64(m)))
+    return m, np.float32(lz), sps.softmax(beta * z64)
+
+
+def _cond_state(rng, B, H, ncap, ccap, D, n, C, dtype="f32"):
+    k, v, _ = rand_tier(rng, B, H, ncap, D, dtype)
+    ck, cv, _ = rand_tier(rng, B, H, ccap, D, dtype)
+    sp = oracle.Tier(k, v, np.asarray(n, np.int32))
+    co = oracle.Tier(ck, cv, np.asarray(C, np.int32))
+    w = rng.uniform(0.0, 1.0, (B * H, ccap)).astype(np.float32)
+    return sp, co, w
+
+
+def pin_condense_merge_is_weighted_average():
+    """MERGE: the new condensed slot is numpy's weighted average of the oldest
+    block's rows, weighted by the calibrated probabilities (scipy softmax);
+    its weight is the block's mass."""
+    rng = np.random.default_rng(32)
+    B, H, ncap, ccap, D, block = 1, 3, 40, 5, 16, 7
+    sp, co, w = _cond_state(rng, B, H, ncap, ccap, D, [40, 33, 7], [0, 2, 4])
+    z = rng.standard_normal((B * H, ncap)).astype(np.float32) * 3
+    beta = np.array([1.0, 0.5, 2.0], np.float32)
+    m = np.zeros(B * H, np.float32)
+    lz = np.zeros(B * H, np.float32)
+    P = []
+    for u in range(B * H):
+        m[u], lz[u], Pu = _calibrated(z[u, :sp.len[u]], float(beta[u]))
+        P.append(Pu)
+    s2, c2, w2, done = oracle.condense(sp, co, w, z, m, lz, beta, block, block, oracle.CONDENSE_MERGE)
+    assert list(done) == [1, 1, 1]
+    for u in range(B * H):
+        C = int(co.len[u])
+        a = P[u][:block]
+        for t_in, t_out in ((sp.k, c2.k), (sp.v, c2.v)):
+            ref = np.average(t_in[0, u, :block].astype(np.float64), axis=0, weights=a).astype(np.float32)
+            _ulp_close(t_out[0, u, C], ref)
+        assert abs(float(w2[u, C]) - a.sum()) <= 1e-6 * a.sum()
+        assert c2.len[u] == C + 1
+        # earlier slots untouched
+        assert np.array_equal(c2.k[0, u, :C], co.k[0, u, :C]) and np.array_equal(w2[u, :C], w[u, :C])
+
+
+def pin_condense_matches_list_model():
+    """A run of condensations against a plain Python model: per unit the sparse
+    tier as a list of rows in age order and the condensed tier as a list of
+    (row, weight); blocks leave from the old end; a full condensed tier first
+    merges its two oldest slots (MERGE, numpy weighted average) or drops its
+    oldest (EVICT); EVICT keeps the block's first highest-scoring token."""
+    rng = np.random.default_rng(33)
+    for policy in (oracle.CONDENSE_MERGE, oracle.CONDENSE_EVICT):
+        B, H, ncap, ccap, D, block, trig = 1, 2, 30, 3, 8, 4, 10
+        sp, co, w = _cond_state(rng, B, H, ncap, ccap, D, [30, 12], [1, 3])
+        model_s = [[(sp.k[0, u, i].copy(), sp.v[0, u, i].copy()) for i in range(sp.len[u])] for u in range(2)]
+        model_c = [[(co.k[0, u, i].copy(), co.v[0, u, i].copy(), np.float64(w[u, i])) for i in range(co.len[u])]
+                   for u in range(2)]
+        for rnd in range(7):
+            z = np.round(rng.standard_normal((2, ncap)) * 2).astype(np.float32)  # ties happen
+            m = np.zeros(2, np.float32)
+            lz = np.zeros(2, np.float32)
+            Ps = []
+            for u in range(2):
+                n = int(sp.len[u])
+                if n:
+                    m[u], lz[u], Pu = _calibrated(z[u, :n], 1.0)
+                else:
+                    Pu = np.zeros(0)
+                Ps.append(Pu)
+            sp, co, w, done = oracle.condense(sp, co, w, z, m, lz, None, block, trig, policy)
+            for u in range(2):
+                if len(model_s[u]) >= max(trig, block):
+                    assert done[u] == 1
+                    blk = model_s[u][:block]
+                    model_s[u] = model_s[u][block:]
+                    a = Ps[u][:block]
+                    if policy == oracle.CONDENSE_MERGE:
+                        if len(model_c[u]) == ccap:
+                            (k0, v0, w0), (k1, v1, w1) = model_c[u][0], model_c[u][1]
+                            ww = np.array([w0, w1])
+                            mk = np.average(np.stack([k0, k1]).astype(np.float64), axis=0, weights=ww)
+                            mv = np.average(np.stack([v0, v1]).astype(np.float64), axis=0, weights=ww)
+                            model_c[u] = [(mk.astype(np.float32), mv.astype(np.float32), w0 + w1)] + model_c[u][2:]
+                        nk = np.average(np.stack([r[0] for r in blk]).astype(np.float64), axis=0, weights=a)
+                        nv = np.average(np.stack([r[1] for r in blk]).astype(np.float64), axis=0, weights=a)
+                        model_c[u].append((nk.astype(np.float32), nv.astype(np.float32), a.sum()))
+                    else:
+                        if len(model_c[u]) == ccap:
+                            model_c[u] = model_c[u][1:]
+                        j = int(np.flatnonzero(z[u, :block] == z[u, :block].max())[0])
+                        model_c[u].append((blk[j][0], blk[j][1], a[j]))
+                else:
+                    assert done[u] == 0
+                assert sp.len[u] == len(model_s[u]) and co.len[u] == len(model_c[u]), (policy, rnd, u)
+                for i, (kk, vv) in enumerate(model_s[u]):
+                    assert np.array_equal(sp.k[0, u, i], kk) and np.array_equal(sp.v[0, u, i], vv)
+                for i, (kk, vv, ww) in enumerate(model_c[u]):
+                    # weights are known to about 1e-7 relative (the model keeps
+                    # float64 masses, the tier float32 ones), and a mean moves
+                    # by at most that times the spread of its rows
+                    for got, want in ((co.k[0, u, i], kk), (co.v[0, u, i], vv)):
+                        err = np.abs(got.astype(np.float64) - np.asarray(want, np.float64))
+                        assert np.all(err <= 1e-6 * (1 + np.abs(want))), (policy, rnd, u, i, err.max())
+                    assert abs(float(w[u, i]) - ww) <= 1e-5 * max(ww, 1e-30), (policy, rnd, u, i)
+
+
+def pin_condense_noop_drop_and_single_slot():
+    """Below the trigger nothing changes; a condensed tier of capacity 0 drops
+    the block; with one slot, MERGE folds the block into it (numpy weighted
+    average of the slot, weighted by its weight, and the block's rows)."""
+    rng = np.random.default_rng(34)
+    sp, co, w = _cond_state(rng, 1, 2, 20, 1, 8, [9, 20], [1, 1])
+    z = rng.standard_normal((2, 20)).astype(np.float32)
+    m = np.array([z[0, :9].max(), z[1].max()], np.float32)
+    lz = np.array([sps.logsumexp(z[0, :9] - m[0]), sps.logsumexp(z[1] - m[1])], np.float32)
+    s2, c2, w2, done = oracle.condense(sp, co, w, z, m, lz, None, 5, 10, oracle.CONDENSE_MERGE)
+    assert list(done) == [0, 1] and list(s2.len) == [9, 15] and list(c2.len) == [1, 1]
+    assert np.array_equal(s2.k[0, 0], sp.k[0, 0]) and np.array_equal(c2.k[0, 0], co.k[0, 0])
+    a = np.concatenate([[np.float64(w[1, 0])], np.exp(z[1, :5].astype(np.float64) - m[1] - np.float64(lz[1]))])
+    rows = np.concatenate([co.k[0, 1, :1], sp.k[0, 1, :5]]).astype(np.float64)
+    _ulp_close(c2.k[0, 1, 0], np.average(rows, axis=0, weights=a).astype(np.float32))
+    assert np.array_equal(s2.k[0, 1, :15], sp.k[0, 1, 5:20])
+    empty = oracle.Tier(np.zeros((1, 2, 0, 8), np.float32), np.zeros((1, 2, 0, 8), np.float32),
+                        np.zeros(2, np.int32))
+    s3, c3, w3, done = oracle.condense(sp, empty, np.zeros((2, 0), np.float32), z, m, lz, None, 5, 5,
+                                       oracle.CONDENSE_EVICT)
+    assert list(done) == [1, 1] and list(s3.len) == [4, 15] and list(c3.len) == [0, 0]
+    assert np.array_equal(s3.v[0, 0, :4], sp.v[0, 0, 5:9])
+
+
+def pin_condense_bf16_merge_exact():
+    """bf16 tiers: each merged element is the nearest bf16 value (ties to even,
+    exact rational arithmetic) to the exact weighted mean of the block, when
+    the mean is not within 1e-12 of a rounding tie."""
+    from fractions import Fraction
+
+    rng = np.random.default_rng(35)
+    sp, co, w = _cond_state(rng, 1, 1, 12, 4, 16, [12], [0], "bf16")
+    z = rng.standard_normal((1, 12)).astype(np.float32)
+    m = np.array([z[0].max()], np.float32)
+    lz = np.array([sps.logsumexp(z[0] - m[0])], np.float32)
+    s2, c2, w2, _ = oracle.condense(sp, co, w, z, m, lz, None, 6, 6, oracle.CONDENSE_MERGE)
+    a = np.exp(z[0, :6].astype(np.float64) - np.float64(m[0]) - np.float64(lz[0]))
+    for t_in, t_out in ((sp.k, c2.k), (sp.v, c2.v)):
+        rows = as_f64(t_in[0, 0, :6])
+        for d in range(16):
+            exact = sum(Fraction(float(a[j])) * Fraction(float(rows[j, d])) for j in range(6)) / \
+                sum(Fraction(float(x)) for x in a)
+            want = _nearest_bf16_exact(float(exact))
+            got = as_f64(t_out[0, 0, 0:1])[0, d]
+            if got != want:
+                # the float64 sums may only move a value that sits at a tie
+                spacing = abs(want) * 2.0 ** -8
+                assert abs(abs(float(exact) - want) - spacing / 2) <= 1e-12 * abs(want), (d, got, want)
+
+
+# ---- Rewrite Cache vs Sparse Loading (TS 2.C Trade-off Management) ------------------------
+
+
+def pin_mti_trigger_and_horizon():
+    """The trigger is a hysteresis on the budget: above L_upper rewrite, below
+    L_lower sparse loading, in between the previous mode; a rewrite of k rows
+    serves the largest H >= 1 with k H within the memory-time allowance
+    (brute force)."""
+    R, S = oracle.MODE_REWRITE, oracle.MODE_SPARSE
+    table = [(5, S, 10, 20, S), (5, R, 10, 20, S), (10, R, 10, 20, R), (10, S, 10, 20, S), (15, R, 10, 20, R),
+             (20, S, 10, 20, S), (21, S, 10, 20, R), (21, R, 10, 20, R), (0, R, 0, 0, R), (1, S, 0, 0, R)]
+    for k, mode, lo, hi, want in table:
+        assert oracle.mti_trigger(k, mode, lo, hi) == want, (k, mode, lo, hi)
+    for k in range(1, 70):
+        for cap in (0, 1, 63, 64, 65, 1000, 4096):
+            best = max([h for h in range(1, 5000) if k * h <= cap] or [1])
+            assert oracle.mti_horizon(k, cap) == best, (k, cap)
+    assert oracle.mti_horizon(0, 100) == 1
+
+
+def _mti_case(seed, dtype="f32"):
+    rng = np.random.default_rng(seed)
+    B, Hkv, G, D, n, W, C = 1, 3, 2, 16, 40, 5, 3
+    q = rand_q(rng, B, Hkv * G, D, dtype)
+    tiers = [oracle.Tier(*rand_tier(rng, B, Hkv, cap, D, dtype)) for cap in (W, n, C)]
+    return rng, q, tiers
+
+
+def pin_mti_reuse_attends_the_rewritten_rows():
+    """A unit whose rewrite still serves attends over dense ++ its rewritten
+    rows ++ condensed (torch SDPA over the concatenation), reports those rows'
+    indices, and counts one step down; the others run the plain step."""
+    rng, q, (dense, sparse, cond) = _mti_case(41)
+    B, Hkv, D, bmax = 1, 3, 16, 12
+    scale = 1 / math.sqrt(D)
+    st = oracle.mti_state(3, bmax, B, Hkv, D, sparse.k)
+    st["left"][:] = [2, 0, 1]
+    st["rw_len"][:] = [7, 0, 12]
+    st["rw_k"][...] = rng.standard_normal(st["rw_k"].shape).astype(np.float32)
+    st["rw_v"][...] = rng.standard_normal(st["rw_v"].shape).astype(np.float32)
+    st["rw_idx"][:] = rng.integers(0, 40, (3, bmax))
+    res, st2 = oracle.step_mti(q, dense, sparse, cond, scale, 0.9, 2, bmax, st, 4, 8, 100)
+    assert list(res["fresh"]) == [0, 1, 0] and list(st2["left"][[0, 2]]) == [1, 0]
+    for u in (0, 2):
+        n = int(st["rw_len"][u])
+        k = np.concatenate([dense.k[0, u], st["rw_k"][0, u, :n], cond.k[0, u]]).astype(np.float64)
+        v = np.concatenate([dense.v[0, u], st["rw_v"][0, u, :n], cond.v[0, u]]).astype(np.float64)
+        qq = torch.from_numpy(q[0, 2 * u:2 * u + 2].astype(np.float64))
+        ref = F.scaled_dot_product_attention(qq[None, :, None, :], torch.from_numpy(k)[None, None].expand(1, 2, -1, -1),
+                                             torch.from_numpy(v)[None, None].expand(1, 2, -1, -1), scale=scale)
+        assert np.allclose(res["out"][0, 2 * u:2 * u + 2], ref[0, :, 0].numpy(), atol=1e-6)
+        assert res["k"][u] == n and np.array_equal(res["idx"][u, :n], st["rw_idx"][u, :n])
+        assert np.all(res["idx"][u, n:] == -1)
+    plain = oracle.step(q, dense, sparse, cond, scale, 0.9, 2, bmax)
+    assert np.array_equal(res["out"][0, 2:4], plain["out"][0, 2:4]) and res["k"][1] == plain["k"][1]
+
+
+def pin_mti_rewrite_copies_the_top_rows():
+    """A fresh unit whose budget crosses L_upper copies its selected rows: the
+    rows of the top-k tokens by (score desc, index asc) from numpy's own sort,
+    in token order (numpy fancy indexing); one whose budget falls below L_lower
+    drops its rewrite."""
+    rng, q, (dense, sparse, cond) = _mti_case(42)
+    B, Hkv, D, bmax = 1, 3, 16, 6
+    scale = 1 / math.sqrt(D)
+    st = oracle.mti_state(3, bmax, B, Hkv, D, sparse.k)
+    st["mode"][:] = [0, 1, 1]
+    st["rw_len"][:] = [0, 3, 3]
+    # budgets: bmin = bmax = 6 makes every fresh budget 6
+    res, st2 = oracle.step_mti(q, dense, sparse, cond, scale, 0.5, bmax, bmax, st, 4, 5, 60)
+    assert list(st2["mode"]) == [1, 1, 1] and list(st2["rw_len"]) == [6, 6, 6] and list(st2["left"]) == [9, 9, 9]
+    qf = q.astype(np.float64).reshape(1, 3, 2, 16)
+    for u in range(3):
+        z = (np.einsum("gd,nd->gn", qf[0, u], sparse.k[0, u].astype(np.float64)) * scale).max(axis=0)
+        top = np.sort(order_desc(z.astype(np.float32))[:6])
+        assert np.array_equal(st2["rw_idx"][u, :6], top)
+        assert np.array_equal(st2["rw_k"][0, u, :6], sparse.k[0, u][top])
+        assert np.array_equal(st2["rw_v"][0, u, :6], sparse.v[0, u][top])
+    res3, st3 = oracle.step_mti(q, dense, sparse, cond, scale, 1e-4, 1, bmax,
+                                st2 | {"left": np.zeros(3, np.int32)}, 4, 5, 60)
+    assert np.all(res3["k"] < 4)
+    assert list(st3["mode"]) == [0, 0, 0] and list(st3["rw_len"]) == [0, 0, 0] and list(st3["left"]) == [0, 0, 0]
+
+
+def pin_mti_state_matches_model():
+    """Many steps with scripted budgets against a plain model of the trigger:
+    per unit a mode and a count of steps left, a rewrite served H(k) steps."""
+    rng, q, (dense, sparse, cond) = _mti_case(43)
+    B, Hkv, D, bmax = 1, 3, 16, 30
+    scale = 1 / math.sqrt(D)
+    lo, hi, cap = 8, 20, 90
+    st = oracle.mti_state(3, bmax, B, Hkv, D, sparse.k)
+    model = [[0, 0, 0] for _ in range(3)]  # mode, left, rows
+    for step_i in range(40):
+        kf = rng.integers(0, 31, 3).astype(np.int32)
+        idf = np.stack([np.sort(rng.choice(40, bmax, replace=False)).astype(np.int32) for _ in range(3)])
+        res, st = oracle.step_mti(q, dense, sparse, cond, scale, 0.9, 1, bmax, st, lo, hi, cap, kf, idf)
+        for u in range(3):
+            mode, left, rows = model[u]
+            if left > 0:
+                assert res["fresh"][u] == 0 and res["k"][u] == rows
+                model[u] = [mode, left - 1, rows]
+            else:
+                assert res["fresh"][u] == 1
+                k = int(kf[u])
+                mode = 1 if k > hi else (0 if k < lo else mode)
+                model[u] = [mode, (max(1, cap // k) - 1) if (mode and k) else 0, k if mode else 0]
+                if mode:
+                    assert np.array_equal(st["rw_idx"][u, :k], idf[u, :k])
+            assert [int(st["mode"][u]), int(st["left"][u]), int(st["rw_len"][u])] == model[u], (step_i, u)
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_") and callable(v)]

@@ -28,7 +28,7 @@ def declared_symbols():
 
 def test_every_declared_symbol_is_exported(hk):
     names = declared_symbols()
-    assert len(names) == 17, names
+    assert len(names) == 21, names
     for n in names:
         assert hasattr(hk.lib, n), n
     nm = os.popen(f"nm -D --defined-only {hk.LIB_PATH}").read()
@@ -129,6 +129,66 @@ def test_append_validates_on_the_host(hk):
     assert call(dense=bad) == "HKV_ERR_INVALID_ARG"
     assert hk.STATUS[hk.lib.hkv_append(C.byref(_prob(hk, D=96).c()), kn, vn, C.byref(d), head, C.byref(s),
                                        None, ws, 256, None)] == "HKV_ERR_UNSUPPORTED"
+
+
+def test_condense_validates_on_the_host(hk):
+    """hkv_condense refuses bad arguments before launching anything."""
+    prob = _prob(hk)
+    s, c = _tier(hk, 1000, addr=0x40000000), _tier(hk, 16)
+    ws, w, z, m, lz = (C.c_void_p(a) for a in (0x500000, 0x600000, 0x700000, 0x800000, 0x900000))
+
+    def call(sparse=s, cond=c, w=w, z=z, zs=1000, m=m, lz=lz, block=16, trig=1000, pol=0, ws=ws, wsb=256):
+        return hk.STATUS[hk.lib.hkv_condense(C.byref(prob.c()), sparse and C.byref(sparse), cond and C.byref(cond),
+                                             w, z, zs, m, lz, block, trig, pol, None, ws, wsb, None)]
+
+    assert call(sparse=None) == "HKV_ERR_INVALID_ARG"
+    assert call(block=0) == "HKV_ERR_INVALID_ARG"
+    assert call(block=1001) == "HKV_ERR_INVALID_ARG"          # more than the sparse capacity
+    assert call(block=hk.CONDENSE_MAX_BLOCK + 1) == "HKV_ERR_INVALID_ARG"
+    assert call(trig=-1) == "HKV_ERR_INVALID_ARG"
+    assert call(pol=2) == "HKV_ERR_INVALID_ARG"
+    assert call(w=None) == "HKV_ERR_INVALID_ARG"              # slots need their weights
+    assert call(m=None) == "HKV_ERR_INVALID_ARG"              # scores: all three or none
+    assert call(zs=999) == "HKV_ERR_INVALID_ARG"
+    assert call(wsb=128) == "HKV_ERR_WORKSPACE"
+    assert call(ws=None) == "HKV_ERR_WORKSPACE"
+
+
+def test_step_mti_validates_on_the_host(hk):
+    """hkv_step_mti refuses bad thresholds, state or outputs before launching anything."""
+    prob = _prob(hk)
+    d, s, c = _tier(hk, 64), _tier(hk, 1000, addr=0x40000000), _tier(hk, 16)
+    code, n = _ws_size(hk, prob, d, s, c)
+    assert code == 0
+    ws = C.c_void_p(0x7000000)
+
+    def mti(**kw):
+        f = dict(L_lower=10, L_upper=20, mti_cap=1000, mode=0x500000, left=0x510000,
+                 rewrite=_tier(hk, 64, addr=0x60000000), rw_idx=0x520000)
+        f.update(kw)
+        return hk._Mti(**f)
+
+    def call(m, **out):
+        o = dict(sel_len=0x800000, idx=0x810000, out=0x820000)
+        o.update(out)
+        so = hk._StepOut(**o)
+        return hk.STATUS[hk.lib.hkv_step_mti(C.byref(prob.c()), C.c_void_p(0x100000), C.byref(d), C.byref(s),
+                                             C.byref(c), m and C.byref(m), C.byref(so), ws, n, None)]
+
+    assert call(None) == "HKV_ERR_INVALID_ARG"
+    assert call(mti(L_lower=30)) == "HKV_ERR_INVALID_ARG"          # L_lower above L_upper
+    assert call(mti(L_lower=-1)) == "HKV_ERR_INVALID_ARG"
+    assert call(mti(mti_cap=-5)) == "HKV_ERR_INVALID_ARG"
+    assert call(mti(left=None)) == "HKV_ERR_INVALID_ARG"
+    assert call(mti(rw_idx=0x520002)) == "HKV_ERR_INVALID_ARG"     # misaligned
+    assert call(mti(rewrite=_tier(hk, 63, addr=0x60000000))) == "HKV_ERR_INVALID_ARG"  # buffer below bmax
+    assert call(mti(), k_out=0x900000, v_out=0x910000) == "HKV_ERR_INVALID_ARG"     # no Rewrite Cache outputs
+    assert call(mti(), beta_fit=0x920000) == "HKV_ERR_INVALID_ARG"                 # no fitted temperature
+    big = _prob(hk, B=600, Hkv=2)
+    code, nb = _ws_size(hk, big, d, s, c)
+    so = hk._StepOut(sel_len=0x800000, idx=0x810000, out=0x820000)
+    assert hk.STATUS[hk.lib.hkv_step_mti(C.byref(big.c()), C.c_void_p(0x100000), C.byref(d), C.byref(s), C.byref(c),
+                                         C.byref(mti()), C.byref(so), ws, nb, None)] == "HKV_ERR_UNSUPPORTED"
 
 
 def test_fit_entry_points_validate_on_the_host(hk):

@@ -73,10 +73,20 @@ def test_calibrate(case):
     Pg = Pg.cpu().numpy()
     assert np.array_equal(m.cpu().numpy(), mr)
     assert np.allclose(lz.cpu().numpy(), lzr, rtol=0, atol=2e-6)
+    # P = w / Z in fp32. The weight is within 2^-22 + 3 2^-24 ln2 x_j relative
+    # (x_j = beta log2e (m - z_j); see gpu_helpers.window), Z (a double sum of
+    # such weights) within 2^-22 + 3 2^-24 ln2 E_P[x], and the rounding of 1/Z
+    # to fp32 and of the product add 2^-23; 1.5 times that, for results in the
+    # normal fp32 range.
+    c = 3 * 2.0 ** -24 * np.log(2)
     for u in range(wl.units):
         n = ln[u]
-        tol = 1e-6 * (2 + beta[u] * (mr[u] - zr[u, :n])) * Pr[u, :n] + 1e-12
-        assert np.all(np.abs(Pg[u, :n] - Pr[u, :n]) <= tol), (name, u)
+        x = beta[u] * np.log2(np.e) * (np.float64(mr[u]) - zr[u, :n].astype(np.float64))
+        ex = float(np.sum(Pr[u, :n].astype(np.float64) * x))
+        rel = 2 * 2.0 ** -22 + c * (x + ex) + 2.0 ** -23
+        tol = 1.5 * rel * Pr[u, :n] + 2e-38
+        err = np.abs(Pg[u, :n] - Pr[u, :n])
+        assert np.all(err <= tol), (name, u, float(np.max(err / np.maximum(Pr[u, :n], 1e-300))))
 
 
 @pytest.mark.parametrize("p", [0.0, 0.3, 0.8, 0.95, 1.0])
@@ -101,10 +111,8 @@ def test_topp_and_compact_identical_scores(case, p):
         assert ws.status() == 0
         kg = sel.cpu().numpy()
         r = oracle.topp(zr, ln, p, wl.bmin, wl.bmax)
-        for u in range(U):
-            if kg[u] != r["k"][u]:
-                amb = abs(r["c_before"][u] - p) < H.AMBIG or abs(r["c_at"][u] - p) < H.AMBIG
-                assert amb and abs(int(kg[u]) - int(r["k"][u])) <= 1, (name, p, u, kg[u], r["k"][u])
+        ok, bad = H.budgets_match(kg, r, p, zr, ln)
+        assert ok, (name, p, bad)
         ct = cut.cpu().numpy()
         assert np.array_equal(ct[:, 1] + ct[:, 2], kg)
         want = oracle.compact(zr, ln, kg, wl.bmax, layout)

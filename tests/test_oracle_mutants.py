@@ -151,3 +151,91 @@ def test_fit_mutant_is_caught(name, monkeypatch):
         except Exception:
             failed = True
     assert failed, f"mutant {name} passed every fitted-temperature pin"
+
+
+# ---- the numpy condensed-tier formation (TS 2.A Tier 3, pipeline step 4) ----
+
+CONDENSE_MUTANTS = {
+    "newest_block_condensed": ("condense", "rows_k, rows_v = _f64(sk[b, h, :block]), _f64(sv[b, h, :block])",
+                               "rows_k, rows_v = _f64(sk[b, h, n - block:n]), _f64(sv[b, h, n - block:n])"),
+    "full_tier_not_shifted": ("condense", "ck[b, h, 1:ccap - 1] = ck[b, h, 2:ccap].copy()",
+                              "ck[b, h, 1:ccap - 1] = ck[b, h, 1:ccap - 1].copy()"),
+    "evict_least_important": ("condense", "jstar = int(np.argmax(zz))", "jstar = int(np.argmin(zz))"),
+    "evict_drops_newest_slot": ("condense", "ck[b, h, 0:ccap - 1] = ck[b, h, 1:ccap].copy()",
+                                "ck[b, h, 0:ccap - 1] = ck[b, h, 0:ccap - 1].copy()"),
+    "sparse_not_moved_down": ("condense", "sk[b, h, :n - block] = sk[b, h, block:n].copy()",
+                              "sk[b, h, :n - block] = sk[b, h, :n - block].copy()"),
+    "trigger_ignored": ("condense", "if n < max(trigger, block, 1):", "if n < max(block, 1):"),
+    "mass_not_kept": ("condense", "w[u, C] = np.float32(_seq_sum(a))", "w[u, C] = np.float32(1.0)"),
+    "beta_ignored": ("condense", "a = np.exp(be * (zz", "a = np.exp(1.0 * (zz"),
+    "unweighted_mean": ("_weighted_mean", "num = num + a[j] * rows[j]", "num = num + rows[j] * (den * 0 + 1)"),
+    "bf16_round_half_up": ("round_to_bf16", "r = np.rint(np.ldexp(x, -sh))", "r = np.floor(np.ldexp(x, -sh) + 0.5)"),
+    "bf16_through_float32": ("round_to_bf16", "f, e = np.frexp(x)",
+                             "x = x.astype(np.float32).astype(np.float64)\n    f, e = np.frexp(x)"),
+}
+
+
+@pytest.mark.filterwarnings("ignore::RuntimeWarning")
+@pytest.mark.parametrize("name", sorted(CONDENSE_MUTANTS))
+def test_condense_mutant_is_caught(name, monkeypatch):
+    import inspect
+    import textwrap
+
+    import oracle
+    from tests import pins
+
+    fn, old, new = CONDENSE_MUTANTS[name]
+    src = textwrap.dedent(inspect.getsource(getattr(oracle, fn)))
+    assert old in src, name
+    ns = dict(vars(oracle))
+    exec(compile(src.replace(old, new), "<mutant>", "exec"), ns)
+    monkeypatch.setattr(oracle, fn, ns[fn])
+    # the module's other functions look helpers up in the module namespace
+    failed = False
+    for pin in (pins.pin_round_to_bf16_is_nearest_even, pins.pin_condense_merge_is_weighted_average,
+                pins.pin_condense_matches_list_model, pins.pin_condense_noop_drop_and_single_slot,
+                pins.pin_condense_bf16_merge_exact):
+        try:
+            pin()
+        except Exception:
+            failed = True
+    assert failed, f"mutant {name} passed every condensation pin"
+
+
+# ---- the numpy Rewrite Cache / Sparse Loading trigger (TS 2.C Trade-off Management) ----
+
+MTI_MUTANTS = {
+    "trigger_inverted": ("mti_trigger", "if k > L_upper:\n        return MODE_REWRITE",
+                         "if k > L_upper:\n        return MODE_SPARSE"),
+    "no_hysteresis": ("mti_trigger", "    return mode", "    return MODE_SPARSE"),
+    "horizon_floor_missing": ("mti_horizon", "max(1, mti_cap // k)", "max(1, -(-mti_cap // k))"),
+    "reuse_not_counted_down": ("step_mti", 'st["left"][u] -= 1', 'st["left"][u] -= 0'),
+    "horizon_counts_the_rewrite_step_twice": ("step_mti", "mti_horizon(ku, mti_cap) - 1", "mti_horizon(ku, mti_cap)"),
+    "rewrite_of_the_wrong_rows": ("step_mti", "rows = idf[u, :ku]", "rows = idf[u, :ku] * 0"),
+    "reuse_attends_plain_step": ("step_mti", "out[b, h * G:(h + 1) * G] = r_out[b, h * G:(h + 1) * G]",
+                                 "out[b, h * G:(h + 1) * G] = plain['out'][b, h * G:(h + 1) * G]"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MTI_MUTANTS))
+def test_mti_mutant_is_caught(name, monkeypatch):
+    import inspect
+    import textwrap
+
+    import oracle
+    from tests import pins
+
+    fn, old, new = MTI_MUTANTS[name]
+    src = textwrap.dedent(inspect.getsource(getattr(oracle, fn)))
+    assert old in src, name
+    ns = dict(vars(oracle))
+    exec(compile(src.replace(old, new), "<mutant>", "exec"), ns)
+    monkeypatch.setattr(oracle, fn, ns[fn])
+    failed = False
+    for pin in (pins.pin_mti_trigger_and_horizon, pins.pin_mti_reuse_attends_the_rewritten_rows,
+                pins.pin_mti_rewrite_copies_the_top_rows, pins.pin_mti_state_matches_model):
+        try:
+            pin()
+        except Exception:
+            failed = True
+    assert failed, f"mutant {name} passed every trigger pin"

@@ -18,15 +18,17 @@ from tests import gpu_helpers as H
 from tests.test_gpu_stages import CASES
 
 
-def _reference_and_inputs(name):
-    """Selection from hkv_step, then the workspace cascade decode over it."""
+def _reference_and_inputs(name, layout=hkv.PAD_MAX):
+    """Selection from hkv_step (index rows in `layout`), then the workspace
+    cascade decode over it."""
     wl = CASES[name]
     x = H.inputs(wl)
-    prob, step_out, ws = H.run_step(wl, x)
+    prob, step_out, ws = H.run_step(wl, x, layout=layout)
     dense, sparse, cond = H.tiers_of(x)
     ref = torch.zeros(wl.B, wl.Hq, wl.D, device=H.dev())
     ref_lse = torch.zeros(wl.B, wl.Hq, device=H.dev())
-    hkv.cascade_decode(prob, x.q, dense, sparse, step_out.idx, step_out.sel_len, cond, ref, ws, lse=ref_lse)
+    hkv.cascade_decode(prob, x.q, dense, sparse, step_out.idx, step_out.sel_len, cond, ref, ws, lse=ref_lse,
+                       offsets=step_out.offsets)
     torch.cuda.synchronize()
     assert ws.status() == 0
     return wl, x, prob, step_out, (dense, sparse, cond), ref, ref_lse
@@ -34,22 +36,27 @@ def _reference_and_inputs(name):
 
 @pytest.mark.gpu
 def test_noalloc_decode_matches_workspace_decode_on_consecutive_calls():
-    # two calls in a row on different problems, then the first problem again:
-    # each must match the workspace entry point whatever the array last held
-    cases = ["bf16_b2_n3000", "fp32_d128_g8", "bf16_b2_n3000"]
-    for call, name in enumerate(cases):
-        wl, x, prob, so, (dense, sparse, cond), ref, ref_lse = _reference_and_inputs(name)
+    # calls in a row on different problems and layouts, the first problem
+    # again, and calls without lse or status: each must match the workspace
+    # entry point whatever the array last held
+    cases = [("bf16_b2_n3000", hkv.PAD_MAX, True), ("fp32_d128_g8", hkv.PAD_MAX, True),
+             ("bf16_ragged", hkv.FLAT_SUM, True), ("bf16_b2_n3000", hkv.PAD_MAX, True),
+             ("bf16_hetero", hkv.FLAT_SUM, False), ("bf16_b2_n3000", hkv.PAD_MAX, False)]
+    for call, (name, layout, extras) in enumerate(cases):
+        wl, x, prob, so, (dense, sparse, cond), ref, ref_lse = _reference_and_inputs(name, layout)
         out = torch.full_like(ref, float("nan"))
-        lse = torch.full_like(ref_lse, float("nan"))
-        status = torch.full((1,), -1, dtype=torch.int32, device=H.dev())
+        lse = torch.full_like(ref_lse, float("nan")) if extras else None
+        status = torch.full((1,), -1, dtype=torch.int32, device=H.dev()) if extras else None
         hkv.cascade_decode_noalloc(prob, x.q, dense, sparse, so.idx, so.sel_len, cond, out, lse=lse,
-                                   status=status)
+                                   offsets=so.offsets, status=status)
         torch.cuda.synchronize()
-        assert int(status.item()) == 0, (call, name, int(status.item()))
+        if status is not None:
+            assert int(status.item()) == 0, (call, name, int(status.item()))
         ok, err = H.attn_close(out.cpu().numpy(), ref.cpu().numpy())
         assert ok, (call, name, "out", err)
-        ok, err = H.attn_close(lse.cpu().numpy(), ref_lse.cpu().numpy())
-        assert ok, (call, name, "lse", err)
+        if lse is not None:
+            ok, err = H.attn_close(lse.cpu().numpy(), ref_lse.cpu().numpy())
+            assert ok, (call, name, "lse", err)
 
 
 def test_noalloc_refuses_problems_beyond_its_array():
