@@ -311,6 +311,177 @@ def config_of(wl, world: int) -> dict:
             "timing": f"CUDA graphs of {GRAPH_STEPS} consecutive steps replayed back to back; CUDA events around the K steps"}
 
 
+# ---- the other workloads, the timeline and the rows beyond the step -----------------
+
+
+def capture(fn, stream):
+    """One call of fn outside capture (warm-up), then fn captured in a CUDA graph."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def replay_ms(g, stream, min_ms=300.0, warm=3) -> float:
+    """Mean device time of one replay of g, timed with CUDA events over enough
+    replays to last about min_ms."""
+    for _ in range(warm):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    one = max(e0.elapsed_time(e1), 1e-3)
+    reps = int(max(5, min(20000, min_ms / one)))
+    e0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def in_step_spans(hkv, prob, x, tiers, out, ws, stream, reps=20) -> dict:
+    """Live in-step times of each kernel of one step: the kernels record their
+    earliest start and latest end in the workspace (hkv_set_timeline); medians
+    over single-step graph replays, relative to the scorer's start (us)."""
+    hkv.set_timeline(True)
+    try:
+        g = capture(lambda: hkv.step(prob, x.q, *tiers, out, ws), stream)
+        hkv.read_timeline(ws)
+        rows = []
+        for _ in range(reps):
+            g.replay()
+            torch.cuda.synchronize()
+            rows.append(hkv.read_timeline(ws))
+        del g
+    finally:
+        hkv.set_timeline(False)
+    spans = {}
+    for kind in rows[0]:
+        rel = [(r[kind][0] - r["score"][0], r[kind][1] - r["score"][0]) for r in rows if kind in r]
+        st = statistics.median(a for a, _ in rel) / 1e3
+        en = statistics.median(b for _, b in rel) / 1e3
+        spans[kind] = {"start_us": round(st, 2), "end_us": round(en, 2), "us": round(en - st, 2)}
+    step = statistics.median((max(b for _, b in r.values()) - r["score"][0]) for r in rows) / 1e3
+    spans["step_us"] = round(step, 2)
+    return spans
+
+
+def oracle_sample(wl, hs, layers: int, seconds: float = 2.0) -> dict:
+    """The oracle on as many units of one layer as fit in about `seconds`,
+    scaled to steps/s of the whole workload (all units of all layers)."""
+    import oracle
+
+    done, t0 = 0, time.perf_counter()
+    while True:
+        oracle_units(wl, hs, [done % wl.units])
+        done += 1
+        dt = time.perf_counter() - t0
+        if dt >= seconds or done >= wl.units:
+            break
+    per_unit = dt / done
+    return {"value": round(1.0 / (per_unit * wl.units * layers), 6), "unit": "steps/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{done} unit(s) of one layer in {dt:.1f} s, scaled to {wl.units} units x {layers} layer(s)"}
+
+
+def workload_entry(hkv, wl, device, stream, p=None, with_oracle=True) -> dict:
+    """Throughput of one workload: all its layers' steps issued back to back on
+    one stream, captured in one CUDA graph and replayed."""
+    peak, peak_kind = peaks()
+    p = wl.p if p is None else p
+    xs = [make_inputs(wl, device, layer) for layer in range(wl.layers)]
+    prob = hkv.Problem(wl.B, wl.Hq, wl.Hkv, wl.D, wl.dtype, p, wl.bmin, wl.bmax)
+    tiers = [[hkv.Tier(t.k, t.v, t.len) for t in (x.dense, x.sparse, x.condensed)] for x in xs]
+    outs = [hkv.StepOutputs.allocate(prob, tiers[0][1], device) for _ in xs]
+    ws = hkv.Workspace(prob, *tiers[0])
+
+    def all_layers():
+        for x, t, o in zip(xs, tiers, outs):
+            hkv.step(prob, x.q, *t, o, ws)
+
+    g = capture(all_layers, stream)
+    ms = replay_ms(g, stream)
+    assert ws.status() == 0, f"device status word set on {wl.name}"
+    nbytes, ks = 0, []
+    for x, o in zip(xs, outs):
+        k = o.sel_len.cpu().numpy()
+        ks.append(k)
+        nbytes += step_bytes(wl, x.sparse.len.cpu().numpy(), x.dense.len.cpu().numpy(),
+                             x.condensed.len.cpu().numpy(), k)
+    ks = np.concatenate(ks)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    e = {"workload": wl.name, "p": p, "layers": wl.layers, "units_per_layer": wl.units,
+         "step_us": round(ms * 1e3, 2), "steps_per_s": round(1e3 / ms, 2),
+         "bytes_per_step": int(nbytes), "kv_gbs": round(gbs, 1),
+         "frac_of_8tbs": round(gbs / NOMINAL_HBM_GBS, 4), "frac_of_peak": round(gbs / peak, 4),
+         "peak_kind": peak_kind,
+         "budgets": {"min": int(ks.min()), "median": int(np.median(ks)), "max": int(ks.max()),
+                     "mean": round(float(ks.mean()), 1)}}
+    if with_oracle:
+        e["cpu_baseline"] = oracle_sample(wl.with_(p=p), host_state(xs[0]), wl.layers)
+    del g
+    return e
+
+
+def mti_entry(hkv, wl, x, prob, tiers, plain_ms, device, stream, horizon=4) -> dict:
+    """Rewrite Cache vs Sparse Loading on one decode state: a fresh step that
+    also rewrites every unit's selection, a step that reuses the rewrites, and
+    the number of reuse steps that pay for a rewrite."""
+    st = hkv.MtiState.allocate(prob, device, 0, 0, horizon * max(wl.bmax, 1))
+    out = hkv.StepOutputs.allocate(prob, tiers[1], device)
+    ws = hkv.Workspace(prob, *tiers)
+
+    def fresh():
+        st.left.zero_()
+        st.mode.zero_()
+        hkv.step_mti(prob, x.q, *tiers, st, out, ws)
+
+    rw_ms = replay_ms(capture(fresh, stream), stream)
+    st.left.fill_(1 << 30)  # every unit keeps reusing the rewrite the last fresh step made
+    reuse_ms = replay_ms(capture(lambda: hkv.step_mti(prob, x.q, *tiers, st, out, ws), stream), stream)
+    assert ws.status() == 0
+    gain = plain_ms - reuse_ms
+    return {"workload": wl.name, "policy": f"L_lower 0, L_upper 0 (every unit rewrites), horizon {horizon}",
+            "plain_step_us": round(plain_ms * 1e3, 2), "rewrite_step_us": round(rw_ms * 1e3, 2),
+            "reuse_step_us": round(reuse_ms * 1e3, 2),
+            "rewrite_cost_us": round((rw_ms - plain_ms) * 1e3, 2),
+            "steps_to_amortize": round((rw_ms - plain_ms) / gain, 3) if gain > 0 else None,
+            "cycle_steps_per_s": round(horizon / (rw_ms + (horizon - 1) * reuse_ms) * 1e3, 1)}
+
+
+def condense_entry(hkv, wl, x, prob, out, device, stream, block=256) -> dict:
+    """One condensation pass with every unit's sparse tier full (MERGE)."""
+    sk, sv, cv, ck = (t.clone() for t in (x.sparse.k, x.sparse.v, x.condensed.v, x.condensed.k))
+    slen0, clen0 = x.sparse.len.clone(), torch.zeros_like(x.condensed.len)
+    slen, clen = slen0.clone(), clen0.clone()
+    sp, co = hkv.Tier(sk, sv, slen), hkv.Tier(ck, cv, clen)
+    w = torch.zeros(wl.units, wl.c_cap, device=device)
+    ws = hkv.Workspace(prob, None, sp, co)
+    z = torch.zeros(wl.units, wl.n_cap, device=device)
+    m = torch.zeros(wl.units, device=device)
+    lz = torch.zeros(wl.units, device=device)
+
+    def once():
+        slen.copy_(slen0)
+        clen.copy_(clen0)
+        hkv.condense(prob, sp, co, w, ws, block, wl.n_cap, hkv.CONDENSE_MERGE, z=z, m=m, logZ=lz)
+
+    ms = replay_ms(capture(once, stream), stream, min_ms=100.0)
+    assert ws.status() == 0
+    e = 2 if wl.dtype == torch.bfloat16 else 4
+    moved = int(slen0.sum().item()) - wl.units * block
+    nbytes = moved * 2 * wl.D * e * 2 + wl.units * block * 2 * wl.D * e
+    return {"workload": wl.name, "block": block, "policy": "merge", "us": round(ms * 1e3, 2),
+            "gbs": round(nbytes / (ms / 1e3) / 1e9, 1), "us_per_step_amortized": round(ms * 1e3 / block, 3)}
+
+
 # ---- our arm ----------------------------------------------------------------------------
 
 
@@ -445,12 +616,19 @@ def run_ours(args):
                 "frac": round(achieved_gbs / peak, 4), "traffic": traffic_from_profile(kernel),
                 "peak_kind": peak_kind, "kernel": kernel, "bytes_per_launch": int(score_bytes),
                 "launch_us": round(score_ms * 1e3, 2)}
+    # the attention again, through the entry point that allocates nothing
+    noalloc_ms = kernel_ms(lambda: [hkv.cascade_decode_noalloc(prob, x.q, *tiers[:2], out.idx, out.sel_len,
+                                                               tiers[2], out.out, lse=out.lse)
+                                    for x, prob, tiers, out in sets], NSETS, stream, args)
+    noalloc_ms = max_over_ranks(noalloc_ms, dist, device)
     kernels = {"step_us": round(launch_ms_max * 1e3, 2), "step_gbs": round(step_gbs, 1),
                "score_us": round(score_ms * 1e3, 2), "attn_us": round(attn_ms * 1e3, 2),
-               "select_compact_us_remainder": round((launch_ms_max - score_ms - attn_ms) * 1e3, 2),
+               "attn_noalloc_us": round(noalloc_ms * 1e3, 2),
                "append_us": round(append_ms * 1e3, 2),
                "fitted_step_us": round(fitted_ms * 1e3, 2),
                "append_bytes": int(append_bytes(wl))}
+    # live in-step spans of every kernel of the step (device timeline)
+    kernels["in_step"] = in_step_spans(hkv, *sets[0][1:2], sets[0][0], sets[0][2], sets[0][3], ws, stream)
 
     # end to end through the public API: per step, copy the step's query and the
     # per-unit lengths from pinned host memory, run, and read the outputs back
@@ -488,8 +666,29 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         base = cpu_baseline(wl, host_state(sets[0][0]), args.cpu_seconds)
 
-    del multi
-    singles.clear()
+    # the other workloads, and the rows beyond the step, on one GPU
+    extras = None
+    if world == 1 and not args.headline_only:
+        x0, prob0, tiers0, out0 = sets[0]
+        extras = {"mti": mti_entry(hkv, wl, x0, prob0, tiers0, launch_ms_max, device, stream),
+                  "condense": condense_entry(hkv, wl, x0, prob0, out0, device, stream)}
+        del multi
+        singles.clear()
+        sets.clear()
+        torch.cuda.empty_cache()
+        oracle_on = not args.no_cpu_baseline
+        per = [workload_entry(hkv, WORKLOADS[1], device, stream, with_oracle=oracle_on)]
+        for wid in (3, 5):
+            per.append(workload_entry(hkv, WORKLOADS[wid], device, stream, with_oracle=oracle_on))
+            torch.cuda.empty_cache()
+        for pp in WORKLOADS[4].p_sweep:
+            per.append(workload_entry(hkv, WORKLOADS[4], device, stream, p=pp, with_oracle=oracle_on))
+            torch.cuda.empty_cache()
+        extras["workloads"] = per
+
+    if extras is None:
+        del multi
+        singles.clear()
     if rank == 0:
         ms = region_ms_max / args.steps
         line = {
@@ -508,6 +707,8 @@ def run_ours(args):
             "clocks": clk,
             "impl": "ours",
         }
+        if extras is not None:
+            line["extras"] = extras
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.destroy_process_group()
@@ -559,6 +760,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="time only the headline workload (no other workloads, trigger or condensation)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

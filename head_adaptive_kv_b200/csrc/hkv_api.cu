@@ -37,7 +37,8 @@ namespace hkv {
 // 1 first stage landed, 2 pipeline done, 3 kernel entry (attention).
 // Per unit u of the fitting kernel, TR_FIT + 16u + i: 0 start, 1 entropy
 // done, 2 scores staged, 3 beta found; 4 holds the number of evaluations.
-[[maybe_unused]] constexpr int TR_SEL = 250000, TR_SW = 0, TR_AW = 20000, TR_FIT = 240000;
+// Per unit u of the merge kernel, TR_MRG + 2u: 0 start, 1 done.
+[[maybe_unused]] constexpr int TR_SEL = 250000, TR_SW = 0, TR_AW = 20000, TR_FIT = 240000, TR_MRG = 260000;
 
 // =============================================================================
 // Kernels
@@ -50,23 +51,28 @@ __global__ void __launch_bounds__(sc_nw(G) * 32, 1) k_score_stream(const __grid_
 {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     using Job = ScoreJob<ES, D, G>;
-    auto &ring = *reinterpret_cast<typename Job::RingT *>(smem_raw);
+    auto &sm = *reinterpret_cast<typename Job::Smem *>(smem_raw);
     const Ctl c = make_ctl(P);
-    ring_init(ring);
+    ring_init(sm.ring);
     allow_dependents();
     wait_prior_grid();  // the previous kernel's results are visible from here on
-    const int64_t R = (int64_t)P.units * P.sparse.cap;
     const int64_t NW = (int64_t)gridDim.x * Job::NW;
     const int64_t g = (int64_t)blockIdx.x * Job::NW + (threadIdx.x >> 5);
-    Job job(P, c, ring, share_begin(g, NW, R), share_begin(g + 1, NW, R));
+    tl_start(P.tl, TL_SCORE);
+    const bool prefix = P.units <= PREFIX_CAP;
+    const int64_t T = prefix ? score_prologue<Job::NW * 32>(P, c, sm.line, sm.red)
+                             : (int64_t)P.units * P.sparse.cap;
+    Job job(P, c, sm.ring, prefix ? &sm.line : nullptr, T, g, NW);
     HKV_TRACE_WARP(TR_SW + 4 * (int)g);
     if (!job.run_single_unit())
-        warp_pipeline(job, ring, c, TR_SW + 4 * (int)g);
+        warp_pipeline(job, sm.ring, c, TR_SW + 4 * (int)g);
+    tl_end(P.tl, TL_SCORE);
 }
 
 // S5 ([TS 2.A] cascade decode over the three tiers; [TS 2.C] Sparse Loading):
-// persistent streaming attention over line A (dense and condensed tokens)
-// and line B (selected sparse tokens); writes one record per warp and unit.
+// persistent streaming attention over line A (dense and condensed tokens, and
+// the rows of reused rewrites), before the wait for the selection, then line B
+// (the selected sparse tokens); writes one record per warp and unit and line.
 template <int ES, int D, int G>
 __global__ void __launch_bounds__(AT_NW * 32, 1) k_attn_stream(const __grid_constant__ Params P)
 {
@@ -77,16 +83,23 @@ __global__ void __launch_bounds__(AT_NW * 32, 1) k_attn_stream(const __grid_cons
     const Ctl c = make_ctl(P);
     ring_init(sm.ring);
     allow_dependents();
+    tl_start(P.tl, TL_ATTN);
+    // line A (dense, reused rewrite and condensed tokens) needs only the
+    // inputs, so it runs before the wait, alongside the selection kernel
     AttnLens lens;
-    attn_read_lengths(P, c, lens);  // inputs only: overlaps the previous kernel's tail
-    wait_prior_grid();
-    HKV_TRACE_WARP(TR_AW + 4 * (blockIdx.x * AT_NW + (threadIdx.x >> 5)) + 3);
-    AttnLine A, B;
-    attn_prologue<ES, D, G>(P, sm, c, red, lens, &A, &B);
+    attn_read_lengths(P, c, lens);
+    const AttnLine A = attn_prologue_a<ES, D, G>(P, sm, red, lens);
     const int64_t g = (int64_t)blockIdx.x * AT_NW + (threadIdx.x >> 5);
-    AttnJob<ES, D, G> job(P, c, sm, A, B, g);
+    AttnJob<ES, D, G> job(P, c, sm, A, g);
     HKV_TRACE_WARP(TR_AW + 4 * (int)g);
-    warp_pipeline(job, sm.ring, c, TR_AW + 4 * (int)g);
+    const uint32_t used = warp_pipeline(job, sm.ring, c, TR_AW + 4 * (int)g);
+    // line B (the selected tokens) after the selection
+    __syncthreads();
+    wait_prior_grid();
+    HKV_TRACE_WARP(TR_AW + 4 * (int)g + 3);
+    job.begin_line_b(attn_prologue_b<ES, D, G>(P, sm, c, red, lens, A));
+    warp_pipeline(job, sm.ring, c, -1, used);
+    tl_end(P.tl, TL_ATTN);
 }
 
 // S5 merge: out and lse of each (unit, query head) from the unit's records on
@@ -97,8 +110,12 @@ __global__ void __launch_bounds__(G * 32) k_merge(const __grid_constant__ Params
     allow_dependents();
     wait_prior_grid();
     const int u = blockIdx.x;
+    HKV_TRACE_AT(TR_MRG + 2 * u);
+    tl_start(P.tl, TL_MERGE);
     const int4 r = __ldcg(reinterpret_cast<const int4 *>(P.rec_range) + u);
     merge_head<D, G>(P, u, threadIdx.x >> 5, r.x, r.y, r.z, r.w);
+    HKV_TRACE_AT(TR_MRG + 2 * u + 1);
+    tl_end(P.tl, TL_MERGE);
 }
 
 // Rewrite Cache ([TS 2.C]): copy the k selected K/V rows of unit u, listed in
@@ -226,6 +243,31 @@ __device__ __forceinline__ void unit_work(const Params &P, USmem &sm, const Ctl 
     }
 }
 
+// A unit that reuses its rewrite this step (hkv_step_mti): its step outputs
+// describe the rewrite's rows (their token indices as of the rewrite), which
+// the attention reads from the rewrite buffer. Its cut, m and logZ are not
+// computed (NaN; kstar -1).
+__device__ void mti_reuse_outputs(const Params &P, const Ctl &c, int u)
+{
+    int k = tier_len(P.rw, u, c);
+    if (k > P.bmax) {
+        raise_flag(c, HKV_DEV_BAD_INDEX);
+        k = P.bmax;
+    }
+    int32_t *row = P.idx + (int64_t)u * P.bmax;
+    for (int i = threadIdx.x; i < P.bmax; i += NT)
+        row[i] = i < k ? __ldcg(P.rw_idx + (int64_t)u * P.bmax + i) : -1;
+    if (threadIdx.x == 0) {
+        P.sel_len[u] = k;
+        if (P.cut)
+            P.cut[u] = hkv_cut{__int_as_float(0x7fc00000), 0, 0, -1};
+        if (P.m_out)
+            P.m_out[u] = __int_as_float(0x7fc00000);
+        if (P.logZ_out)
+            P.logZ_out[u] = __int_as_float(0x7fc00000);
+    }
+}
+
 // S2-S4 per unit, one CTA per (sequence, KV head). Units of up to ZSTAGE
 // tokens work on a copy of their scores in shared memory.
 //  do_select  ([TS 2.B] calibration, [Abstract]/[TS 2.A] Top-p budget with the
@@ -244,19 +286,23 @@ __global__ void __launch_bounds__(NT) k_unit(const __grid_constant__ Params P)
     allow_dependents();
     wait_prior_grid();
     HKV_TRACE_AT(TR_SEL + 16 * u);
+    tl_start(P.tl, TL_UNIT);
     const int n = tier_len(P.sparse, u, c);
     const float *zg = P.z + (int64_t)u * P.z_stride;
-    if (P.have_range && P.do_select && P.do_compact && n <= ZSTAGE) {
+    if (P.mti_left != nullptr && __ldcg(P.mti_left + u) > 0) {
+        mti_reuse_outputs(P, c, u);  // the unit reuses its rewrite: nothing to select
+    } else if (P.have_range && P.do_select && P.do_compact && n <= ZSTAGE) {
         // hkv_step: the range is known, so the first sweep stages the scores
         unit_work<ES, true>(P, sm, c, u, n, sm.zs, zg);
-        return;
+    } else {
+        const bool staged = stage_scores(zg, n, sm);
+        HKV_TRACE_AT(TR_SEL + 16 * u + 6);
+        if (staged)
+            unit_work<ES, true>(P, sm, c, u, n, sm.zs);
+        else
+            unit_work<ES, false>(P, sm, c, u, n, zg);
     }
-    const bool staged = stage_scores(zg, n, sm);
-    HKV_TRACE_AT(TR_SEL + 16 * u + 6);
-    if (staged)
-        unit_work<ES, true>(P, sm, c, u, n, sm.zs);
-    else
-        unit_work<ES, false>(P, sm, c, u, n, zg);
+    tl_end(P.tl, TL_UNIT);
 }
 
 // S2 standalone ([TS 2.B]) for unit u: m, logZ and optionally the calibrated
@@ -317,6 +363,7 @@ __global__ void __cluster_dims__(FIT_CTAS, 1, 1) __launch_bounds__(NT, 1) k_fit(
     FitCluster cl;
     allow_dependents();
     wait_prior_grid();
+    tl_start(P.tl, TL_FIT);
     const int n = tier_len(P.sparse, u, c);
     HKV_TRACE_IF(cl.rank == 0 && threadIdx.x == 0, TR_FIT + 16 * u);
     float target;
@@ -343,6 +390,7 @@ __global__ void __cluster_dims__(FIT_CTAS, 1, 1) __launch_bounds__(NT, 1) k_fit(
     }
     // no CTA leaves while another may still read its shared memory
     cooperative_groups::this_cluster().sync();
+    tl_end(P.tl, TL_FIT);
 }
 
 // FLAT_SUM rows and Rewrite Cache copies after the step's PAD_MAX compaction
@@ -354,6 +402,7 @@ __global__ void __launch_bounds__(NT) k_flatten(const __grid_constant__ Params P
     const Ctl c = make_ctl(P);
     const int u = blockIdx.x;
     wait_prior_grid();
+    tl_start(P.tl, TL_FLAT);
     const int n = tier_len(P.sparse, u, c);
     const int k = max(0, min(__ldcg(P.sel_len + u), min(n, P.bmax)));
     const int32_t *src = P.idx + (int64_t)u * P.bmax;
@@ -366,6 +415,7 @@ __global__ void __launch_bounds__(NT) k_flatten(const __grid_constant__ Params P
     }
     if (P.k_out != nullptr)
         rewrite_rows(P, u, src, k, off, ES, c, n);
+    tl_end(P.tl, TL_FLAT);
 }
 
 // =============================================================================
@@ -375,6 +425,10 @@ __global__ void __launch_bounds__(NT) k_flatten(const __grid_constant__ Params P
 std::atomic<uint64_t> g_launches{0};
 std::atomic<uint64_t> g_wait_ns{1000000000ull};
 std::atomic<int32_t> g_withhold{0};
+std::atomic<int32_t> g_timeline{0};
+
+// Timeline words: the last 128 bytes of the workspace's 256-byte control area.
+constexpr size_t TL_OFFSET = 128;
 
 struct WsLayout {
     size_t ctl, urange, rec_range, part, idxbuf, zbuf, logits, total;
@@ -497,6 +551,7 @@ static Params base_params(const hkv_problem *p, const WsLayout &L, char *ws, con
     P.wait_ns = g_wait_ns.load();
     P.withhold = g_withhold.load();
     P.ctl = reinterpret_cast<uint32_t *>(ws + L.ctl);
+    P.tl = g_timeline.load() ? reinterpret_cast<unsigned long long *>(ws + L.ctl + TL_OFFSET) : nullptr;
     P.rec_range = reinterpret_cast<int32_t *>(ws + L.rec_range);
     P.part = reinterpret_cast<float *>(ws + L.part);
     P.part_slots = L.part_slots;
@@ -632,7 +687,7 @@ template <int ES, int D, int G>
 struct RunScore {
     static hkv_status run(const Params &P, cudaStream_t s, bool pdl)
     {
-        return launch_stream(k_score_stream<ES, D, G>, sc_nw(G) * 32, sizeof(typename ScoreJob<ES, D, G>::RingT),
+        return launch_stream(k_score_stream<ES, D, G>, sc_nw(G) * 32, sizeof(typename ScoreJob<ES, D, G>::Smem),
                              1 << 20, s, P, pdl);
     }
 };
@@ -699,6 +754,251 @@ bool aligned(const void *p, uintptr_t a) { return ((uintptr_t)p & (a - 1)) == 0;
 
 }  // namespace
 
+namespace hkv {
+
+// ---- Rewrite Cache vs Sparse Loading ([TS 2.C] Trade-off Management) --------
+//
+// After the step's attention, per unit: a unit that reused its rewrite counts
+// one step down; any other unit (it was scored and selected) takes the trigger
+// on its fresh budget k -- Rewrite Cache when k > L_upper, Sparse Loading when
+// k < L_lower, the previous mode in between -- and under Rewrite Cache copies
+// its k selected K and V rows into the rewrite buffer, which then serves
+// H(k) = max(1, floor(mti_cap / k)) steps in all (this one included): a
+// rewrite of k rows kept H steps holds k H <= mti_cap row-steps of memory.
+// A cluster of MTI_CTAS CTAs per unit splits the rows; they meet once, before
+// the unit's state (read by all of them) is updated.
+
+constexpr int MTI_CTAS = 4;
+constexpr int MTI_NT = 256;
+
+struct MtiP {
+    const char *sk, *sv;                   // sparse tier
+    int64_t ssb, ssh, sst;                 // byte strides
+    char *rk, *rv;                         // rewrite buffer
+    int64_t rsb, rsh, rst;
+    const int32_t *idx, *sel_len, *slen;   // the step's PAD_MAX rows and budgets; sparse lengths
+    int32_t *mode, *left, *rw_len, *rw_idx;
+    int32_t Hkv, bmax, rowb, ncap, L_lower, L_upper;
+    int64_t mti_cap;
+    uint32_t *status;
+    unsigned long long *tl;
+};
+
+__global__ void __cluster_dims__(MTI_CTAS, 1, 1) __launch_bounds__(MTI_NT) k_mti(const __grid_constant__ MtiP M)
+{
+    auto cluster = cooperative_groups::this_cluster();
+    const int r = (int)cluster.block_rank();
+    const int u = blockIdx.x / MTI_CTAS;
+    wait_prior_grid();  // the step's attention has read the state and the buffer
+    tl_start(M.tl, TL_MTI);
+    const int left0 = __ldcg(M.left + u);
+    if (left0 > 0) {  // reused this step
+        cluster.sync();
+        if (r == 0 && threadIdx.x == 0)
+            M.left[u] = left0 - 1;
+        tl_end(M.tl, TL_MTI);
+        return;
+    }
+    const int k = max(0, min(__ldcg(M.sel_len + u), M.bmax));
+    const int mode0 = __ldcg(M.mode + u);
+    const int mode1 = k > M.L_upper ? 1 : (k < M.L_lower ? 0 : (mode0 != 0 ? 1 : 0));
+    if (mode1) {
+        // rows [k r / MTI_CTAS, k (r + 1) / MTI_CTAS) of the selection, in 16-byte chunks
+        const int b = u / M.Hkv, h = u - b * M.Hkv;
+        const int n = max(0, min(__ldcg(M.slen + u), M.ncap));
+        const int i0 = k * r / MTI_CTAS, i1 = k * (r + 1) / MTI_CTAS;
+        const int ch = M.rowb / 16;
+        const int32_t *row = M.idx + (int64_t)u * M.bmax;
+        for (int x = threadIdx.x; x < (i1 - i0) * 2 * ch; x += MTI_NT) {
+            const int i = i0 + x / (2 * ch), q = x % (2 * ch);
+            const bool isk = q < ch;
+            int j = __ldcg(row + i);
+            if (j < 0 || j >= n) {
+                atomicOr(M.status, HKV_DEV_BAD_INDEX);
+                j = 0;
+            }
+            const char *src = (isk ? M.sk : M.sv) + (int64_t)b * M.ssb + (int64_t)h * M.ssh + (int64_t)j * M.sst;
+            char *dst = (isk ? M.rk : M.rv) + (int64_t)b * M.rsb + (int64_t)h * M.rsh + (int64_t)i * M.rst;
+            const int off = (isk ? q : q - ch) * 16;
+            *reinterpret_cast<uint4 *>(dst + off) = __ldcs(reinterpret_cast<const uint4 *>(src + off));
+            if (q == 0)
+                M.rw_idx[(int64_t)u * M.bmax + i] = __ldcg(row + i);
+        }
+    }
+    cluster.sync();
+    if (r == 0 && threadIdx.x == 0) {
+        M.mode[u] = mode1;
+        if (mode1) {
+            const int64_t H = k > 0 ? max((int64_t)1, min(M.mti_cap / k, (int64_t)1 << 30)) : 1;
+            M.rw_len[u] = k;
+            M.left[u] = (int32_t)(H - 1);
+        } else {
+            M.rw_len[u] = 0;
+            M.left[u] = 0;
+        }
+    }
+    tl_end(M.tl, TL_MTI);
+}
+
+}  // namespace hkv
+
+namespace {
+
+// The decode step (hkv_step), and with `mti` the step under the Rewrite Cache /
+// Sparse Loading trigger (hkv_step_mti).
+hkv_status step_impl(const hkv_problem *prob, const void *q, const hkv_tier *dense, const hkv_tier *sparse,
+                     const hkv_tier *condensed, const hkv_step_out *o, const hkv_mti *mti, void *ws, size_t ws_bytes,
+                     hkv_stream_t stream)
+{
+    WsLayout L;
+    Params P;
+    if (sparse == nullptr || o == nullptr)
+        return HKV_ERR_INVALID_ARG;
+    hkv_status s = prologue(prob, dense, sparse, condensed, true, ws, ws_bytes, &L, &P);
+    if (s != HKV_OK)
+        return s;
+    if (q == nullptr || !aligned(q, 16) || o->out == nullptr || o->sel_len == nullptr || o->idx == nullptr)
+        return HKV_ERR_INVALID_ARG;
+    const bool flat = prob->layout == HKV_LAYOUT_FLAT_SUM;
+    if (flat && o->offsets == nullptr)
+        return HKV_ERR_INVALID_ARG;
+    const bool rewrite = o->k_out != nullptr || o->v_out != nullptr;
+    if (rewrite && (o->k_out == nullptr || o->v_out == nullptr || !aligned(o->k_out, 16) || !aligned(o->v_out, 16)))
+        return HKV_ERR_INVALID_ARG;
+    if (o->z && !aligned(o->z, 4))
+        return HKV_ERR_INVALID_ARG;
+    if ((o->h_attn != nullptr && o->beta_fit == nullptr) || (o->beta_fit && !aligned(o->beta_fit, 4)) ||
+        (o->h_attn && !aligned(o->h_attn, 4)))
+        return HKV_ERR_INVALID_ARG;
+    if (mti != nullptr) {
+        // the rewrite buffer is the Rewrite Cache here; a fitted temperature
+        // would need the scores that reusing units skip
+        if (rewrite || o->beta_fit != nullptr)
+            return HKV_ERR_INVALID_ARG;
+        if (mti->L_lower < 0 || mti->L_upper < mti->L_lower || mti->mti_cap < 0 || mti->mode == nullptr ||
+            mti->left == nullptr || mti->rw_idx == nullptr || !aligned(mti->mode, 4) || !aligned(mti->left, 4) ||
+            !aligned(mti->rw_idx, 4))
+            return HKV_ERR_INVALID_ARG;
+        if ((s = check_tier(&mti->rewrite, prob, true)) != HKV_OK)
+            return s;
+        if (mti->rewrite.cap < prob->bmax || (prob->bmax > 0 && mti->rewrite.len == nullptr))
+            return HKV_ERR_INVALID_ARG;
+        // units and lines small enough for the attention's exact (prefix) layout
+        const int64_t span = (int64_t)(dense ? dense->cap : 0) + mti->rewrite.cap + (condensed ? condensed->cap : 0) +
+                             std::min(prob->bmax, sparse->cap);
+        if ((int64_t)P.units > PREFIX_CAP || (int64_t)P.units * span >= (1ll << 31))
+            return HKV_ERR_UNSUPPORTED;
+    }
+    if (P.units == 0)
+        return HKV_OK;
+    char *wsb = static_cast<char *>(ws);
+    const cudaStream_t st = (cudaStream_t)stream;
+    P.q = static_cast<const char *>(q);
+    P.z = o->z ? o->z : reinterpret_cast<float *>(wsb + L.zbuf);
+    P.z_stride = o->z ? sparse->cap : L.z_stride;
+    P.sel_len = o->sel_len;
+    P.cut = o->cut;
+    P.idx = flat ? reinterpret_cast<int32_t *>(wsb + L.idxbuf) : o->idx;  // PAD_MAX rows for the attention
+    P.idx_user = o->idx;
+    P.offsets = o->offsets;
+    P.out = o->out;
+    P.lse = o->lse;
+    P.m_out = o->m;
+    P.logZ_out = o->logZ;
+    P.k_out = static_cast<char *>(o->k_out);
+    P.v_out = static_cast<char *>(o->v_out);
+    P.logit = reinterpret_cast<float *>(wsb + L.logits);  // scorer -> attention of the selected tokens
+    P.layout = HKV_LAYOUT_PAD_MAX;  // the three kernels work on PAD_MAX rows
+    if (mti != nullptr) {
+        P.mti_left = mti->left;
+        P.rw = tier_p(&mti->rewrite);
+        P.rw_idx = mti->rw_idx;
+        P.attn_prefix = 1;
+    }
+    // 1. scores, and the score range of each unit (launched in stream order:
+    // as a programmatic dependent of the previous step its CTAs would sit on
+    // SMs the previous attention is leaving, which measured slower)
+    const bool scored = sparse->cap > 0;
+    Params S = P;
+    S.urange = reinterpret_cast<uint32_t *>(wsb + L.urange);
+    if (scored && (s = dispatch<RunScore>(prob, S, st, false)) != HKV_OK)
+        return s;
+    // 1b. optionally the fitted inverse temperature of every unit, from the
+    // scorer's logit records and scores; the selection then uses it
+    Params U = S;
+    if (o->beta_fit != nullptr) {
+        Params F = S;
+        F.urange = nullptr;
+        F.beta_out = o->beta_fit;
+        F.h_out = o->h_attn;
+        if ((s = dispatch<RunFit>(prob, F, st, scored)) != HKV_OK)
+            return s;
+        U.inv_temp = o->beta_fit;
+    }
+    // 2. calibration, Top-p budget, cut and compaction, per unit
+    U.have_range = scored;
+    U.do_select = 1;
+    U.do_compact = 1;
+    if ((s = launch_unit(prob, U, st, true)) != HKV_OK)
+        return s;
+    // 3. attention over the three tiers and the merge of each unit
+    if ((s = dispatch<RunAttn>(prob, P, st, true)) != HKV_OK)
+        return s;
+    if (flat || rewrite) {
+        P.layout = prob->layout;
+        s = prob->dtype == HKV_BF16 ? launch(k_flatten<2>, P.units, NT, 0, st, P, true)
+                                    : launch(k_flatten<4>, P.units, NT, 0, st, P, true);
+        if (s != HKV_OK)
+            return s;
+    }
+    if (mti == nullptr)
+        return HKV_OK;
+    // 4. the trigger, and the rewrites it asks for
+    const int es = es_of(prob->dtype);
+    MtiP M{};
+    M.sk = static_cast<const char *>(sparse->k);
+    M.sv = static_cast<const char *>(sparse->v);
+    M.ssb = sparse->stride_b * es;
+    M.ssh = sparse->stride_h * es;
+    M.sst = sparse->stride_t * es;
+    M.rk = static_cast<char *>(const_cast<void *>(mti->rewrite.k));
+    M.rv = static_cast<char *>(const_cast<void *>(mti->rewrite.v));
+    M.rsb = mti->rewrite.stride_b * es;
+    M.rsh = mti->rewrite.stride_h * es;
+    M.rst = mti->rewrite.stride_t * es;
+    M.idx = P.idx;
+    M.sel_len = o->sel_len;
+    M.slen = sparse->len;
+    M.mode = mti->mode;
+    M.left = mti->left;
+    M.rw_len = const_cast<int32_t *>(mti->rewrite.len);
+    M.rw_idx = mti->rw_idx;
+    M.Hkv = prob->Hkv;
+    M.bmax = prob->bmax;
+    M.rowb = prob->D * es;
+    M.ncap = sparse->cap;
+    M.L_lower = mti->L_lower;
+    M.L_upper = mti->L_upper;
+    M.mti_cap = mti->mti_cap;
+    M.status = P.ctl;
+    M.tl = P.tl;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(P.units * MTI_CTAS));
+    cfg.blockDim = dim3(MTI_NT);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, k_mti, M) != cudaSuccess)
+        return HKV_ERR_CUDA;
+    g_launches.fetch_add(1);
+    return HKV_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char *hkv_status_string(hkv_status s)
@@ -722,6 +1022,31 @@ hkv_status hkv_set_wait_limit_ns(uint64_t ns)
     if (ns == 0)
         return HKV_ERR_INVALID_ARG;
     g_wait_ns.store(ns);
+    return HKV_OK;
+}
+
+hkv_status hkv_set_timeline(int32_t on)
+{
+    g_timeline.store(on ? 1 : 0);
+    return HKV_OK;
+}
+
+hkv_status hkv_read_timeline(void *ws, uint64_t *start_end, hkv_stream_t stream)
+{
+    if (ws == nullptr || ((uintptr_t)ws & 255))
+        return HKV_ERR_WORKSPACE;
+    if (start_end == nullptr)
+        return HKV_ERR_INVALID_ARG;
+    unsigned long long w[16];
+    cudaStream_t s = (cudaStream_t)stream;
+    char *tl = static_cast<char *>(ws) + TL_OFFSET;
+    if (cudaMemcpyAsync(w, tl, sizeof w, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess || cudaMemsetAsync(tl, 0, sizeof w, s) != cudaSuccess)
+        return HKV_ERR_CUDA;
+    for (int k = 0; k < HKV_TL_KINDS; ++k) {
+        start_end[2 * k] = w[k] ? ~w[k] : 0;
+        start_end[2 * k + 1] = w[8 + k];
+    }
     return HKV_OK;
 }
 
@@ -895,81 +1220,16 @@ hkv_status hkv_step(const hkv_problem *prob, const void *q, const hkv_tier *dens
                     const hkv_tier *condensed, const hkv_step_out *o, void *ws, size_t ws_bytes,
                     hkv_stream_t stream)
 {
-    WsLayout L;
-    Params P;
-    if (sparse == nullptr || o == nullptr)
+    return step_impl(prob, q, dense, sparse, condensed, o, nullptr, ws, ws_bytes, stream);
+}
+
+hkv_status hkv_step_mti(const hkv_problem *prob, const void *q, const hkv_tier *dense, const hkv_tier *sparse,
+                        const hkv_tier *condensed, const hkv_mti *mti, const hkv_step_out *o, void *ws,
+                        size_t ws_bytes, hkv_stream_t stream)
+{
+    if (mti == nullptr)
         return HKV_ERR_INVALID_ARG;
-    hkv_status s = prologue(prob, dense, sparse, condensed, true, ws, ws_bytes, &L, &P);
-    if (s != HKV_OK)
-        return s;
-    if (q == nullptr || !aligned(q, 16) || o->out == nullptr || o->sel_len == nullptr || o->idx == nullptr)
-        return HKV_ERR_INVALID_ARG;
-    const bool flat = prob->layout == HKV_LAYOUT_FLAT_SUM;
-    if (flat && o->offsets == nullptr)
-        return HKV_ERR_INVALID_ARG;
-    const bool rewrite = o->k_out != nullptr || o->v_out != nullptr;
-    if (rewrite && (o->k_out == nullptr || o->v_out == nullptr || !aligned(o->k_out, 16) || !aligned(o->v_out, 16)))
-        return HKV_ERR_INVALID_ARG;
-    if (o->z && !aligned(o->z, 4))
-        return HKV_ERR_INVALID_ARG;
-    if ((o->h_attn != nullptr && o->beta_fit == nullptr) || (o->beta_fit && !aligned(o->beta_fit, 4)) ||
-        (o->h_attn && !aligned(o->h_attn, 4)))
-        return HKV_ERR_INVALID_ARG;
-    if (P.units == 0)
-        return HKV_OK;
-    char *wsb = static_cast<char *>(ws);
-    const cudaStream_t st = (cudaStream_t)stream;
-    P.q = static_cast<const char *>(q);
-    P.z = o->z ? o->z : reinterpret_cast<float *>(wsb + L.zbuf);
-    P.z_stride = o->z ? sparse->cap : L.z_stride;
-    P.sel_len = o->sel_len;
-    P.cut = o->cut;
-    P.idx = flat ? reinterpret_cast<int32_t *>(wsb + L.idxbuf) : o->idx;  // PAD_MAX rows for the attention
-    P.idx_user = o->idx;
-    P.offsets = o->offsets;
-    P.out = o->out;
-    P.lse = o->lse;
-    P.m_out = o->m;
-    P.logZ_out = o->logZ;
-    P.k_out = static_cast<char *>(o->k_out);
-    P.v_out = static_cast<char *>(o->v_out);
-    P.logit = reinterpret_cast<float *>(wsb + L.logits);  // scorer -> attention of the selected tokens
-    P.layout = HKV_LAYOUT_PAD_MAX;  // the three kernels work on PAD_MAX rows
-    // 1. scores, and the score range of each unit (launched in stream order:
-    // as a programmatic dependent of the previous step its CTAs would sit on
-    // SMs the previous attention is leaving, which measured slower)
-    const bool scored = sparse->cap > 0;
-    Params S = P;
-    S.urange = reinterpret_cast<uint32_t *>(wsb + L.urange);
-    if (scored && (s = dispatch<RunScore>(prob, S, st, false)) != HKV_OK)
-        return s;
-    // 1b. optionally the fitted inverse temperature of every unit, from the
-    // scorer's logit records and scores; the selection then uses it
-    Params U = S;
-    if (o->beta_fit != nullptr) {
-        Params F = S;
-        F.urange = nullptr;
-        F.beta_out = o->beta_fit;
-        F.h_out = o->h_attn;
-        if ((s = dispatch<RunFit>(prob, F, st, scored)) != HKV_OK)
-            return s;
-        U.inv_temp = o->beta_fit;
-    }
-    // 2. calibration, Top-p budget, cut and compaction, per unit
-    U.have_range = scored;
-    U.do_select = 1;
-    U.do_compact = 1;
-    if ((s = launch_unit(prob, U, st, true)) != HKV_OK)
-        return s;
-    // 3. attention over the three tiers and the merge of each unit
-    if ((s = dispatch<RunAttn>(prob, P, st, true)) != HKV_OK)
-        return s;
-    if (!flat && !rewrite)
-        return HKV_OK;
-    P.layout = prob->layout;
-    if (prob->dtype == HKV_BF16)
-        return launch(k_flatten<2>, P.units, NT, 0, st, P, true);
-    return launch(k_flatten<4>, P.units, NT, 0, st, P, true);
+    return step_impl(prob, q, dense, sparse, condensed, o, mti, ws, ws_bytes, stream);
 }
 
 hkv_status hkv_attention_entropy(const hkv_problem *prob, const void *q, const hkv_tier *sparse, float *h, void *ws,
@@ -1045,16 +1305,22 @@ constexpr int NOALLOC_MAX_DEVICES = 64;
 static std::mutex g_noalloc_mu;
 static void *g_noalloc_ptr[NOALLOC_MAX_DEVICES];
 
-// Device address of the scratch on the current device, looked up once per
-// device (the first call on a device does this; it must not run under stream
-// capture).
-static hkv_status noalloc_scratch(void **ptr)
+// Device address of the scratch in the current device's context. A call made
+// outside stream capture looks it up afresh (cudaGetSymbolAddress, which also
+// loads the module on first use), so an address never outlives the context
+// it belongs to (a cudaDeviceReset, another primary context); a call under
+// capture, where loading a module is not allowed, uses the address that the
+// last call outside capture on this device found.
+static hkv_status noalloc_scratch(cudaStream_t stream, void **ptr)
 {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= NOALLOC_MAX_DEVICES)
         return HKV_ERR_CUDA;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess)
+        return HKV_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (g_noalloc_ptr[dev] == nullptr) {
+    if (cap == cudaStreamCaptureStatusNone || g_noalloc_ptr[dev] == nullptr) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
             return HKV_ERR_CUDA;
@@ -1102,7 +1368,7 @@ extern "C" hkv_status hkv_cascade_decode_noalloc(const hkv_problem *prob, const 
         return status ? (cudaMemsetAsync(status, 0, sizeof(uint32_t), st) == cudaSuccess ? HKV_OK : HKV_ERR_CUDA)
                       : HKV_OK;
     void *scratch = nullptr;
-    if ((s = noalloc_scratch(&scratch)) != HKV_OK)
+    if ((s = noalloc_scratch(st, &scratch)) != HKV_OK)
         return s;
     char *base = static_cast<char *>(scratch);
     Params P = base_params(prob, L, base, dense, sparse, condensed);
@@ -1266,6 +1532,387 @@ extern "C" hkv_status hkv_append(const hkv_problem *prob, const void *k_new, con
     cfg.blockDim = dim3(APPEND_WARPS * 32);
     cfg.stream = (cudaStream_t)stream;
     if (cudaLaunchKernelEx(&cfg, k_append, A) != cudaSuccess)
+        return HKV_ERR_CUDA;
+    g_launches.fetch_add(1);
+    return HKV_OK;
+}
+
+// =============================================================================
+// Condensed-tier formation ([TS 2.A] Tier 3 "the oldest blocks are further
+// compressed into constant-sized storage via eviction or weighted merging";
+// pipeline step 4)
+//
+// A unit whose sparse tier holds at least max(trigger, block) tokens gives up
+// its oldest `block` tokens (sparse slots 0 .. block-1; the tier is in age
+// order). They become one condensed slot after the existing ones: under MERGE
+// the weighted mean of the block's K and V rows, weighted by the tokens'
+// calibrated probabilities a_j = exp(beta (z_j - m) - logZ) under the step's
+// scores, with weight sum_j a_j; under EVICT a copy of the block's most
+// important token (largest score, the older one on ties) with weight a_j. A
+// full condensed tier first merges its two oldest slots (MERGE; a one-slot tier
+// folds the block into its slot) or drops its oldest slot (EVICT). The sparse
+// tier then moves down by `block` rows. Means are float64 sums in slot order
+// (multiply, then add: no fused multiply-add), divided once and rounded once to
+// the element type, nearest with ties to even.
+//
+// Each unit is worked by a cluster of COND_CTAS CTAs; CTA r owns bytes
+// [r RB / COND_CTAS, (r+1) RB / COND_CTAS) of every K and V row (RB bytes per
+// row), for the mean and for the move alike, so the CTAs never touch the same
+// byte. They meet once, at a cluster barrier before the lengths and weights
+// (read by all of them at the start) are updated.
+// =============================================================================
+
+namespace hkv {
+
+constexpr int COND_CTAS = 4;
+constexpr int COND_NT = 256;
+constexpr int COND_STAGE = 32768;  // bytes one CTA moves per batch (its K and V slices)
+
+struct CondP {
+    char *sk, *sv, *ck, *cv;               // tier storage, written in place
+    int64_t ssb, ssh, sst, csb, csh, cst;  // byte strides
+    int32_t ncap, ccap;
+    int32_t *slen, *clen, *done;
+    float *cw;                             // [units, ccap] condensed-slot weights
+    const float *z, *m, *logZ, *inv_temp;
+    int64_t z_stride;
+    int32_t Hkv, units, D, es, block, trigger, policy;
+    uint32_t *status;
+};
+
+struct __align__(16) CondSmem {
+    double a[HKV_CONDENSE_MAX_BLOCK];  // the block's weights
+    unsigned char stage[COND_STAGE];   // one batch of the move
+    int32_t jstar;
+};
+
+// The bf16 value nearest x, ties to an even last mantissa bit, from the double
+// directly (a detour through float would round twice): integer rounding of the
+// 53-bit significand to 8 bits, or to the fixed 2^-133 spacing below 2^-126.
+__device__ __forceinline__ uint16_t bf16_from_double(double x)
+{
+    const unsigned long long bits = (unsigned long long)__double_as_longlong(x);
+    const uint16_t sign = (uint16_t)((bits >> 48) & 0x8000u);
+    const unsigned long long mag = bits & 0x7fffffffffffffffull;
+    if (mag >= 0x7ff0000000000000ull)  // inf or NaN
+        return (uint16_t)(sign | 0x7f80u | (mag > 0x7ff0000000000000ull ? 0x40u : 0u));
+    const int e = (int)(mag >> 52) - 1023;
+    if (e < -134)  // below a quarter of the smallest bf16 step: 0 (double subnormals included)
+        return sign;
+    const unsigned long long sig = (mag & 0xfffffffffffffull) | (1ull << 52);
+    // drop s low bits: 45 for a normal bf16 (8 significant bits kept), more below 2^-126
+    const int s = e >= -126 ? 45 : 45 + (-126 - e);
+    unsigned long long keep = sig >> s;
+    const unsigned long long rem = sig & ((1ull << s) - 1ull), half = 1ull << (s - 1);
+    if (rem > half || (rem == half && (keep & 1ull)))
+        ++keep;
+    if (e < -126)  // subnormal (or the smallest normal, if rounding carried): keep is the whole pattern
+        return (uint16_t)(sign | (uint16_t)keep);
+    int ee = e;
+    if (keep == 256ull) {
+        keep = 128ull;
+        ++ee;
+    }
+    if (ee > 127)
+        return (uint16_t)(sign | 0x7f80u);
+    return (uint16_t)(sign | (uint16_t)((ee + 127) << 7) | (uint16_t)(keep & 0x7fu));
+}
+
+__device__ __forceinline__ double cond_load(const char *row, int e, int es)
+{
+    if (es == 2)
+        return (double)__uint_as_float((uint32_t)(*reinterpret_cast<const uint16_t *>(row + 2 * e)) << 16);
+    return (double)*reinterpret_cast<const float *>(row + 4 * e);
+}
+
+__device__ __forceinline__ void cond_store(char *row, int e, int es, double v)
+{
+    if (es == 2)
+        *reinterpret_cast<uint16_t *>(row + 2 * e) = bf16_from_double(v);
+    else
+        *reinterpret_cast<float *>(row + 4 * e) = __double2float_rn(v);
+}
+
+__device__ __forceinline__ void cond_copy_elem(char *dst, const char *src, int e, int es)
+{
+    if (es == 2)
+        *reinterpret_cast<uint16_t *>(dst + 2 * e) = *reinterpret_cast<const uint16_t *>(src + 2 * e);
+    else
+        *reinterpret_cast<uint32_t *>(dst + 4 * e) = *reinterpret_cast<const uint32_t *>(src + 4 * e);
+}
+
+__global__ void __cluster_dims__(COND_CTAS, 1, 1) __launch_bounds__(COND_NT)
+    k_condense(const __grid_constant__ CondP P)
+{
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    CondSmem &sm = *reinterpret_cast<CondSmem *>(smem_raw);
+    auto cluster = cooperative_groups::this_cluster();
+    const int r = (int)cluster.block_rank();
+    const int u = blockIdx.x / COND_CTAS;
+    const int b = u / P.Hkv, h = u - b * P.Hkv;
+    const int n = __ldcg(P.slen + u);
+    const int C0 = P.ccap > 0 ? __ldcg(P.clen + u) : 0;
+    if (n < 0 || n > P.ncap || C0 < 0 || C0 > P.ccap) {  // a corrupt unit is left as it is
+        if (r == 0 && threadIdx.x == 0) {
+            atomicOr(P.status, HKV_DEV_LEN_CLAMPED);
+            if (P.done)
+                P.done[u] = 0;
+        }
+        return;
+    }
+    const int blk = P.block;
+    if (n < max(max(P.trigger, blk), 1)) {
+        if (r == 0 && threadIdx.x == 0 && P.done)
+            P.done[u] = 0;
+        return;
+    }
+    char *sk = P.sk + (int64_t)b * P.ssb + (int64_t)h * P.ssh;
+    char *sv = P.sv + (int64_t)b * P.ssb + (int64_t)h * P.ssh;
+    char *ck = P.ccap > 0 ? P.ck + (int64_t)b * P.csb + (int64_t)h * P.csh : nullptr;
+    char *cv = P.ccap > 0 ? P.cv + (int64_t)b * P.csb + (int64_t)h * P.csh : nullptr;
+    float *cw = P.ccap > 0 ? P.cw + (int64_t)u * P.ccap : nullptr;
+
+    // the block's weights (and, for EVICT, its first highest-scoring token)
+    double beta = 1.0;
+    if (P.inv_temp != nullptr) {
+        const float bt = __ldcg(P.inv_temp + u);
+        if (!(bt >= 0.0f) || isinf(bt)) {
+            if (r == 0 && threadIdx.x == 0)
+                atomicOr(P.status, HKV_DEV_BAD_TEMP);
+        } else {
+            beta = (double)bt;
+        }
+    }
+    const float *zu = P.z != nullptr ? P.z + (int64_t)u * P.z_stride : nullptr;
+    const double mu = zu ? (double)__ldcg(P.m + u) : 0.0, lz = zu ? (double)__ldcg(P.logZ + u) : 0.0;
+    for (int j = threadIdx.x; j < blk; j += COND_NT)
+        sm.a[j] = zu ? exp(__dsub_rn(__dmul_rn(beta, __dsub_rn((double)__ldcg(zu + j), mu)), lz)) : 1.0;
+    if (threadIdx.x == 0)
+        sm.jstar = 0;
+    __syncthreads();
+    if (P.policy == HKV_CONDENSE_EVICT && zu != nullptr) {
+        // first maximum: the largest (score, -index) pair
+        unsigned long long best = 0ull;
+        for (int j = threadIdx.x; j < blk; j += COND_NT) {
+            const unsigned long long key = ((unsigned long long)(~score_key(__ldcg(zu + j))) << 32) |
+                                           (uint32_t)(0x7fffffff - j);
+            best = key > best ? key : best;
+        }
+        for (int o = 16; o > 0; o >>= 1) {
+            const unsigned long long y = __shfl_xor_sync(0xffffffffu, best, o);
+            best = y > best ? y : best;
+        }
+        __shared__ unsigned long long wbest[COND_NT / 32];
+        if ((threadIdx.x & 31) == 0)
+            wbest[threadIdx.x >> 5] = best;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            unsigned long long m_ = 0ull;
+            for (int w = 0; w < COND_NT / 32; ++w)
+                m_ = wbest[w] > m_ ? wbest[w] : m_;
+            sm.jstar = 0x7fffffff - (int)(uint32_t)m_;
+        }
+        __syncthreads();
+    }
+
+    // this CTA's elements of a row: NE of K, then NE of V
+    const int NE = P.D / COND_CTAS;
+    const int e0 = r * NE;
+    int C = C0;             // slot of the new condensed entry
+    bool fold = false;      // one-slot MERGE tier: the old slot joins the block's mean
+    if (P.ccap > 0) {
+        const bool full = C0 >= P.ccap;
+        if (P.policy == HKV_CONDENSE_MERGE && full && P.ccap >= 2) {
+            const double w0 = (double)cw[0], w1 = (double)cw[1];
+            const bool eq = !(__dadd_rn(__dadd_rn(0.0, w0), w1) > 0.0);
+            const double a0 = eq ? 1.0 : w0, a1 = eq ? 1.0 : w1;
+            for (int t = threadIdx.x; t < 2 * NE; t += COND_NT) {
+                char *base = t < NE ? ck : cv;
+                const int e = e0 + (t < NE ? t : t - NE);
+                const double x0 = cond_load(base, e, P.es), x1 = cond_load(base + P.cst, e, P.es);
+                double num = __dadd_rn(0.0, __dmul_rn(a0, x0));  // sums start at +0, as in any plain loop
+                num = __dadd_rn(num, __dmul_rn(a1, x1));
+                const double den = __dadd_rn(__dadd_rn(0.0, a0), a1);
+                cond_store(base, e, P.es, __ddiv_rn(num, den));
+                for (int i = 1; i + 1 < P.ccap; ++i)  // the later slots move down by one
+                    cond_copy_elem(base + (int64_t)i * P.cst, base + (int64_t)(i + 1) * P.cst, e, P.es);
+            }
+            C = P.ccap - 1;
+        } else if (P.policy == HKV_CONDENSE_MERGE && full) {
+            fold = true;
+            C = 0;
+        } else if (full) {  // EVICT: the oldest slot goes
+            for (int t = threadIdx.x; t < 2 * NE; t += COND_NT) {
+                char *base = t < NE ? ck : cv;
+                const int e = e0 + (t < NE ? t : t - NE);
+                for (int i = 0; i + 1 < P.ccap; ++i)
+                    cond_copy_elem(base + (int64_t)i * P.cst, base + (int64_t)(i + 1) * P.cst, e, P.es);
+            }
+            C = P.ccap - 1;
+        }
+        if (P.policy == HKV_CONDENSE_MERGE) {
+            // weights in slot order: the folded slot's first, then the block's
+            const double wf = fold ? (double)cw[0] : 0.0;
+            double S = fold ? __dadd_rn(0.0, wf) : 0.0;
+            for (int j = 0; j < blk; ++j)
+                S = __dadd_rn(S, sm.a[j]);
+            const bool eq = !(S > 0.0);
+            for (int t = threadIdx.x; t < 2 * NE; t += COND_NT) {
+                const bool isk = t < NE;
+                const char *src = isk ? sk : sv;
+                char *dst = (isk ? ck : cv) + (int64_t)C * P.cst;
+                const int e = e0 + (isk ? t : t - NE);
+                double num = 0.0, den = 0.0;
+                if (fold) {
+                    const double a_ = eq ? 1.0 : wf;
+                    num = __dadd_rn(num, __dmul_rn(a_, cond_load(dst, e, P.es)));
+                    den = __dadd_rn(den, a_);
+                }
+#pragma unroll 4
+                for (int j = 0; j < blk; ++j) {
+                    const double a_ = eq ? 1.0 : sm.a[j];
+                    num = __dadd_rn(num, __dmul_rn(a_, cond_load(src + (int64_t)j * P.sst, e, P.es)));
+                    den = __dadd_rn(den, a_);
+                }
+                cond_store(dst, e, P.es, __ddiv_rn(num, den));
+            }
+        } else {
+            const int js = sm.jstar;
+            for (int t = threadIdx.x; t < 2 * NE; t += COND_NT) {
+                const bool isk = t < NE;
+                const int e = e0 + (isk ? t : t - NE);
+                cond_copy_elem((isk ? ck : cv) + (int64_t)C * P.cst, (isk ? sk : sv) + (int64_t)js * P.sst, e, P.es);
+            }
+        }
+    }
+    __syncthreads();  // the block's rows are read; the move may overwrite them
+
+    // the sparse tier moves down by blk rows: batches staged in shared memory
+    // (a batch's rows are all read before any is written, and a later batch
+    // reads only rows above everything written so far)
+    const int QB = NE * P.es;          // this CTA's bytes of one row of K (and of V)
+    const int QC = QB / 16;            // ... in 16-byte chunks
+    const int rows_per_batch = COND_STAGE / (2 * QB);
+    const int left = n - blk;
+    for (int r0 = 0; r0 < left; r0 += rows_per_batch) {
+        const int rows = min(rows_per_batch, left - r0);
+        const int chunks = rows * 2 * QC;
+        for (int c = threadIdx.x; c < chunks; c += COND_NT) {
+            const int row = c / (2 * QC), q = c - row * 2 * QC;
+            const bool isk = q < QC;
+            const char *src = (isk ? sk : sv) + (int64_t)(r0 + blk + row) * P.sst + e0 * P.es + (isk ? q : q - QC) * 16;
+            *reinterpret_cast<uint4 *>(sm.stage + c * 16) = __ldcs(reinterpret_cast<const uint4 *>(src));
+        }
+        __syncthreads();
+        for (int c = threadIdx.x; c < chunks; c += COND_NT) {
+            const int row = c / (2 * QC), q = c - row * 2 * QC;
+            const bool isk = q < QC;
+            char *dst = (isk ? sk : sv) + (int64_t)(r0 + row) * P.sst + e0 * P.es + (isk ? q : q - QC) * 16;
+            *reinterpret_cast<uint4 *>(dst) = *reinterpret_cast<const uint4 *>(sm.stage + c * 16);
+        }
+        __syncthreads();
+    }
+    // every CTA of the unit has read the lengths and weights: update them
+    cluster.sync();
+    if (r == 0 && threadIdx.x == 0) {
+        P.slen[u] = n - blk;
+        if (P.ccap > 0) {
+            if (P.policy == HKV_CONDENSE_MERGE) {
+                if (C0 >= P.ccap && P.ccap >= 2) {
+                    cw[0] = __double2float_rn(__dadd_rn(__dadd_rn(0.0, (double)cw[0]), (double)cw[1]));
+                    for (int i = 1; i + 1 < P.ccap; ++i)
+                        cw[i] = cw[i + 1];
+                }
+                double S = fold ? __dadd_rn(0.0, (double)cw[0]) : 0.0;
+                for (int j = 0; j < blk; ++j)
+                    S = __dadd_rn(S, sm.a[j]);
+                cw[C] = __double2float_rn(S);
+            } else {
+                if (C0 >= P.ccap)
+                    for (int i = 0; i + 1 < P.ccap; ++i)
+                        cw[i] = cw[i + 1];
+                cw[C] = __double2float_rn(sm.a[sm.jstar]);
+            }
+            P.clen[u] = C + 1;
+        }
+        if (P.done)
+            P.done[u] = 1;
+    }
+}
+
+}  // namespace hkv
+
+extern "C" hkv_status hkv_condense(const hkv_problem *prob, const hkv_tier *sparse, const hkv_tier *condensed,
+                                   float *cond_w, const float *z, int64_t z_stride, const float *m,
+                                   const float *logZ, int32_t block, int32_t trigger,
+                                   hkv_condense_policy policy, int32_t *done, void *ws, size_t ws_bytes,
+                                   hkv_stream_t stream)
+{
+    hkv_status s = check_problem(prob);
+    if (s != HKV_OK)
+        return s;
+    if (sparse == nullptr)
+        return HKV_ERR_INVALID_ARG;
+    if ((s = check_tier(sparse, prob, true)) != HKV_OK || (s = check_tier(condensed, prob, true)) != HKV_OK)
+        return s;
+    if (ws == nullptr || !aligned(ws, 256) || ws_bytes < 256)
+        return HKV_ERR_WORKSPACE;
+    const int ncap = sparse->cap, ccap = condensed ? condensed->cap : 0;
+    if (block < 1 || block > HKV_CONDENSE_MAX_BLOCK || block > ncap || trigger < 0 ||
+        (policy != HKV_CONDENSE_MERGE && policy != HKV_CONDENSE_EVICT))
+        return HKV_ERR_INVALID_ARG;
+    if (ccap > 0 && (cond_w == nullptr || !aligned(cond_w, 4)))
+        return HKV_ERR_INVALID_ARG;
+    const bool scores = z != nullptr || m != nullptr || logZ != nullptr;
+    if (scores && (z == nullptr || m == nullptr || logZ == nullptr || !aligned(z, 4) || z_stride < ncap))
+        return HKV_ERR_INVALID_ARG;
+    if (done != nullptr && !aligned(done, 4))
+        return HKV_ERR_INVALID_ARG;
+    const int64_t units = (int64_t)prob->B * prob->Hkv;
+    if (units == 0 || ncap == 0)
+        return HKV_OK;
+    const int es = es_of(prob->dtype);
+    CondP P{};
+    P.sk = static_cast<char *>(const_cast<void *>(sparse->k));
+    P.sv = static_cast<char *>(const_cast<void *>(sparse->v));
+    P.ssb = sparse->stride_b * es;
+    P.ssh = sparse->stride_h * es;
+    P.sst = sparse->stride_t * es;
+    P.slen = const_cast<int32_t *>(sparse->len);
+    if (ccap > 0) {
+        P.ck = static_cast<char *>(const_cast<void *>(condensed->k));
+        P.cv = static_cast<char *>(const_cast<void *>(condensed->v));
+        P.csb = condensed->stride_b * es;
+        P.csh = condensed->stride_h * es;
+        P.cst = condensed->stride_t * es;
+        P.clen = const_cast<int32_t *>(condensed->len);
+    }
+    P.ncap = ncap;
+    P.ccap = ccap;
+    P.cw = cond_w;
+    P.z = scores ? z : nullptr;
+    P.m = scores ? m : nullptr;
+    P.logZ = scores ? logZ : nullptr;
+    P.z_stride = z_stride;
+    P.inv_temp = prob->inv_temp;
+    P.done = done;
+    P.Hkv = prob->Hkv;
+    P.units = (int32_t)units;
+    P.D = prob->D;
+    P.es = es;
+    P.block = block;
+    P.trigger = trigger;
+    P.policy = (int32_t)policy;
+    P.status = static_cast<uint32_t *>(ws);
+    const size_t smem = sizeof(CondSmem);
+    if ((s = prepare((const void *)k_condense, COND_NT, smem, nullptr)) != HKV_OK)
+        return s;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(units * COND_CTAS));
+    cfg.blockDim = dim3(COND_NT);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = (cudaStream_t)stream;
+    if (cudaLaunchKernelEx(&cfg, k_condense, P) != cudaSuccess)
         return HKV_ERR_CUDA;
     g_launches.fetch_add(1);
     return HKV_OK;

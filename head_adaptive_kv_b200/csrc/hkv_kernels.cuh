@@ -84,7 +84,36 @@ struct Params {
     const float *h_target;
     float *h_out, *beta_out;
     uint64_t wait_ns;
+    // Rewrite Cache vs Sparse Loading (hkv_step_mti; nullptr elsewhere): steps
+    // each unit's rewrite still serves (> 0: the unit reuses it this step),
+    // the rewrite buffer (rows in its len) and the token indices of its rows
+    const int32_t *mti_left;
+    TierP rw;
+    const int32_t *rw_idx;
+    // kernel timeline (hkv_set_timeline; nullptr when off): per kernel kind,
+    // the complement of its earliest start and its latest end (global timer)
+    unsigned long long *tl;
 };
+
+// Kernel kinds of the timeline (index of their start word; the end word is 8 on).
+enum : int { TL_SCORE = 0, TL_UNIT = 1, TL_ATTN = 2, TL_MERGE = 3, TL_FLAT = 4, TL_FIT = 5, TL_MTI = 6 };
+
+// A CTA's start and end on the timeline: starts are kept as complements under
+// atomicMax, so that zeroed words mean "nothing recorded" for both.
+__device__ __forceinline__ void tl_start(unsigned long long *tl, int kind)
+{
+    if (tl != nullptr && threadIdx.x == 0)
+        atomicMax(tl + kind, ~(unsigned long long)global_ns());
+}
+
+__device__ __forceinline__ void tl_end(unsigned long long *tl, int kind)
+{
+    if (tl != nullptr) {
+        __syncthreads();
+        if (threadIdx.x == 0)
+            atomicMax(tl + 8 + kind, (unsigned long long)global_ns());
+    }
+}
 
 __device__ __forceinline__ Ctl make_ctl(const Params &P) { return Ctl{P.ctl, P.wait_ns}; }
 
@@ -225,16 +254,20 @@ __device__ __forceinline__ void ring_init(R &r)
 // Up to NS stages are in flight. If a wait runs out (status word set), the
 // warp stops consuming, waits (bounded) for the copies it started, and returns.
 template <class Job, class R>
-__device__ void warp_pipeline(Job &job, R &ring, const Ctl &c, int tslot = -1)
+__device__ uint32_t warp_pipeline(Job &job, R &ring, const Ctl &c, int tslot = -1, uint32_t start = 0)
 {
+    // start: stages the warp already pushed through its ring (slot i % NS,
+    // phase parity (i / NS) & 1 for the i-th stage overall)
     constexpr int NS = Job::NS;
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    uint32_t issued = 0, consumed = 0;
+    uint32_t issued = start, consumed = start;
     StageDesc d;
-    while (issued < (uint32_t)NS && job.next(d)) {
-        if (issued < 12)
-            HKV_TRACE_WARP(tslot < 0 ? -1 : TRACE_STAGES + tslot * 8 + 2 * (int)issued);
-        job.issue(d, (int)issued);
+    if (start > 0 && lane == 0)
+        fence_proxy_async_smem();  // the warp's reads of its slots before the copies that refill them
+    while (issued < start + (uint32_t)NS && job.next(d)) {
+        if (issued - start < 12)
+            HKV_TRACE_WARP(tslot < 0 ? -1 : TRACE_STAGES + tslot * 8 + 2 * (int)(issued - start));
+        job.issue(d, (int)(issued % NS));
         ++issued;
     }
     bool ok = true;
@@ -244,10 +277,10 @@ __device__ void warp_pipeline(Job &job, R &ring, const Ctl &c, int tslot = -1)
             ok = false;
             break;
         }
-        if (consumed == 0)
+        if (consumed == start)
             HKV_TRACE_WARP(tslot < 0 ? -1 : tslot + 1);
-        if (consumed < 12)
-            HKV_TRACE_WARP(tslot < 0 ? -1 : TRACE_STAGES + tslot * 8 + 2 * (int)consumed + 1);
+        if (consumed - start < 12)
+            HKV_TRACE_WARP(tslot < 0 ? -1 : TRACE_STAGES + tslot * 8 + 2 * (int)(consumed - start) + 1);
         const StageDesc cd = ring.desc[w][j];
         job.consume(cd, ring.slot[w][j]);
         __syncwarp();
@@ -255,8 +288,8 @@ __device__ void warp_pipeline(Job &job, R &ring, const Ctl &c, int tslot = -1)
         if (job.next(d)) {
             if (lane == 0)
                 fence_proxy_async_smem();  // this warp's reads of the slot before the copies that refill it
-            if (issued < 12)
-                HKV_TRACE_WARP(tslot < 0 ? -1 : TRACE_STAGES + tslot * 8 + 2 * (int)issued);
+            if (issued - start < 12)
+                HKV_TRACE_WARP(tslot < 0 ? -1 : TRACE_STAGES + tslot * 8 + 2 * (int)(issued - start));
             job.issue(d, j);
             ++issued;
         }
@@ -271,6 +304,7 @@ __device__ void warp_pipeline(Job &job, R &ring, const Ctl &c, int tslot = -1)
     }
     __syncwarp();
     HKV_TRACE_WARP(tslot < 0 ? -1 : tslot + 2);
+    return issued;
 }
 
 // ---- warp butterfly over the LPR lanes of a row: NV partial sums per lane ->
@@ -377,20 +411,66 @@ __device__ __forceinline__ int64_t share_owner(int64_t t, int64_t NW, int64_t T)
 
 // ---- scoring ([TS 2.B] max-pooled attention logits; [TS 2.A] Tier 2) --------
 //
-// Work line: the sparse tier's capacity rows of all units, unit-major; a warp
-// scores the rows of its share that lie below the unit's length. In hkv_step
-// each warp also folds the range of the scores it wrote into its units'
-// range words (atomic max of order keys), which the selection starts from.
+// Work line: the rows each unit has to score, unit-major, cut into equal
+// static shares, one per warp. With at most PREFIX_CAP units the line holds
+// exactly those rows (a unit's length, or none for a unit that reuses a
+// rewrite this step): every CTA sums the units' counts in shared memory. With
+// more units the line is the capacity rows of all units, and rows past a
+// unit's length are skipped. In hkv_step each warp also folds the range of
+// the scores it wrote into its units' range words (atomic max of order keys),
+// which the selection starts from.
+
+// Rows unit u scores this step: its sparse length, or 0 when it reuses a rewrite.
+__device__ __forceinline__ int score_len(const Params &P, int u, const Ctl &c)
+{
+    if (P.mti_left != nullptr && __ldcg(P.mti_left + u) > 0)
+        return 0;
+    return tier_len(P.sparse, u, c);
+}
+
+struct ScoreLineSmem {
+    int64_t pre[PREFIX_CAP + 1];  // line position of each unit's first row
+};
+
+// Prefix layout: the units' line positions in shared memory. Returns the rows on the line.
+template <int NTH>
+__device__ int64_t score_prologue(const Params &P, const Ctl &c, ScoreLineSmem &L, unsigned long long *red)
+{
+    constexpr int UPT = (PREFIX_CAP + NTH - 1) / NTH;
+    unsigned long long carry = 0;
+#pragma unroll
+    for (int i = 0; i < UPT; ++i) {
+        if (i * NTH >= P.units)
+            break;  // uniform over the CTA
+        const int u = i * NTH + threadIdx.x;
+        const int n = u < P.units ? score_len(P, u, c) : 0;
+        unsigned long long tot;
+        const unsigned long long ex = block_exclusive_scan<NTH>((unsigned long long)n, red, &tot);
+        if (u < P.units)
+            L.pre[u] = (int64_t)(carry + ex);
+        carry += tot;
+    }
+    if (threadIdx.x == 0)
+        L.pre[P.units] = (int64_t)carry;
+    __syncthreads();
+    return (int64_t)carry;
+}
 
 template <int ES, int D, int G>
 struct ScoreJob {
     using Gm = Geo<ES, D, G>;
     static constexpr int NS = sc_stages(G), NW = sc_nw(G);
     using RingT = Ring<NW, SC_SLOT, NS>;
+    struct Smem {
+        RingT ring;
+        ScoreLineSmem line;
+        unsigned long long red[NW];
+    };
 
     const Params &P;
     const Ctl &c;
     RingT &ring;
+    const ScoreLineSmem *L;  // prefix layout (nullptr: capacity layout)
     uint64_t policy;
     int w, lane;
     // generator: the share's next row is row j of unit u; `left` rows remain
@@ -402,25 +482,52 @@ struct ScoreJob {
     float2 qv[G][Gm::NP];
     float tmax = -INFINITY, tmin = INFINITY;
 
-    __device__ ScoreJob(const Params &P_, const Ctl &c_, RingT &ring_, int64_t r0, int64_t r1)
-        : P(P_), c(c_), ring(ring_), policy(evict_first_policy()), w(threadIdx.x >> 5), lane(threadIdx.x & 31)
+    // Rows unit x holds on the line.
+    __device__ __forceinline__ int span(int x) const
     {
-        const int cap = max(P.sparse.cap, 1);
-        u = (int)(r0 / cap);
-        j = (int)(r0 - (int64_t)u * cap);
+        return L ? (int)(L->pre[x + 1] - L->pre[x]) : P.sparse.cap;
+    }
+
+    __device__ ScoreJob(const Params &P_, const Ctl &c_, RingT &ring_, const ScoreLineSmem *L_, int64_t T,
+                        int64_t g, int64_t nw)
+        : P(P_), c(c_), ring(ring_), L(L_), policy(evict_first_policy()), w(threadIdx.x >> 5), lane(threadIdx.x & 31)
+    {
+        const int64_t r0 = share_begin(g, nw, T), r1 = share_begin(g + 1, nw, T);
         left = r1 - r0;
+        if (L != nullptr) {
+            // the unit holding line position r0 (the last with pre[u] <= r0)
+            int lo = 0, hi = P.units - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (L->pre[mid] <= r0)
+                    lo = mid;
+                else
+                    hi = mid - 1;
+            }
+            u = lo;
+            j = (int)(r0 - L->pre[u]);
+        } else {
+            const int cap = max(P.sparse.cap, 1);
+            u = (int)(r0 / cap);
+            j = (int)(r0 - (int64_t)u * cap);
+        }
+    }
+
+    __device__ __forceinline__ void enter(int x)
+    {
+        if (x != gu) {  // length and K rows of a new unit
+            gu = x;
+            gn = L ? span(x) : score_len(P, x, c);
+            const int b = x / P.Hkv, h = x % P.Hkv;
+            kbase = P.sparse.k + ((int64_t)b * P.sparse.sb + (int64_t)h * P.sparse.sh) * ES;
+        }
     }
 
     __device__ __forceinline__ bool next(StageDesc &d)
     {
         while (left > 0) {
-            if (u != gu) {  // length and K rows of a new unit
-                gu = u;
-                gn = tier_len(P.sparse, u, c);
-                const int b = u / P.Hkv, h = u % P.Hkv;
-                kbase = P.sparse.k + ((int64_t)b * P.sparse.sb + (int64_t)h * P.sparse.sh) * ES;
-            }
-            const int seg = (int)min(left, (int64_t)(P.sparse.cap - j));  // rows of unit u left in the share
+            enter(u);
+            const int seg = (int)min(left, (int64_t)(span(u) - j));  // rows of unit u left in the share
             const int vend = min(j + seg, gn);
             if (j >= vend) {
                 left -= seg;
@@ -468,18 +575,18 @@ struct ScoreJob {
         __syncwarp();
     }
 
-    // A share inside one unit whose rows are all present (the common case):
-    // the stages follow from their number alone, so the warp runs this short
-    // loop instead of warp_pipeline's general generator. Returns false when
-    // the share does not qualify.
+    // A static share inside one unit whose rows are all present (the common
+    // case): the stages follow from their number alone, so the warp runs this
+    // short loop instead of warp_pipeline's general generator, and leaves the
+    // job at the end of its static share. Returns false (having done nothing)
+    // when the share does not qualify or a wait ran out.
     __device__ __forceinline__ bool run_single_unit()
     {
         if (left <= 0 || P.withhold)
             return false;
-        const int cap = P.sparse.cap;
-        if ((int64_t)j + left > cap)
+        if ((int64_t)j + left > span(u))
             return false;
-        const int n = tier_len(P.sparse, u, c);
+        const int n = L ? span(u) : score_len(P, u, c);
         if (j + (int)left > n)
             return false;
         gu = u;
@@ -503,7 +610,8 @@ struct ScoreJob {
                 // let the copies already started land before returning
                 for (int i = sidx; i < nst && i < sidx + NS; ++i)
                     mbar_wait_bounded(&ring.full[w][i % NS], (i / NS) & 1u, c.wait_ns);
-                return true;
+                left = 0;
+                return false;
             }
             consume(stage(sidx), ring.slot[w][slot]);
             __syncwarp();
@@ -513,6 +621,7 @@ struct ScoreJob {
                 copy_stage(stage(sidx + NS), slot);
             }
         }
+        left = 0;
         return true;
     }
 
@@ -810,7 +919,7 @@ struct AttnSmem {
     // attn_prefix (every line shorter than 2^31): start of each unit on line A
     // and on line B, and each unit's dense, sparse, selected and condensed counts
     int32_t pre[2][PREFIX_CAP + 1];
-    int32_t uW[PREFIX_CAP], uN[PREFIX_CAP], uK[PREFIX_CAP], uC[PREFIX_CAP];
+    int32_t uW[PREFIX_CAP], uN[PREFIX_CAP], uR[PREFIX_CAP];  // dense, sparse and rewrite-buffer rows
 };
 
 // A line of the attention work: the units' spans laid end to end and the
@@ -837,7 +946,7 @@ struct AttnJob {
     // generator
     int line = 0;
     int64_t t = 0, t_end = 0;
-    int gu = -1, gW = 0, gk = 0, gtot = 0, last_unit = -1;
+    int gu = -1, gW = 0, gR = 0, gk = 0, gtot = 0, last_unit = -1;
     int64_t gS = 0, gspan = 0;
     const int32_t *gidx = nullptr;
     int gn = 0;
@@ -849,13 +958,21 @@ struct AttnJob {
     bool had = false;
     int q_unit = -1;
 
-    __device__ AttnJob(const Params &P_, const Ctl &c_, SM &sm_, const AttnLine &A, const AttnLine &B, int64_t g_)
+    // Line A first; line B once begin_line_b gives it (the budgets it needs
+    // are known only after the selection kernel).
+    __device__ AttnJob(const Params &P_, const Ctl &c_, SM &sm_, const AttnLine &A, int64_t g_)
         : P(P_), c(c_), sm(sm_), policy(evict_first_policy()), w(threadIdx.x >> 5), lane(threadIdx.x & 31), g(g_)
     {
         ln[0] = A;
-        ln[1] = B;
+        ln[1] = AttnLine{0, 0, 0};
         start_line(0);
         st.reset();
+    }
+
+    __device__ __forceinline__ void begin_line_b(const AttnLine &B)
+    {
+        ln[1] = B;
+        start_line(1);
     }
 
     __device__ __forceinline__ void start_line(int l)
@@ -886,35 +1003,34 @@ struct AttnJob {
         gS = unit_start(u);
         gspan = unit_start(u + 1) - gS;
         int C;
-        if (P.attn_prefix) {  // counts the prologue checked and kept
+        if (P.attn_prefix) {  // counts the prologue checked and kept; spans are exact
             gW = sm.uW[u];
             gn = sm.uN[u];
-            gk = sm.uK[u];
-            C = sm.uC[u];
+            gR = sm.uR[u];
+            gk = sm.pre[1][u + 1] - sm.pre[1][u];
+            C = sm.pre[0][u + 1] - sm.pre[0][u] - gW - gR;
         } else {
             gW = tier_len(P.dense, u, c);
             gn = tier_len(P.sparse, u, c);
+            gR = 0;
             gk = unit_budget(P, u, gn, c);
             C = tier_len(P.cond, u, c);
         }
-        // tokens of the unit on this line: dense ++ condensed (A) or the selection (B)
-        gtot = line == 0 ? gW + C : gk;
+        // tokens of the unit on this line: dense ++ rewrite buffer ++ condensed
+        // (A) or the selection (B)
+        gtot = line == 0 ? gW + gR + C : gk;
         if (line == 1 && gk > 0)
             gidx = P.layout == HKV_LAYOUT_FLAT_SUM ? P.idx + __ldcg(P.offsets + u) : P.idx + (int64_t)u * P.bmax;
     }
 
     // Stages never cross a unit or a tier. Line A positions a < W are dense
-    // rows, the rest condensed rows a - W; line B positions are selection
-    // entries.
+    // rows, then R rows of a reused rewrite buffer, then condensed rows
+    // a - W - R; line B positions are selection entries.
     __device__ __forceinline__ bool next(StageDesc &d)
     {
         for (;;) {
-            if (t >= t_end) {
-                if (line == 1)
-                    return false;
-                start_line(1);
-                continue;
-            }
+            if (t >= t_end)
+                return false;  // the end of this line's share
             if (gu < 0 || t >= gS + gspan) {
                 int u = gu + 1;
                 if (gu < 0) {  // first unit of the share: binary search
@@ -949,9 +1065,9 @@ struct AttnJob {
             }
             int cnt, flags;
             if (line == 0) {
-                const int tier_end = a < gW ? gW : vend;
+                const int tier_end = a < gW ? gW : (a < gW + gR ? gW + gR : vend);
                 cnt = min(Gm::ATOK, min(vend, tier_end) - a);
-                const bool contiguous = a < gW ? P.dense.st == D : P.cond.st == D;
+                const bool contiguous = a < gW ? P.dense.st == D : (a < gW + gR ? P.rw.st == D : P.cond.st == D);
                 flags = contiguous ? 0 : SD_GATHER;
             } else {
                 cnt = min(Gm::ATOK, vend - a);
@@ -963,6 +1079,21 @@ struct AttnJob {
             t = last ? gS + seg_end : t + cnt;
             return true;
         }
+    }
+
+    // The tier and row of line-A position a of the current unit.
+    __device__ __forceinline__ const TierP &line_a_tier(int a, int *row) const
+    {
+        if (a < gW) {
+            *row = a;
+            return P.dense;
+        }
+        if (a < gW + gR) {
+            *row = a - gW;
+            return P.rw;
+        }
+        *row = a - gW - gR;
+        return P.cond;
     }
 
     // Source rows of line position a of the current unit (lane-level).
@@ -1001,9 +1132,9 @@ struct AttnJob {
             if (lane == 0) {
                 mbar_arrive_expect_tx(bar, (uint32_t)(2 * d.count * Gm::ROWB));
                 if (d.count > 0) {
-                    const bool dn = d.start < gW;
-                    const TierP &Tt = dn ? P.dense : P.cond;
-                    const int64_t off = row_offset(Tt, b, h, dn ? d.start : d.start - gW);
+                    int r;
+                    const TierP &Tt = line_a_tier(d.start, &r);
+                    const int64_t off = row_offset(Tt, b, h, r);
                     bulk_g2s(dst, Tt.k + off, d.count * Gm::ROWB, bar, policy);
                     bulk_g2s(dst + AT_SLOT / 2, Tt.v + off, d.count * Gm::ROWB, bar, policy);
                 }
@@ -1056,10 +1187,9 @@ struct AttnJob {
                 ks = P.sparse.k + off;
                 vs = P.sparse.v + off;
             } else {
-                const int a = d.start + lane;
-                const bool dn = a < gW;
-                const TierP &Tt = dn ? P.dense : P.cond;
-                off = row_offset(Tt, b, h, dn ? a : a - gW);
+                int r;
+                const TierP &Tt = line_a_tier(d.start + lane, &r);
+                off = row_offset(Tt, b, h, r);
                 ks = Tt.k + off;
                 vs = Tt.v + off;
             }
@@ -1135,7 +1265,7 @@ struct AttnJob {
 // thread reads the input lengths of its units (attn_prefix).
 constexpr int AT_UPT = PREFIX_CAP / (AT_NW * 32);  // units per thread
 struct AttnLens {
-    int W[AT_UPT], N[AT_UPT], C[AT_UPT];
+    int W[AT_UPT], N[AT_UPT], C[AT_UPT], R[AT_UPT];  // R: rows of a reused rewrite, -1 when not reused
 };
 
 __device__ __forceinline__ void attn_read_lengths(const Params &P, const Ctl &c, AttnLens &L)
@@ -1149,65 +1279,92 @@ __device__ __forceinline__ void attn_read_lengths(const Params &P, const Ctl &c,
         L.W[i] = ok ? tier_len(P.dense, u, c) : 0;
         L.N[i] = ok ? tier_len(P.sparse, u, c) : 0;
         L.C[i] = ok ? tier_len(P.cond, u, c) : 0;
+        L.R[i] = ok && P.mti_left != nullptr && __ldcg(P.mti_left + u) > 0 ? tier_len(P.rw, u, c) : -1;
     }
 }
 
-// Part 2 (after the wait): the budgets, the two lines and, with attn_prefix,
-// each unit's start on each line and its counts in shared memory; CTA 0 also
-// writes every unit's record slots (rec_range[u] = first and last slot on line
-// A, then on line B; first > last when empty) for k_merge.
+// Part 2 (before the wait, from the inputs alone): line A -- with
+// attn_prefix each unit's start on it and its dense, sparse and rewrite-buffer
+// counts in shared memory.
 template <int ES, int D, int G>
-__device__ void attn_prologue(const Params &P, AttnSmem<ES, D, G> &sm, const Ctl &c, unsigned long long *red,
-                              const AttnLens &Ln, AttnLine *A, AttnLine *B)
+__device__ AttnLine attn_prologue_a(const Params &P, AttnSmem<ES, D, G> &sm, unsigned long long *red,
+                                    const AttnLens &Ln)
 {
     constexpr int NTA = AT_NW * 32;
     const int64_t NWt = (int64_t)gridDim.x * AT_NW;
-    int64_t TA, TB;
+    int64_t TA;
     if (P.attn_prefix) {
-        unsigned long long ca = 0, cb = 0;
+        unsigned long long ca = 0;
 #pragma unroll
         for (int i = 0; i < AT_UPT; ++i) {
             if (i * NTA >= P.units)
                 break;  // uniform over the CTA
             const int u = i * NTA + threadIdx.x;
-            unsigned long long ta = 0, tb = 0;
+            unsigned long long ta = 0;
             if (u < P.units) {
-                const int k = unit_budget(P, u, Ln.N[i], c);
+                // a unit that reuses its rewrite attends its rows on line A
+                const int R = Ln.R[i] >= 0 ? Ln.R[i] : 0;
                 sm.uW[u] = Ln.W[i];
                 sm.uN[u] = Ln.N[i];
-                sm.uK[u] = k;
-                sm.uC[u] = Ln.C[i];
-                ta = (unsigned long long)(Ln.W[i] + Ln.C[i]);
-                tb = (unsigned long long)k;
+                sm.uR[u] = R;
+                ta = (unsigned long long)(Ln.W[i] + R + Ln.C[i]);
             }
-            // both prefixes in one scan (each line is shorter than 2^31)
             unsigned long long sum;
-            const unsigned long long ex = block_exclusive_scan<NTA>((tb << 32) | ta, red, &sum);
-            if (u < P.units) {
-                sm.pre[0][u] = (int32_t)(ca + (ex & 0xffffffffull));
-                sm.pre[1][u] = (int32_t)(cb + (ex >> 32));
-            }
-            ca += sum & 0xffffffffull;
-            cb += sum >> 32;
+            const unsigned long long ex = block_exclusive_scan<NTA>(ta, red, &sum);
+            if (u < P.units)
+                sm.pre[0][u] = (int32_t)(ca + ex);
+            ca += sum;
         }
-        if (threadIdx.x == 0) {
+        if (threadIdx.x == 0)
             sm.pre[0][P.units] = (int32_t)ca;
-            sm.pre[1][P.units] = (int32_t)cb;
-        }
         __syncthreads();
         TA = (int64_t)ca;
-        TB = (int64_t)cb;
     } else {
         TA = (int64_t)P.units * (P.dense.cap + P.cond.cap);
+    }
+    return AttnLine{TA, min(NWt, TA), 0};
+}
+
+// Part 3 (after the wait): the budgets and line B -- with attn_prefix each
+// unit's start on it; CTA 0 also writes every unit's record slots
+// (rec_range[u] = first and last slot on line A, then on line B; first > last
+// when empty) for k_merge.
+template <int ES, int D, int G>
+__device__ AttnLine attn_prologue_b(const Params &P, AttnSmem<ES, D, G> &sm, const Ctl &c, unsigned long long *red,
+                                    const AttnLens &Ln, const AttnLine &A)
+{
+    constexpr int NTA = AT_NW * 32;
+    const int64_t NWt = (int64_t)gridDim.x * AT_NW;
+    int64_t TB;
+    if (P.attn_prefix) {
+        unsigned long long cb = 0;
+#pragma unroll
+        for (int i = 0; i < AT_UPT; ++i) {
+            if (i * NTA >= P.units)
+                break;  // uniform over the CTA
+            const int u = i * NTA + threadIdx.x;
+            unsigned long long tb = 0;
+            if (u < P.units)  // a unit that reuses its rewrite has no selection on line B
+                tb = Ln.R[i] >= 0 ? 0ull : (unsigned long long)unit_budget(P, u, Ln.N[i], c);
+            unsigned long long sum;
+            const unsigned long long ex = block_exclusive_scan<NTA>(tb, red, &sum);
+            if (u < P.units)
+                sm.pre[1][u] = (int32_t)(cb + ex);
+            cb += sum;
+        }
+        if (threadIdx.x == 0)
+            sm.pre[1][P.units] = (int32_t)cb;
+        __syncthreads();
+        TB = (int64_t)cb;
+    } else {
         TB = (int64_t)P.units * min(P.bmax, P.sparse.cap);
     }
-    *A = AttnLine{TA, min(NWt, TA), 0};
-    *B = AttnLine{TB, min(NWt, TB), NWt + P.units};
+    const AttnLine B{TB, min(NWt, TB), NWt + P.units};
     if (blockIdx.x == 0) {
         for (int u = threadIdx.x; u < P.units; u += NTA) {
             int r[4];
             for (int l = 0; l < 2; ++l) {
-                const AttnLine &L = l ? *B : *A;
+                const AttnLine &L = l ? B : A;
                 int64_t s0, s1;
                 if (P.attn_prefix) {
                     s0 = sm.pre[l][u];
@@ -1228,6 +1385,7 @@ __device__ void attn_prologue(const Params &P, AttnSmem<ES, D, G> &sm, const Ctl
             *reinterpret_cast<int4 *>(P.rec_range + 4 * u) = make_int4(r[0], r[1], r[2], r[3]);
         }
     }
+    return B;
 }
 
 // =============================================================================

@@ -22,6 +22,8 @@ STATUS = {0: "HKV_OK", 1: "HKV_ERR_INVALID_ARG", 2: "HKV_ERR_UNSUPPORTED", 3: "H
           4: "HKV_ERR_TIMEOUT", 5: "HKV_ERR_DEVICE", 6: "HKV_ERR_WORKSPACE"}
 DEV_LEN_CLAMPED, DEV_TIMEOUT, DEV_BAD_TEMP, DEV_BAD_INDEX, DEV_BAD_P = 0x1, 0x2, 0x4, 0x8, 0x10
 DEV_SPARSE_FULL = 0x20
+CONDENSE_MERGE, CONDENSE_EVICT = 0, 1
+CONDENSE_MAX_BLOCK = 8192
 
 
 class HkvError(RuntimeError):
@@ -68,13 +70,17 @@ def _load():
         "hkv_compact": [P, P, i64, P, P, P, P, P, P, P, P, sz, P],
         "hkv_cascade_decode": [P, P, P, P, P, P, P, P, P, P, P, sz, P],
         "hkv_step": [P, P, P, P, P, P, P, sz, P],
+        "hkv_step_mti": [P, P, P, P, P, P, P, P, sz, P],
         "hkv_cascade_decode_noalloc": [P, P, P, P, P, P, P, P, P, P, P, P],
         "hkv_append": [P, P, P, P, P, P, P, P, sz, P],
+        "hkv_condense": [P, P, P, P, P, i64, P, P, i32, i32, i32, P, P, sz, P],
         "hkv_attention_entropy": [P, P, P, P, P, sz, P],
         "hkv_fit_temperature": [P, P, i64, P, P, P, P, sz, P],
         "hkv_get_status": [P, C.POINTER(C.c_uint32), P],
         "hkv_set_wait_limit_ns": [C.c_uint64],
         "hkv_debug_withhold_publish": [i32],
+        "hkv_set_timeline": [i32],
+        "hkv_read_timeline": [P, C.POINTER(C.c_uint64), P],
         "hkv_launch_count": [],
         "hkv_status_string": [i32],
     }
@@ -284,6 +290,50 @@ def step(prob: Problem, q: torch.Tensor, dense: Optional[Tier], sparse: Tier, co
                         C.byref(out.c()), ws.ptr, ws.nbytes, _stream(stream)), "hkv_step")
 
 
+class _Mti(C.Structure):
+    _fields_ = [("L_lower", C.c_int32), ("L_upper", C.c_int32), ("mti_cap", C.c_int64), ("mode", C.c_void_p),
+                ("left", C.c_void_p), ("rewrite", _Tier), ("rw_idx", C.c_void_p)]
+
+
+@dataclass
+class MtiState:
+    """Rewrite Cache / Sparse Loading trigger: thresholds, memory-time allowance
+    and the per-unit state (mode, left), the rewrite buffer (a Tier of capacity
+    >= bmax whose len holds the rows each unit's rewrite keeps) and the token
+    indices of those rows (rw_idx, int32 [B*Hkv*bmax])."""
+
+    L_lower: int
+    L_upper: int
+    mti_cap: int
+    mode: torch.Tensor
+    left: torch.Tensor
+    rewrite: Tier
+    rw_idx: torch.Tensor
+
+    def c(self) -> _Mti:
+        for t in (self.mode, self.left, self.rw_idx):
+            if t.dtype != torch.int32 or not t.is_contiguous():
+                raise TypeError("mode, left and rw_idx must be contiguous int32")
+        return _Mti(int(self.L_lower), int(self.L_upper), int(self.mti_cap), self.mode.data_ptr(),
+                    self.left.data_ptr(), self.rewrite.c(), self.rw_idx.data_ptr())
+
+    @staticmethod
+    def allocate(prob: "Problem", device, L_lower: int, L_upper: int, mti_cap: int) -> "MtiState":
+        U, dev = prob.units, torch.device(device)
+        z = lambda: torch.zeros(U, dtype=torch.int32, device=dev)
+        buf = lambda: torch.zeros(prob.B, prob.Hkv, max(prob.bmax, 1), prob.D, dtype=prob.dtype, device=dev)
+        return MtiState(L_lower, L_upper, mti_cap, z(), z(), Tier(buf(), buf(), z()),
+                        torch.zeros(U * max(prob.bmax, 1), dtype=torch.int32, device=dev))
+
+
+def step_mti(prob: "Problem", q: torch.Tensor, dense: Optional[Tier], sparse: Tier, condensed: Optional[Tier],
+             mti: MtiState, out: "StepOutputs", ws: "Workspace", stream=None):
+    """hkv_step under the Rewrite Cache / Sparse Loading trigger (see hkv_step_mti)."""
+    _check(lib.hkv_step_mti(C.byref(prob.c()), _ptr(q), _tref(dense), C.byref(sparse.c()), _tref(condensed),
+                            C.byref(mti.c()), C.byref(out.c()), ws.ptr, ws.nbytes, _stream(stream)),
+           "hkv_step_mti")
+
+
 def cascade_decode_noalloc(prob: Problem, q: torch.Tensor, dense: Optional[Tier], sparse: Optional[Tier],
                            idx: Optional[torch.Tensor], sel_len: Optional[torch.Tensor],
                            condensed: Optional[Tier], out: torch.Tensor, lse: Optional[torch.Tensor] = None,
@@ -315,6 +365,25 @@ def append(prob: Problem, k_new: torch.Tensor, v_new: torch.Tensor, dense: Optio
                           _tref(sparse), _ptr(dropped), ws.ptr, ws.nbytes, _stream(stream)), "hkv_append")
 
 
+def condense(prob: Problem, sparse: Tier, condensed: Optional[Tier], cond_w: Optional[torch.Tensor],
+             ws: Workspace, block: int, trigger: int, policy: int = CONDENSE_MERGE,
+             z: Optional[torch.Tensor] = None, m: Optional[torch.Tensor] = None,
+             logZ: Optional[torch.Tensor] = None, done: Optional[torch.Tensor] = None, stream=None):
+    """Condensed-tier formation, in place on the tiers' K, V and lengths and on
+    cond_w (fp32 [B*Hkv, condensed cap]): units whose sparse tier holds at
+    least max(trigger, block) tokens turn their oldest `block` tokens into one
+    condensed slot (MERGE: weighted mean; EVICT: the most important token),
+    weighted by the calibrated probabilities of the step's scores z (with its
+    m and logZ; all three or none). done: optional int32 [B*Hkv]."""
+    if cond_w is not None and (cond_w.dtype != torch.float32 or not cond_w.is_contiguous()):
+        raise ValueError("cond_w must be a contiguous fp32 tensor [B*Hkv, condensed cap]")
+    if z is not None and (z.dtype != torch.float32 or z.dim() != 2 or z.stride(1) != 1):
+        raise ValueError("z must be fp32 [B*Hkv, >= sparse cap] with contiguous rows")
+    _check(lib.hkv_condense(C.byref(prob.c()), C.byref(sparse.c()), _tref(condensed), _ptr(cond_w), _ptr(z),
+                            0 if z is None else z.stride(0), _ptr(m), _ptr(logZ), int(block), int(trigger),
+                            int(policy), _ptr(done), ws.ptr, ws.nbytes, _stream(stream)), "hkv_condense")
+
+
 def _f32_vector(t: torch.Tensor, n: int, what: str):
     if t.dtype != torch.float32 or t.dim() != 1 or t.stride(0) != 1 or t.numel() < n:
         raise ValueError(f"{what} must be a contiguous fp32 vector of at least {n} elements")
@@ -341,6 +410,22 @@ def fit_temperature(prob: Problem, z: torch.Tensor, sparse: Tier, h_target: torc
 
 def set_wait_limit_ns(ns: int):
     _check(lib.hkv_set_wait_limit_ns(int(ns)), "hkv_set_wait_limit_ns")
+
+
+TL_KINDS = ("score", "select", "attention", "merge", "layout", "fit", "trigger")
+
+
+def set_timeline(on: bool):
+    """Record the step kernels' start and end times in their workspace (see hkv_set_timeline)."""
+    _check(lib.hkv_set_timeline(1 if on else 0), "hkv_set_timeline")
+
+
+def read_timeline(ws: Workspace, stream=None) -> dict:
+    """Read and clear a workspace's kernel timeline: {kind: (start_ns, end_ns)}
+    for the kinds that ran since the last read."""
+    buf = (C.c_uint64 * (2 * len(TL_KINDS)))()
+    _check(lib.hkv_read_timeline(ws.ptr, buf, _stream(stream)), "hkv_read_timeline")
+    return {k: (int(buf[2 * i]), int(buf[2 * i + 1])) for i, k in enumerate(TL_KINDS) if buf[2 * i + 1]}
 
 
 def debug_withhold_publish(on: bool):

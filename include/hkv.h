@@ -227,6 +227,52 @@ hkv_status hkv_step(const hkv_problem *prob, const void *q, const hkv_tier *dens
                     const hkv_step_out *out, void *ws, size_t ws_bytes,
                     hkv_stream_t stream);
 
+/* State and thresholds of the trade-off between Rewrite Cache and Sparse
+ * Loading ([TS 2.C] Trade-off Management: a Memory-Time Integral weighs the
+ * upfront cost of rewriting against the per-step decoding gains, and budget
+ * thresholds L_lower and L_upper trigger sparse loading or full rewriting;
+ * [TS 4]: the rewrite overhead is amortized within a few decoding steps).
+ * Every per-unit array is caller-owned device memory, zero before the first
+ * step (all units start in Sparse Loading with no rewrite). */
+typedef struct {
+    int32_t L_lower, L_upper;  /* budget thresholds (tokens), 0 <= L_lower <= L_upper: a fresh budget
+                                  k > L_upper switches the unit to Rewrite Cache, k < L_lower to Sparse
+                                  Loading, and a budget in between keeps the unit's mode */
+    int64_t mti_cap;           /* memory-time allowance of one rewrite, in row-steps: a rewrite of k
+                                  rows serves H(k) = max(1, floor(mti_cap / k)) steps, the step that
+                                  made it included */
+    int32_t *mode;             /* device [B*Hkv]: 0 Sparse Loading, 1 Rewrite Cache (read, written) */
+    int32_t *left;             /* device [B*Hkv]: further steps the unit's rewrite serves (read, written) */
+    hkv_tier rewrite;          /* the rewrite buffer: K, V [B, Hkv, cap >= bmax, D] (written), len =
+                                  device [B*Hkv] rows it holds (written) */
+    int32_t *rw_idx;           /* device [B*Hkv*bmax]: token indices of the rewritten rows (written) */
+} hkv_mti;
+
+/* The decode step under the Rewrite Cache / Sparse Loading trigger ([TS 2.C]
+ * Rewrite Cache: selected rows moved to contiguous ranges; Sparse Loading: rows
+ * read through the indices; Trade-off Management). Per unit u at each call:
+ * - left[u] > 0 (the unit reuses its rewrite): the unit is not scored or
+ *   selected; its attention runs over dense ++ rewrite rows [0, rewrite.len[u])
+ *   ++ condensed, read as contiguous rows; its outputs report sel_len[u] =
+ *   rewrite.len[u] and, in idx, the rows' token indices as of the rewrite;
+ *   cut, m and logZ are NaN (kstar -1); afterwards left[u] -= 1.
+ * - left[u] == 0: the unit is scored, selected and attended exactly as by
+ *   hkv_step (Sparse Loading of the fresh selection). Then its mode follows the
+ *   trigger on the fresh budget k (above), and under Rewrite Cache its k
+ *   selected K and V rows are copied to rewrite rows 0 .. k-1 (bit copies,
+ *   token order), rw_idx gets their indices, rewrite.len[u] = k and
+ *   left[u] = H(k) - 1; under Sparse Loading rewrite.len[u] = left[u] = 0.
+ * Other arguments and outputs as for hkv_step, except that out->k_out/v_out
+ * and out->beta_fit must be NULL. At most 1024 units (HKV_ERR_UNSUPPORTED
+ * beyond). A rewrite keeps the rows it copied: a token that ages into the
+ * sparse tier, or a condensation (hkv_condense) of the unit, takes effect for
+ * the unit at its next fresh step; set left[u] = 0 to force one. One more
+ * kernel than hkv_step (the trigger and the copies), a cluster of four CTAs
+ * per unit. */
+hkv_status hkv_step_mti(const hkv_problem *prob, const void *q, const hkv_tier *dense, const hkv_tier *sparse,
+                        const hkv_tier *condensed, const hkv_mti *mti, const hkv_step_out *out, void *ws,
+                        size_t ws_bytes, hkv_stream_t stream);
+
 /* KV append with the dense-window roll ([TS 2.A] Cascade Cache Hierarchy,
  * pipeline step 1: the new token joins the dense window of recent tokens, and
  * the token that leaves the window moves to the sparse tier). One kernel, one
@@ -292,6 +338,53 @@ hkv_status hkv_fit_temperature(const hkv_problem *prob, const float *z, int64_t 
                                const hkv_tier *sparse, const float *h_target, float *beta,
                                void *ws, size_t ws_bytes, hkv_stream_t stream);
 
+/* Condensed-tier formation ([TS 2.A] Tier 3: "the oldest blocks are further
+ * compressed into constant-sized storage via eviction or weighted merging";
+ * pipeline step 4, "eviction or merging of the oldest blocks"). One kernel, a
+ * cluster of four CTAs per unit. A unit u whose sparse tier holds
+ * n >= max(trigger, block) tokens gives up its oldest `block` tokens (sparse
+ * slots 0 .. block-1: the tier is in age order, as hkv_append keeps it); they
+ * become ONE condensed slot, written after the existing slots:
+ *   HKV_CONDENSE_MERGE: the slot's K and V rows are the weighted means of the
+ *     block's rows, weighted by the tokens' calibrated probabilities
+ *     a_j = exp(beta_u (z_j - m_u) - logZ_u) under the step's scores (beta_u
+ *     from prob->inv_temp, 1 when NULL), and the slot's weight is sum_j a_j. A
+ *     full condensed tier first merges its two oldest slots the same way
+ *     (weighted by their weights; the result weighs their sum) and moves the
+ *     later slots down; a tier of one slot folds the block into that slot.
+ *   HKV_CONDENSE_EVICT: the slot is a bit copy of the block's most important
+ *     token (largest z_j, the older one on ties), weighing a_j; the rest of
+ *     the block is dropped. A full condensed tier first drops its oldest slot.
+ * Weights that sum to zero, or no scores (z, m, logZ all NULL), mean equal
+ * weights (and EVICT keeps the oldest token). Means are float64 sums in slot
+ * order, each product and sum rounded separately, divided once and rounded
+ * once to the element type (nearest, ties to even; bf16 straight from the
+ * double). The sparse tier then moves down by `block` rows (age order kept)
+ * and its length drops by `block`; a condensed tier of capacity 0 just loses
+ * the block. The cost is a read and a write of the unit's remaining sparse
+ * rows; it is paid once per `block` appends when the call runs after each
+ * step with trigger = the sparse capacity.
+ * - sparse, condensed: tiers as elsewhere (condensed may be NULL or empty);
+ *   THIS CALL WRITES through their k, v and len pointers.
+ * - cond_w: device fp32 [B*Hkv, condensed->cap], the slots' weights, read and
+ *   written (required when the condensed tier has slots; start with zeros or
+ *   the weights of slots filled some other way).
+ * - z (z_stride >= sparse->cap), m, logZ: device fp32, the scores of the
+ *   sparse tier and each unit's max and log normaliser from the last step
+ *   (hkv_step's z, m and logZ outputs); all three or none.
+ * - block: 1 .. min(HKV_CONDENSE_MAX_BLOCK, sparse->cap); trigger >= 0.
+ * - done: device int32 [B*Hkv] or NULL; 1 where the unit gave up a block.
+ * - A unit whose lengths are outside [0, cap] is left as it is and sets
+ *   HKV_DEV_LEN_CLAMPED; a negative or NaN inverse temperature uses 1 and
+ *   sets HKV_DEV_BAD_TEMP.
+ * - ws: any workspace of at least 256 bytes (only its status word is used). */
+typedef enum { HKV_CONDENSE_MERGE = 0, HKV_CONDENSE_EVICT = 1 } hkv_condense_policy;
+#define HKV_CONDENSE_MAX_BLOCK 8192
+hkv_status hkv_condense(const hkv_problem *prob, const hkv_tier *sparse, const hkv_tier *condensed,
+                        float *cond_w, const float *z, int64_t z_stride, const float *m, const float *logZ,
+                        int32_t block, int32_t trigger, hkv_condense_policy policy, int32_t *done,
+                        void *ws, size_t ws_bytes, hkv_stream_t stream);
+
 /* Capacity, in bytes, of the device scratch array behind
  * hkv_cascade_decode_noalloc (one array per GPU that loads the library, held
  * until the process exits). */
@@ -313,9 +406,13 @@ hkv_status hkv_fit_temperature(const hkv_problem *prob, const float *z, int64_t 
  *   that example); a problem with too many units for even one CTA (about 1000
  *   units at G = 4, D = 128) is refused with HKV_ERR_WORKSPACE before anything
  *   is launched: use hkv_cascade_decode with a workspace for those.
- * - Set-up: the first call on each device looks up the array's device address
- *   and sets the kernel's shared-memory attribute. Make that first call outside
- *   any stream capture.
+ * - Set-up: a call made outside stream capture looks up the array's device
+ *   address in the current context (the first one on a device also loads the
+ *   module and sets the kernel's shared-memory attribute); a call under
+ *   capture reuses the address found by the last call outside capture on that
+ *   device. So make the first call on each device, and the first after a
+ *   cudaDeviceReset (which also discards the array's contents), outside any
+ *   stream capture.
  * - Sharing: every call on a device uses the same array, which keeps the last
  *   call's contents. Each call zeroes the one word that must start at zero
  *   (the status word) on `stream` before its kernels run; everything else is
@@ -346,6 +443,20 @@ hkv_status hkv_get_status(void *ws, uint32_t *flags, hkv_stream_t stream);
 /* Upper bound, in nanoseconds, of every spin-wait inside the library's kernels
  * (default 1e9). Takes effect at the next launch. */
 hkv_status hkv_set_wait_limit_ns(uint64_t ns);
+
+/* Kernel timeline, a measurement aid: while on (it takes effect at the next
+ * launch), the step's kernels record, in the workspace they run with, the
+ * earliest start and the latest end of each kernel kind (device global
+ * timer, nanoseconds; one atomic per CTA at each end). Kinds: 0 scoring,
+ * 1 per-unit selection and compaction, 2 attention, 3 merge, 4 layout (FLAT_SUM
+ * rows, Rewrite Cache copies), 5 fitted temperature, 6 the rewrite trigger. */
+#define HKV_TL_KINDS 7
+hkv_status hkv_set_timeline(int32_t on);
+
+/* Read and clear the timeline of a workspace. Synchronises `stream`.
+ * start_end: host [2*HKV_TL_KINDS], start then end per kind; 0 and 0 for a
+ * kind that did not run since the last read (or since hkv_workspace_init). */
+hkv_status hkv_read_timeline(void *ws, uint64_t *start_end, hkv_stream_t stream);
 
 /* Fault injection for tests: when nonzero, the streaming kernels (scoring and
  * attention, hkv_step included) never arm their copy stages, so each consumer's
