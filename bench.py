@@ -424,6 +424,8 @@ def workload_entry(hkv, wl, device, stream, p=None, with_oracle=True) -> dict:
          "peak_kind": peak_kind,
          "budgets": {"min": int(ks.min()), "median": int(np.median(ks)), "max": int(ks.max()),
                      "mean": round(float(ks.mean()), 1)}}
+    # live in-step kernel spans of the first layer's step
+    e["in_step"] = in_step_spans(hkv, prob, xs[0], tiers[0], outs[0], ws, stream, reps=5)
     if with_oracle:
         e["cpu_baseline"] = oracle_sample(wl.with_(p=p), host_state(xs[0]), wl.layers)
     del g

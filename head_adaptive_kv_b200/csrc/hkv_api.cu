@@ -38,7 +38,11 @@ namespace hkv {
 // Per unit u of the fitting kernel, TR_FIT + 16u + i: 0 start, 1 entropy
 // done, 2 scores staged, 3 beta found; 4 holds the number of evaluations.
 // Per unit u of the merge kernel, TR_MRG + 2u: 0 start, 1 done.
-[[maybe_unused]] constexpr int TR_SEL = 250000, TR_SW = 0, TR_AW = 20000, TR_FIT = 240000, TR_MRG = 260000;
+// Per attention warp g, TR_AB + 2g: line B start (after the wait and its
+// layout), line B done (merges included); TR_LB + 4g: line B's pipeline
+// (first landing, end, and the stages at TRACE_STAGES + 8 (TR_LB + 4g)).
+[[maybe_unused]] constexpr int TR_SEL = 250000, TR_SW = 0, TR_AW = 20000, TR_FIT = 240000, TR_MRG = 260000,
+                               TR_AB = 30000, TR_LB = 8000;
 
 // =============================================================================
 // Kernels
@@ -98,7 +102,9 @@ __global__ void __launch_bounds__(AT_NW * 32, 1) k_attn_stream(const __grid_cons
     wait_prior_grid();
     HKV_TRACE_WARP(TR_AW + 4 * (int)g + 3);
     job.begin_line_b(attn_prologue_b<ES, D, G>(P, sm, c, red, lens, A));
-    warp_pipeline(job, sm.ring, c, -1, used);
+    HKV_TRACE_WARP(TR_AB + 2 * (int)g);
+    warp_pipeline(job, sm.ring, c, TR_LB + 4 * (int)g, used);
+    HKV_TRACE_WARP(TR_AB + 2 * (int)g + 1);
     tl_end(P.tl, TL_ATTN);
 }
 
@@ -108,8 +114,8 @@ template <int D, int G>
 __global__ void __launch_bounds__(G * 32) k_merge(const __grid_constant__ Params P)
 {
     allow_dependents();
-    wait_prior_grid();
     const int u = blockIdx.x;
+    wait_prior_grid();
     HKV_TRACE_AT(TR_MRG + 2 * u);
     tl_start(P.tl, TL_MERGE);
     const int4 r = __ldcg(reinterpret_cast<const int4 *>(P.rec_range) + u);
@@ -158,6 +164,20 @@ __device__ __forceinline__ void write_offsets(const Params &P, int u, int64_t of
     }
 }
 
+// The V rows of unit u's sparse tier, for RowPrefetch (the step only).
+template <int ES>
+__device__ __forceinline__ RowPrefetch v_prefetch(const Params &P, int u)
+{
+    RowPrefetch r;
+    if (P.prefetch_v && P.sparse.v != nullptr) {
+        const int b = u / P.Hkv, h = u % P.Hkv;
+        r.base = P.sparse.v + ((int64_t)b * P.sparse.sb + (int64_t)h * P.sparse.sh) * ES;
+        r.stride = P.sparse.st * ES;
+        r.bytes = (uint32_t)(P.D * ES);
+    }
+    return r;
+}
+
 // S2-S4 of unit u, scores at zu (in shared memory when ZS).
 // zg_stage (ZS only): the unit's scores are still in global memory there and
 // the fast path stages them during its first sweep.
@@ -204,7 +224,7 @@ __device__ __forceinline__ void unit_work(const Params &P, USmem &sm, const Ctl 
             Selection s;
             if (P.do_compact &&
                 select_compact_fast(zu, n, m, zlo, beta, pu, P.bmin, P.bmax, sm, s, P.idx + (int64_t)u * P.bmax,
-                                    P.bmax, TR_SEL + 16 * u, zg_stage)) {
+                                    P.bmax, TR_SEL + 16 * u, zg_stage, v_prefetch<ES>(P, u))) {
                 publish(s);
                 HKV_TRACE_AT(TR_SEL + 16 * u + 5);
                 return;
@@ -235,7 +255,7 @@ __device__ __forceinline__ void unit_work(const Params &P, USmem &sm, const Ctl 
         write_offsets(P, u, off);
     }
     int32_t *row = P.idx + off;
-    compact_unit<ZS>(zu, n, key, n_tie, k, row, flat ? k : P.bmax, sm.red, TR_SEL + 16 * u);
+    compact_unit<ZS>(zu, n, key, n_tie, k, row, flat ? k : P.bmax, sm.red, TR_SEL + 16 * u, v_prefetch<ES>(P, u));
     HKV_TRACE_AT(TR_SEL + 16 * u + 5);
     if (P.k_out != nullptr && !P.do_select) {
         __syncthreads();
@@ -277,7 +297,7 @@ __device__ void mti_reuse_outputs(const Params &P, const Ctl &c, int u)
 //             order from the cut -- PAD_MAX rows, or FLAT_SUM (standalone) --
 //             and, standalone, the Rewrite Cache copy when k_out is given.
 template <int ES>
-__global__ void __launch_bounds__(NT) k_unit(const __grid_constant__ Params P)
+__global__ void __launch_bounds__(NT, 1) k_unit(const __grid_constant__ Params P)
 {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     USmem &sm = *reinterpret_cast<USmem *>(smem_raw);
@@ -701,8 +721,13 @@ struct RunAttn {
         const int max_ctas = (P.part_slots / 2 - P.units) / AT_NW;
         if (max_ctas < 1)
             return HKV_ERR_WORKSPACE;
+        // with fewer units than SMs, line A goes to the CTAs that start while
+        // the selection kernel (one CTA per unit) runs
+        const int sms = sm_count();
+        Params Q = P;
+        Q.attn_a_ctas = (pdl && P.units < sms) ? sms - P.units : (1 << 30);
         hkv_status st = launch_stream(k_attn_stream<ES, D, G>, AT_NW * 32, sizeof(AttnSmem<ES, D, G>), max_ctas, s,
-                                      P, pdl);
+                                      Q, pdl);
         if (st != HKV_OK)
             return st;
         return launch(k_merge<D, G>, P.units, G * 32, 0, s, P, true);
@@ -939,6 +964,7 @@ hkv_status step_impl(const hkv_problem *prob, const void *q, const hkv_tier *den
     U.have_range = scored;
     U.do_select = 1;
     U.do_compact = 1;
+    U.prefetch_v = 1;
     if ((s = launch_unit(prob, U, st, true)) != HKV_OK)
         return s;
     // 3. attention over the three tiers and the merge of each unit

@@ -174,6 +174,12 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         : "memory");
 }
 
+// Start bringing the 128-byte line holding `src` into L2.
+__device__ __forceinline__ void prefetch_l2_line(const void *src)
+{
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(src));
+}
+
 // 16-byte asynchronous copy global -> shared, cached in L2 only.
 __device__ __forceinline__ void cp_async16(void *dst, const void *src)
 {

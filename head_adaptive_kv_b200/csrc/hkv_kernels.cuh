@@ -26,6 +26,7 @@
 
 namespace hkv {
 
+
 constexpr int SC_SLOT = 8192;             // scoring: bytes per stage (K rows)
 // scoring: warps per CTA and ring slots per warp (192 KB of slots per CTA);
 // eight query heads per group keep twice the query registers per lane, so
@@ -76,8 +77,10 @@ struct Params {
     float *part;          // [part_slots * part_stride] attention records
     int32_t part_slots;   // record slots: 2 x (streaming warps of the attention grid + units)
     int32_t attn_prefix;  // attention partition over actual tokens (units <= PREFIX_CAP, lines < 2^31), else over capacity
+    int32_t attn_a_ctas;  // attention CTAs that share line A (the first ones, which start while the selection runs)
     int32_t have_range;   // per-unit kernel: urange holds the units' score ranges
     int32_t do_select, do_compact;  // per-unit kernel: which steps to run
+    int32_t prefetch_v;   // per-unit kernel: bring the selected tokens' V rows into L2 (the attention follows)
     int32_t withhold;     // fault injection: streaming warps never arm their stages
     // fitted temperature: per-unit entropy target in (nullptr: from the logit
     // records), target out, fitted inverse temperature out
@@ -205,11 +208,18 @@ struct Geo {
     static constexpr int NV = NB * G;                     // partial sums per lane before reduction
     static constexpr int REP = LPR / NV;                  // lanes holding the same sum afterwards
     static constexpr int SROWS = SC_SLOT / ROWB;          // rows per scoring stage
-    static constexpr int ATOK = (AT_SLOT / 2) / ROWB;     // tokens per attention stage
+    static constexpr int ATOK = (AT_SLOT / 2) / ROWB;     // tokens per attention stage (K and V rows)
+    // a stage of selected tokens read with the scorer's logits holds no K rows:
+    // room for 32 logit records, then BTOK V rows from byte VOFF_B (fewer,
+    // fuller stages: a warp's share of the selection is only a few stages long)
+    static constexpr int VOFF_B = 32 * logit_floats(G) * 4;
+    static constexpr int BTOK0 = (AT_SLOT - VOFF_B) / ROWB;
+    static constexpr int BTOK = BTOK0 < 32 ? BTOK0 : 32;
     static constexpr int DPL = D / 32;                    // PV: head-dim elements per lane
     static_assert(G >= 1 && G <= LPR, "group size must not exceed lanes per row");
     static_assert(ATOK * G <= SC_FLOATS && ATOK <= 32, "stage sizes");
     static_assert(ATOK * logit_floats(G) * 4 <= AT_SLOT / 2, "logit records of a stage");
+    static_assert(BTOK * G <= SC_FLOATS && BTOK >= ATOK && VOFF_B % 16 == 0, "stages of selected tokens");
     static_assert(SITERS % NB == 0 && AITERS % NB == 0 && LPR % NV == 0, "iteration batches");
 };
 
@@ -802,7 +812,7 @@ __device__ __forceinline__ void attn_stage(const Params &P, const unsigned char 
             st.o[g][e].x *= alpha[g];
             st.o[g][e].y *= alpha[g];
         }
-    const unsigned char *vbase = stage + AT_SLOT / 2 + lane * Gm::DPL * ES;
+    const unsigned char *vbase = stage + (from_logits ? Gm::VOFF_B : AT_SLOT / 2) + lane * Gm::DPL * ES;
 #pragma unroll 2
     for (int r = 0; r < nt; ++r) {
         float2 vv[NPV];
@@ -1070,7 +1080,7 @@ struct AttnJob {
                 const bool contiguous = a < gW ? P.dense.st == D : (a < gW + gR ? P.rw.st == D : P.cond.st == D);
                 flags = contiguous ? 0 : SD_GATHER;
             } else {
-                cnt = min(Gm::ATOK, vend - a);
+                cnt = min(P.logit != nullptr ? Gm::BTOK : Gm::ATOK, vend - a);
                 flags = P.logit != nullptr ? SD_LOGIT : SD_GATHER;
             }
             const bool last = a + cnt >= vend;
@@ -1163,7 +1173,7 @@ struct AttnJob {
                 const char *v_ = reinterpret_cast<const char *>(
                     (uintptr_t)__shfl_sync(0xffffffffu, (unsigned long long)(uintptr_t)vs, r & 31));
                 if (r < d.count)
-                    cp_async16(dst + AT_SLOT / 2 + r * Gm::ROWB + cc * 16, v_ + cc * 16);
+                    cp_async16(dst + Gm::VOFF_B + r * Gm::ROWB + cc * 16, v_ + cc * 16);
             }
             if (lane < d.count)
 #pragma unroll
@@ -1322,7 +1332,13 @@ __device__ AttnLine attn_prologue_a(const Params &P, AttnSmem<ES, D, G> &sm, uns
     } else {
         TA = (int64_t)P.units * (P.dense.cap + P.cond.cap);
     }
-    return AttnLine{TA, min(NWt, TA), 0};
+    // line A goes to the first attn_a_ctas CTAs only: with fewer units than
+    // SMs those start on the SMs the selection kernel leaves free and finish
+    // line A while it runs; the others start when it ends, and go straight to
+    // line B
+    const int64_t NWa = (int64_t)min((int)gridDim.x, max(1, P.attn_a_ctas)) * AT_NW;
+    (void)NWt;
+    return AttnLine{TA, min(NWa, TA), 0};
 }
 
 // Part 3 (after the wait): the budgets and line B -- with attn_prefix each
@@ -1564,6 +1580,9 @@ __device__ __forceinline__ void sweep_stage(const float *zg, float *zs, int n, F
 {
     const bool vec = (((uintptr_t)zg) & 15) == 0;
     const int nq = (n + 3) >> 2;
+    // a batch's loads all in flight and stored, then f over the thread's own
+    // scores read back in one rolled loop (a single copy of f's code: these
+    // kernels run it once per unit and are otherwise bound by instruction fetch)
     for (int base = 0; base < nq; base += NT * SWEEP_Q) {
         float4 v[SWEEP_Q];
 #pragma unroll
@@ -1583,10 +1602,11 @@ __device__ __forceinline__ void sweep_stage(const float *zg, float *zs, int n, F
             const int j = 4 * (base + i * NT + (int)threadIdx.x);
             if (j < n)
                 reinterpret_cast<float4 *>(zs)[j >> 2] = v[i];  // j < n <= ZSTAGE, j a multiple of 4
-            f(v[i].x, j, j < n);
-            f(v[i].y, j + 1, j + 1 < n);
-            f(v[i].z, j + 2, j + 2 < n);
-            f(v[i].w, j + 3, j + 3 < n);
+        }
+#pragma unroll 1
+        for (int x = 0; x < 4 * SWEEP_Q; ++x) {
+            const int j = 4 * (base + (x >> 2) * NT + (int)threadIdx.x) + (x & 3);
+            f(j < n ? lds1(zs + j) : 0.f, j, j < n);
         }
     }
 }
@@ -1972,6 +1992,19 @@ __device__ Selection select_unit(const float *zu, int n, float m, float zlo, flo
 }
 
 // =============================================================================
+// S2-S4 fused, lean, for a unit whose scores are staged in shared memory as
+// the first sweep reads them (hkv_step): the same budget, cut and PAD_MAX row
+// as select_unit followed by compact_unit, in three sweeps over the scores --
+// (A) stage them and build the bin counts, the bins' exact fixed-point masses
+// and Z; (B) gather the tokens of the few bins that can hold the cut and count,
+// per warp segment, the tokens in the bins before each; (C) write the
+// selection in index order -- with one scan of the bins between A and B, and
+// sorts of the needed bins between B and C. Returns false, having written
+// nothing, when a needed bin outgrows its buffer; the caller then takes
+// select_unit and compact_unit on the staged scores.
+// =============================================================================
+
+// =============================================================================
 // S2-S4 fused for a unit whose scores are staged in shared memory (hkv_step):
 // the same budget and cut as select_unit followed by compact_unit, with fewer
 // passes over the unit. After the count histogram (sweep 1, which also sums
@@ -2100,9 +2133,25 @@ __device__ int list_candidates_warp(const float *zs, int n, const BinFn &bins, i
     return (int)tot;
 }
 
+// The V rows of a unit's selected tokens, brought into L2 as the compaction
+// finds them (the step's attention gathers them next). base nullptr: none.
+struct RowPrefetch {
+    const char *base = nullptr;
+    int64_t stride = 0;  // bytes between rows
+    uint32_t bytes = 0;  // bytes of a row
+    __device__ __forceinline__ void operator()(int j) const
+    {
+        if (base == nullptr)
+            return;
+        const uintptr_t a = reinterpret_cast<uintptr_t>(base + (int64_t)j * stride);
+        for (uintptr_t l = a & ~(uintptr_t)127; l < a + bytes; l += 128)
+            prefetch_l2_line(reinterpret_cast<const void *>(l));
+    }
+};
+
 __device__ bool select_compact_fast(const float *zs, int n, float m, float zlo, float beta, float p, int bmin,
                                     int bmax, USmem &sm, Selection &r, int32_t *row, int pad, int tb,
-                                    const float *zg = nullptr)
+                                    const float *zg = nullptr, const RowPrefetch &pf = RowPrefetch{})
 {
     const float bl2 = beta * LOG2E;
     const BinFn bins = make_bins(m, zlo);
@@ -2217,12 +2266,14 @@ __device__ bool select_compact_fast(const float *zs, int n, float m, float zlo, 
                 if ((uint32_t)(e >> 32) < cut_key) {
                     const uint32_t j = (uint32_t)e;
                     atomicOr(&sm.bits[j >> 5], 1u << (j & 31));
+                    pf((int)j);
                 }
             }
             const int n_tie = k - n_above;
             for (int i = threadIdx.x; i < n_tie; i += NT) {
                 const uint32_t j = (uint32_t)sm.binbuf[tie0 + i];
                 atomicOr(&sm.bits[j >> 5], 1u << (j & 31));
+                pf((int)j);
             }
             __syncthreads();
             // expansion in index order: thread t takes a contiguous run of words
@@ -2278,7 +2329,7 @@ __device__ __forceinline__ float zload(const float *zu, int j)
 
 template <bool ZS>
 __device__ void compact_unit(const float *zu, int n, uint32_t cut_key, int n_tie, int k, int32_t *row, int pad,
-                             unsigned long long *red, int tb = -1)
+                             unsigned long long *red, int tb = -1, const RowPrefetch &pf = RowPrefetch{})
 {
     constexpr int NW = NT / 32;
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -2313,8 +2364,10 @@ __device__ void compact_unit(const float *zu, int n, uint32_t cut_key, int n_tie
             const uint32_t eq_taken_before = min(eq_rank, (uint32_t)n_tie);
             const bool take = ((mlt >> lane) & 1u) || (((meq >> lane) & 1u) && eq_rank < (uint32_t)n_tie);
             const uint32_t pos = lt_before + __popc(mlt & lower) + eq_taken_before;
-            if (take && pos < (uint32_t)k)  // a caller's inconsistent cut stays in the row
+            if (take && pos < (uint32_t)k) {  // a caller's inconsistent cut stays in the row
                 row[pos] = j;
+                pf(j);
+            }
             lt_before += __popc(mlt);
             eq_before += __popc(meq);
         }
