@@ -109,17 +109,58 @@ __global__ void __launch_bounds__(AT_NW * 32, 1) k_attn_stream(const __grid_cons
 }
 
 // S5 merge: out and lse of each (unit, query head) from the unit's records on
-// both attention lines, in slot order (one warp per query head).
+// both attention lines, in slot order. Warp w takes head w % G and the
+// (w / G)-th of merge_split(G) contiguous parts of the records; the parts of a
+// head are then combined in part order.
 template <int D, int G>
-__global__ void __launch_bounds__(G * 32) k_merge(const __grid_constant__ Params P)
+__global__ void __launch_bounds__(MERGE_WARPS * 32) k_merge(const __grid_constant__ Params P)
 {
+    constexpr int S = merge_split(G), DPL = D / 32;
+    __shared__ float pm[MERGE_WARPS], pl[MERGE_WARPS], po[MERGE_WARPS][D];
     allow_dependents();
     const int u = blockIdx.x;
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, g = w % G, part = w / G;
     wait_prior_grid();
     HKV_TRACE_AT(TR_MRG + 2 * u);
     tl_start(P.tl, TL_MERGE);
     const int4 r = __ldcg(reinterpret_cast<const int4 *>(P.rec_range) + u);
-    merge_head<D, G>(P, u, threadIdx.x >> 5, r.x, r.y, r.z, r.w);
+    const int na = r.y >= r.x ? r.y - r.x + 1 : 0, nb = r.w >= r.z ? r.w - r.z + 1 : 0;
+    const int tot = na + nb;
+    float M, L, O[DPL];
+    merge_records<D, G>(P, g, r.x, na, r.z, part * tot / S, (part + 1) * tot / S, M, L, O);
+#pragma unroll
+    for (int e = 0; e < DPL; ++e)
+        po[w][lane * DPL + e] = O[e];
+    if (lane == 0) {
+        pm[w] = M;
+        pl[w] = L;
+    }
+    __syncthreads();
+    if (part == 0) {
+        for (int q = 1; q < S; ++q) {
+            const int x = q * G + g;
+            const float mq = pm[x];
+            if (mq == -INFINITY)
+                continue;
+            const float Mn = fmaxf(M, mq);
+            const float a = (M == -INFINITY) ? 0.0f : ex2(M - Mn);
+            const float f = ex2(mq - Mn);
+            L = L * a + pl[x] * f;
+#pragma unroll
+            for (int e = 0; e < DPL; ++e)
+                O[e] = O[e] * a + po[x][lane * DPL + e] * f;
+            M = Mn;
+        }
+        // no tokens at all: out 0, lse -inf
+        const int b = u / P.Hkv, h = u % P.Hkv;
+        const int hq = h * G + g;
+        float *orow = P.out + ((int64_t)b * P.Hq + hq) * D + lane * DPL;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e)
+            orow[e] = (M == -INFINITY) ? 0.0f : O[e] / L;
+        if (lane == 0 && P.lse != nullptr)
+            P.lse[(int64_t)b * P.Hq + hq] = (M == -INFINITY) ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
+    }
     HKV_TRACE_AT(TR_MRG + 2 * u + 1);
     tl_end(P.tl, TL_MERGE);
 }
@@ -730,7 +771,7 @@ struct RunAttn {
                                       Q, pdl);
         if (st != HKV_OK)
             return st;
-        return launch(k_merge<D, G>, P.units, G * 32, 0, s, P, true);
+        return launch(k_merge<D, G>, P.units, MERGE_WARPS * 32, 0, s, P, true);
     }
 };
 

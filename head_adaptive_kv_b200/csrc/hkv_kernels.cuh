@@ -860,27 +860,30 @@ __device__ __forceinline__ void attn_stage(const Params &P, const unsigned char 
 // Record layout (part_stride floats): o[G][D] (unnormalised, log2 domain
 // weights), then m[G], then l[G]. m = -inf marks a record without tokens.
 
-// Output of head g of unit u from the records in slots [a0, a1] and [b0, b1]
-// (fixed order), by one warp: lane l owns head-dim elements l*DPL ..
-// l*DPL + DPL - 1. No tokens at all gives out = 0 and lse = -inf.
+// Merge of query head g over records t_lo .. t_hi - 1 of a unit's list: its
+// na line-A records in slots a0 .. a0 + na - 1, then its line-B records from
+// slot b0 (fixed order), by one warp. Lane l owns head-dim elements l*DPL ..
+// l*DPL + DPL - 1 of the partial (M, L, O); M = -inf when no record holds a
+// token.
 template <int D, int G>
-__device__ void merge_head(const Params &P, int u, int g, int a0, int a1, int b0, int b1)
+__device__ void merge_records(const Params &P, int g, int a0, int na, int b0, int t_lo, int t_hi, float &M, float &L,
+                              float (&O)[D / 32])
 {
     constexpr int DPL = D / 32;
     constexpr int RS = part_stride(D, G);
     const int lane = threadIdx.x & 31;
-    float M = -INFINITY, L = 0.f, O[DPL];
+    M = -INFINITY;
+    L = 0.f;
 #pragma unroll
     for (int e = 0; e < DPL; ++e)
         O[e] = 0.f;
-    constexpr int RB = 16;  // records loaded together
-    const int na = a1 >= a0 ? a1 - a0 + 1 : 0, nb = b1 >= b0 ? b1 - b0 + 1 : 0;
-    for (int t0 = 0; t0 < na + nb; t0 += RB) {
+    constexpr int RB = 8;  // records loaded together
+    for (int t0 = t_lo; t0 < t_hi; t0 += RB) {
         float mt[RB], lt[RB], ot[RB][DPL];
 #pragma unroll
         for (int r = 0; r < RB; ++r) {
             const int t = t0 + r;
-            const bool ok = t < na + nb;
+            const bool ok = t < t_hi;
             const int slot = t < na ? a0 + t : b0 + (t - na);
             const float *pr = P.part + (int64_t)(ok ? slot : 0) * RS;
             mt[r] = ok ? __ldcg(pr + G * D + g) : -INFINITY;
@@ -912,15 +915,12 @@ __device__ void merge_head(const Params &P, int u, int g, int a0, int a1, int b0
             M = Mn;
         }
     }
-    const int b = u / P.Hkv, h = u % P.Hkv;
-    const int hq = h * G + g;
-    float *orow = P.out + ((int64_t)b * P.Hq + hq) * D + lane * DPL;
-#pragma unroll
-    for (int e = 0; e < DPL; ++e)
-        orow[e] = (M == -INFINITY) ? 0.0f : O[e] / L;
-    if (lane == 0 && P.lse != nullptr)
-        P.lse[(int64_t)b * P.Hq + hq] = (M == -INFINITY) ? -INFINITY : (M + log2f(L)) * 0.6931471805599453f;
 }
+
+// Warps of the merge kernel: MERGE_SPLIT(G) warps per query head, each merging
+// a contiguous part of the unit's records; the parts are then combined in order.
+constexpr int MERGE_WARPS = 16;
+__host__ __device__ constexpr int merge_split(int G) { return MERGE_WARPS / G; }
 
 template <int ES, int D, int G>
 struct AttnSmem {
