@@ -113,7 +113,7 @@ __global__ void __launch_bounds__(AT_NW * 32, 1) k_attn_stream(const __grid_cons
 // (w / G)-th of merge_split(G) contiguous parts of the records; the parts of a
 // head are then combined in part order.
 template <int D, int G>
-__global__ void __launch_bounds__(MERGE_WARPS * 32) k_merge(const __grid_constant__ Params P)
+__global__ void __launch_bounds__(MERGE_WARPS * 32, 1) k_merge(const __grid_constant__ Params P)
 {
     constexpr int S = merge_split(G), DPL = D / 32;
     __shared__ float pm[MERGE_WARPS], pl[MERGE_WARPS], po[MERGE_WARPS][D];
@@ -987,7 +987,9 @@ hkv_status step_impl(const hkv_problem *prob, const void *q, const hkv_tier *den
     const bool scored = sparse->cap > 0;
     Params S = P;
     S.urange = reinterpret_cast<uint32_t *>(wsb + L.urange);
-    if (scored && (s = dispatch<RunScore>(prob, S, st, false)) != HKV_OK)
+    // the scorer waits for the previous kernel before reading anything; PDL
+    // only hides its launch behind that kernel's tail
+    if (scored && (s = dispatch<RunScore>(prob, S, st, true)) != HKV_OK)
         return s;
     // 1b. optionally the fitted inverse temperature of every unit, from the
     // scorer's logit records and scores; the selection then uses it

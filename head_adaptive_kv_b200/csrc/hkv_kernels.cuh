@@ -39,7 +39,10 @@ constexpr int AT_STAGES = 3;              // attention: ring slots per warp
 constexpr int SC_FLOATS = 256;            // per-warp logits of one attention stage
 constexpr bool ATTN_UNROLL_QK = true;     // attention: unroll the logit batches of a full stage
 constexpr int PREFIX_CAP = 1024;          // attention: units whose token prefixes fit in shared memory
-constexpr int SEL_THREADS = 512;          // per-unit kernels
+#ifndef HKV_SEL_THREADS
+#define HKV_SEL_THREADS 512
+#endif
+constexpr int SEL_THREADS = HKV_SEL_THREADS;  // per-unit kernels
 constexpr float LOG2E = 1.4426950408889634f;
 
 struct TierP {
@@ -2203,18 +2206,20 @@ __device__ bool select_compact_fast(const float *zs, int n, float m, float zlo, 
         } else if (p <= 0.0f) {
             kstar = 0;
         } else {
-            for (int i = threadIdx.x; i < ncand; i += NT) {
-                const float z = key_score((uint32_t)(sm.cand[i] >> 32));
-                sred_add(&sm.mass[bins(z)], wfix(z, m, bl2));
-            }
-            __syncthreads();
+            // the mass of all listed tokens first (an exact integer sum): the
+            // per-bin masses are needed only when it reaches the target
+            unsigned long long part = 0;
+            for (int i = threadIdx.x; i < ncand; i += NT)
+                part += wfix(key_score((uint32_t)(sm.cand[i] >> 32)), m, bl2);
+            const unsigned long long through = block_sum_u64<NT>(part, sm.red);
             const double t = ceil((double)p * r.Z * 1099511627776.0);
             const unsigned long long T = t < 1.0 ? 1ull : (unsigned long long)t;
-            unsigned long long part = 0;
-            for (int i = threadIdx.x; i <= b_hi; i += NT)
-                part += sm.mass[i];
-            const unsigned long long through = block_sum_u64<NT>(part, sm.red);
             if (through >= T) {
+                for (int i = threadIdx.x; i < ncand; i += NT) {
+                    const float z = key_score((uint32_t)(sm.cand[i] >> 32));
+                    sred_add(&sm.mass[bins(z)], wfix(z, m, bl2));
+                }
+                __syncthreads();
                 unsigned long long mb_c, mb_m;
                 const int b_m = find_crossing(sm.cnt, mass, SBINS, true, T, &mb_c, &mb_m, sm);
                 const int cb = load_sorted_bin(b_m, ncand, bins, sm);
@@ -2231,9 +2236,12 @@ __device__ bool select_compact_fast(const float *zs, int n, float m, float zlo, 
         HKV_TRACE_AT(tb < 0 ? -1 : tb + 8);
         if (k > 0) {
             if (!(mass_cut && k == kstar)) {
-                // the clamp decides: the token of rank k
-                unsigned long long kb_c, kb_m;
-                const int b_k = find_crossing(sm.cnt, mass, SBINS, false, (unsigned long long)k, &kb_c, &kb_m, sm);
+                // the clamp decides: the token of rank k (at bmax, the bin
+                // the listing already found)
+                unsigned long long kb_c = hb_c, kb_m = 0;
+                const int b_k = k == r_hi ? b_hi
+                                          : find_crossing(sm.cnt, mass, SBINS, false, (unsigned long long)k, &kb_c,
+                                                          &kb_m, sm);
                 HKV_TRACE_AT(tb < 0 ? -1 : tb + 9);
                 const int cb = load_sorted_bin(b_k, ncand, bins, sm);
                 HKV_TRACE_AT(tb < 0 ? -1 : tb + 10);
