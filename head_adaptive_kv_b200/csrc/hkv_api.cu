@@ -257,7 +257,7 @@ __device__ __forceinline__ void unit_work(const Params &P, USmem &sm, const Ctl 
                 if (P.m_out)
                     P.m_out[u] = m;
                 if (P.logZ_out)
-                    P.logZ_out[u] = n > 0 ? (float)log(s.Z) : -INFINITY;
+                    P.logZ_out[u] = n > 0 ? (float)log(s.Z()) : -INFINITY;
             }
         };
         if constexpr (ZS) {
@@ -367,8 +367,9 @@ __global__ void __launch_bounds__(NT, 1) k_unit(const __grid_constant__ Params P
 }
 
 // S2 standalone ([TS 2.B]) for unit u: m, logZ and optionally the calibrated
-// probabilities. Z is summed exactly as the selection sums it, so m and logZ
-// match hkv_step's bit for bit.
+// probabilities. Z is summed exactly as the selection sums it (the 40-bit
+// fixed-point weights, an exact integer sum), so m and logZ match hkv_step's
+// bit for bit.
 template <bool ZS>
 __device__ __forceinline__ void calibrate_unit(const Params &P, USmem &sm, const Ctl &c, int u, int n,
                                                const float *zu)
@@ -376,12 +377,12 @@ __device__ __forceinline__ void calibrate_unit(const Params &P, USmem &sm, const
     float m, zlo;
     unit_range<ZS>(zu, n, &m, &zlo, sm);
     const float bl2 = unit_beta(P, u, c) * LOG2E;
-    double part = 0.0;
+    unsigned long long part = 0;
     sweep_scores<ZS>(zu, n, [&](float z, int, bool valid) {
         if (valid)
-            part += (double)wcal(z, m, bl2);
+            part += wfix(z, m, bl2);
     });
-    const double Z = block_sum_f64<NT>(part, sm.redd);
+    const double Z = (double)block_sum_u64<NT>(part, sm.red) * (1.0 / 1099511627776.0);
     if (P.P_out != nullptr && n > 0) {
         const float inv = (float)(1.0 / Z);
         float *Pu = P.P_out + (int64_t)u * P.z_stride;

@@ -404,24 +404,4 @@ __device__ __forceinline__ float block_max(float v, float *scratch)
     return r;
 }
 
-// Sum of a double over the CTA in a fixed order (deterministic).
-template <int NT>
-__device__ __forceinline__ double block_sum_f64(double v, double *scratch)
-{
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    constexpr int NW = NT / 32;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0)
-        scratch[warp] = v;
-    __syncthreads();
-    double r = 0.0;
-#pragma unroll
-    for (int i = 0; i < NW; ++i)
-        r += scratch[i];
-    __syncthreads();
-    return r;
-}
-
 }  // namespace hkv

@@ -1492,20 +1492,22 @@ struct __align__(16) USmem {  // shared memory of the per-unit kernels
     unsigned long long binbuf[BIN_CAP];  // the tokens of one bin, sorted (staged fast path)
     uint32_t bits[ZSTAGE / 32];          // selected tokens (staged fast path)
     unsigned long long red[NT / 32];
-    double redd[NT / 32];
     float redf[NT / 32];
     int32_t bc[8];
     unsigned long long bcl[4];
 };
 
+// Bin of a score: (m - z) s rounded to the nearest integer, clamped to
+// [0, SBINS - 1]; -inf and NaN land in the last bin. Any bin map that does not
+// decrease as z falls serves the selection (the cut itself is exact), so the
+// rounding is done with the fp32 add of 1.5 * 2^23 (whose low mantissa bits
+// are then the integer) instead of conversion instructions.
 struct BinFn {
     float m, s;
     __device__ __forceinline__ int operator()(float z) const
     {
-        if (z == -INFINITY)
-            return SBINS - 1;
-        const float t = fminf(floorf((m - z) * s), (float)(SBINS - 1));
-        return (int)t;
+        const float t = fmaxf(fminf((m - z) * s, (float)(SBINS - 1)), 0.0f);
+        return (__float_as_int(t + 12582912.0f) & 0x7fffff) ^ 0x400000;
     }
 };
 
@@ -1522,8 +1524,16 @@ struct Selection {
     int32_t k, kstar;
     hkv_cut cut;
     uint32_t key;                 // order key of the cut (unused when k = 0)
-    double Z;                     // normaliser sum_j exp(beta (z_j - m))
+    unsigned long long Zq;        // normaliser sum_j exp(beta (z_j - m)) in 40-bit fixed point
+    __device__ __forceinline__ double Z() const { return (double)Zq * (1.0 / 1099511627776.0); }
 };
+
+// Top-p target in fixed point: ceil(p Z 2^40), at least 1, for Z = Zq 2^-40.
+__device__ __forceinline__ unsigned long long mass_target(float p, unsigned long long Zq)
+{
+    const double t = ceil((double)p * (double)Zq);
+    return t < 1.0 ? 1ull : (unsigned long long)t;
+}
 
 // Largest and smallest finite score of a unit.
 template <bool ZS, class SM>
@@ -1584,8 +1594,7 @@ __device__ __forceinline__ void sweep_stage(const float *zg, float *zs, int n, F
     const bool vec = (((uintptr_t)zg) & 15) == 0;
     const int nq = (n + 3) >> 2;
     // a batch's loads all in flight and stored, then f over the thread's own
-    // scores read back in one rolled loop (a single copy of f's code: these
-    // kernels run it once per unit and are otherwise bound by instruction fetch)
+    // quads read back in a rolled loop (one copy of the quad's four calls of f)
     for (int base = 0; base < nq; base += NT * SWEEP_Q) {
         float4 v[SWEEP_Q];
 #pragma unroll
@@ -1607,9 +1616,14 @@ __device__ __forceinline__ void sweep_stage(const float *zg, float *zs, int n, F
                 reinterpret_cast<float4 *>(zs)[j >> 2] = v[i];  // j < n <= ZSTAGE, j a multiple of 4
         }
 #pragma unroll 1
-        for (int x = 0; x < 4 * SWEEP_Q; ++x) {
-            const int j = 4 * (base + (x >> 2) * NT + (int)threadIdx.x) + (x & 3);
-            f(j < n ? lds1(zs + j) : 0.f, j, j < n);
+        for (int i = 0; i < SWEEP_Q; ++i) {
+            // the quad back from shared memory (zeros past n were stored with it)
+            const int j = 4 * (base + i * NT + (int)threadIdx.x);
+            const float4 q4 = j < n ? lds4(zs + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            f(q4.x, j, j < n);
+            f(q4.y, j + 1, j + 1 < n);
+            f(q4.z, j + 2, j + 2 < n);
+            f(q4.w, j + 3, j + 3 < n);
         }
     }
 }
@@ -1856,15 +1870,16 @@ __device__ Selection select_unit(const float *zu, int n, float m, float zlo, flo
     }
     __syncthreads();
     const auto mass = [&](int b) { return sm.mass[b]; };
-    // sweep 1: bin counts and the normaliser
-    double zsum = 0.0;
+    // sweep 1: bin counts and the normaliser (an exact sum of the fixed-point
+    // weights the prefix masses add up, so it does not depend on the order)
+    unsigned long long zsum = 0;
     sweep_scores<ZS>(zu, n, [&](float z, int, bool valid) {
         if (!valid)
             return;
-        zsum += (double)wcal(z, m, bl2);
+        zsum += wfix(z, m, bl2);
         sred_add(&sm.cnt[bins(z)], 1u);
     });
-    r.Z = block_sum_f64<NT>(zsum, sm.redd);
+    r.Zq = block_sum_u64<NT>(zsum, sm.red);
     HKV_TRACE_AT(tb < 0 ? -1 : tb + 1);
 
     // sweep 2: mass of the bins up to b_hi (the bin of rank min(n, bmax)) and
@@ -1906,8 +1921,7 @@ __device__ Selection select_unit(const float *zu, int n, float m, float zlo, flo
     else if (p <= 0.0f)
         kstar = 0;
     else {
-        const double t = ceil((double)p * r.Z * 1099511627776.0);
-        unsigned long long T = t < 1.0 ? 1ull : (unsigned long long)t;
+        unsigned long long T = mass_target(p, r.Zq);
         unsigned long long part = 0;
         for (int i = threadIdx.x; i <= b_hi; i += NT)
             part += mass(i);
@@ -2054,7 +2068,7 @@ __device__ int load_sorted_bin(int b, int ncand, const BinFn &bins, USmem &sm)
 // Append the (key, index) of every staged token with bin <= b_hi to sm.cand,
 // at positions from a block scan of per-thread counts (no shared counter):
 // one sweep counts, the second writes. Returns the number listed.
-__device__ int list_candidates(const float *zs, int n, const BinFn &bins, int b_hi, USmem &sm)
+__device__ int list_candidates(const float *zs, int n, const BinFn &bins, int b_hi, USmem &sm, int base = 0)
 {
     unsigned long long mine = 0;
     sweep_scores<true>(zs, n, [&](float z, int, bool valid) { mine += (valid && bins(z) <= b_hi) ? 1u : 0u; });
@@ -2062,7 +2076,7 @@ __device__ int list_candidates(const float *zs, int n, const BinFn &bins, int b_
     int at = (int)block_exclusive_scan<NT>(mine, sm.red, &tot);
     sweep_scores<true>(zs, n, [&](float z, int j, bool valid) {
         if (valid && bins(z) <= b_hi)
-            sm.cand[at++] = ((unsigned long long)score_key(z) << 32) | (uint32_t)j;
+            sm.cand[at++] = ((unsigned long long)score_key(z) << 32) | (uint32_t)(base + j);
     });
     __syncthreads();
     return (int)tot;
@@ -2072,8 +2086,9 @@ __device__ int list_candidates(const float *zs, int n, const BinFn &bins, int b_
 // of the staged scores four tokens per lane at a time and appends its hits to
 // its own region of sm.cand (CAND_CAP / warps entries, no atomics); the regions
 // are then closed up into one list. Returns the number listed, or -1 (and
-// nothing usable in sm.cand) when a region overflows.
-__device__ int list_candidates_warp(const float *zs, int n, const BinFn &bins, int b_hi, USmem &sm)
+// nothing usable in sm.cand) when a region overflows. Token j of zs is listed
+// as index base + j.
+__device__ int list_candidates_warp(const float *zs, int n, const BinFn &bins, int b_hi, USmem &sm, int base = 0)
 {
     constexpr int NW = NT / 32, REG = CAND_CAP / NW;
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -2103,7 +2118,7 @@ __device__ int list_candidates_warp(const float *zs, int n, const BinFn &bins, i
             const unsigned m = __ballot_sync(0xffffffffu, hit);
             const int at = cnt + __popc(m & lower);
             if (hit && at < REG)
-                reg[at] = ((unsigned long long)score_key(a[e]) << 32) | (uint32_t)(j + e);
+                reg[at] = ((unsigned long long)score_key(a[e]) << 32) | (uint32_t)(base + j + e);
             cnt += __popc(m);
         }
     }
@@ -2152,6 +2167,147 @@ struct RowPrefetch {
     }
 };
 
+// From the listed tokens (sm.cand[0, ncand): every token of bins 0 .. b_hi,
+// b_hi the bin of rank r_hi = min(n, bmax), hb_c the tokens before it) and the
+// unit's bin counts: the budget, its cut and, when k > 0, the bitmap of the
+// selected tokens in sm.bits (n bits, token j at bit j). The selected tokens'
+// rows are handed to pf. Returns false when the crossing bin holds more than
+// BIN_CAP tokens (the caller falls back to the general path).
+__device__ bool cut_bitmap(int n, int ncand, int b_hi, unsigned long long hb_c, int r_hi, float m, float bl2,
+                           const BinFn &bins, float p, int bmin, int bmax, USmem &sm, Selection &r, int tb,
+                           const RowPrefetch &pf)
+{
+    const auto mass = [&](int b) { return sm.mass[b]; };
+    int kstar = -1, pos = -1;
+    bool mass_cut = false;
+    unsigned long long before_c = 0;
+    if (p >= 1.0f) {
+        kstar = n;
+    } else if (p <= 0.0f) {
+        kstar = 0;
+    } else {
+        // the mass of all listed tokens first (an exact integer sum): the
+        // per-bin masses are needed only when it reaches the target
+        unsigned long long part = 0;
+        for (int i = threadIdx.x; i < ncand; i += NT)
+            part += wfix(key_score((uint32_t)(sm.cand[i] >> 32)), m, bl2);
+        const unsigned long long through = block_sum_u64<NT>(part, sm.red);
+        const unsigned long long T = mass_target(p, r.Zq);
+        if (through >= T) {
+            for (int i = threadIdx.x; i < SBINS; i += NT)
+                sm.mass[i] = 0;
+            __syncthreads();
+            for (int i = threadIdx.x; i < ncand; i += NT) {
+                const float z = key_score((uint32_t)(sm.cand[i] >> 32));
+                sred_add(&sm.mass[bins(z)], wfix(z, m, bl2));
+            }
+            __syncthreads();
+            unsigned long long mb_c, mb_m;
+            const int b_m = find_crossing(sm.cnt, mass, SBINS, true, T, &mb_c, &mb_m, sm);
+            const int cb = load_sorted_bin(b_m, ncand, bins, sm);
+            if (cb < 0)
+                return false;
+            pos = sort_and_locate(cb, true, T, mb_m, m, bl2, sm, sm.binbuf);
+            kstar = (int)mb_c + pos + 1;
+            before_c = mb_c;
+            mass_cut = true;
+        }
+    }
+    int k = kstar < 0 ? bmax : min(kstar, bmax);
+    k = min(max(k, bmin), n);
+    HKV_TRACE_AT(tb < 0 ? -1 : tb + 8);
+    uint32_t cut_key = 0u;
+    int n_above = 0;
+    if (k > 0) {
+        if (!(mass_cut && k == kstar)) {
+            // the clamp decides: the token of rank k (at bmax, the bin the
+            // listing already found)
+            unsigned long long kb_c = hb_c, kb_m = 0;
+            const int b_k = k == r_hi ? b_hi
+                                      : find_crossing(sm.cnt, mass, SBINS, false, (unsigned long long)k, &kb_c, &kb_m,
+                                                      sm);
+            HKV_TRACE_AT(tb < 0 ? -1 : tb + 9);
+            const int cb = load_sorted_bin(b_k, ncand, bins, sm);
+            HKV_TRACE_AT(tb < 0 ? -1 : tb + 10);
+            if (cb < 0)
+                return false;
+            pos = sort_and_locate(cb, false, (unsigned long long)k - kb_c, 0, m, bl2, sm, sm.binbuf);
+            HKV_TRACE_AT(tb < 0 ? -1 : tb + 14);
+            before_c = kb_c;
+        }
+        cut_key = (uint32_t)(sm.binbuf[pos] >> 32);
+        if (threadIdx.x == 0) {
+            int first = pos;
+            while (first > 0 && (uint32_t)(sm.binbuf[first - 1] >> 32) == cut_key)
+                --first;
+            sm.bc[4] = first;
+        }
+        __syncthreads();
+        const int tie0 = sm.bc[4];
+        n_above = (int)before_c + tie0;
+        HKV_TRACE_AT(tb < 0 ? -1 : tb + 3);
+        // bitmap of the selection: listed tokens above the cut, and the first
+        // n_tie ties (consecutive in binbuf, by index)
+        const int nwords = (n + 31) >> 5;
+        for (int i = threadIdx.x; i < nwords; i += NT)
+            sm.bits[i] = 0u;
+        __syncthreads();
+        for (int i = threadIdx.x; i < ncand; i += NT) {
+            const unsigned long long e = sm.cand[i];
+            if ((uint32_t)(e >> 32) < cut_key) {
+                const uint32_t j = (uint32_t)e;
+                atomicOr(&sm.bits[j >> 5], 1u << (j & 31));
+                pf((int)j);
+            }
+        }
+        const int n_tie = k - n_above;
+        for (int i = threadIdx.x; i < n_tie; i += NT) {
+            const uint32_t j = (uint32_t)sm.binbuf[tie0 + i];
+            atomicOr(&sm.bits[j >> 5], 1u << (j & 31));
+            pf((int)j);
+        }
+        __syncthreads();
+    }
+    r.k = k;
+    r.kstar = kstar;
+    r.key = cut_key;
+    r.cut.z_cut = key_score(cut_key);
+    r.cut.n_above = n_above;
+    r.cut.n_tie = k - n_above;
+    r.cut.kstar = kstar;
+    if (k == 0)
+        r.cut = hkv_cut{0.0f, 0, 0, kstar};
+    return true;
+}
+
+// The set bits of bits[w_begin, w_end) in index order, written as token
+// indices (32 w + bit) to row[at0 ...], positions below k only: thread t takes
+// a contiguous run of words, a block scan gives each run its first position.
+__device__ void expand_bits(const uint32_t *bits, int w_begin, int w_end, int at0, int k, int32_t *row, USmem &sm)
+{
+    const int nw = max(0, w_end - w_begin);
+    const int wpt = (nw + NT - 1) / NT;
+    const int w0 = w_begin + threadIdx.x * wpt, w1 = min(w_end, w0 + wpt);
+    unsigned long long cntw = 0;
+    for (int i = w0; i < w1; ++i)
+        cntw += __popc(bits[i]);
+    unsigned long long tot;
+    int at = at0 + (int)block_exclusive_scan<NT>(cntw, sm.red, &tot);
+    for (int i = w0; i < w1; ++i) {
+        uint32_t b = bits[i];
+        while (b) {
+            const int bit = __ffs(b) - 1;
+            if (at < k)
+                row[at] = i * 32 + bit;
+            ++at;
+            b &= b - 1u;
+        }
+    }
+}
+
+// Selection and PAD_MAX compaction of one unit in one go, its n <= ZSTAGE
+// scores staged in shared memory (zs; or staged from zg during the first sweep).
+// Returns false (nothing written) when a list or bin outgrows shared memory.
 __device__ bool select_compact_fast(const float *zs, int n, float m, float zlo, float beta, float p, int bmin,
                                     int bmax, USmem &sm, Selection &r, int32_t *row, int pad, int tb,
                                     const float *zg = nullptr, const RowPrefetch &pf = RowPrefetch{})
@@ -2159,31 +2315,26 @@ __device__ bool select_compact_fast(const float *zs, int n, float m, float zlo, 
     const float bl2 = beta * LOG2E;
     const BinFn bins = make_bins(m, zlo);
     r = Selection{};
-    for (int i = threadIdx.x; i < SBINS; i += NT) {
+    for (int i = threadIdx.x; i < SBINS; i += NT)
         sm.cnt[i] = 0;
-        sm.mass[i] = 0;
-    }
     __syncthreads();
     const auto mass = [&](int b) { return sm.mass[b]; };
-    // sweep 1: bin counts and the normaliser (staging the scores when they
-    // still are in global memory at zg)
-    double zsum = 0.0;
+    // sweep 1: bin counts and the normaliser (an exact sum of the fixed-point
+    // weights the prefix masses add up, so it does not depend on the order),
+    // staging the scores when they still are in global memory at zg
+    unsigned long long zsum = 0;
     const auto count = [&](float z, int, bool valid) {
         if (!valid)
             return;
-        zsum += (double)wcal(z, m, bl2);
+        zsum += wfix(z, m, bl2);
         sred_add(&sm.cnt[bins(z)], 1u);
     };
     if (zg != nullptr)
         sweep_stage(zg, sm.zs, n, count);
     else
         sweep_scores<true>(zs, n, count);
-    r.Z = block_sum_f64<NT>(zsum, sm.redd);
+    r.Zq = block_sum_u64<NT>(zsum, sm.red);
     HKV_TRACE_AT(tb < 0 ? -1 : tb + 1);
-    int k = 0, kstar = 0;
-    uint32_t cut_key = 0u;
-    int n_above = 0;
-    int tie0 = 0;  // first tie in sm.binbuf
     if (n > 0) {
         const int r_hi = min(n, max(bmax, 1));
         unsigned long long hb_c, hb_m;
@@ -2196,125 +2347,25 @@ __device__ bool select_compact_fast(const float *zs, int n, float m, float zlo, 
         if (list_candidates_warp(zs, n, bins, b_hi, sm) < 0)
             list_candidates(zs, n, bins, b_hi, sm);
         HKV_TRACE_AT(tb < 0 ? -1 : tb + 2);
-        // Top-p budget from the listed tokens' bin masses
-        kstar = -1;
-        bool mass_cut = false;
-        int pos = -1;
-        unsigned long long before_c = 0;
-        if (p >= 1.0f) {
-            kstar = n;
-        } else if (p <= 0.0f) {
-            kstar = 0;
-        } else {
-            // the mass of all listed tokens first (an exact integer sum): the
-            // per-bin masses are needed only when it reaches the target
-            unsigned long long part = 0;
-            for (int i = threadIdx.x; i < ncand; i += NT)
-                part += wfix(key_score((uint32_t)(sm.cand[i] >> 32)), m, bl2);
-            const unsigned long long through = block_sum_u64<NT>(part, sm.red);
-            const double t = ceil((double)p * r.Z * 1099511627776.0);
-            const unsigned long long T = t < 1.0 ? 1ull : (unsigned long long)t;
-            if (through >= T) {
-                for (int i = threadIdx.x; i < ncand; i += NT) {
-                    const float z = key_score((uint32_t)(sm.cand[i] >> 32));
-                    sred_add(&sm.mass[bins(z)], wfix(z, m, bl2));
-                }
+        if (!cut_bitmap(n, ncand, b_hi, hb_c, r_hi, m, bl2, bins, p, bmin, bmax, sm, r, tb, pf))
+            return false;
+        if (r.k > 0) {
+            // the row is built in shared memory (the candidate list is no longer
+            // needed) and then written out with coalesced stores
+            int32_t *buf = reinterpret_cast<int32_t *>(sm.cand);
+            const bool in_smem = r.k <= 2 * CAND_CAP;
+            expand_bits(sm.bits, 0, (n + 31) >> 5, 0, r.k, in_smem ? buf : row, sm);
+            if (in_smem) {
                 __syncthreads();
-                unsigned long long mb_c, mb_m;
-                const int b_m = find_crossing(sm.cnt, mass, SBINS, true, T, &mb_c, &mb_m, sm);
-                const int cb = load_sorted_bin(b_m, ncand, bins, sm);
-                if (cb < 0)
-                    return false;
-                pos = sort_and_locate(cb, true, T, mb_m, m, bl2, sm, sm.binbuf);
-                kstar = (int)mb_c + pos + 1;
-                before_c = mb_c;
-                mass_cut = true;
+                for (int i = threadIdx.x; i < r.k; i += NT)
+                    row[i] = buf[i];
             }
         }
-        k = kstar < 0 ? bmax : min(kstar, bmax);
-        k = min(max(k, bmin), n);
-        HKV_TRACE_AT(tb < 0 ? -1 : tb + 8);
-        if (k > 0) {
-            if (!(mass_cut && k == kstar)) {
-                // the clamp decides: the token of rank k (at bmax, the bin
-                // the listing already found)
-                unsigned long long kb_c = hb_c, kb_m = 0;
-                const int b_k = k == r_hi ? b_hi
-                                          : find_crossing(sm.cnt, mass, SBINS, false, (unsigned long long)k, &kb_c,
-                                                          &kb_m, sm);
-                HKV_TRACE_AT(tb < 0 ? -1 : tb + 9);
-                const int cb = load_sorted_bin(b_k, ncand, bins, sm);
-                HKV_TRACE_AT(tb < 0 ? -1 : tb + 10);
-                HKV_TRACE_VAL(tb < 0 ? -1 : tb + 15, cb);
-                if (cb < 0)
-                    return false;
-                pos = sort_and_locate(cb, false, (unsigned long long)k - kb_c, 0, m, bl2, sm, sm.binbuf);
-                HKV_TRACE_AT(tb < 0 ? -1 : tb + 14);
-                before_c = kb_c;
-            }
-            cut_key = (uint32_t)(sm.binbuf[pos] >> 32);
-            if (threadIdx.x == 0) {
-                int first = pos;
-                while (first > 0 && (uint32_t)(sm.binbuf[first - 1] >> 32) == cut_key)
-                    --first;
-                sm.bc[4] = first;
-            }
-            __syncthreads();
-            tie0 = sm.bc[4];
-            n_above = (int)before_c + tie0;
-            HKV_TRACE_AT(tb < 0 ? -1 : tb + 3);
-            // bitmap of the selection: listed tokens above the cut, and the
-            // first n_tie ties (consecutive in binbuf, by index)
-            const int nwords = (n + 31) >> 5;
-            for (int i = threadIdx.x; i < nwords; i += NT)
-                sm.bits[i] = 0u;
-            __syncthreads();
-            for (int i = threadIdx.x; i < ncand; i += NT) {
-                const unsigned long long e = sm.cand[i];
-                if ((uint32_t)(e >> 32) < cut_key) {
-                    const uint32_t j = (uint32_t)e;
-                    atomicOr(&sm.bits[j >> 5], 1u << (j & 31));
-                    pf((int)j);
-                }
-            }
-            const int n_tie = k - n_above;
-            for (int i = threadIdx.x; i < n_tie; i += NT) {
-                const uint32_t j = (uint32_t)sm.binbuf[tie0 + i];
-                atomicOr(&sm.bits[j >> 5], 1u << (j & 31));
-                pf((int)j);
-            }
-            __syncthreads();
-            // expansion in index order: thread t takes a contiguous run of words
-            const int wpt = (nwords + NT - 1) / NT;
-            const int w0 = threadIdx.x * wpt, w1 = min(nwords, w0 + wpt);
-            unsigned long long cntw = 0;
-            for (int i = w0; i < w1; ++i)
-                cntw += __popc(sm.bits[i]);
-            unsigned long long tot;
-            int at = (int)block_exclusive_scan<NT>(cntw, sm.red, &tot);
-            for (int i = w0; i < w1; ++i) {
-                uint32_t b = sm.bits[i];
-                while (b) {
-                    const int bit = __ffs(b) - 1;
-                    if (at < k)
-                        row[at] = i * 32 + bit;
-                    ++at;
-                    b &= b - 1u;
-                }
-            }
-        }
+    } else {
+        r.cut = hkv_cut{0.0f, 0, 0, 0};
     }
-    for (int i = k + threadIdx.x; i < pad; i += NT)
+    for (int i = r.k + threadIdx.x; i < pad; i += NT)
         row[i] = -1;
-    r.k = k;
-    r.kstar = kstar;
-    r.key = cut_key;
-    r.cut.z_cut = key_score(cut_key);
-    r.cut.n_above = n_above;
-    r.cut.n_tie = k - n_above;
-    r.cut.kstar = kstar;
-    if (k == 0)
-        r.cut = hkv_cut{0.0f, 0, 0, kstar};
     __syncthreads();
     return true;
 }

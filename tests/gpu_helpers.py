@@ -25,10 +25,12 @@ ATOL, RTOL = 2e-3, 1e-2
 # exponent, rounded three times in fp32, is off by at most 3 2^-24 |x|
 # (x = (z - m) beta log2 e), which moves w by ln 2 times that. Summed over a
 # unit, the weights' error is at most Z (2^-22 + 3 2^-24 ln 2 E_P|x|), E_P the
-# calibrated mean. The GPU compares the exact integer sum of 40-bit fixed-point
-# weights with ceil(p Z 2^40), Z a double sum of the same weights, so its test
-# C_k >= p can differ from the exact one only within
-#     2 (2^-22 + 3 2^-24 ln 2 E_P|x|) + (k + 1) 2^-40
+# calibrated mean. The GPU compares the exact integer sum of the first k
+# weights, each floored to 40-bit fixed point, with ceil(p Z 2^40), where Z 2^40
+# is the exact integer sum of all n such weights (so Z is low by at most
+# n 2^-40, and Z >= 1 as the maximum's weight is exactly 1). Its test C_k >= p
+# can therefore differ from the exact one only within
+#     2 (2^-22 + 3 2^-24 ln 2 E_P|x|) + (k + 1 + n) 2^-40
 # of p; window() takes 1.5 times that (second-order terms, the oracle's own
 # fp64 sums) and never less than AMBIG_FLOOR.
 AMBIG_FLOOR = 1e-6
@@ -46,7 +48,7 @@ def window(z_row: np.ndarray, n: int, beta: float, k: int) -> float:
     x = beta * math.log2(math.e) * (z.max() - z)
     P = sps.softmax(beta * z)
     ex = float(np.sum(P * x))
-    w = 1.5 * (2 * (2.0 ** -22 + 3 * 2.0 ** -24 * math.log(2) * ex) + (k + 1) * 2.0 ** -40)
+    w = 1.5 * (2 * (2.0 ** -22 + 3 * 2.0 ** -24 * math.log(2) * ex) + (k + 1 + n) * 2.0 ** -40)
     w = max(w, AMBIG_FLOOR)
     AMBIG_TALLY["max_window"] = max(AMBIG_TALLY["max_window"], w)
     return w

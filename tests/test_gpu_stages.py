@@ -74,16 +74,16 @@ def test_calibrate(case):
     assert np.array_equal(m.cpu().numpy(), mr)
     assert np.allclose(lz.cpu().numpy(), lzr, rtol=0, atol=2e-6)
     # P = w / Z in fp32. The weight is within 2^-22 + 3 2^-24 ln2 x_j relative
-    # (x_j = beta log2e (m - z_j); see gpu_helpers.window), Z (a double sum of
-    # such weights) within 2^-22 + 3 2^-24 ln2 E_P[x], and the rounding of 1/Z
-    # to fp32 and of the product add 2^-23; 1.5 times that, for results in the
-    # normal fp32 range.
+    # (x_j = beta log2e (m - z_j); see gpu_helpers.window), Z (the exact sum of
+    # such weights floored to 40-bit fixed point) within 2^-22 + 3 2^-24 ln2
+    # E_P[x] + n 2^-40, and the rounding of 1/Z to fp32 and of the product add
+    # 2^-23; 1.5 times that, for results in the normal fp32 range.
     c = 3 * 2.0 ** -24 * np.log(2)
     for u in range(wl.units):
         n = ln[u]
         x = beta[u] * np.log2(np.e) * (np.float64(mr[u]) - zr[u, :n].astype(np.float64))
         ex = float(np.sum(Pr[u, :n].astype(np.float64) * x))
-        rel = 2 * 2.0 ** -22 + c * (x + ex) + 2.0 ** -23
+        rel = 2 * 2.0 ** -22 + c * (x + ex) + 2.0 ** -23 + n * 2.0 ** -40
         tol = 1.5 * rel * Pr[u, :n] + 2e-38
         err = np.abs(Pg[u, :n] - Pr[u, :n])
         assert np.all(err <= tol), (name, u, float(np.max(err / np.maximum(Pr[u, :n], 1e-300))))
