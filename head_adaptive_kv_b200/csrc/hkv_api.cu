@@ -366,6 +366,84 @@ __global__ void __launch_bounds__(NT, 1) k_unit(const __grid_constant__ Params P
     tl_end(P.tl, TL_UNIT);
 }
 
+// hkv_step's S2-S4 for units too long to stage in one CTA, each split over a
+// cluster of UNIT_CLUSTER CTAs (used when the clusters all fit the SMs at
+// once): the same selection and PAD_MAX rows as k_unit. Units that reuse a
+// rewrite, units short enough for one CTA, and units whose lists or cut bin
+// outgrow shared memory are done by rank 0 alone, as k_unit does them.
+constexpr int UNIT_CLUSTER = 4;
+
+template <int ES>
+__global__ void __cluster_dims__(UNIT_CLUSTER, 1, 1) __launch_bounds__(NT, 1)
+    k_unit_cluster(const __grid_constant__ Params P)
+{
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    USmem &sm = *reinterpret_cast<USmem *>(smem_raw);
+    const Ctl c = make_ctl(P);
+    const int u = blockIdx.x / UNIT_CLUSTER;
+    const int rank = (int)cooperative_groups::this_cluster().block_rank();
+    allow_dependents();
+    wait_prior_grid();
+    const int tb = rank == 0 ? TR_SEL + 16 * u : -1;
+    HKV_TRACE_AT(tb);
+    tl_start(P.tl, TL_UNIT);
+    const int n = tier_len(P.sparse, u, c);
+    const float *zg = P.z + (int64_t)u * P.z_stride;
+    if (P.mti_left != nullptr && __ldcg(P.mti_left + u) > 0) {
+        if (rank == 0)
+            mti_reuse_outputs(P, c, u);  // the unit reuses its rewrite: nothing to select
+    } else if (n <= ZSTAGE || cluster_chunk<UNIT_CLUSTER>(n) > ZSTAGE) {
+        if (rank == 0) {
+            if (n <= ZSTAGE) {
+                unit_work<ES, true>(P, sm, c, u, n, sm.zs, zg);
+            } else {
+                const bool staged = stage_scores(zg, n, sm);
+                if (staged)
+                    unit_work<ES, true>(P, sm, c, u, n, sm.zs);
+                else
+                    unit_work<ES, false>(P, sm, c, u, n, zg);
+            }
+        }
+    } else {
+        // every rank reads the scorer's range words; rank 0 resets them for
+        // the next step once the cluster is done with the unit
+        if (threadIdx.x == 0) {
+            const uint32_t kmax = __ldcg(P.urange + 2 * u), kmin = __ldcg(P.urange + 2 * u + 1);
+            sm.redf[0] = kmax ? ord_val(kmax) : -INFINITY;
+            sm.redf[1] = kmin ? ord_val(~kmin) : INFINITY;
+        }
+        __syncthreads();
+        const float m = sm.redf[0], zlo = sm.redf[1];
+        __syncthreads();
+        HKV_TRACE_AT(tb < 0 ? -1 : tb + 4);
+        const float beta = unit_beta(P, u, c), pu = unit_p(P, u, c);
+        Selection s;
+        const int st = select_compact_cluster<UNIT_CLUSTER>(zg, n, m, zlo, beta, pu, P.bmin, P.bmax, sm, s,
+                                                            P.idx + (int64_t)u * P.bmax, P.bmax, tb,
+                                                            v_prefetch<ES>(P, u), rank);
+        if (rank == 0) {
+            if (st != 0) {
+                // the general path, alone (it reads and resets the range words)
+                unit_work<ES, false>(P, sm, c, u, n, zg);
+            } else {
+                if (threadIdx.x == 0) {
+                    P.sel_len[u] = s.k;
+                    if (P.cut)
+                        P.cut[u] = s.cut;
+                    if (P.m_out)
+                        P.m_out[u] = m;
+                    if (P.logZ_out)
+                        P.logZ_out[u] = (float)log(s.Z());
+                    P.urange[2 * u] = 0;
+                    P.urange[2 * u + 1] = 0;
+                }
+                HKV_TRACE_AT(tb + 5);
+            }
+        }
+    }
+    tl_end(P.tl, TL_UNIT);
+}
+
 // S2 standalone ([TS 2.B]) for unit u: m, logZ and optionally the calibrated
 // probabilities. Z is summed exactly as the selection sums it (the 40-bit
 // fixed-point weights, an exact integer sum), so m and logZ match hkv_step's
@@ -622,6 +700,7 @@ static Params base_params(const hkv_problem *p, const WsLayout &L, char *ws, con
     const int64_t span = (int64_t)(dense ? dense->cap : 0) + std::min(p->bmax, sparse ? sparse->cap : 0) +
                          (cond ? cond->cap : 0);
     P.attn_prefix = P.units <= PREFIX_CAP && (int64_t)P.units * span < (1ll << 31);
+    P.unit_ctas = P.units;
     return P;
 }
 
@@ -767,7 +846,7 @@ struct RunAttn {
         // the selection kernel (one CTA per unit) runs
         const int sms = sm_count();
         Params Q = P;
-        Q.attn_a_ctas = (pdl && P.units < sms) ? sms - P.units : (1 << 30);
+        Q.attn_a_ctas = (pdl && P.unit_ctas < sms) ? sms - P.unit_ctas : (1 << 30);
         hkv_status st = launch_stream(k_attn_stream<ES, D, G>, AT_NW * 32, sizeof(AttnSmem<ES, D, G>), max_ctas, s,
                                       Q, pdl);
         if (st != HKV_OK)
@@ -784,8 +863,13 @@ struct RunFit {
     }
 };
 
-static hkv_status launch_unit(const hkv_problem *prob, const Params &P, cudaStream_t s, bool pdl)
+static hkv_status launch_unit(const hkv_problem *prob, const Params &P, cudaStream_t s, bool pdl,
+                              bool split = false)
 {
+    if (split)
+        return prob->dtype == HKV_BF16
+                   ? launch(k_unit_cluster<2>, UNIT_CLUSTER * P.units, NT, sizeof(USmem), s, P, pdl)
+                   : launch(k_unit_cluster<4>, UNIT_CLUSTER * P.units, NT, sizeof(USmem), s, P, pdl);
     if (prob->dtype == HKV_BF16)
         return launch(k_unit<2>, P.units, NT, sizeof(USmem), s, P, pdl);
     return launch(k_unit<4>, P.units, NT, sizeof(USmem), s, P, pdl);
@@ -1009,8 +1093,13 @@ hkv_status step_impl(const hkv_problem *prob, const void *q, const hkv_tier *den
     U.do_select = 1;
     U.do_compact = 1;
     U.prefetch_v = 1;
-    if ((s = launch_unit(prob, U, st, true)) != HKV_OK)
+    // units longer than one CTA can stage are split over a cluster of CTAs
+    // when the clusters all fit the SMs at once (one wave: the step waits for
+    // the selection's latency, and one CTA would sweep such a unit from L2)
+    const bool split = scored && sparse->cap > ZSTAGE && UNIT_CLUSTER * P.units <= sm_count();
+    if ((s = launch_unit(prob, U, st, true, split)) != HKV_OK)
         return s;
+    P.unit_ctas = split ? UNIT_CLUSTER * P.units : P.units;
     // 3. attention over the three tiers and the merge of each unit
     if ((s = dispatch<RunAttn>(prob, P, st, true)) != HKV_OK)
         return s;

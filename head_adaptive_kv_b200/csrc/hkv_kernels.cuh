@@ -81,6 +81,7 @@ struct Params {
     int32_t part_slots;   // record slots: 2 x (streaming warps of the attention grid + units)
     int32_t attn_prefix;  // attention partition over actual tokens (units <= PREFIX_CAP, lines < 2^31), else over capacity
     int32_t attn_a_ctas;  // attention CTAs that share line A (the first ones, which start while the selection runs)
+    int32_t unit_ctas;    // CTAs of the selection kernel before the attention (units, or more when split)
     int32_t have_range;   // per-unit kernel: urange holds the units' score ranges
     int32_t do_select, do_compact;  // per-unit kernel: which steps to run
     int32_t prefetch_v;   // per-unit kernel: bring the selected tokens' V rows into L2 (the attention follows)
@@ -1495,6 +1496,14 @@ struct __align__(16) USmem {  // shared memory of the per-unit kernels
     float redf[NT / 32];
     int32_t bc[8];
     unsigned long long bcl[4];
+    // a unit split over a cluster (select_compact_cluster): this CTA's part of
+    // the bin counts, its normaliser and listed mass, tokens listed, a listing
+    // overflow, tokens selected, and (rank 0) the cut every rank applies
+    uint32_t cnt_part[SBINS];
+    unsigned long long z_part, t_part;
+    int32_t c_part, over_part, sel_part;
+    int32_t pub_k, pub_kstar, pub_n_above, pub_fallback, pub_tie_last;
+    uint32_t pub_key;
 };
 
 // Bin of a score: (m - z) s rounded to the nearest integer, clamped to
@@ -2281,9 +2290,10 @@ __device__ bool cut_bitmap(int n, int ncand, int b_hi, unsigned long long hb_c, 
 }
 
 // The set bits of bits[w_begin, w_end) in index order, written as token
-// indices (32 w + bit) to row[at0 ...], positions below k only: thread t takes
+// indices (index_base + 32 w + bit) to row[at0 ...], positions below k only: thread t takes
 // a contiguous run of words, a block scan gives each run its first position.
-__device__ void expand_bits(const uint32_t *bits, int w_begin, int w_end, int at0, int k, int32_t *row, USmem &sm)
+__device__ void expand_bits(const uint32_t *bits, int w_begin, int w_end, int at0, int k, int32_t *row, USmem &sm,
+                            int index_base = 0)
 {
     const int nw = max(0, w_end - w_begin);
     const int wpt = (nw + NT - 1) / NT;
@@ -2298,7 +2308,7 @@ __device__ void expand_bits(const uint32_t *bits, int w_begin, int w_end, int at
         while (b) {
             const int bit = __ffs(b) - 1;
             if (at < k)
-                row[at] = i * 32 + bit;
+                row[at] = index_base + i * 32 + bit;
             ++at;
             b &= b - 1u;
         }
@@ -2368,6 +2378,275 @@ __device__ bool select_compact_fast(const float *zs, int n, float m, float zlo, 
         row[i] = -1;
     __syncthreads();
     return true;
+}
+
+// Rank 0 of a cluster: every listed token of bin b, from the lists of all C
+// ranks, into sm.binbuf (unordered). Returns their number, or -1 when the bin
+// holds more than BIN_CAP tokens.
+template <int C>
+__device__ int gather_bin_cluster(int b, const BinFn &bins, USmem &sm, USmem *const (&peers)[C])
+{
+    const int cb = (int)sm.cnt[b];
+    if (cb > BIN_CAP)
+        return -1;
+    if (threadIdx.x == 0)
+        sm.bc[3] = 0;
+    __syncthreads();
+    const int lane = threadIdx.x & 31;
+#pragma unroll 1
+    for (int q = 0; q < C; ++q) {
+        const USmem &src = *peers[q];
+        const int cq = src.c_part;
+        for (int base = 0; base < cq; base += NT) {
+            const int i = base + threadIdx.x;
+            const unsigned long long e = i < cq ? src.cand[i] : 0ull;
+            const bool hit = i < cq && bins(key_score((uint32_t)(e >> 32))) == b;
+            const unsigned mask = __ballot_sync(0xffffffffu, hit);
+            if (mask != 0) {
+                const int leader = __ffs(mask) - 1;
+                int at = 0;
+                if (lane == leader)
+                    at = satom_add(&sm.bc[3], __popc(mask));
+                at = __shfl_sync(0xffffffffu, at, leader);
+                if (hit && at + __popc(mask & ((1u << lane) - 1u)) < BIN_CAP)
+                    sm.binbuf[at + __popc(mask & ((1u << lane) - 1u))] = e;
+            }
+        }
+    }
+    __syncthreads();
+    return min(sm.bc[3], cb);
+}
+
+// A unit too long to stage in one CTA, split over a cluster of C CTAs (all of
+// them run this function): rank r stages tokens [r c, r c + c) of the unit's
+// scores (c a multiple of 128, c <= ZSTAGE), counts and lists its part, and
+// the parts meet in distributed shared memory. The cut is found by rank 0 from
+// the summed bin counts and masses and the one bin that holds it, gathered from
+// every rank's list; each rank then marks and expands its own part of the
+// selection, after the selected tokens of the ranks before it. Every branch
+// around a cluster barrier depends only on values all ranks hold alike (the
+// summed counts, the published cut), so all ranks pass the same barriers, and
+// the last one keeps every CTA's shared memory alive while others read it.
+// Returns 0 when done (r valid on rank 0), 1 when rank 0 must redo the unit on
+// the general path (a part's list or the cut's bin too large; nothing written).
+template <int C>
+__host__ __device__ constexpr int cluster_chunk(int n)
+{
+    return ((n + C - 1) / C + 127) / 128 * 128;
+}
+
+template <int C>
+__device__ int select_compact_cluster(const float *zg, int n, float m, float zlo, float beta, float p, int bmin,
+                                      int bmax, USmem &sm, Selection &r, int32_t *row, int pad, int tb,
+                                      const RowPrefetch &pf, int rank)
+{
+    namespace cg = cooperative_groups;
+    auto cl = cg::this_cluster();
+    USmem *peers[C];
+#pragma unroll
+    for (int q = 0; q < C; ++q)
+        peers[q] = cl.map_shared_rank(&sm, q);
+    const float bl2 = beta * LOG2E;
+    const BinFn bins = make_bins(m, zlo);
+    const int chunk = cluster_chunk<C>(n);
+    const int j0 = min(n, rank * chunk), nl = min(n, j0 + chunk) - j0;
+    r = Selection{};
+    for (int i = threadIdx.x; i < SBINS; i += NT)
+        sm.cnt_part[i] = 0;
+    __syncthreads();
+    // this part's bin counts and normaliser, staging its scores
+    unsigned long long zsum = 0;
+    sweep_stage(zg + j0, sm.zs, nl, [&](float z, int, bool valid) {
+        if (!valid)
+            return;
+        zsum += wfix(z, m, bl2);
+        sred_add(&sm.cnt_part[bins(z)], 1u);
+    });
+    const unsigned long long zp = block_sum_u64<NT>(zsum, sm.red);
+    if (threadIdx.x == 0)
+        sm.z_part = zp;
+    cl.sync();  // 1: parts counted
+    for (int i = threadIdx.x; i < SBINS; i += NT) {
+        uint32_t t = 0;
+#pragma unroll
+        for (int q = 0; q < C; ++q)
+            t += peers[q]->cnt_part[i];
+        sm.cnt[i] = t;
+    }
+#pragma unroll
+    for (int q = 0; q < C; ++q)
+        r.Zq += peers[q]->z_part;
+    __syncthreads();
+    HKV_TRACE_AT(tb < 0 ? -1 : tb + 1);
+    const auto mass = [&](int b) { return sm.mass[b]; };
+    const int r_hi = min(n, max(bmax, 1));
+    unsigned long long hb_c, hb_m;
+    const int b_hi = find_crossing(sm.cnt, mass, SBINS, false, (unsigned long long)r_hi, &hb_c, &hb_m, sm);
+    // this part's tokens of bins 0 .. b_hi, and their mass
+    int c = -1;
+    {
+        unsigned long long mine = 0;
+        sweep_scores<true>(sm.zs, nl, [&](float z, int, bool valid) { mine += (valid && bins(z) <= b_hi) ? 1u : 0u; });
+        unsigned long long tot;
+        const int at0 = (int)block_exclusive_scan<NT>(mine, sm.red, &tot);
+        if (tot <= (unsigned long long)CAND_CAP) {
+            int at = at0;
+            sweep_scores<true>(sm.zs, nl, [&](float z, int j, bool valid) {
+                if (valid && bins(z) <= b_hi)
+                    sm.cand[at++] = ((unsigned long long)score_key(z) << 32) | (uint32_t)(j0 + j);
+            });
+            c = (int)tot;
+        }
+    }
+    __syncthreads();
+    unsigned long long tpart = 0;
+    for (int i = threadIdx.x; i < max(c, 0); i += NT)
+        tpart += wfix(key_score((uint32_t)(sm.cand[i] >> 32)), m, bl2);
+    tpart = block_sum_u64<NT>(tpart, sm.red);
+    if (threadIdx.x == 0) {
+        sm.c_part = max(c, 0);
+        sm.over_part = c < 0 ? 1 : 0;
+        sm.t_part = tpart;
+    }
+    cl.sync();  // 2: parts listed
+    bool fallback = false;
+    unsigned long long through = 0;
+#pragma unroll
+    for (int q = 0; q < C; ++q) {
+        fallback |= peers[q]->over_part != 0;
+        through += peers[q]->t_part;
+    }
+    HKV_TRACE_AT(tb < 0 ? -1 : tb + 2);
+    if (!fallback) {
+        const unsigned long long T = mass_target(p, r.Zq);
+        const bool mass_case = p > 0.0f && p < 1.0f && through >= T;  // alike in every rank
+        if (mass_case) {
+            // per-bin masses of this part's listed tokens (exact integer sums)
+            for (int i = threadIdx.x; i < SBINS; i += NT)
+                sm.mass[i] = 0;
+            __syncthreads();
+            for (int i = threadIdx.x; i < sm.c_part; i += NT) {
+                const float z = key_score((uint32_t)(sm.cand[i] >> 32));
+                sred_add(&sm.mass[bins(z)], wfix(z, m, bl2));
+            }
+            __syncthreads();
+            cl.sync();  // 3: part masses
+        }
+        if (rank == 0) {
+            int kstar = p >= 1.0f ? n : (p <= 0.0f ? 0 : -1), pos = -1;
+            bool mass_cut = false, bad = false;
+            unsigned long long before_c = 0;
+            if (mass_case) {
+                for (int i = threadIdx.x; i <= b_hi; i += NT) {
+                    unsigned long long t = sm.mass[i];
+#pragma unroll
+                    for (int q = 1; q < C; ++q)
+                        t += peers[q]->mass[i];
+                    sm.mass[i] = t;
+                }
+                __syncthreads();
+                unsigned long long mb_c, mb_m;
+                const int b_m = find_crossing(sm.cnt, mass, SBINS, true, T, &mb_c, &mb_m, sm);
+                const int cb = gather_bin_cluster<C>(b_m, bins, sm, peers);
+                if (cb < 0) {
+                    bad = true;
+                } else {
+                    pos = sort_and_locate(cb, true, T, mb_m, m, bl2, sm, sm.binbuf);
+                    kstar = (int)mb_c + pos + 1;
+                    before_c = mb_c;
+                    mass_cut = true;
+                }
+            }
+            int k = kstar < 0 ? bmax : min(kstar, bmax);
+            k = min(max(k, bmin), n);
+            uint32_t cut_key = 0u;
+            int n_above = 0, tie_last = -1;
+            if (!bad && k > 0) {
+                if (!(mass_cut && k == kstar)) {
+                    unsigned long long kb_c = hb_c, kb_m = 0;
+                    const int b_k = k == r_hi ? b_hi
+                                              : find_crossing(sm.cnt, mass, SBINS, false, (unsigned long long)k,
+                                                              &kb_c, &kb_m, sm);
+                    const int cb = gather_bin_cluster<C>(b_k, bins, sm, peers);
+                    if (cb < 0)
+                        bad = true;
+                    else
+                        pos = sort_and_locate(cb, false, (unsigned long long)k - kb_c, 0, m, bl2, sm, sm.binbuf);
+                    before_c = kb_c;
+                }
+                if (!bad) {
+                    cut_key = (uint32_t)(sm.binbuf[pos] >> 32);
+                    if (threadIdx.x == 0) {
+                        int first = pos;
+                        while (first > 0 && (uint32_t)(sm.binbuf[first - 1] >> 32) == cut_key)
+                            --first;
+                        sm.bc[4] = first;
+                    }
+                    __syncthreads();
+                    const int tie0 = sm.bc[4];
+                    n_above = (int)before_c + tie0;
+                    // the selected ties are the first k - n_above by index:
+                    // those up to the index of the last of them
+                    tie_last = k > n_above ? (int)(uint32_t)sm.binbuf[tie0 + (k - n_above) - 1] : -1;
+                }
+            }
+            r.k = k;
+            r.kstar = kstar;
+            r.key = cut_key;
+            r.cut.z_cut = key_score(cut_key);
+            r.cut.n_above = n_above;
+            r.cut.n_tie = k - n_above;
+            r.cut.kstar = kstar;
+            if (k == 0)
+                r.cut = hkv_cut{0.0f, 0, 0, kstar};
+            if (threadIdx.x == 0) {
+                sm.pub_fallback = bad ? 1 : 0;
+                sm.pub_k = k;
+                sm.pub_key = cut_key;
+                sm.pub_tie_last = tie_last;
+            }
+            __syncthreads();
+        }
+        cl.sync();  // 4: the cut published
+        const USmem &r0 = *peers[0];
+        fallback = r0.pub_fallback != 0;
+        const int k = r0.pub_k;
+        const uint32_t key = r0.pub_key;
+        const int tie_last = r0.pub_tie_last;
+        if (!fallback && k > 0) {
+            // this part's selected tokens as a bitmap over its own positions
+            const int nwl = (nl + 31) >> 5;
+            for (int i = threadIdx.x; i < nwl; i += NT)
+                sm.bits[i] = 0u;
+            __syncthreads();
+            for (int i = threadIdx.x; i < sm.c_part; i += NT) {
+                const unsigned long long e = sm.cand[i];
+                const uint32_t kk = (uint32_t)(e >> 32);
+                const int j = (int)(uint32_t)e;
+                if (kk < key || (kk == key && j <= tie_last)) {
+                    atomicOr(&sm.bits[(j - j0) >> 5], 1u << ((j - j0) & 31));
+                    pf(j);
+                }
+            }
+            __syncthreads();
+            unsigned long long sc = 0;
+            for (int i = threadIdx.x; i < nwl; i += NT)
+                sc += __popc(sm.bits[i]);
+            sc = block_sum_u64<NT>(sc, sm.red);
+            if (threadIdx.x == 0)
+                sm.sel_part = (int)sc;
+            cl.sync();  // 5: parts' selected counts
+            int at0 = 0;
+            for (int q = 0; q < rank; ++q)
+                at0 += peers[q]->sel_part;
+            expand_bits(sm.bits, 0, nwl, at0, k, row, sm, j0);
+        }
+        if (rank == 0 && !fallback)
+            for (int i = k + threadIdx.x; i < pad; i += NT)
+                row[i] = -1;
+    }
+    cl.sync();  // 6: no CTA leaves while another may still read its shared memory
+    return fallback ? 1 : 0;
 }
 
 // =============================================================================
