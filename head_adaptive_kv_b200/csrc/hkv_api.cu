@@ -367,20 +367,17 @@ __global__ void __launch_bounds__(NT, 1) k_unit(const __grid_constant__ Params P
 }
 
 // hkv_step's S2-S4 for units too long to stage in one CTA, each split over a
-// cluster of UNIT_CLUSTER CTAs (used when the clusters all fit the SMs at
-// once): the same selection and PAD_MAX rows as k_unit. Units that reuse a
-// rewrite, units short enough for one CTA, and units whose lists or cut bin
-// outgrow shared memory are done by rank 0 alone, as k_unit does them.
-constexpr int UNIT_CLUSTER = 4;
-
-template <int ES>
-__global__ void __cluster_dims__(UNIT_CLUSTER, 1, 1) __launch_bounds__(NT, 1)
-    k_unit_cluster(const __grid_constant__ Params P)
+// cluster of C CTAs: the same selection and PAD_MAX rows as k_unit. Units
+// that reuse a rewrite, units short enough for one CTA, and units whose lists
+// or cut bin outgrow shared memory are done by rank 0 alone, as k_unit does
+// them (the other ranks then leave at once).
+template <int ES, int C>
+__global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(NT, 1) k_unit_cluster(const __grid_constant__ Params P)
 {
     extern __shared__ __align__(128) unsigned char smem_raw[];
     USmem &sm = *reinterpret_cast<USmem *>(smem_raw);
     const Ctl c = make_ctl(P);
-    const int u = blockIdx.x / UNIT_CLUSTER;
+    const int u = blockIdx.x / C;
     const int rank = (int)cooperative_groups::this_cluster().block_rank();
     allow_dependents();
     wait_prior_grid();
@@ -392,7 +389,7 @@ __global__ void __cluster_dims__(UNIT_CLUSTER, 1, 1) __launch_bounds__(NT, 1)
     if (P.mti_left != nullptr && __ldcg(P.mti_left + u) > 0) {
         if (rank == 0)
             mti_reuse_outputs(P, c, u);  // the unit reuses its rewrite: nothing to select
-    } else if (n <= ZSTAGE || cluster_chunk<UNIT_CLUSTER>(n) > ZSTAGE) {
+    } else if (n <= ZSTAGE || cluster_chunk<C>(n) > ZSTAGE) {
         if (rank == 0) {
             if (n <= ZSTAGE) {
                 unit_work<ES, true>(P, sm, c, u, n, sm.zs, zg);
@@ -418,9 +415,9 @@ __global__ void __cluster_dims__(UNIT_CLUSTER, 1, 1) __launch_bounds__(NT, 1)
         HKV_TRACE_AT(tb < 0 ? -1 : tb + 4);
         const float beta = unit_beta(P, u, c), pu = unit_p(P, u, c);
         Selection s;
-        const int st = select_compact_cluster<UNIT_CLUSTER>(zg, n, m, zlo, beta, pu, P.bmin, P.bmax, sm, s,
-                                                            P.idx + (int64_t)u * P.bmax, P.bmax, tb,
-                                                            v_prefetch<ES>(P, u), rank);
+        const int st = select_compact_cluster<C>(zg, n, m, zlo, beta, pu, P.bmin, P.bmax, sm, s,
+                                                 P.idx + (int64_t)u * P.bmax, P.bmax, tb, v_prefetch<ES>(P, u),
+                                                 rank);
         if (rank == 0) {
             if (st != 0) {
                 // the general path, alone (it reads and resets the range words)
@@ -863,13 +860,16 @@ struct RunFit {
     }
 };
 
-static hkv_status launch_unit(const hkv_problem *prob, const Params &P, cudaStream_t s, bool pdl,
-                              bool split = false)
+// split: CTAs per unit (1, 2 or 4)
+static hkv_status launch_unit(const hkv_problem *prob, const Params &P, cudaStream_t s, bool pdl, int split = 1)
 {
-    if (split)
-        return prob->dtype == HKV_BF16
-                   ? launch(k_unit_cluster<2>, UNIT_CLUSTER * P.units, NT, sizeof(USmem), s, P, pdl)
-                   : launch(k_unit_cluster<4>, UNIT_CLUSTER * P.units, NT, sizeof(USmem), s, P, pdl);
+    const bool bf = prob->dtype == HKV_BF16;
+    if (split == 4)
+        return bf ? launch(k_unit_cluster<2, 4>, 4 * P.units, NT, sizeof(USmem), s, P, pdl)
+                  : launch(k_unit_cluster<4, 4>, 4 * P.units, NT, sizeof(USmem), s, P, pdl);
+    if (split == 2)
+        return bf ? launch(k_unit_cluster<2, 2>, 2 * P.units, NT, sizeof(USmem), s, P, pdl)
+                  : launch(k_unit_cluster<4, 2>, 2 * P.units, NT, sizeof(USmem), s, P, pdl);
     if (prob->dtype == HKV_BF16)
         return launch(k_unit<2>, P.units, NT, sizeof(USmem), s, P, pdl);
     return launch(k_unit<4>, P.units, NT, sizeof(USmem), s, P, pdl);
@@ -1094,12 +1094,18 @@ hkv_status step_impl(const hkv_problem *prob, const void *q, const hkv_tier *den
     U.do_compact = 1;
     U.prefetch_v = 1;
     // units longer than one CTA can stage are split over a cluster of CTAs
-    // when the clusters all fit the SMs at once (one wave: the step waits for
-    // the selection's latency, and one CTA would sweep such a unit from L2)
-    const bool split = scored && sparse->cap > ZSTAGE && UNIT_CLUSTER * P.units <= sm_count();
+    // (one CTA would sweep such a unit from L2 several times): four when all
+    // the clusters fit the SMs at once, else two when two CTAs can stage it
+    int split = 1;
+    if (scored && sparse->cap > ZSTAGE) {
+        if (4 * P.units <= sm_count() && cluster_chunk<4>(sparse->cap) <= ZSTAGE)
+            split = 4;
+        else if (cluster_chunk<2>(sparse->cap) <= ZSTAGE)
+            split = 2;
+    }
     if ((s = launch_unit(prob, U, st, true, split)) != HKV_OK)
         return s;
-    P.unit_ctas = split ? UNIT_CLUSTER * P.units : P.units;
+    P.unit_ctas = split * P.units;
     // 3. attention over the three tiers and the merge of each unit
     if ((s = dispatch<RunAttn>(prob, P, st, true)) != HKV_OK)
         return s;

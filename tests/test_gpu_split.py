@@ -1,5 +1,6 @@
 """Units too long for one CTA to stage (more than 24576 sparse tokens), split
-over a cluster of CTAs inside hkv_step when the clusters fit the SMs at once.
+over a cluster of CTAs inside hkv_step: four per unit when the clusters all fit
+the SMs at once, else two.
 
 Each CTA of the cluster counts and lists its part of the unit; the parts meet
 in distributed shared memory, one CTA finds the cut, and every CTA writes its
@@ -27,6 +28,8 @@ SPLIT_CASES = {
     # fp32 keys, D 64, four query heads per KV head
     "fp32_long_d64": WORKLOADS[2].with_(B=1, Hq=8, Hkv=2, D=64, dtype=torch.float32, n_cap=30000, bmin=1,
                                         bmax=3000),
+    # 40 units: too many for clusters of four on the SMs at once, so pairs
+    "bf16_ragged_pairs": WORKLOADS[3].with_(B=5, n_cap=30000, ctx_range=(320, 30320), bmin=8, bmax=4000),
 }
 
 
