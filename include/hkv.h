@@ -161,8 +161,9 @@ hkv_status hkv_score(const hkv_problem *prob, const void *q, const hkv_tier *spa
  * Z = sum_j exp(beta (z_j - m)), logZ = ln Z, and optionally
  * P[u*z_stride + j] = exp(beta (z_j - m)) / Z. sparse supplies the lengths
  * (its K/V are not read). m, logZ: device [B*Hkv]; P may be NULL. An empty unit
- * gives m = -inf, logZ = -inf. Z is summed in double precision in a fixed
- * order, exactly as hkv_topp_select and hkv_step sum it. */
+ * gives m = -inf, logZ = -inf. Z is the exact integer sum of the weights
+ * floored to 40-bit fixed point (so it is low by at most n 2^-40, with Z >= 1),
+ * exactly as hkv_topp_select and hkv_step sum it. */
 hkv_status hkv_calibrate(const hkv_problem *prob, const float *z, int64_t z_stride,
                          const hkv_tier *sparse, float *P, float *m, float *logZ,
                          void *ws, size_t ws_bytes, hkv_stream_t stream);
@@ -170,9 +171,9 @@ hkv_status hkv_calibrate(const hkv_problem *prob, const float *z, int64_t z_stri
 /* S3 Top-p budget ([Abstract], [TS 2.A], [TS 2.B]): per unit the budget
  * sel_len[u] = min(n, max(bmin, min(k*, bmax))), k* the fewest tokens (score
  * descending, lower index first) whose calibrated mass is at least p, and the
- * cut that identifies the set. Prefix masses are exact sums of 40-bit
- * fixed-point weights and Z a fixed-order double sum, so the result is
- * deterministic. sparse supplies the lengths.
+ * cut that identifies the set. Prefix masses and Z are exact sums of the same
+ * 40-bit fixed-point weights, so the result does not depend on the order of
+ * summation and is deterministic. sparse supplies the lengths.
  * sel_len, cut: device [B*Hkv]. */
 hkv_status hkv_topp_select(const hkv_problem *prob, const float *z, int64_t z_stride,
                            const hkv_tier *sparse, int32_t *sel_len, hkv_cut *cut,
@@ -205,16 +206,18 @@ hkv_status hkv_cascade_decode(const hkv_problem *prob, const void *q,
                               hkv_stream_t stream);
 
 /* S1..S5 in one call ([TS 2.A] pipeline steps 2 and 3 plus decoding): four
- * kernels on `stream`, all but the first launched as programmatic dependents
- * of the one before. (1) A persistent streaming kernel scores every sparse
+ * kernels on `stream`, each launched as a programmatic dependent of the
+ * kernel before it (the first waits for that kernel before reading anything). (1) A persistent streaming kernel scores every sparse
  * token (the same kernel as hkv_score), also writing each token's per-head
  * logits and each unit's score range into the workspace; (2) one CTA per unit
+ * (a cluster of four, or two, for units of more than 24576 sparse tokens)
  * calibrates, takes the Top-p budget and the cut, and compacts the unit's
- * indices into PAD_MAX rows; (3) a persistent streaming kernel attends over
- * the dense and condensed tokens and over the selected tokens, whose rows it
- * reads through the indices ([TS 2.C] Sparse Loading) together with the
- * scorer's logits (so their K rows are not read again); (4) a merge kernel
- * combines each unit's partial softmax records. A FLAT_SUM layout or
+ * indices into PAD_MAX rows, starting each selected V row's way into L2; (3) a
+ * persistent streaming kernel attends over the dense and condensed tokens
+ * (before it waits for (2)) and over the selected tokens, whose rows it reads
+ * through the indices ([TS 2.C] Sparse Loading) together with the scorer's
+ * logits (so their K rows are not read again); (4) a merge kernel combines
+ * each unit's partial softmax records. A FLAT_SUM layout or
  * k_out/v_out (the Rewrite Cache copy) adds a kernel at the end; out->beta_fit
  * adds one between (1) and (2) that fits each unit's inverse temperature from
  * the scorer's per-head logits and scores (hkv_attention_entropy and
@@ -314,7 +317,7 @@ hkv_status hkv_append(const hkv_problem *prob, const void *k_new, const void *v_
  * of each head's raw attention softmax_j(scale * q_g . k_j) over the sparse
  * tokens j < len[u]; 0 for an empty unit. Two kernels: the scorer (the same as
  * hkv_score, here writing each token's per-head logits into the workspace)
- * and one CTA per unit summing in double precision.
+ * and a cluster of two CTAs per unit summing in double precision.
  * q: device [B, Hq, D]; h: device [B*Hkv] fp32. */
 hkv_status hkv_attention_entropy(const hkv_problem *prob, const void *q, const hkv_tier *sparse,
                                  float *h, void *ws, size_t ws_bytes, hkv_stream_t stream);
