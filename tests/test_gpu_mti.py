@@ -20,12 +20,17 @@ pytestmark = pytest.mark.gpu
 STEPS = 8
 
 
-def _case():
-    wl = WORKLOADS[2].with_(B=2, Hq=8, Hkv=4, n_cap=3000, w_cap=32, c_cap=8, bmin=16, bmax=1024, p=0.95)
+def _case(long=False):
+    # long: units beyond what one CTA stages, so the selection runs split over
+    # clusters of CTAs, and reusing units leave their clusters idle
+    wl = WORKLOADS[2].with_(B=2, Hq=8, Hkv=4, n_cap=30000 if long else 3000, w_cap=32, c_cap=8, bmin=16,
+                            bmax=16384 if long else 1024, p=0.95)
     x = make_inputs(wl, H.dev(), 5)
     g = torch.Generator(device=H.dev()).manual_seed(9)
     qs = [torch.randn(x.q.shape, generator=g, device=H.dev()).to(wl.dtype) for _ in range(STEPS)]
-    pu = np.linspace(0.3, 0.99, wl.units).astype(np.float32)  # budgets spread over the units
+    # budgets spread over the units, below the clamp
+    pu = np.linspace(0.005, 0.3, wl.units) if long else np.linspace(0.3, 0.99, wl.units)
+    pu = pu.astype(np.float32)
     return wl, x, qs, pu
 
 
@@ -44,8 +49,9 @@ def _host_state(st: hkv.MtiState):
             "rw_idx": st.rw_idx.cpu().numpy().reshape(len(st.mode), -1)}
 
 
-def test_step_mti_matches_oracle_over_steps_and_in_a_graph():
-    wl, x, qs, pu = _case()
+@pytest.mark.parametrize("long", [False, True])
+def test_step_mti_matches_oracle_over_steps_and_in_a_graph(long):
+    wl, x, qs, pu = _case(long)
     lo, hi, cap = _thresholds(wl, x, pu)
     prob = H.problem_of(wl, p_unit=torch.from_numpy(pu).to(H.dev()))
     tiers = H.tiers_of(x)

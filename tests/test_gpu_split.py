@@ -9,10 +9,12 @@ ragged lengths, flat and spiky heads, bf16 and fp32, short units in the same
 launch) and on a unit whose cut falls in a block of identical keys, which no
 part can list and which therefore goes back to the one-CTA general path. Each
 is checked end to end against the oracle, as the other step tests are."""
+import numpy as np
 import pytest
 import torch
 
-from head_adaptive_kv_b200.workloads import WORKLOADS
+from head_adaptive_kv_b200 import hkv
+from head_adaptive_kv_b200.workloads import WORKLOADS, to_host_bits
 from tests import gpu_helpers as H
 from tests.test_gpu_step import check_step
 
@@ -54,3 +56,31 @@ def test_split_step_with_a_block_of_identical_keys():
         prob, out, ws = H.run_step(wl, x, p=p)
         assert ws.status() == 0
         check_step(wl, x, out, p, wl.bmin, wl.bmax, tag=f"tied p={p}")
+
+
+def test_split_step_flat_sum_and_rewrite():
+    """The split path's rows through the FLAT_SUM layout and the Rewrite Cache
+    copy: the same budgets and rows as PAD_MAX, offsets the scan of the
+    budgets, and the copied K/V rows bit for bit."""
+    wl = SPLIT_CASES["bf16_long_ragged"]
+    x = H.inputs(wl)
+    _, pad, _ = H.run_step(wl, x, rewrite=True)
+    _, flat, ws = H.run_step(wl, x, layout=hkv.FLAT_SUM, rewrite=True)
+    assert ws.status() == 0
+    U = wl.units
+    k = pad.sel_len.cpu().numpy()
+    assert np.array_equal(k, flat.sel_len.cpu().numpy())
+    offs = flat.offsets.cpu().numpy()
+    assert list(offs) == [0] + list(np.cumsum(k))
+    rows = pad.idx.cpu().numpy().reshape(U, wl.bmax)
+    fl = flat.idx.cpu().numpy()
+    kf = to_host_bits(flat.k_out)
+    vf = to_host_bits(flat.v_out)
+    ks = to_host_bits(x.sparse.k).reshape(U, -1, wl.D)
+    vs = to_host_bits(x.sparse.v).reshape(U, -1, wl.D)
+    for u in range(U):
+        r = rows[u, : k[u]]
+        assert np.array_equal(fl[offs[u]: offs[u + 1]], r)
+        assert np.array_equal(kf[offs[u]: offs[u + 1]], ks[u, r])
+        assert np.array_equal(vf[offs[u]: offs[u + 1]], vs[u, r])
+    assert torch.equal(pad.out, flat.out)
