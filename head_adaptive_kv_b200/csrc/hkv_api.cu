@@ -39,7 +39,7 @@ namespace hkv {
 // done, 2 scores staged, 3 beta found; 4 holds the number of evaluations.
 // Per unit u of the merge kernel, TR_MRG + 2u: 0 start, 1 done.
 // Per attention warp g, TR_AB + 2g: line B start (after the wait and its
-// layout), line B done (merges included); TR_LB + 4g: line B's pipeline
+// layout), line B done; TR_LB + 4g: line B's pipeline
 // (first landing, end, and the stages at TRACE_STAGES + 8 (TR_LB + 4g)).
 [[maybe_unused]] constexpr int TR_SEL = 250000, TR_SW = 0, TR_AW = 20000, TR_FIT = 240000, TR_MRG = 260000,
                                TR_AB = 30000, TR_LB = 8000;

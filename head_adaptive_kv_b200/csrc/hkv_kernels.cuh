@@ -39,10 +39,7 @@ constexpr int AT_STAGES = 3;              // attention: ring slots per warp
 constexpr int SC_FLOATS = 256;            // per-warp logits of one attention stage
 constexpr bool ATTN_UNROLL_QK = true;     // attention: unroll the logit batches of a full stage
 constexpr int PREFIX_CAP = 1024;          // attention: units whose token prefixes fit in shared memory
-#ifndef HKV_SEL_THREADS
-#define HKV_SEL_THREADS 512
-#endif
-constexpr int SEL_THREADS = HKV_SEL_THREADS;  // per-unit kernels
+constexpr int SEL_THREADS = 512;          // per-unit kernels
 constexpr float LOG2E = 1.4426950408889634f;
 
 struct TierP {
