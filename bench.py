@@ -634,47 +634,75 @@ def run_ours(args):
 
     # end to end through the public API: per step, copy the step's query and the
     # per-unit lengths from pinned host memory, run, and read the outputs back
-    # into pinned host memory, all in stream order on the step's stream (the
-    # host does not wait for a step before issuing the next: a decode loop's
-    # calls and copies pipeline on the stream, as an engine's would). The
-    # inputs sit in one device buffer and the outputs in another, so each
-    # direction is one copy per step. (Copies on a second stream into two
-    # alternating buffers measured slower: the loop is bound by the host's
-    # issue rate, and the extra events cost more than the copies' overlap.)
+    # into pinned host memory. The host does not wait for a step before issuing
+    # the next (it issues a step in about a third of the step's device time),
+    # and the copies run on two copy streams into and out of two alternating
+    # buffers, so step i + 1's inputs travel in and step i - 1's outputs travel
+    # back while step i runs; events order each buffer's reuse. Each direction
+    # is one copy per step: the inputs sit in one device buffer and the
+    # outputs in another.
     x, prob, tiers, out = sets[0]
     lens = [t.len for t in (x.dense, x.sparse, x.condensed)]
     q_bytes = x.q.numel() * x.q.element_size()
     in_bytes = q_bytes + sum(t.numel() * 4 for t in lens)
-    dev_in = torch.empty(in_bytes, dtype=torch.uint8, device=device)
-    q_in = dev_in[:q_bytes].view(x.q.dtype).view(x.q.shape)
-    q_in.copy_(x.q)
-    lens_in, at = [], q_bytes
-    for t in lens:
-        lens_in.append(dev_in[at:at + t.numel() * 4].view(torch.int32))
-        lens_in[-1].copy_(t)
-        at += t.numel() * 4
-    host_in = dev_in.cpu().pin_memory()
-    tiers_in = [hkv.Tier(t.k, t.v, ln) for t, ln in zip(tiers, lens_in)]
     n_out, n_lse = out.out.numel(), out.lse.numel()
     out_bytes = (n_out + n_lse + out.sel_len.numel()) * 4
-    dev_out = torch.empty(out_bytes, dtype=torch.uint8, device=device)
-    out_e2e = hkv.StepOutputs(sel_len=dev_out[(n_out + n_lse) * 4:].view(torch.int32), idx=out.idx,
-                              out=dev_out[:n_out * 4].view(torch.float32).view(out.out.shape),
-                              lse=dev_out[n_out * 4:(n_out + n_lse) * 4].view(torch.float32).view(out.lse.shape))
-    host_out = torch.empty(out_bytes, dtype=torch.uint8).pin_memory()
+    bufs = []
+    for _ in range(2):
+        dev_in = torch.empty(in_bytes, dtype=torch.uint8, device=device)
+        q_in = dev_in[:q_bytes].view(x.q.dtype).view(x.q.shape)
+        q_in.copy_(x.q)
+        lens_in, at = [], q_bytes
+        for t in lens:
+            lens_in.append(dev_in[at:at + t.numel() * 4].view(torch.int32))
+            lens_in[-1].copy_(t)
+            at += t.numel() * 4
+        dev_out = torch.empty(out_bytes, dtype=torch.uint8, device=device)
+        oe = hkv.StepOutputs(sel_len=dev_out[(n_out + n_lse) * 4:].view(torch.int32), idx=out.idx,
+                             out=dev_out[:n_out * 4].view(torch.float32).view(out.out.shape),
+                             lse=dev_out[n_out * 4:(n_out + n_lse) * 4].view(torch.float32).view(out.lse.shape))
+        bufs.append({"in": dev_in, "q": q_in, "tiers": [hkv.Tier(t.k, t.v, ln) for t, ln in zip(tiers, lens_in)],
+                     "out": dev_out, "o": oe, "ready": torch.cuda.Event(), "done": torch.cuda.Event(),
+                     "read": torch.cuda.Event(), "host_out": torch.empty(out_bytes, dtype=torch.uint8).pin_memory()})
+    host_in = bufs[0]["in"].cpu().pin_memory()
+    s_in, s_out = torch.cuda.Stream(device=device), torch.cuda.Stream(device=device)
     e2e_steps = min(args.steps, 500)
     barrier(dist, device)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    s_in.wait_event(e0)
+    s_out.wait_event(e0)
+
+    def load(i):  # step i's inputs, once step i - 2 has read the buffer
+        bf = bufs[i % 2]
+        if i >= 2:
+            s_in.wait_event(bf["done"])
+        with torch.cuda.stream(s_in):
+            bf["in"].copy_(host_in, non_blocking=True)
+        bf["ready"].record(s_in)
+
+    load(0)
     for i in range(e2e_steps):
-        dev_in.copy_(host_in, non_blocking=True)
-        hkv.step(prob, q_in, *tiers_in, out_e2e, ws)
-        host_out.copy_(dev_out, non_blocking=True)
+        bf = bufs[i % 2]
+        if i + 1 < e2e_steps:
+            load(i + 1)
+        stream.wait_event(bf["ready"])
+        if i >= 2:
+            stream.wait_event(bf["read"])  # step i - 2's outputs are back on the host
+        hkv.step(prob, bf["q"], *bf["tiers"], bf["o"], ws)
+        bf["done"].record(stream)
+        s_out.wait_event(bf["done"])
+        with torch.cuda.stream(s_out):
+            bf["host_out"].copy_(bf["out"], non_blocking=True)
+        bf["read"].record(s_out)
+    for bf in bufs:
+        stream.wait_event(bf["read"])
     e1.record(stream)
     torch.cuda.synchronize()
-    assert torch.equal(host_out[(n_out + n_lse) * 4:].view(torch.int32), out.sel_len.cpu())
+    for bf in bufs:
+        assert torch.equal(bf["host_out"][(n_out + n_lse) * 4:].view(torch.int32), out.sel_len.cpu())
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, device)
     h2d, d2h = in_bytes, out_bytes
     e2e = {"value": round(whole_job_value(wl.units, wl.units, world, e2e_ms / 1e3, e2e_steps), 2),
