@@ -205,26 +205,13 @@ __device__ __forceinline__ void write_offsets(const Params &P, int u, int64_t of
     }
 }
 
-// The V rows of unit u's sparse tier, for RowPrefetch (the step only).
-template <int ES>
-__device__ __forceinline__ RowPrefetch v_prefetch(const Params &P, int u)
-{
-    RowPrefetch r;
-    if (P.prefetch_v && P.sparse.v != nullptr) {
-        const int b = u / P.Hkv, h = u % P.Hkv;
-        r.base = P.sparse.v + ((int64_t)b * P.sparse.sb + (int64_t)h * P.sparse.sh) * ES;
-        r.stride = P.sparse.st * ES;
-        r.bytes = (uint32_t)(P.D * ES);
-    }
-    return r;
-}
-
 // S2-S4 of unit u, scores at zu (in shared memory when ZS).
 // zg_stage (ZS only): the unit's scores are still in global memory there and
-// the fast path stages them during its first sweep.
+// the fast path stages them during its first sweep. zs_in_flight (ZS only):
+// they are landing in shared memory from this thread's cp.async copies.
 template <int ES, bool ZS>
 __device__ __forceinline__ void unit_work(const Params &P, USmem &sm, const Ctl &c, int u, int n, const float *zu,
-                                          const float *zg_stage = nullptr)
+                                          const float *zg_stage = nullptr, bool zs_in_flight = false)
 {
     int k, n_tie;
     uint32_t key;
@@ -265,7 +252,7 @@ __device__ __forceinline__ void unit_work(const Params &P, USmem &sm, const Ctl 
             Selection s;
             if (P.do_compact &&
                 select_compact_fast(zu, n, m, zlo, beta, pu, P.bmin, P.bmax, sm, s, P.idx + (int64_t)u * P.bmax,
-                                    P.bmax, TR_SEL + 16 * u, zg_stage, v_prefetch<ES>(P, u))) {
+                                    P.bmax, TR_SEL + 16 * u, zg_stage, zs_in_flight)) {
                 publish(s);
                 HKV_TRACE_AT(TR_SEL + 16 * u + 5);
                 return;
@@ -296,7 +283,7 @@ __device__ __forceinline__ void unit_work(const Params &P, USmem &sm, const Ctl 
         write_offsets(P, u, off);
     }
     int32_t *row = P.idx + off;
-    compact_unit<ZS>(zu, n, key, n_tie, k, row, flat ? k : P.bmax, sm.red, TR_SEL + 16 * u, v_prefetch<ES>(P, u));
+    compact_unit<ZS>(zu, n, key, n_tie, k, row, flat ? k : P.bmax, sm.red, TR_SEL + 16 * u);
     HKV_TRACE_AT(TR_SEL + 16 * u + 5);
     if (P.k_out != nullptr && !P.do_select) {
         __syncthreads();
@@ -348,10 +335,21 @@ __global__ void __launch_bounds__(NT, 1) k_unit(const __grid_constant__ Params P
     wait_prior_grid();
     HKV_TRACE_AT(TR_SEL + 16 * u);
     tl_start(P.tl, TL_UNIT);
-    const int n = tier_len(P.sparse, u, c);
     const float *zg = P.z + (int64_t)u * P.z_stride;
+    // hkv_step: with the range known and every unit short enough to stage,
+    // the scores start landing in shared memory before the length and the
+    // range words are read
+    const bool early = P.have_range && P.do_select && P.do_compact && P.sparse.cap <= ZSTAGE &&
+                       (reinterpret_cast<uintptr_t>(zg) & 15) == 0;
+    if (early)
+        stage_scores_async(zg, P.sparse.cap, sm.zs);
+    const int n = tier_len(P.sparse, u, c);
     if (P.mti_left != nullptr && __ldcg(P.mti_left + u) > 0) {
+        if (early)
+            cp_async_wait_all();
         mti_reuse_outputs(P, c, u);  // the unit reuses its rewrite: nothing to select
+    } else if (early) {
+        unit_work<ES, true>(P, sm, c, u, n, sm.zs, nullptr, true);
     } else if (P.have_range && P.do_select && P.do_compact && n <= ZSTAGE) {
         // hkv_step: the range is known, so the first sweep stages the scores
         unit_work<ES, true>(P, sm, c, u, n, sm.zs, zg);
@@ -416,8 +414,7 @@ __global__ void __cluster_dims__(C, 1, 1) __launch_bounds__(NT, 1) k_unit_cluste
         const float beta = unit_beta(P, u, c), pu = unit_p(P, u, c);
         Selection s;
         const int st = select_compact_cluster<C>(zg, n, m, zlo, beta, pu, P.bmin, P.bmax, sm, s,
-                                                 P.idx + (int64_t)u * P.bmax, P.bmax, tb, v_prefetch<ES>(P, u),
-                                                 rank);
+                                                 P.idx + (int64_t)u * P.bmax, P.bmax, tb, rank);
         if (rank == 0) {
             if (st != 0) {
                 // the general path, alone (it reads and resets the range words)
@@ -1092,7 +1089,6 @@ hkv_status step_impl(const hkv_problem *prob, const void *q, const hkv_tier *den
     U.have_range = scored;
     U.do_select = 1;
     U.do_compact = 1;
-    U.prefetch_v = 1;
     // units longer than one CTA can stage are split over a cluster of CTAs
     // (one CTA would sweep such a unit from L2 several times): four when all
     // the clusters fit the SMs at once, else two when two CTAs can stage it

@@ -174,17 +174,15 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
         : "memory");
 }
 
-// Start bringing the 128-byte line holding `src` into L2.
-__device__ __forceinline__ void prefetch_l2_line(const void *src)
-{
-    asm volatile("prefetch.global.L2 [%0];" ::"l"(src));
-}
-
 // 16-byte asynchronous copy global -> shared, cached in L2 only.
 __device__ __forceinline__ void cp_async16(void *dst, const void *src)
 {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src) : "memory");
 }
+
+// Wait until this thread's earlier cp.async copies have landed (a barrier
+// then makes every thread's copies visible to the CTA).
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // Arrive on `bar` once this thread's earlier cp.async copies have landed (the
 // pending count is raised first, so the phase waits for them).

@@ -81,7 +81,6 @@ struct Params {
     int32_t unit_ctas;    // CTAs of the selection kernel before the attention (units, or more when split)
     int32_t have_range;   // per-unit kernel: urange holds the units' score ranges
     int32_t do_select, do_compact;  // per-unit kernel: which steps to run
-    int32_t prefetch_v;   // per-unit kernel: bring the selected tokens' V rows into L2 (the attention follows)
     int32_t withhold;     // fault injection: streaming warps never arm their stages
     // fitted temperature: per-unit entropy target in (nullptr: from the logit
     // records), target out, fitted inverse temperature out
@@ -1591,6 +1590,18 @@ __device__ bool stage_scores(const float *zu, int n, SM &sm)
     return true;
 }
 
+// Start copying a unit's first cnt <= ZSTAGE scores (zg 16-byte aligned) into
+// shared memory: cp.async for the whole quads, plain loads and stores for the
+// rest. The copies land after cp_async_wait_all and a barrier.
+__device__ __forceinline__ void stage_scores_async(const float *zg, int cnt, float *zs)
+{
+    const int nq = cnt >> 2;
+    for (int q = threadIdx.x; q < nq; q += NT)
+        cp_async16(zs + 4 * q, zg + 4 * q);
+    for (int j = 4 * nq + threadIdx.x; j < cnt; j += NT)
+        zs[j] = __ldcg(zg + j);
+}
+
 // A sweep over a unit's scores in global memory that also stages them in
 // shared memory: thread t takes the same quads in the same order as
 // sweep_scores<true>, so sums taken in call order match it bit for bit.
@@ -2089,11 +2100,11 @@ __device__ int list_candidates(const float *zs, int n, const BinFn &bins, int b_
 }
 
 // One-sweep version of list_candidates: warp w walks its contiguous segment
-// of the staged scores four tokens per lane at a time and appends its hits to
-// its own region of sm.cand (CAND_CAP / warps entries, no atomics); the regions
-// are then closed up into one list. Returns the number listed, or -1 (and
-// nothing usable in sm.cand) when a region overflows. Token j of zs is listed
-// as index base + j.
+// of the staged scores 128 tokens at a time (four per lane, a lane's tokens 32
+// apart) and appends its hits to its own region of sm.cand (CAND_CAP / warps
+// entries, no atomics); the regions are then closed up into one list, in
+// index order. Returns the number listed, or -1 (and nothing usable in
+// sm.cand) when a region overflows. Token j of zs is listed as index base + j.
 __device__ int list_candidates_warp(const float *zs, int n, const BinFn &bins, int b_hi, USmem &sm, int base = 0)
 {
     constexpr int NW = NT / 32, REG = CAND_CAP / NW;
@@ -2105,26 +2116,20 @@ __device__ int list_candidates_warp(const float *zs, int n, const BinFn &bins, i
     int cnt = 0;
 #pragma unroll 1
     for (int jb = j0; jb < j1; jb += 128) {
-        const int j = jb + 4 * lane;
         float a[4];
-        if (j + 4 <= j1) {
-            const float4 v = lds4(zs + j);
-            a[0] = v.x;
-            a[1] = v.y;
-            a[2] = v.z;
-            a[3] = v.w;
-        } else {
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-                a[e] = j + e < j1 ? lds1(zs + j + e) : 0.f;
+        for (int e = 0; e < 4; ++e) {
+            const int j = jb + 32 * e + lane;
+            a[e] = j < j1 ? lds1(zs + j) : 0.f;
         }
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-            const bool hit = j + e < j1 && bins(a[e]) <= b_hi;
+            const int j = jb + 32 * e + lane;
+            const bool hit = j < j1 && bins(a[e]) <= b_hi;
             const unsigned m = __ballot_sync(0xffffffffu, hit);
             const int at = cnt + __popc(m & lower);
             if (hit && at < REG)
-                reg[at] = ((unsigned long long)score_key(a[e]) << 32) | (uint32_t)(base + j + e);
+                reg[at] = ((unsigned long long)score_key(a[e]) << 32) | (uint32_t)(base + j);
             cnt += __popc(m);
         }
     }
@@ -2157,31 +2162,17 @@ __device__ int list_candidates_warp(const float *zs, int n, const BinFn &bins, i
     return (int)tot;
 }
 
-// The V rows of a unit's selected tokens, brought into L2 as the compaction
-// finds them (the step's attention gathers them next). base nullptr: none.
-struct RowPrefetch {
-    const char *base = nullptr;
-    int64_t stride = 0;  // bytes between rows
-    uint32_t bytes = 0;  // bytes of a row
-    __device__ __forceinline__ void operator()(int j) const
-    {
-        if (base == nullptr)
-            return;
-        const uintptr_t a = reinterpret_cast<uintptr_t>(base + (int64_t)j * stride);
-        for (uintptr_t l = a & ~(uintptr_t)127; l < a + bytes; l += 128)
-            prefetch_l2_line(reinterpret_cast<const void *>(l));
-    }
-};
-
 // From the listed tokens (sm.cand[0, ncand): every token of bins 0 .. b_hi,
 // b_hi the bin of rank r_hi = min(n, bmax), hb_c the tokens before it) and the
-// unit's bin counts: the budget, its cut and, when k > 0, the bitmap of the
-// selected tokens in sm.bits (n bits, token j at bit j). The selected tokens'
-// rows are handed to pf. Returns false when the crossing bin holds more than
-// BIN_CAP tokens (the caller falls back to the general path).
+// unit's bin counts: the budget and its cut. When k > 0, *tie_last receives
+// the index of the last selected token of the cut key (the selection is every
+// token with a key below the cut's, and those of the cut key up to that
+// index), and with `bitmap` the selected tokens are also marked in sm.bits
+// (n bits, token j at bit j). Returns false when the crossing bin holds more
+// than BIN_CAP tokens (the caller falls back to the general path).
 __device__ bool cut_bitmap(int n, int ncand, int b_hi, unsigned long long hb_c, int r_hi, float m, float bl2,
                            const BinFn &bins, float p, int bmin, int bmax, USmem &sm, Selection &r, int tb,
-                           const RowPrefetch &pf)
+                           bool bitmap, uint32_t *tie_last)
 {
     const auto mass = [&](int b) { return sm.mass[b]; };
     int kstar = -1, pos = -1;
@@ -2251,28 +2242,31 @@ __device__ bool cut_bitmap(int n, int ncand, int b_hi, unsigned long long hb_c, 
         __syncthreads();
         const int tie0 = sm.bc[4];
         n_above = (int)before_c + tie0;
+        // the selected ties are the first k - n_above of the cut key in the
+        // sorted bin (by index); the last of them sits at pos
+        *tie_last = (uint32_t)sm.binbuf[pos];
         HKV_TRACE_AT(tb < 0 ? -1 : tb + 3);
-        // bitmap of the selection: listed tokens above the cut, and the first
-        // n_tie ties (consecutive in binbuf, by index)
-        const int nwords = (n + 31) >> 5;
-        for (int i = threadIdx.x; i < nwords; i += NT)
-            sm.bits[i] = 0u;
-        __syncthreads();
-        for (int i = threadIdx.x; i < ncand; i += NT) {
-            const unsigned long long e = sm.cand[i];
-            if ((uint32_t)(e >> 32) < cut_key) {
-                const uint32_t j = (uint32_t)e;
-                atomicOr(&sm.bits[j >> 5], 1u << (j & 31));
-                pf((int)j);
+        if (bitmap) {
+            // bitmap of the selection: listed tokens above the cut, and the
+            // first n_tie ties (consecutive in binbuf, by index)
+            const int nwords = (n + 31) >> 5;
+            for (int i = threadIdx.x; i < nwords; i += NT)
+                sm.bits[i] = 0u;
+            __syncthreads();
+            for (int i = threadIdx.x; i < ncand; i += NT) {
+                const unsigned long long e = sm.cand[i];
+                if ((uint32_t)(e >> 32) < cut_key) {
+                    const uint32_t j = (uint32_t)e;
+                    atomicOr(&sm.bits[j >> 5], 1u << (j & 31));
+                }
             }
+            const int n_tie = k - n_above;
+            for (int i = threadIdx.x; i < n_tie; i += NT) {
+                const uint32_t j = (uint32_t)sm.binbuf[tie0 + i];
+                atomicOr(&sm.bits[j >> 5], 1u << (j & 31));
+            }
+            __syncthreads();
         }
-        const int n_tie = k - n_above;
-        for (int i = threadIdx.x; i < n_tie; i += NT) {
-            const uint32_t j = (uint32_t)sm.binbuf[tie0 + i];
-            atomicOr(&sm.bits[j >> 5], 1u << (j & 31));
-            pf((int)j);
-        }
-        __syncthreads();
     }
     r.k = k;
     r.kstar = kstar;
@@ -2312,18 +2306,58 @@ __device__ void expand_bits(const uint32_t *bits, int w_begin, int w_end, int at
     }
 }
 
+// The selected tokens of a candidate list in index order (sm.cand[0, ncand),
+// as list_candidates_warp leaves it): every entry whose key is below cut_key,
+// and those of cut_key with an index up to tie_last, written in list order to
+// row[0, k). Warp w takes a contiguous part of the list, 32 entries a step; a
+// block scan of the warps' counts places the parts.
+__device__ void compact_list(int ncand, uint32_t cut_key, uint32_t tie_last, int k, int32_t *row, USmem &sm)
+{
+    constexpr int NW = NT / 32;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int seg = ((ncand + NW - 1) / NW + 31) / 32 * 32;
+    const int i0 = min(ncand, w * seg), i1 = min(ncand, i0 + seg);
+    const auto take = [&](int i) {
+        if (i >= i1)
+            return false;
+        const unsigned long long e = sm.cand[i];
+        const uint32_t kk = (uint32_t)(e >> 32);
+        return kk < cut_key || (kk == cut_key && (uint32_t)e <= tie_last);
+    };
+    int cnt = 0;
+#pragma unroll 1
+    for (int i = i0 + lane; i - lane < i1; i += 32)
+        cnt += __popc(__ballot_sync(0xffffffffu, take(i)));
+    unsigned long long tot;
+    const unsigned long long ex = block_exclusive_scan<NT>(lane == 0 ? (unsigned long long)cnt : 0ull, sm.red, &tot);
+    int at = (int)__shfl_sync(0xffffffffu, (unsigned int)ex, 0);
+    const unsigned lower = (1u << lane) - 1u;
+#pragma unroll 1
+    for (int i = i0 + lane; i - lane < i1; i += 32) {
+        const bool t = take(i);
+        const unsigned msk = __ballot_sync(0xffffffffu, t);
+        const int pos = at + __popc(msk & lower);
+        if (t && pos < k)
+            row[pos] = (int32_t)(uint32_t)sm.cand[i];
+        at += __popc(msk);
+    }
+}
+
 // Selection and PAD_MAX compaction of one unit in one go, its n <= ZSTAGE
-// scores staged in shared memory (zs; or staged from zg during the first sweep).
+// scores staged in shared memory (zs; or staged from zg during the first sweep;
+// or, zs_in_flight, still landing from this thread's cp.async copies).
 // Returns false (nothing written) when a list or bin outgrows shared memory.
 __device__ bool select_compact_fast(const float *zs, int n, float m, float zlo, float beta, float p, int bmin,
                                     int bmax, USmem &sm, Selection &r, int32_t *row, int pad, int tb,
-                                    const float *zg = nullptr, const RowPrefetch &pf = RowPrefetch{})
+                                    const float *zg = nullptr, bool zs_in_flight = false)
 {
     const float bl2 = beta * LOG2E;
     const BinFn bins = make_bins(m, zlo);
     r = Selection{};
     for (int i = threadIdx.x; i < SBINS; i += NT)
         sm.cnt[i] = 0;
+    if (zs_in_flight)
+        cp_async_wait_all();
     __syncthreads();
     const auto mass = [&](int b) { return sm.mass[b]; };
     // sweep 1: bin counts and the normaliser (an exact sum of the fixed-point
@@ -2349,16 +2383,21 @@ __device__ bool select_compact_fast(const float *zs, int n, float m, float zlo, 
         const int ncand = (int)hb_c + (int)sm.cnt[b_hi];
         if (ncand > CAND_CAP)
             return false;
-        // the tokens of bins 0 .. b_hi: one sweep, or two when a warp's share
-        // of them outgrows its region
-        if (list_candidates_warp(zs, n, bins, b_hi, sm) < 0)
+        // the tokens of bins 0 .. b_hi: one sweep, in index order, or two
+        // (in another order) when a warp's share of them outgrows its region
+        const bool ordered = list_candidates_warp(zs, n, bins, b_hi, sm) >= 0;
+        if (!ordered)
             list_candidates(zs, n, bins, b_hi, sm);
         HKV_TRACE_AT(tb < 0 ? -1 : tb + 2);
-        if (!cut_bitmap(n, ncand, b_hi, hb_c, r_hi, m, bl2, bins, p, bmin, bmax, sm, r, tb, pf))
+        uint32_t tie_last = 0;
+        if (!cut_bitmap(n, ncand, b_hi, hb_c, r_hi, m, bl2, bins, p, bmin, bmax, sm, r, tb, !ordered, &tie_last))
             return false;
-        if (r.k > 0) {
-            // the row is built in shared memory (the candidate list is no longer
-            // needed) and then written out with coalesced stores
+        if (r.k > 0 && ordered) {
+            // the selected entries of the list, already in index order
+            compact_list(ncand, r.key, tie_last, r.k, row, sm);
+        } else if (r.k > 0) {
+            // the row is built in shared memory from the bitmap (the candidate
+            // list is no longer needed) and then written out with coalesced stores
             int32_t *buf = reinterpret_cast<int32_t *>(sm.cand);
             const bool in_smem = r.k <= 2 * CAND_CAP;
             expand_bits(sm.bits, 0, (n + 31) >> 5, 0, r.k, in_smem ? buf : row, sm);
@@ -2435,7 +2474,7 @@ __host__ __device__ constexpr int cluster_chunk(int n)
 template <int C>
 __device__ int select_compact_cluster(const float *zg, int n, float m, float zlo, float beta, float p, int bmin,
                                       int bmax, USmem &sm, Selection &r, int32_t *row, int pad, int tb,
-                                      const RowPrefetch &pf, int rank)
+                                      int rank)
 {
     namespace cg = cooperative_groups;
     auto cl = cg::this_cluster();
@@ -2622,7 +2661,6 @@ __device__ int select_compact_cluster(const float *zg, int n, float m, float zlo
                 const int j = (int)(uint32_t)e;
                 if (kk < key || (kk == key && j <= tie_last)) {
                     atomicOr(&sm.bits[(j - j0) >> 5], 1u << ((j - j0) & 31));
-                    pf(j);
                 }
             }
             __syncthreads();
@@ -2664,7 +2702,7 @@ __device__ __forceinline__ float zload(const float *zu, int j)
 
 template <bool ZS>
 __device__ void compact_unit(const float *zu, int n, uint32_t cut_key, int n_tie, int k, int32_t *row, int pad,
-                             unsigned long long *red, int tb = -1, const RowPrefetch &pf = RowPrefetch{})
+                             unsigned long long *red, int tb = -1)
 {
     constexpr int NW = NT / 32;
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -2701,7 +2739,6 @@ __device__ void compact_unit(const float *zu, int n, uint32_t cut_key, int n_tie
             const uint32_t pos = lt_before + __popc(mlt & lower) + eq_taken_before;
             if (take && pos < (uint32_t)k) {  // a caller's inconsistent cut stays in the row
                 row[pos] = j;
-                pf(j);
             }
             lt_before += __popc(mlt);
             eq_before += __popc(meq);
