@@ -219,11 +219,14 @@ __device__ __forceinline__ void unit_work(const Params &P, USmem &sm, const Ctl 
         float m, zlo;
         if (P.have_range) {
             // the scorer's range words of the unit (key 0: no score), reset
-            // for the next step once read
+            // for the next step once read (zs_in_flight: k_unit has put them
+            // in sm.redf already)
             if (threadIdx.x == 0) {
-                const uint32_t kmax = __ldcg(P.urange + 2 * u), kmin = __ldcg(P.urange + 2 * u + 1);
-                sm.redf[0] = kmax ? ord_val(kmax) : -INFINITY;
-                sm.redf[1] = kmin ? ord_val(~kmin) : INFINITY;
+                if (!zs_in_flight) {
+                    const uint32_t kmax = __ldcg(P.urange + 2 * u), kmin = __ldcg(P.urange + 2 * u + 1);
+                    sm.redf[0] = kmax ? ord_val(kmax) : -INFINITY;
+                    sm.redf[1] = kmin ? ord_val(~kmin) : INFINITY;
+                }
                 P.urange[2 * u] = 0;
                 P.urange[2 * u + 1] = 0;
             }
@@ -337,13 +340,23 @@ __global__ void __launch_bounds__(NT, 1) k_unit(const __grid_constant__ Params P
     tl_start(P.tl, TL_UNIT);
     const float *zg = P.z + (int64_t)u * P.z_stride;
     // hkv_step: with the range known and every unit short enough to stage,
-    // the scores start landing in shared memory before the length and the
-    // range words are read
+    // the length and the range words are requested first, then the scores'
+    // copy into shared memory (which the loads would otherwise queue behind)
     const bool early = P.have_range && P.do_select && P.do_compact && P.sparse.cap <= ZSTAGE &&
                        (reinterpret_cast<uintptr_t>(zg) & 15) == 0;
-    if (early)
-        stage_scores_async(zg, P.sparse.cap, sm.zs);
+    uint32_t kmax = 0, kmin = 0;
+    if (early && threadIdx.x == 0) {
+        kmax = __ldcg(P.urange + 2 * u);
+        kmin = __ldcg(P.urange + 2 * u + 1);
+    }
     const int n = tier_len(P.sparse, u, c);
+    if (early) {
+        stage_scores_async(zg, P.sparse.cap, sm.zs);
+        if (threadIdx.x == 0) {
+            sm.redf[0] = kmax ? ord_val(kmax) : -INFINITY;
+            sm.redf[1] = kmin ? ord_val(~kmin) : INFINITY;
+        }
+    }
     if (P.mti_left != nullptr && __ldcg(P.mti_left + u) > 0) {
         if (early)
             cp_async_wait_all();

@@ -1502,17 +1502,18 @@ struct __align__(16) USmem {  // shared memory of the per-unit kernels
     uint32_t pub_key;
 };
 
-// Bin of a score: (m - z) s rounded to the nearest integer, clamped to
-// [0, SBINS - 1]; -inf and NaN land in the last bin. Any bin map that does not
-// decrease as z falls serves the selection (the cut itself is exact), so the
-// rounding is done with the fp32 add of 1.5 * 2^23 (whose low mantissa bits
-// are then the integer) instead of conversion instructions.
+// Bin of a score: m s - z s (one fused multiply-add, with m s rounded once)
+// rounded to the nearest integer, clamped to [0, SBINS - 1]; -inf and NaN land
+// in the last bin. Any bin map that does not decrease as z falls serves the
+// selection (the cut itself is exact), so the rounding is done with the fp32
+// add of 1.5 * 2^23 (after which the float's bits are 0x4B400000 plus the
+// integer) instead of conversion instructions.
 struct BinFn {
-    float m, s;
+    float ms, s;
     __device__ __forceinline__ int operator()(float z) const
     {
-        const float t = fmaxf(fminf((m - z) * s, (float)(SBINS - 1)), 0.0f);
-        return (__float_as_int(t + 12582912.0f) & 0x7fffff) ^ 0x400000;
+        const float t = fmaxf(fminf(fmaf(-z, s, ms), (float)(SBINS - 1)), 0.0f);
+        return __float_as_int(t + 12582912.0f) - 0x4B400000;
     }
 };
 
@@ -1520,8 +1521,8 @@ __device__ __forceinline__ BinFn make_bins(float m, float zlo)
 {
     const float R = m - zlo;
     BinFn f;
-    f.m = m;
     f.s = (R > 0.0f && isfinite(R)) ? (float)SBINS / R : 0.0f;
+    f.ms = m * f.s;
     return f;
 }
 
