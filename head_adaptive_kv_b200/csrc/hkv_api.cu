@@ -335,6 +335,10 @@ __global__ void __launch_bounds__(NT, 1) k_unit(const __grid_constant__ Params P
     const Ctl c = make_ctl(P);
     const int u = blockIdx.x;
     allow_dependents();
+    // the unit's length is an input of the step (no kernel of the step writes
+    // it, and the kernels that do, the append and the condensation, let their
+    // dependents start only when they end): read before the wait
+    const int n = tier_len(P.sparse, u, c);
     wait_prior_grid();
     HKV_TRACE_AT(TR_SEL + 16 * u);
     tl_start(P.tl, TL_UNIT);
@@ -349,7 +353,6 @@ __global__ void __launch_bounds__(NT, 1) k_unit(const __grid_constant__ Params P
         kmax = __ldcg(P.urange + 2 * u);
         kmin = __ldcg(P.urange + 2 * u + 1);
     }
-    const int n = tier_len(P.sparse, u, c);
     if (early) {
         stage_scores_async(zg, P.sparse.cap, sm.zs);
         if (threadIdx.x == 0) {

@@ -212,11 +212,14 @@ hkv_status hkv_cascade_decode(const hkv_problem *prob, const void *q,
  * logits and each unit's score range into the workspace; (2) one CTA per unit
  * (a cluster of four, or two, for units of more than 24576 sparse tokens)
  * calibrates, takes the Top-p budget and the cut, and compacts the unit's
- * indices into PAD_MAX rows, starting each selected V row's way into L2; (3) a
+ * indices into PAD_MAX rows; (3) a
  * persistent streaming kernel attends over the dense and condensed tokens
  * (before it waits for (2)) and over the selected tokens, whose rows it reads
  * through the indices ([TS 2.C] Sparse Loading) together with the scorer's
- * logits (so their K rows are not read again); (4) a merge kernel combines
+ * logits (so their K rows are not read again); (2) and (3) read the tiers'
+ * lengths before their waits, so the lengths must be final when the call is
+ * made (this library's append and condensation let no dependent start before
+ * they end); (4) a merge kernel combines
  * each unit's partial softmax records. A FLAT_SUM layout or
  * k_out/v_out (the Rewrite Cache copy) adds a kernel at the end; out->beta_fit
  * adds one between (1) and (2) that fits each unit's inverse temperature from
