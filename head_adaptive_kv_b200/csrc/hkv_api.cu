@@ -68,7 +68,7 @@ __global__ void __launch_bounds__(sc_nw(G) * 32, 1) k_score_stream(const __grid_
                              : (int64_t)P.units * P.sparse.cap;
     Job job(P, c, sm.ring, prefix ? &sm.line : nullptr, T, g, NW);
     HKV_TRACE_WARP(TR_SW + 4 * (int)g);
-    if (!job.run_single_unit())
+    if (!job.run_static_share())
         warp_pipeline(job, sm.ring, c, TR_SW + 4 * (int)g);
     tl_end(P.tl, TL_SCORE);
 }

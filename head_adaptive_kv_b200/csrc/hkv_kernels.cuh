@@ -585,35 +585,53 @@ struct ScoreJob {
         __syncwarp();
     }
 
-    // A static share inside one unit whose rows are all present (the common
-    // case): the stages follow from their number alone, so the warp runs this
-    // short loop instead of warp_pipeline's general generator, and leaves the
-    // job at the end of its static share. Returns false (having done nothing)
-    // when the share does not qualify or a wait ran out.
-    __device__ __forceinline__ bool run_single_unit()
+    // A static share inside one unit, or across the end of one unit into the
+    // next, whose rows are all present (the common case): the stages of its
+    // one or two segments follow from their sizes alone, numbered on through
+    // the warp's ring, so the warp runs this short loop instead of
+    // warp_pipeline's general generator, and leaves the job at the end of its
+    // static share. Returns false (having done nothing) when the share does
+    // not qualify or a wait ran out.
+    __device__ __forceinline__ bool run_static_share()
     {
         if (left <= 0 || P.withhold)
             return false;
-        if ((int64_t)j + left > span(u))
+        // segment 0: rows [j, j + rows0) of unit u; segment 1: rows
+        // [0, rows1) of unit u + 1 (rows1 = 0: none)
+        const int span0 = span(u);
+        const int rows0 = (int)min(left, (int64_t)(span0 - j));
+        const int rows1 = (int)(left - rows0);
+        if (rows0 <= 0 || (rows1 > 0 && (u + 1 >= P.units || rows1 > span(u + 1))))
             return false;
-        const int n = L ? span(u) : score_len(P, u, c);
-        if (j + (int)left > n)
+        if (j + rows0 > (L ? span0 : score_len(P, u, c)))
             return false;
-        gu = u;
-        gn = n;
-        {
-            const int b = u / P.Hkv, h = u % P.Hkv;
-            kbase = P.sparse.k + ((int64_t)b * P.sparse.sb + (int64_t)h * P.sparse.sh) * ES;
-        }
-        const int j0 = j, rows = (int)left;
-        const int nst = (rows + Gm::SROWS - 1) / Gm::SROWS;
+        if (rows1 > 0 && rows1 > (L ? span(u + 1) : score_len(P, u + 1, c)))
+            return false;
+        const auto unit_k = [&](int x) {
+            const int b = x / P.Hkv, h = x % P.Hkv;
+            return P.sparse.k + ((int64_t)b * P.sparse.sb + (int64_t)h * P.sparse.sh) * ES;
+        };
+        const char *kb0 = unit_k(u);
+        const char *kb1 = rows1 > 0 ? unit_k(u + 1) : kb0;
+        const int u0 = u, j0 = j;
+        const int nst0 = (rows0 + Gm::SROWS - 1) / Gm::SROWS;
+        const int nst = nst0 + (rows1 + Gm::SROWS - 1) / Gm::SROWS;
         const auto stage = [&](int sidx) {
-            const int st0 = j0 + sidx * Gm::SROWS;
-            return StageDesc{u, st0, min(Gm::SROWS, j0 + rows - st0),
-                             (sidx == 0 ? SD_FIRST : 0) | (sidx == nst - 1 ? SD_LAST : 0)};
+            if (sidx < nst0) {
+                const int st0 = j0 + sidx * Gm::SROWS;
+                return StageDesc{u0, st0, min(Gm::SROWS, j0 + rows0 - st0),
+                                 (sidx == 0 ? SD_FIRST : 0) | (sidx == nst0 - 1 ? SD_LAST : 0)};
+            }
+            const int s1 = sidx - nst0, st0 = s1 * Gm::SROWS;
+            return StageDesc{u0 + 1, st0, min(Gm::SROWS, rows1 - st0),
+                             (s1 == 0 ? SD_FIRST : 0) | (sidx == nst - 1 ? SD_LAST : 0)};
+        };
+        const auto copy = [&](int sidx, int slot) {
+            kbase = sidx < nst0 ? kb0 : kb1;
+            copy_stage(stage(sidx), slot);
         };
         for (int sidx = 0; sidx < NS && sidx < nst; ++sidx)
-            copy_stage(stage(sidx), sidx);
+            copy(sidx, sidx);
         for (int sidx = 0; sidx < nst; ++sidx) {
             const int slot = sidx % NS;
             if (!mbar_wait(&ring.full[w][slot], (sidx / NS) & 1u, c)) {
@@ -628,9 +646,10 @@ struct ScoreJob {
             if (sidx + NS < nst) {
                 if (lane == 0)
                     fence_proxy_async_smem();
-                copy_stage(stage(sidx + NS), slot);
+                copy(sidx + NS, slot);
             }
         }
+        gu = rows1 > 0 ? u0 + 1 : u0;
         left = 0;
         return true;
     }
