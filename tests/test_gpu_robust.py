@@ -133,3 +133,25 @@ def test_withheld_publish_times_out_and_context_survives():
     prob, out, ws2 = H.run_step(WL, x)
     assert ws2.status() == 0
     check_step(WL, x, out, WL.p, WL.bmin, WL.bmax, tag="after timeout")
+
+
+def test_candidates_crowded_into_one_warp_segment():
+    """A unit whose best 2000 scores are its first 2000 tokens: the warps that
+    list the candidates each take a contiguous segment of the unit, so the
+    first two segments hold far more candidates than a warp's region, the
+    one-sweep list gives up, and the two-sweep list (in another order) with
+    the bitmap row takes over. Budgets, cuts, rows and outputs still match the
+    oracle; the other units take the one-sweep path in the same launch."""
+    wl = WORKLOADS[2].with_(B=1, Hq=8, Hkv=2, n_cap=16000, bmin=1, bmax=2048)
+    x = H.inputs(wl)
+    g = torch.Generator(device="cpu").manual_seed(7)
+    k = x.sparse.k[0, 0]
+    # keys along the unit's first query head, longer than the others: the top scores
+    q0 = x.q[0, 0].float().cpu()
+    scale_k = float(k.float().norm(dim=1).mean())
+    noise = 0.05 * torch.randn(2000, wl.D, generator=g)
+    k[:2000] = (q0 / q0.norm() * (1.5 * scale_k) + noise).to(k.dtype).to(k.device)
+    for p in (0.5, 0.95, 1.0):
+        prob, out, ws = H.run_step(wl, x, p=p)
+        assert ws.status() == 0
+        check_step(wl, x, out, p, wl.bmin, wl.bmax, tag=f"crowded p={p}")
