@@ -24,6 +24,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <cudaTypedefs.h>
+
 #include "hkv_kernels.cuh"
 
 namespace hkv {
@@ -590,6 +592,46 @@ static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 static int es_of(hkv_dtype d) { return d == HKV_BF16 ? 2 : 4; }
 
+// The driver's tensor-map encoder, looked up once through the runtime
+// (nullptr when the driver does not provide it).
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }();
+    return fn;
+}
+
+// The sparse tier's V rows as a 2-D tensor map for the attention's four-row
+// gathers: every unit's cap rows one after another (row u cap + j), D
+// elements a row, a box of one row. False (no map) unless the tier is laid
+// out exactly that way: rows of D contiguous elements, units back to back.
+static bool encode_vmap(const hkv_problem *p, const hkv_tier *t, CUtensorMap *m)
+{
+    const auto enc = tensor_map_encoder();
+    if (enc == nullptr || t == nullptr || t->v == nullptr || t->cap <= 0)
+        return false;
+    const int64_t D = p->D;
+    if (t->stride_t != D || t->stride_h != (int64_t)t->cap * D || t->stride_b != (int64_t)p->Hkv * t->cap * D)
+        return false;
+    const int64_t rows = (int64_t)p->B * p->Hkv * t->cap;
+    if (rows >= (1ll << 31) || (reinterpret_cast<uintptr_t>(t->v) & 15) != 0)
+        return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)(D * es_of(p->dtype))};
+    const cuuint32_t box[2] = {(cuuint32_t)D, 1};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, p->dtype == HKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+               const_cast<void *>(t->v), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static hkv_status check_tier(const hkv_tier *t, const hkv_problem *p, bool need_v)
 {
     if (t == nullptr)
@@ -1072,6 +1114,7 @@ hkv_status step_impl(const hkv_problem *prob, const void *q, const hkv_tier *den
     P.k_out = static_cast<char *>(o->k_out);
     P.v_out = static_cast<char *>(o->v_out);
     P.logit = reinterpret_cast<float *>(wsb + L.logits);  // scorer -> attention of the selected tokens
+    P.vmap_ok = encode_vmap(prob, sparse, &P.vmap) ? 1 : 0;  // four-row gathers of the selected V rows
     P.layout = HKV_LAYOUT_PAD_MAX;  // the three kernels work on PAD_MAX rows
     if (mti != nullptr) {
         P.mti_left = mti->left;

@@ -96,6 +96,11 @@ struct Params {
     // kernel timeline (hkv_set_timeline; nullptr when off): per kernel kind,
     // the complement of its earliest start and its latest end (global timer)
     unsigned long long *tl;
+    // hkv_step with a plainly laid out sparse tier (vmap_ok): its V rows as a
+    // 2-D tensor map (row u cap + j = token j of unit u, D elements, box one
+    // row high), for the attention's four-row TMA gathers of selected rows
+    int32_t vmap_ok;
+    CUtensorMap vmap;
 };
 
 // Kernel kinds of the timeline (index of their start word; the end word is 8 on).
@@ -214,7 +219,7 @@ struct Geo {
     // fuller stages: a warp's share of the selection is only a few stages long)
     static constexpr int VOFF_B = 32 * logit_floats(G) * 4;
     static constexpr int BTOK0 = (AT_SLOT - VOFF_B) / ROWB;
-    static constexpr int BTOK = BTOK0 < 32 ? BTOK0 : 32;
+    static constexpr int BTOK = (BTOK0 < 32 ? BTOK0 : 32) / 4 * 4;  // whole groups of four rows
     static constexpr int DPL = D / 32;                    // PV: head-dim elements per lane
     static_assert(G >= 1 && G <= LPR, "group size must not exceed lanes per row");
     static_assert(ATOK * G <= SC_FLOATS && ATOK <= 32, "stage sizes");
@@ -1178,10 +1183,39 @@ struct AttnJob {
             // in 16-byte cp.async chunks spread over the warp (random rows
             // stream faster this way than as one bulk copy per row)
             const char *vs = nullptr, *ls = nullptr;
+            int grow = 0;  // the lane's row on the V tensor map
             if (lane < d.count) {
                 const int jj = sparse_row(d);
                 vs = P.sparse.v + row_offset(P.sparse, b, h, jj);
                 ls = reinterpret_cast<const char *>(P.logit + ((int64_t)u * P.sparse.cap + jj) * logit_floats(G));
+                grow = u * P.sparse.cap + jj;
+            }
+            if (P.vmap_ok) {
+                // the logit records by cp.async (each lane's copies counted on
+                // the barrier first), then the V rows in groups of four by the
+                // TMA: lane i < ng gathers rows 4i .. 4i + 3, a short last group
+                // repeating its last row into the slack of the slot
+                if (lane < d.count)
+#pragma unroll
+                    for (int i = 0; i < LB / 16; ++i)
+                        cp_async16(dst + lane * LB + i * 16, ls + i * 16);
+                cp_async_arrive(bar);
+                __syncwarp();
+                const int ng = (d.count + 3) >> 2;
+                if (lane == 0)
+                    mbar_arrive_expect_tx(bar, (uint32_t)(ng * 4 * Gm::ROWB));
+                __syncwarp();
+                int r[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    r[k] = __shfl_sync(0xffffffffu, grow, min(4 * lane + k, max(d.count - 1, 0)) & 31);
+                if (lane < ng) {
+                    fence_proxy_async_smem();  // this lane's copy after the warp's reads of the slot
+                    tma_gather4(dst + Gm::VOFF_B + 4 * lane * Gm::ROWB, &P.vmap, r[0], r[1], r[2], r[3], bar);
+                }
+                __syncwarp();
+                prefetch_index(d);
+                return;
             }
             constexpr int CH = Gm::ROWB / 16;  // chunks of a V row
             static_assert(CH <= 32 && 32 % CH == 0, "row chunks");
