@@ -215,8 +215,9 @@ hkv_status hkv_cascade_decode(const hkv_problem *prob, const void *q,
  * indices into PAD_MAX rows; (3) a
  * persistent streaming kernel attends over the dense and condensed tokens
  * (before it waits for (2)) and over the selected tokens, whose rows it reads
- * through the indices ([TS 2.C] Sparse Loading) together with the scorer's
- * logits (so their K rows are not read again); (2) and (3) read the tiers'
+ * through the indices ([TS 2.C] Sparse Loading; four V rows per TMA gather
+ * when the sparse tier's rows are contiguous and its units back to back)
+ * together with the scorer's logits (so their K rows are not read again); (2) and (3) read the tiers'
  * lengths before their waits, so the lengths must be final when the call is
  * made (this library's append and condensation let no dependent start before
  * they end); (4) a merge kernel combines
