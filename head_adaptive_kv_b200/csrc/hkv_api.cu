@@ -346,8 +346,8 @@ __global__ void __launch_bounds__(NT, 1) k_unit(const __grid_constant__ Params P
     tl_start(P.tl, TL_UNIT);
     const float *zg = P.z + (int64_t)u * P.z_stride;
     // hkv_step: with the range known and every unit short enough to stage,
-    // the length and the range words are requested first, then the scores'
-    // copy into shared memory (which the loads would otherwise queue behind)
+    // the range words are requested first, then the scores' copy into shared
+    // memory (which the loads would otherwise queue behind)
     const bool early = P.have_range && P.do_select && P.do_compact && P.sparse.cap <= ZSTAGE &&
                        (reinterpret_cast<uintptr_t>(zg) & 15) == 0;
     uint32_t kmax = 0, kmin = 0;
@@ -607,29 +607,40 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
     return fn;
 }
 
-// The sparse tier's V rows as a 2-D tensor map for the attention's four-row
-// gathers: every unit's cap rows one after another (row u cap + j), D
-// elements a row, a box of one row. False (no map) unless the tier is laid
-// out exactly that way: rows of D contiguous elements, units back to back.
-static bool encode_vmap(const hkv_problem *p, const hkv_tier *t, CUtensorMap *m)
+// The sparse tier's K or V rows (rows_base: its k or v) as a 2-D tensor map
+// for the attention's four-row gathers: every unit's cap rows one after
+// another (row u cap + j), D elements a row, a box of one row. False (no map)
+// unless the tier is laid out exactly that way: rows of D contiguous
+// elements, units back to back.
+static bool encode_rows_map(const hkv_problem *p, const hkv_tier *t, const void *rows_base, CUtensorMap *m)
 {
     const auto enc = tensor_map_encoder();
-    if (enc == nullptr || t == nullptr || t->v == nullptr || t->cap <= 0)
+    if (enc == nullptr || t == nullptr || rows_base == nullptr || t->cap <= 0)
         return false;
     const int64_t D = p->D;
     if (t->stride_t != D || t->stride_h != (int64_t)t->cap * D || t->stride_b != (int64_t)p->Hkv * t->cap * D)
         return false;
     const int64_t rows = (int64_t)p->B * p->Hkv * t->cap;
-    if (rows >= (1ll << 31) || (reinterpret_cast<uintptr_t>(t->v) & 15) != 0)
+    if (rows >= (1ll << 31) || (reinterpret_cast<uintptr_t>(rows_base) & 15) != 0)
         return false;
     const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {(cuuint64_t)(D * es_of(p->dtype))};
     const cuuint32_t box[2] = {(cuuint32_t)D, 1};
     const cuuint32_t estr[2] = {1, 1};
     return enc(m, p->dtype == HKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
-               const_cast<void *>(t->v), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               const_cast<void *>(rows_base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The attention calls: both maps of the sparse tier, for four-row gathers of
+// the selected tokens' K and V rows (neither when either cannot be made).
+static void set_row_maps(const hkv_problem *p, const hkv_tier *sparse, Params &P)
+{
+    const bool ok = sparse != nullptr && encode_rows_map(p, sparse, sparse->k, &P.kmap) &&
+                    encode_rows_map(p, sparse, sparse->v, &P.vmap);
+    P.kmap_ok = ok ? 1 : 0;
+    P.vmap_ok = ok ? 1 : 0;
 }
 
 static hkv_status check_tier(const hkv_tier *t, const hkv_problem *p, bool need_v)
@@ -1114,7 +1125,7 @@ hkv_status step_impl(const hkv_problem *prob, const void *q, const hkv_tier *den
     P.k_out = static_cast<char *>(o->k_out);
     P.v_out = static_cast<char *>(o->v_out);
     P.logit = reinterpret_cast<float *>(wsb + L.logits);  // scorer -> attention of the selected tokens
-    P.vmap_ok = encode_vmap(prob, sparse, &P.vmap) ? 1 : 0;  // four-row gathers of the selected V rows
+    P.vmap_ok = encode_rows_map(prob, sparse, sparse->v, &P.vmap) ? 1 : 0;  // four-row gathers of selected V rows
     P.layout = HKV_LAYOUT_PAD_MAX;  // the three kernels work on PAD_MAX rows
     if (mti != nullptr) {
         P.mti_left = mti->left;
@@ -1433,6 +1444,7 @@ hkv_status hkv_cascade_decode(const hkv_problem *prob, const void *q, const hkv_
     P.sel_len = const_cast<int32_t *>(sel_len);
     P.out = out;
     P.lse = lse;
+    set_row_maps(prob, sparse, P);
     return dispatch<RunAttn>(prob, P, (cudaStream_t)stream, false);
 }
 
@@ -1605,6 +1617,7 @@ extern "C" hkv_status hkv_cascade_decode_noalloc(const hkv_problem *prob, const 
     // the status word must start at zero; the previous call may have left it set
     if (cudaMemsetAsync(base, 0, sizeof(uint32_t), st) != cudaSuccess)
         return HKV_ERR_CUDA;
+    set_row_maps(prob, sparse, P);
     if ((s = dispatch<RunAttn>(prob, P, st, false)) != HKV_OK)
         return s;
     if (status != nullptr &&

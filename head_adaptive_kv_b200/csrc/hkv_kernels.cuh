@@ -96,11 +96,13 @@ struct Params {
     // kernel timeline (hkv_set_timeline; nullptr when off): per kernel kind,
     // the complement of its earliest start and its latest end (global timer)
     unsigned long long *tl;
-    // hkv_step with a plainly laid out sparse tier (vmap_ok): its V rows as a
-    // 2-D tensor map (row u cap + j = token j of unit u, D elements, box one
-    // row high), for the attention's four-row TMA gathers of selected rows
-    int32_t vmap_ok;
-    CUtensorMap vmap;
+    // a plainly laid out sparse tier: its V rows (vmap_ok; hkv_step and the
+    // attention calls) and K rows (kmap_ok; the attention calls, which gather
+    // both) as 2-D tensor maps (row u cap + j = token j of unit u, D elements,
+    // box one row high), for the attention's four-row TMA gathers of selected
+    // rows
+    int32_t vmap_ok, kmap_ok;
+    CUtensorMap vmap, kmap;
 };
 
 // Kernel kinds of the timeline (index of their start word; the end word is 8 on).
@@ -225,6 +227,7 @@ struct Geo {
     static_assert(ATOK * G <= SC_FLOATS && ATOK <= 32, "stage sizes");
     static_assert(ATOK * logit_floats(G) * 4 <= AT_SLOT / 2, "logit records of a stage");
     static_assert(BTOK * G <= SC_FLOATS && BTOK >= ATOK && VOFF_B % 16 == 0, "stages of selected tokens");
+    static_assert(ATOK % 4 == 0, "K and V stages in whole groups of four rows");
     static_assert(SITERS % NB == 0 && AITERS % NB == 0 && LPR % NV == 0, "iteration batches");
 };
 
@@ -1236,6 +1239,31 @@ struct AttnJob {
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(bar);
+            prefetch_index(d);
+            return;
+        }
+        if (lineb && P.kmap_ok && P.vmap_ok) {
+            // selected tokens' K and V rows in groups of four by the TMA, after
+            // lane 0 has armed the slot for all of them: lane i < ng gathers
+            // rows 4i .. 4i + 3 of both maps (a short last group repeats its
+            // last row; a stage holds at most ATOK rows, a multiple of four)
+            int grow = 0;
+            if (lane < d.count)
+                grow = u * P.sparse.cap + sparse_row(d);
+            const int ng = (d.count + 3) >> 2;
+            if (lane == 0)
+                mbar_arrive_expect_tx(bar, (uint32_t)(ng * 4 * 2 * Gm::ROWB));
+            __syncwarp();
+            int r[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                r[k] = __shfl_sync(0xffffffffu, grow, min(4 * lane + k, max(d.count - 1, 0)) & 31);
+            if (lane < ng) {
+                fence_proxy_async_smem();  // this lane's copies after the warp's reads of the slot
+                tma_gather4(dst + 4 * lane * Gm::ROWB, &P.kmap, r[0], r[1], r[2], r[3], bar);
+                tma_gather4(dst + AT_SLOT / 2 + 4 * lane * Gm::ROWB, &P.vmap, r[0], r[1], r[2], r[3], bar);
+            }
+            __syncwarp();
             prefetch_index(d);
             return;
         }
