@@ -987,6 +987,7 @@ namespace hkv {
 
 constexpr int MTI_CTAS = 4;
 constexpr int MTI_NT = 256;
+constexpr int MTI_BATCH = 8;  // rewrite copy: 16-byte chunks a thread has in flight
 
 struct MtiP {
     const char *sk, *sv;                   // sparse tier
@@ -1026,20 +1027,36 @@ __global__ void __cluster_dims__(MTI_CTAS, 1, 1) __launch_bounds__(MTI_NT) k_mti
         const int i0 = k * r / MTI_CTAS, i1 = k * (r + 1) / MTI_CTAS;
         const int ch = M.rowb / 16;
         const int32_t *row = M.idx + (int64_t)u * M.bmax;
-        for (int x = threadIdx.x; x < (i1 - i0) * 2 * ch; x += MTI_NT) {
-            const int i = i0 + x / (2 * ch), q = x % (2 * ch);
-            const bool isk = q < ch;
-            int j = __ldcg(row + i);
-            if (j < 0 || j >= n) {
-                atomicOr(M.status, HKV_DEV_BAD_INDEX);
-                j = 0;
+        // MTI_BATCH chunks a thread, all loads in flight before the stores
+        const int total = (i1 - i0) * 2 * ch;
+        for (int x0 = threadIdx.x; x0 < total; x0 += MTI_NT * MTI_BATCH) {
+            uint4 val[MTI_BATCH];
+            char *dst[MTI_BATCH];
+#pragma unroll
+            for (int e = 0; e < MTI_BATCH; ++e) {
+                const int x = x0 + e * MTI_NT;
+                dst[e] = nullptr;
+                if (x >= total)
+                    continue;
+                const int i = i0 + x / (2 * ch), q = x % (2 * ch);
+                const bool isk = q < ch;
+                const int j0 = __ldcg(row + i);
+                int j = j0;
+                if (j < 0 || j >= n) {
+                    atomicOr(M.status, HKV_DEV_BAD_INDEX);
+                    j = 0;
+                }
+                const char *src = (isk ? M.sk : M.sv) + (int64_t)b * M.ssb + (int64_t)h * M.ssh + (int64_t)j * M.sst;
+                const int off = (isk ? q : q - ch) * 16;
+                val[e] = __ldcs(reinterpret_cast<const uint4 *>(src + off));
+                dst[e] = (isk ? M.rk : M.rv) + (int64_t)b * M.rsb + (int64_t)h * M.rsh + (int64_t)i * M.rst + off;
+                if (q == 0)
+                    M.rw_idx[(int64_t)u * M.bmax + i] = j0;
             }
-            const char *src = (isk ? M.sk : M.sv) + (int64_t)b * M.ssb + (int64_t)h * M.ssh + (int64_t)j * M.sst;
-            char *dst = (isk ? M.rk : M.rv) + (int64_t)b * M.rsb + (int64_t)h * M.rsh + (int64_t)i * M.rst;
-            const int off = (isk ? q : q - ch) * 16;
-            *reinterpret_cast<uint4 *>(dst + off) = __ldcs(reinterpret_cast<const uint4 *>(src + off));
-            if (q == 0)
-                M.rw_idx[(int64_t)u * M.bmax + i] = __ldcg(row + i);
+#pragma unroll
+            for (int e = 0; e < MTI_BATCH; ++e)
+                if (dst[e] != nullptr)
+                    *reinterpret_cast<uint4 *>(dst[e]) = val[e];
         }
     }
     cluster.sync();
